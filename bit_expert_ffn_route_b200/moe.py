@@ -1,0 +1,176 @@
+"""Thin ctypes binding of ``libmoe.so`` (include/moe.h).
+
+Argument marshalling only: every step of the expert pass runs in the CUDA
+library.  Tensors are torch CUDA tensors; their device pointers and the current
+stream are passed straight through.  Loading fails loudly when the library is
+missing — there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import synth
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+MOE_Q2_32, MOE_Q3_32, MOE_Q3_S256 = 0, 1, 2
+
+EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_size", "moe_workspace_size",
+           "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
+           "moe_status_string"]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({_lib_status_string(status)})")
+
+
+class moe_pool(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("n_slots", ctypes.c_int32), ("shared_slot", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("slot_stride_codes", ctypes.c_uint64), ("slot_stride_scales", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libmoe.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m bit_expert_ffn_route_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        for name in ("moe_slot_code_bytes", "moe_slot_scale_bytes"):
+            getattr(L, name).restype = sz
+            getattr(L, name).argtypes = [i, i, i]
+        L.moe_route_workspace_size.restype = sz
+        L.moe_route_workspace_size.argtypes = [i, i, i, i]
+        L.moe_workspace_size.restype = sz
+        L.moe_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.moe_expert_out_size.restype = sz
+        L.moe_expert_out_size.argtypes = [i, i, i]
+        L.moe_route_topk.restype = i
+        L.moe_route_topk.argtypes = [P, i, i, P, P, i, i, P, P, P, P, sz, P]
+        L.moe_expert_forward.restype = i
+        L.moe_expert_forward.argtypes = [ctypes.POINTER(moe_pool), P, i, P, i, P, i, P, sz, P, P, P, sz, P]
+        L.moe_combine.restype = i
+        L.moe_combine.argtypes = [P, P, i, i, i, P, P, P, P]
+        L.moe_dequantize.restype = i
+        L.moe_dequantize.argtypes = [ctypes.POINTER(moe_pool), i, i, P, P]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_status_string.argtypes = [i]
+        _lib = L
+    return _lib
+
+
+def _lib_status_string(s):
+    try:
+        return lib().moe_status_string(int(s)).decode()
+    except Exception:
+        return "?"
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, st):
+    if st != MOE_OK:
+        raise MoeError(fn, st)
+
+
+def make_pool(pool: synth.PoolData, shared_slot: int) -> moe_pool:
+    return moe_pool(pool.fmt, pool.d_model, pool.d_ff, pool.n_slots, int(shared_slot), 0,
+                    pool.codes.data_ptr(), pool.scales.data_ptr(), pool.stride_codes, pool.stride_scales)
+
+
+def route_workspace_size(T, D, E, k) -> int:
+    return int(lib().moe_route_workspace_size(T, D, E, k))
+
+
+def workspace_size(T, D, F, E, k, fmt) -> int:
+    return int(lib().moe_workspace_size(T, D, F, E, k, fmt))
+
+
+def expert_out_size(T, D, k) -> int:
+    return int(lib().moe_expert_out_size(T, D, k))
+
+
+def alloc_ws(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled, 256-byte aligned device scratch buffer."""
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def moe_route_topk(x, Wr, bias, k, ids, gates, ws, logits=None, stream=None):
+    T, D = x.shape
+    E = Wr.shape[0]
+    st = lib().moe_route_topk(_p(x), T, D, _p(Wr), _p(bias), E, k, _p(ids), _p(gates), _p(logits),
+                              _p(ws), ws.numel(), _stream(stream))
+    _check("moe_route_topk", st)
+
+
+def moe_expert_forward(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_list, miss_count, ws, stream=None):
+    T = x.shape[0]
+    E = slot_table.shape[0]
+    st = lib().moe_expert_forward(ctypes.byref(pool), _p(slot_table), E, _p(x), T, _p(ids), k,
+                                  _p(expert_out), expert_out.numel(), _p(miss_list), _p(miss_count),
+                                  _p(ws), ws.numel(), _stream(stream))
+    _check("moe_expert_forward", st)
+
+
+def moe_combine(expert_out, gates, T, D, k, out, miss_partial=None, residual=None, stream=None):
+    st = lib().moe_combine(_p(expert_out), _p(gates), T, D, k, _p(miss_partial), _p(residual), _p(out),
+                           _stream(stream))
+    _check("moe_combine", st)
+
+
+def moe_dequantize(pool: moe_pool, slot, matrix, out, stream=None):
+    _check("moe_dequantize", lib().moe_dequantize(ctypes.byref(pool), slot, matrix, _p(out), _stream(stream)))
+
+
+class Layer:
+    """Buffers and calls for one MoE layer at a fixed token count: the three
+    C-ABI calls in order on one stream.  Buffers are allocated once here (the
+    library itself never allocates)."""
+
+    def __init__(self, pool: synth.PoolData, shared_slot, slot_table, Wr, bias, k, T, device="cuda"):
+        self.pool_data = pool
+        self.pool = make_pool(pool, shared_slot)
+        self.slot_table, self.Wr, self.bias, self.k, self.T = slot_table, Wr, bias, k, T
+        D, E = Wr.shape[1], Wr.shape[0]
+        self.D, self.E = D, E
+        self.ids = torch.empty(T, k, dtype=torch.int32, device=device)
+        self.gates = torch.empty(T, k, dtype=torch.float32, device=device)
+        self.logits = torch.empty(T, E, dtype=torch.float32, device=device)
+        self.route_ws = alloc_ws(route_workspace_size(T, D, E, k), device)
+        self.ws = alloc_ws(workspace_size(T, D, pool.d_ff, E, k, pool.fmt), device)
+        self.expert_out = alloc_ws(expert_out_size(T, D, k), device)
+        self.miss_list = torch.empty(max(T * k, 1), 3, dtype=torch.int32, device=device)
+        self.miss_count = torch.zeros(1, dtype=torch.int32, device=device)
+        self.out = torch.empty(T, D, dtype=torch.bfloat16, device=device)
+
+    def __call__(self, x, miss_partial=None, residual=None, out=None, stream=None, with_logits=False):
+        out = self.out if out is None else out
+        moe_route_topk(x, self.Wr, self.bias, self.k, self.ids, self.gates, self.route_ws,
+                       logits=self.logits if with_logits else None, stream=stream)
+        moe_expert_forward(self.pool, self.slot_table, x, self.ids, self.k, self.expert_out, self.miss_list,
+                           self.miss_count, self.ws, stream=stream)
+        moe_combine(self.expert_out, self.gates, x.shape[0], self.D, self.k, out, miss_partial=miss_partial,
+                    residual=residual, stream=stream)
+        return out

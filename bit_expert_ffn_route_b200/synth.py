@@ -10,10 +10,13 @@ ours and is stated here:
 * router weights ``Wr``: bf16 of N(0, 0.02);
 * router bias (optional): ``b[e] = -alpha * s * ln(rank(e))`` where ``rank`` is a
   seeded permutation of 1..E (a Zipf(s) popularity prior, strength ``alpha``);
+* weights of zero mean and standard deviation ~``weight_std`` (default 0.02):
 * Q2_32 / Q3_32 codes: uniform random bytes (so every code is uniform);
-  ``s = fp16(0.02 * (0.5 + U))``, ``m = fp16(-1.5 s)`` (Q2) or ``fp16(-3.5 s)`` (Q3);
+  ``s = fp16(c * (0.5 + U))`` with ``c = weight_std / sqrt(1.25)`` (Q2, codes 0..3)
+  or ``weight_std / sqrt(5.25)`` (Q3, codes 0..7); ``m = fp16(-1.5 s)`` (Q2) or
+  ``fp16(-3.5 s)`` (Q3), centring the codes;
 * Q3_S256 codes and 6-bit sub-scales: uniform random bytes;
-  ``d = fp16(4.6e-4 * (0.5 + U))`` (weights of std ~0.02).
+  ``d = fp16(weight_std / 43.3 * (0.5 + U))`` (43.3 = rms of (sc - 32)(q - 4)).
 
 Layout of one slot (bytes, each region 256-byte padded):
   codes : gate plane [F][D/bw][cb] | up plane [F][D/bw][cb] | down plane [D][F/bw][cb]
@@ -119,7 +122,7 @@ def _random_bytes(n: int, g: torch.Generator, device) -> torch.Tensor:
 
 
 def make_pool(fmt: int, D: int, F: int, n_slots: int, seed: int, device="cpu",
-              pool_id: int = 0, chunk_slots: int = 512) -> PoolData:
+              pool_id: int = 0, chunk_slots: int = 512, weight_std: float = 0.02) -> PoolData:
     """Generate ``n_slots`` experts in the pool format (see module docstring)."""
     cb = slot_code_bytes(fmt, D, F)
     sb = slot_scale_bytes(fmt, D, F)
@@ -137,11 +140,12 @@ def make_pool(fmt: int, D: int, F: int, n_slots: int, seed: int, device="cpu",
         u = torch.rand(n, n_blocks, generator=g, device=device, dtype=torch.float32)
         if fmt == Q3_S256:
             sc = _random_bytes(n * n_blocks * 12, g, device).view(n, n_blocks * 12)
-            d = (4.6e-4 * (0.5 + u)).to(torch.float16)
+            d = (weight_std / 43.3 * (0.5 + u)).to(torch.float16)
             sv[c0:c1, :n_blocks * 12] = sc
             sv[c0:c1, n_blocks * 12:n_blocks * 14] = d.view(torch.uint8).view(n, n_blocks * 2)
         else:
-            s = (0.02 * (0.5 + u)).to(torch.float16)
+            c = weight_std / (1.25 ** 0.5 if fmt == Q2_32 else 5.25 ** 0.5)
+            s = (c * (0.5 + u)).to(torch.float16)
             m = (-(1.5 if fmt == Q2_32 else 3.5) * s.float()).to(torch.float16)
             sm = torch.stack([s, m], dim=-1)            # s at the lower address
             sv[c0:c1, :sb] = sm.view(torch.uint8).view(n, sb)

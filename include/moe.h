@@ -1,0 +1,202 @@
+/*
+ * moe.h — C ABI of the B200 routed-MoE expert pass.
+ *
+ * One MoE layer of a 512-expert, top-10 + 1-shared model, split in three
+ * calls that the caller chains on one CUDA stream:
+ *
+ *   moe_route_topk      router logits, top-k expert ids and gates
+ *   moe_expert_forward  expert-cache slot lookup (miss list out), then the
+ *                       SwiGLU FFNs of every resident selected expert and of
+ *                       the shared expert, over 2-/3-bit block-quantised
+ *                       weights dequantised on the fly
+ *   moe_combine         gate-weighted sum of the expert outputs + shared
+ *                       expert (+ caller's partial for the misses) (+ residual)
+ *
+ * Sources: 512 routed experts per layer, 10 routed + 1 shared per token
+ * (wiselychen RTX 5090 report, "30 秒定位"; greenbean-ai "Strata 如何讓 12GB
+ * 顯卡跑 Qwen3.8-Flash-Next", §一).  The GPU runs the routing and the shared
+ * expert, hot experts live in a VRAM cache and misses are computed elsewhere
+ * (greenbean-ai §二; wiselychen report §2 "專家快取與 CPU／GPU 分工").  Weights
+ * are 2-3.5 bit block-quantised (wiselychen report §1; greenbean-ai §四).
+ * The SwiGLU form, the block layouts, the router normalisation and every
+ * other detail the pages leave open are readings, stated at each declaration.
+ *
+ * Conventions for every call:
+ *  - Pointers named x, Wr, ids, gates, logits, slot_table, expert_out,
+ *    miss_list, miss_count, miss_partial, residual, out, ws and the pool's
+ *    codes/scales are DEVICE pointers; the caller allocates and owns them.
+ *    The library never allocates, frees or synchronises.
+ *  - bf16 and fp16 values are passed as uint16_t bit patterns.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *    Argument and shape errors are returned synchronously and launch nothing;
+ *    a failed launch returns MOE_ERR_CUDA.
+ *  - Results are deterministic: no floating-point atomics, fixed summation
+ *    orders; two identical calls give identical bits.
+ *  - T == 0 is valid and launches nothing (miss_count is still zeroed).
+ *  - Path: T <= 4 is the decode path (1 token + up to 3 draft tokens);
+ *    T > 4 is the prefill path.  Both compute the same function.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Identical to cudaStream_t. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,   /* null pointer, bad size, misaligned pointer */
+    MOE_ERR_UNSUPPORTED = -2,   /* shape outside the limits below */
+    MOE_ERR_WORKSPACE = -3,     /* ws / expert_out smaller than the size query */
+    MOE_ERR_CUDA = -4,          /* a CUDA call or launch failed */
+    MOE_ERR_TIMEOUT = -5        /* a bounded device-side wait gave up */
+} moe_status;
+
+/*
+ * Block formats (reading; the pages name Q2_0, IQ2_XS, IQ3_XXS ~3.06 bpw and
+ * IQ3_S ~3.44 bpw without defining them).  Blocks run along the reduction
+ * dimension K of every matrix.
+ *   MOE_Q2_32  : 32 weights/block; 8 code bytes, weight j = bits [2j,2j+2) of
+ *                the block's little-endian bit stream; fp16 s, fp16 m;
+ *                w = fmaf(s, q, m).                        3.0 bits/weight
+ *   MOE_Q3_32  : as Q2_32 with 12 code bytes, weight j = bits [3j,3j+3).
+ *                                                          4.0 bits/weight
+ *   MOE_Q3_S256: 256 weights/super-block; 96 code bytes, weight i = bits
+ *                [3i,3i+3); 12 bytes of 6-bit sub-scales sc_j, j = 0..15, one
+ *                per 16 weights, sub-block j = bits [6j,6j+6); fp16 d;
+ *                w = d * (sc_j - 32) * (q - 4).            3.4375 bits/weight
+ */
+typedef enum moe_qformat { MOE_Q2_32 = 0, MOE_Q3_32 = 1, MOE_Q3_S256 = 2 } moe_qformat;
+
+/*
+ * A slot-mapped pool of quantised experts in device memory (the VRAM expert
+ * cache of the wiselychen report §2).  Every slot holds one expert: gate Wg
+ * [d_ff x d_model], up Wu [d_ff x d_model], down Wd [d_model x d_ff].
+ *   codes  + s*slot_stride_codes : code planes gate | up | down, each row-major
+ *                                  [rows][K/bw blocks][code bytes per block]
+ *   scales + s*slot_stride_scales: Q2_32/Q3_32: (s, m) fp16 pairs (s first),
+ *                                  planes gate | up | down, same block order;
+ *                                  Q3_S256: 12-byte sub-scale planes gate | up |
+ *                                  down, then fp16 d planes gate | up | down.
+ * Strides are multiples of 256 bytes and at least moe_slot_code_bytes /
+ * moe_slot_scale_bytes; codes and scales are 256-byte aligned.  shared_slot
+ * is the always-resident shared expert of this layer.
+ */
+typedef struct moe_pool {
+    int32_t fmt;          /* moe_qformat */
+    int32_t d_model;      /* D */
+    int32_t d_ff;         /* F */
+    int32_t n_slots;
+    int32_t shared_slot;
+    int32_t reserved;     /* must be 0 */
+    const void* codes;
+    const void* scales;
+    uint64_t slot_stride_codes;
+    uint64_t slot_stride_scales;
+} moe_pool;
+
+/*
+ * Shape limits (MOE_ERR_UNSUPPORTED otherwise):
+ *   D % 256 == 0, 256 <= D <= 8192;  F % 128 == 0, 128 <= F <= 4096 (Q3_S256:
+ *   F % 256 == 0);  1 <= k <= 16;  k <= E <= 1024;  0 <= T <= 65536.
+ */
+
+/* Bytes of one slot's codes / scale data (unpadded). */
+size_t moe_slot_code_bytes(int fmt, int d_model, int d_ff);
+size_t moe_slot_scale_bytes(int fmt, int d_model, int d_ff);
+
+/* Workspace bytes for moe_route_topk / moe_expert_forward at these shapes. */
+size_t moe_route_workspace_size(int T, int D, int E, int k);
+size_t moe_workspace_size(int T, int D, int F, int E, int k, int fmt);
+/* Bytes of the expert_out buffer moe_expert_forward fills and moe_combine reads. */
+size_t moe_expert_out_size(int T, int D, int k);
+
+/*
+ * Router logits, top-k and gates (greenbean-ai §二: routing runs on the GPU;
+ * wiselychen report "30 秒定位": top-10 of 512).
+ *   x      bf16 [T][D] row-major, 16-byte aligned
+ *   Wr     bf16 [E][D] row-major, 16-byte aligned
+ *   bias   fp32 [E] or NULL (added to the logits before selection)
+ *   ids    int32 [T][k] out: expert ids in rank order (larger logit first,
+ *          equal logits: lower id first)
+ *   gates  fp32 [T][k] out: exp(l_r - l_0) / sum_{r'<k} exp(l_r' - l_0)
+ *          (reading: softmax restricted to the selected experts; sums to 1)
+ *   logits fp32 [T][E] out, or NULL.  Decode path: the canonical-order
+ *          values below.  Prefill path: tensor-core values within the bound
+ *          |l - canonical| <= 2^-18 * D * |x_t|_2 * |Wr_e|_2.
+ *   ws     device scratch of moe_route_workspace_size bytes, 256-byte
+ *          aligned.  Its first 4 bytes must be zero before the first call
+ *          with this buffer (e.g. zero it once at allocation); every completed
+ *          call leaves them zero.  Calls sharing one ws must not overlap on
+ *          the device.
+ * The selection and the gates use logits in a canonical fp32 order: 32
+ * partial sums, lane L accumulating fmaf over elements 256c + 8L + j (c
+ * ascending, j = 0..7), then added pairwise (L with L+16, then +8, +4, +2,
+ * +1), then + bias.  The ids are therefore reproducible bit for bit.
+ */
+moe_status moe_route_topk(const uint16_t* x, int T, int D, const uint16_t* Wr,
+                          const float* bias, int E, int k, int32_t* ids, float* gates,
+                          float* logits, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Slot lookup, miss list and expert FFNs.
+ *   slot_table int32 [E]: expert id -> slot, -1 = not resident.  Any entry
+ *          outside [0, n_slots) is treated as a miss.
+ *   x      bf16 [T][D];  ids int32 [T][k] (from moe_route_topk or the caller;
+ *          an id outside [0, E) is treated as a miss)
+ *   expert_out   device buffer of moe_expert_out_size(T, D, k) bytes, 256-byte
+ *          aligned: filled with one output row per (token, rank) hit and one
+ *          per token for the shared expert, plus the row map moe_combine reads.
+ *          Opaque to the caller.
+ *   miss_list    int32 [T*k][3] out: (token, rank, expert) per miss, token-major
+ *          then rank order (wiselychen report §2: misses go to the CPU, which
+ *          computes them in place; here they are returned to the caller)
+ *   miss_count   int32 [1] out
+ *   ws     scratch of moe_workspace_size bytes, 256-byte aligned, contents
+ *          need not be initialised.
+ * Per expert (reading; the pages do not give the FFN form):
+ *   h = bf16( silu(Wg x) * (Wu x) ),  y = Wd h,  fp32 accumulation.
+ * Missed experts are not computed.
+ */
+moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, int E,
+                              const uint16_t* x, int T, const int32_t* ids, int k,
+                              void* expert_out, size_t expert_out_bytes,
+                              int32_t* miss_list, int32_t* miss_count,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Gate-weighted combine:
+ *   out[t] = bf16( sum_{r<k, hit} gates[t][r] * y[t][r] + y_shared[t]
+ *                  (+ miss_partial[t]) (+ residual[t]) )
+ * summed in that order in fp32.  Gates are not renormalised over the hits
+ * (reading: the caller adds the missed experts' contribution through
+ * miss_partial, e.g. from a CPU pass over miss_list).
+ *   expert_out   as filled by moe_expert_forward with the same T, D, k
+ *   gates  fp32 [T][k];  miss_partial fp32 [T][D] or NULL;
+ *   residual     bf16 [T][D] or NULL;  out bf16 [T][D] (may alias residual)
+ */
+moe_status moe_combine(const void* expert_out, const float* gates, int T, int D, int k,
+                       const float* miss_partial, const uint16_t* residual,
+                       uint16_t* out, moe_stream_t stream);
+
+/*
+ * Test hook: dequantise one matrix of one slot to fp32, row-major
+ * (matrix 0 = gate [F][D], 1 = up [F][D], 2 = down [D][F]).  Exact:
+ * Q2_32/Q3_32 w = fmaf(s, q, m); Q3_S256 w = d*(sc-32)*(q-4).
+ */
+moe_status moe_dequantize(const moe_pool* pool, int slot, int matrix, float* out,
+                          moe_stream_t stream);
+
+/* Static text for a status code. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

@@ -350,32 +350,36 @@ int orc_moe_layer(const orc_pool* P, const int32_t* slot_table, int E, int k,
     int n_miss = (rc == 0) ? orc_slot_lookup(ids, T, k, slot_table, E, P->n_slots, slots, miss_list) : -1;
     if (rc != 0 || n_miss < 0) { free(logits); free(ids); free(gates); free(slots); return -1; }
 
+    /* Every (token, rank) hit and every token's shared expert is evaluated on
+     * its own (independently, in parallel); the sum per token then runs in the
+     * fixed order: ranks ascending, shared, miss_partial, residual. */
     int failed = 0;
+    const int per_tok = k + 1;
+    double* ys = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * per_tok * D);
+    if (!ys) { free(logits); free(ids); free(gates); free(slots); return -1; }
 #ifdef _OPENMP
     int nt = n_threads > 0 ? n_threads : 1;
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nt) reduction(+ : failed)
 #endif
-    for (int t = 0; t < T; ++t) {
-        double* acc = (double*)calloc((size_t)D, sizeof(double));
-        double* y = (double*)malloc(sizeof(double) * (size_t)D);
-        if (!acc || !y) { free(acc); free(y); failed += 1; continue; }
-        const uint16_t* xt = x + (size_t)t * D;
-        for (int r = 0; r < k; ++r) {
-            int s = slots[(size_t)t * k + r];
-            if (s < 0) continue;
-            if (orc_expert(P, s, xt, NULL, y) != 0) { failed += 1; break; }
-            double g = gates[(size_t)t * k + r];
-            for (int d = 0; d < D; ++d) acc[d] += g * y[d];
-        }
-        if (orc_expert(P, P->shared_slot, xt, NULL, y) != 0) failed += 1;
+    for (int pr = 0; pr < T * per_tok; ++pr) {
+        int t = pr / per_tok, r = pr % per_tok;
+        int s = (r < k) ? slots[(size_t)t * k + r] : P->shared_slot;
+        if (s < 0) continue;
+        if (orc_expert(P, s, x + (size_t)t * D, NULL, ys + (size_t)pr * D) != 0) failed += 1;
+    }
+    for (int t = 0; t < T && !failed; ++t) {
         for (int d = 0; d < D; ++d) {
-            double v = acc[d] + y[d];
+            double v = 0.0;
+            for (int r = 0; r < k; ++r)
+                if (slots[(size_t)t * k + r] >= 0)
+                    v += gates[(size_t)t * k + r] * ys[((size_t)t * per_tok + r) * D + d];
+            v += ys[((size_t)t * per_tok + k) * D + d];
             if (miss_partial) v += (double)miss_partial[(size_t)t * D + d];
             if (residual) v += (double)bf16_to_f32(residual[(size_t)t * D + d]);
             out[(size_t)t * D + d] = orc_bf16_rne(v);
         }
-        free(acc); free(y);
     }
+    free(ys);
     (void)n_threads;
     if (logits_out) memcpy(logits_out, logits, sizeof(float) * (size_t)T * E);
     if (ids_out) memcpy(ids_out, ids, sizeof(int32_t) * (size_t)T * k);

@@ -1,0 +1,112 @@
+"""The C-ABI library loads and exports every symbol include/moe.h declares;
+size queries and argument checks behave as documented (no GPU needed: these
+calls return before touching the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from bit_expert_ffn_route_b200 import build, moe, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return moe.lib()
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(moe.EXPORTS)
+
+
+@pytest.mark.parametrize("fmt", [synth.Q2_32, synth.Q3_32, synth.Q3_S256])
+def test_slot_sizes_agree(L, fmt):
+    for D, F in [(3072, 512), (256, 256)]:
+        assert L.moe_slot_code_bytes(fmt, D, F) == synth.slot_code_bytes(fmt, D, F) == oracle.slot_code_bytes(fmt, D, F)
+        assert L.moe_slot_scale_bytes(fmt, D, F) == synth.slot_scale_bytes(fmt, D, F) == oracle.slot_scale_bytes(fmt, D, F)
+    assert L.moe_slot_code_bytes(7, 3072, 512) == 0
+
+
+def test_size_queries(L):
+    assert L.moe_expert_out_size(4, 3072, 10) >= 4 * 11 * 3072 * 4
+    assert L.moe_route_workspace_size(4, 3072, 512, 10) >= 256
+    assert L.moe_workspace_size(4, 3072, 512, 512, 10, 0) > 0
+    assert L.moe_workspace_size(4, 3000, 512, 512, 10, 0) == 0      # D % 256 != 0
+    assert L.moe_route_workspace_size(4, 3072, 512, 17) == 0        # k > 16
+
+
+def test_status_strings(L):
+    for s in (0, -1, -2, -3, -4, -5):
+        assert L.moe_status_string(s)
+
+
+def _fake(addr=1 << 20):
+    return ctypes.c_void_p(addr)
+
+
+def test_route_argument_errors(L):
+    f = _fake()
+    # shape errors first
+    assert L.moe_route_topk(f, 4, 3000, f, None, 512, 10, f, f, None, f, 1 << 20, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_route_topk(f, 4, 3072, f, None, 512, 0, f, f, None, f, 1 << 20, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route_topk(f, 4, 3072, f, None, 8, 10, f, f, None, f, 1 << 20, None) == moe.MOE_ERR_UNSUPPORTED
+    # null / misaligned pointers
+    assert L.moe_route_topk(None, 4, 3072, f, None, 512, 10, f, f, None, f, 1 << 20, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route_topk(_fake((1 << 20) + 2), 4, 3072, f, None, 512, 10, f, f, None, f, 1 << 20, None) == moe.MOE_ERR_INVALID_ARG
+    # workspace too small
+    assert L.moe_route_topk(f, 4, 3072, f, None, 512, 10, f, f, None, f, 16, None) == moe.MOE_ERR_WORKSPACE
+    # T == 0 is a no-op
+    assert L.moe_route_topk(None, 0, 3072, None, None, 512, 10, None, None, None, None, 0, None) == moe.MOE_OK
+
+
+def _pool(fmt=0, D=3072, F=512, n=4, shared=0, stride_c=None, stride_s=None):
+    f = fmt if fmt in (0, 1, 2) else 0
+    sc = stride_c if stride_c is not None else -(-synth.slot_code_bytes(f, D, F) // 256) * 256
+    ss = stride_s if stride_s is not None else -(-synth.slot_scale_bytes(f, D, F) // 256) * 256
+    return moe.moe_pool(fmt, D, F, n, shared, 0, 1 << 30, 1 << 31, sc, ss)
+
+
+def test_forward_argument_errors(L):
+    f = _fake()
+    fw = lambda pool, T=4, E=512, k=10, eo=1 << 30, ws=1 << 30: L.moe_expert_forward(
+        ctypes.byref(pool), f, E, f, T, f, k, f, eo, f, f, f, ws, None)
+    assert fw(_pool(fmt=5)) == moe.MOE_ERR_INVALID_ARG
+    assert fw(_pool(shared=4)) == moe.MOE_ERR_INVALID_ARG
+    assert fw(_pool(D=3000)) == moe.MOE_ERR_UNSUPPORTED
+    assert fw(_pool(F=200)) == moe.MOE_ERR_UNSUPPORTED
+    assert fw(_pool(fmt=2, F=384)) == moe.MOE_ERR_UNSUPPORTED
+    assert fw(_pool(stride_c=256)) == moe.MOE_ERR_INVALID_ARG          # stride below slot size
+    assert fw(_pool(stride_c=1769472 + 8)) == moe.MOE_ERR_INVALID_ARG  # not a multiple of 256
+    assert fw(_pool(), k=17) == moe.MOE_ERR_UNSUPPORTED
+    assert fw(_pool(), eo=16) == moe.MOE_ERR_WORKSPACE
+    assert fw(_pool(), ws=16) == moe.MOE_ERR_WORKSPACE
+    bad = _pool()
+    bad.reserved = 1
+    assert fw(bad) == moe.MOE_ERR_INVALID_ARG
+    # null miss_count
+    assert L.moe_expert_forward(ctypes.byref(_pool()), f, 512, f, 4, f, 10, f, 1 << 30, f, None, f, 1 << 30,
+                                None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_combine_and_dequant_argument_errors(L):
+    f = _fake()
+    assert L.moe_combine(f, f, 4, 3000, 10, None, None, f, None) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_combine(None, f, 4, 3072, 10, None, None, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(f, f, -1, 3072, 10, None, None, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(None, None, 0, 3072, 10, None, None, None, None) == moe.MOE_OK
+    assert L.moe_dequantize(ctypes.byref(_pool()), 4, 0, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_dequantize(ctypes.byref(_pool()), 0, 3, f, None) == moe.MOE_ERR_INVALID_ARG
