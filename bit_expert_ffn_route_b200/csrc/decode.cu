@@ -10,23 +10,25 @@
 // Work: "pairs" q = t*k + r (token t's rank-r expert) plus the shared expert.
 // The first pair of each distinct resident slot "owns" that expert and serves
 // every token that selected it, so each expert's bytes are read once.
-// Kernel 1 (gate|up) writes h = bf16(silu(Wg x) * (Wu x)); kernel 2 (down)
+// Phase 1 (gate|up) writes h = bf16(silu(Wg x) * (Wu x)); phase 2 (down)
 // writes y = Wd h as fp32 rows of expert_out.
 //
-// Both kernels are persistent (one CTA per SM): a producer warp streams work
-// items (a block of matrix rows of one expert: codes + scales, contiguous in
-// the pool) into a ring of shared-memory stages with bulk copies (TMA),
-// completing on mbarriers; eight consumer warps compute from shared memory.
-// Programmatic dependent launch lets kernel 2 start, resolve its work and
-// prefetch its weights while kernel 1 finishes.
+// One persistent kernel (one CTA per SM) runs both phases: a producer warp
+// streams work items (a block of matrix rows of one expert: codes + scales,
+// contiguous in the pool) into a ring of shared-memory stages with bulk copies
+// (TMA), completing on mbarriers; sixteen consumer warps compute from shared
+// memory.  Programmatic dependent launch overlaps its prologue with the router.
 //
 // Inner product without dequantising each weight: for a block with scale s
 // and min m, sum_j (s q_j + m) x_j = s * sum_j q_j x_j + m * sum_j x_j.  Each
-// code is turned into the float 2^(23-p) + q by OR-ing it, at mantissa bit p,
-// into the exponent of 2^(23-p) (one logic op per code); then
-// sum_j q_j x_j = sum_j x_j f_j - sum_j x_j 2^(23-p_j), the last sum being a
-// per-block constant of the token computed once.
+// code, left at mantissa bit p_j of its word, is OR-ed into 1.0f (one logic op
+// per code, one shared constant): f_j = 1 + q_j 2^(p_j - 23), exactly.  The
+// staged activations are pre-scaled, x'_j = x_j 2^(23 - p_j) (exact), so that
+// sum_j x'_j f_j = sum_j x'_j + sum_j q_j x_j, the first sum being a per-block
+// constant of the token computed once.
 #include <cuda_fp16.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -35,13 +37,13 @@
 namespace moe {
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;        // + one producer warp
 constexpr int kXStride = 36;                     // floats per 32-weight chunk: 32 x + 4 constants
 constexpr int kMaxPairs = kDecodeMaxT * kMaxTopK + 1;
-constexpr int kMaxStages = 4;
-constexpr int kSmemBudget = 200 * 1024;
+constexpr int kMaxStages = 8;
+constexpr int kSmemBudget = 220 * 1024;
 
 // ---------------------------------------------------------------- code decode
 // Q2_32: code j of a 32-bit word sits at bits [2j, 2j+2).  Shifting the word by
@@ -52,7 +54,7 @@ MOE_DEVINL float q2_code(const uint32_t* w, int i) {
     const int j = i & 15;
     const uint32_t src = j == 0 ? (word << 21) : (j <= 5 ? (word << 11) : (j <= 10 ? (word << 1) : (word >> 9)));
     const int p = q2_pos(j);
-    return __uint_as_float((src & (3u << p)) | ((uint32_t)(150 - p) << 23));
+    return __uint_as_float((src & (3u << p)) | 0x3f800000u);
 }
 // Q3 (32 codes in 3 words, code i at stream bits [3i, 3i+3)): groups of three
 // codes are moved to bits 14..22, so code i sits at bit 14 + 3*(i % 3).
@@ -73,12 +75,60 @@ MOE_DEVINL float q3_code(const uint32_t* w, int i) {
         default: src = w[2] >> 12; break;
     }
     const int p = q3_pos(i);
-    return __uint_as_float((src & (7u << p)) | ((uint32_t)(150 - p) << 23));
+    return __uint_as_float((src & (7u << p)) | 0x3f800000u);
 }
-template <int FMT>
-MOE_DEVINL float code_f(const uint32_t* w, int i) {
-    if constexpr (FMT == MOE_Q2_32) return q2_code(w, i);
-    else return q3_code(w, i);
+// Compile-time loop: f(std::integral_constant<int, I>) for I in [B, E).
+template <int B, int E, typename Fn>
+MOE_DEVINL void static_for(Fn&& fn) {
+    if constexpr (B < E) {
+        fn(std::integral_constant<int, B>{});
+        static_for<B + 1, E>(fn);
+    }
+}
+
+// 1.0f as a register operand the compiler cannot fold: `(src & mask) | one`
+// must stay one 3-input logic op (lop3 encodes a single immediate, so two
+// immediates would cost two logic ops per code on the half-rate ALU pipe).
+MOE_DEVINL uint32_t opaque_one() {
+    uint32_t v;
+    asm volatile("mov.b32 %0, 0x3f800000;" : "=r"(v));
+    return v;
+}
+template <uint32_t MASK>
+MOE_DEVINL float and_or(uint32_t src, uint32_t one) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(src), "n"(MASK), "r"(one));   // (a & b) | c
+    return __uint_as_float(r);
+}
+
+// Code I of a chunk as 1 + q 2^(p-23), with I a compile-time constant so that
+// the shift and mask are immediates.
+template <int FMT, int I>
+MOE_DEVINL float code_c(const uint32_t* w, uint32_t one) {
+    if constexpr (FMT == MOE_Q2_32) {
+        constexpr int j = I & 15;
+        constexpr int sh = j == 0 ? 21 : (j <= 5 ? 11 : (j <= 10 ? 1 : -9));
+        constexpr int p = j == 0 ? 21 : (j <= 5 ? 2 * j + 11 : (j <= 10 ? 2 * j + 1 : 2 * j - 9));
+        const uint32_t word = w[I >> 4];
+        const uint32_t src = sh >= 0 ? (word << (sh >= 0 ? sh : 0)) : (word >> (sh < 0 ? -sh : 0));
+        return and_or<(3u << p)>(src, one);
+    } else {
+        constexpr int g = I / 3;
+        constexpr int p = 14 + 3 * (I % 3);
+        uint32_t src;
+        if constexpr (g == 0) src = w[0] << 14;
+        else if constexpr (g == 1) src = w[0] << 5;
+        else if constexpr (g == 2) src = w[0] >> 4;
+        else if constexpr (g == 3) src = __funnelshift_r(w[0], w[1], 13);
+        else if constexpr (g == 4) src = w[1] << 10;
+        else if constexpr (g == 5) src = w[1] << 1;
+        else if constexpr (g == 6) src = w[1] >> 8;
+        else if constexpr (g == 7) src = __funnelshift_r(w[1], w[2], 17);
+        else if constexpr (g == 8) src = w[2] << 6;
+        else if constexpr (g == 9) src = w[2] >> 3;
+        else src = w[2] >> 12;
+        return and_or<(7u << p)>(src, one);
+    }
 }
 template <int FMT>
 MOE_DEVINL int code_pos(int i) {
@@ -86,16 +136,7 @@ MOE_DEVINL int code_pos(int i) {
     else return q3_pos(i);
 }
 
-MOE_DEVINL float2 ffma2(float2 a, float2 b, float2 c) {
-    unsigned long long ra, rb, rc, rd;
-    asm("mov.b64 %0, {%1,%2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
-    asm("mov.b64 %0, {%1,%2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
-    asm("mov.b64 %0, {%1,%2};" : "=l"(rc) : "f"(c.x), "f"(c.y));
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(rd) : "l"(ra), "l"(rb), "l"(rc));
-    float2 d;
-    asm("mov.b64 {%0,%1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
-    return d;
-}
+MOE_DEVINL float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 MOE_DEVINL void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
 
@@ -156,44 +197,66 @@ struct DecodeParams {
     int32_t* miss_count;
     uint16_t* hbuf;        // [kMaxPairs][4][F]
     uint32_t* err;
+    uint32_t* done;        // [kMaxPairs + 1]: per-owner gate|up completion counters + CTA ticket
     int rf;                // gate|up: features per item
     int rd;                // down: rows per item
     int ns_gu, ns_dn;      // pipeline stages
 };
+
+constexpr int kMaxE = 1024;
 
 struct Shared {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
     Owner owners[kMaxPairs];
     int slot_of[kMaxPairs];
+    int table[kMaxE];          // the slot table, staged before the dependency wait
     int n_owners;
-    int cur_owner;
 };
 
-MOE_DEVINL int lookup_slot(const DecodeParams& prm, int e) {
-    int s = (e >= 0 && e < prm.E) ? __ldg(prm.slot_table + e) : -1;
-    return (s < 0 || s >= prm.P.n_slots) ? -1 : s;
+// The slot table is an input of the layer, not produced by the router: stage it
+// while the router may still run.
+__device__ void stage_table(const DecodeParams& prm, Shared& sh) {
+    for (int e = threadIdx.x; e < prm.E; e += blockDim.x) {
+        const int s = __ldg(prm.slot_table + e);
+        sh.table[e] = (s < 0 || s >= prm.P.n_slots) ? -1 : s;
+    }
 }
 
-// One warp: resolve every pair's slot, the owners (first pair of each distinct
-// resident slot, in pair order, then the shared expert) and, with `book`, the
-// row map, miss list and miss count.
+// Work items.  Owner 0 (the shared expert, which serves every token and so
+// costs about twice as much per row) is cut into half-size items, so that
+// equal item counts are roughly equal work:
+//   gate|up: 2*nfb shared items of rf/2 features, then nfb items of rf per owner
+//   down   : 2*nrb shared items of rd/2 rows,     then nrb items of rd per owner
+struct ItemPos { int u, row0, nrows; };
+MOE_DEVINL ItemPos item_pos(int i, int per_owner, int rows) {
+    ItemPos p;
+    if (i < 2 * per_owner) { p.u = 0; p.nrows = rows / 2; p.row0 = i * p.nrows; }
+    else { const int r = i - 2 * per_owner; p.u = 1 + r / per_owner; p.nrows = rows; p.row0 = (r % per_owner) * rows; }
+    return p;
+}
+MOE_DEVINL int items_of(int n_owners, int per_owner) { return 2 * per_owner + (n_owners - 1) * per_owner; }
+
+MOE_DEVINL int lookup_slot(const DecodeParams& prm, const Shared& sh, int e) {
+    return (e >= 0 && e < prm.E) ? sh.table[e] : -1;
+}
+
+// One warp: resolve every pair's slot and the owners — owner 0 is the shared
+// expert, then the first pair of each distinct resident slot in pair order —
+// and, with `book`, the row map, miss list and miss count.
 __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, bool book) {
     const int lane = threadIdx.x & 31;
     const int T = prm.T, k = prm.k, n = T * k;   // n <= 64
-    int e0 = -1, e1 = -1;
-    for (int q = lane; q < n; q += 32) {
-        const int e = __ldg(prm.ids + q);
-        sh.slot_of[q] = lookup_slot(prm, e);
-        if (q < 32) e0 = e; else e1 = e;
-    }
-    __syncwarp();
-    const int s0 = lane < n ? sh.slot_of[lane] : -1;
-    const int s1 = lane + 32 < n ? sh.slot_of[lane + 32] : -1;
+    const int e0 = lane < n ? __ldg(prm.ids + lane) : -1;
+    const int e1 = lane + 32 < n ? __ldg(prm.ids + lane + 32) : -1;
+    const int s0 = lane < n ? lookup_slot(prm, sh, e0) : -1;
+    const int s1 = lane + 32 < n ? lookup_slot(prm, sh, e1) : -1;
+    if (lane < n) sh.slot_of[lane] = s0;
+    if (lane + 32 < n) sh.slot_of[lane + 32] = s1;
     const uint32_t miss0 = __ballot_sync(0xffffffffu, lane < n && s0 < 0);
     const uint32_t miss1 = __ballot_sync(0xffffffffu, lane + 32 < n && s1 < 0);
+    const uint32_t below = (1u << lane) - 1u;
     if (book) {
-        const uint32_t below = (1u << lane) - 1u;
         if (lane < n) {
             const int t = lane / k, r = lane % k;
             prm.rowmap[t * (k + 1) + r] = s0 >= 0 ? t * (k + 1) + r : -1;
@@ -213,69 +276,70 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, bool book) {
         if (lane < T) prm.rowmap[lane * (k + 1) + k] = lane * (k + 1) + k;
         if (lane == 0) prm.miss_count[0] = __popc(miss0) + __popc(miss1);
     }
-    // owners: lane handles pairs p = lane and p = lane + 32
-    bool own[2] = {false, false};
-    uint32_t rm[2][kDecodeMaxT];
+    __syncwarp();
+    // lane handles pairs p = lane (h = 0) and p = lane + 32 (h = 1)
+    uint32_t rm0[kDecodeMaxT] = {0, 0, 0, 0}, rm1[kDecodeMaxT] = {0, 0, 0, 0};
+    bool own0 = lane < n && s0 >= 0, own1 = lane + 32 < n && s1 >= 0;
+    uint64_t eq0 = 0, eq1 = 0;                 // pairs q with the same slot
+#pragma unroll 8
+    for (int q = 0; q < n; ++q) {
+        const int sq = sh.slot_of[q];
+        if (sq == s0) eq0 |= 1ull << q;
+        if (sq == s1) eq1 |= 1ull << q;
+    }
+    if (own0 && (eq0 & ((1ull << lane) - 1ull))) own0 = false;
+    if (own1 && (eq1 & ((1ull << (lane + 32)) - 1ull))) own1 = false;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int p = lane + 32 * h;
-        const int sp = h == 0 ? s0 : s1;
-#pragma unroll
-        for (int t = 0; t < kDecodeMaxT; ++t) rm[h][t] = 0;
-        if (p < n && sp >= 0) {
-            bool first = true;
-            for (int t = 0; t < T; ++t)
-                for (int r = 0; r < k; ++r) {
-                    const int q = t * k + r;
-                    if (sh.slot_of[q] == sp) {
-                        if (q < p) first = false;
-                        rm[h][t] |= 1u << r;
-                    }
-                }
-            own[h] = first;
+    for (int t = 0; t < kDecodeMaxT; ++t) {
+        if (t < T) {
+            rm0[t] = (uint32_t)(eq0 >> (t * k)) & ((1u << k) - 1u);
+            rm1[t] = (uint32_t)(eq1 >> (t * k)) & ((1u << k) - 1u);
         }
     }
-    const uint32_t b0 = __ballot_sync(0xffffffffu, own[0]);
-    const uint32_t b1 = __ballot_sync(0xffffffffu, own[1]);
+    const uint32_t b0 = __ballot_sync(0xffffffffu, own0);
+    const uint32_t b1 = __ballot_sync(0xffffffffu, own1);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        if (own[h]) {
-            const int idx = (h == 0) ? __popc(b0 & ((1u << lane) - 1u)) : __popc(b0) + __popc(b1 & ((1u << lane) - 1u));
-            Owner o;
+        const bool own = h == 0 ? own0 : own1;
+        if (own) {
+            const int idx = h == 0 ? 1 + __popc(b0 & below) : 1 + __popc(b0) + __popc(b1 & below);
+            Owner& o = sh.owners[idx];
+            int nt = 0;
+#pragma unroll
+            for (int t = 0; t < kDecodeMaxT; ++t) {
+                const uint32_t m = h == 0 ? rm0[t] : rm1[t];
+                if (t < T && m) { o.tok[nt] = t; o.rmask[nt] = m; ++nt; }
+            }
+            o.ntok = nt;
             o.slot = h == 0 ? s0 : s1;
-            o.ntok = 0;
-            for (int t = 0; t < T; ++t)
-                if (rm[h][t]) { o.tok[o.ntok] = t; o.rmask[o.ntok] = rm[h][t]; ++o.ntok; }
-            sh.owners[idx] = o;
         }
     }
+    if (lane < T) { sh.owners[0].tok[lane] = lane; sh.owners[0].rmask[lane] = 1u << k; }
     if (lane == 0) {
-        const int idx = __popc(b0) + __popc(b1);
-        Owner o;
-        o.slot = prm.P.shared_slot;
-        o.ntok = T;
-        for (int t = 0; t < T; ++t) { o.tok[t] = t; o.rmask[t] = 1u << k; }
-        sh.owners[idx] = o;
-        sh.n_owners = idx + 1;
+        sh.owners[0].slot = prm.P.shared_slot;
+        sh.owners[0].ntok = T;
+        sh.n_owners = 1 + __popc(b0) + __popc(b1);
     }
     __syncwarp();
 }
 
 // ---------------------------------------------------------------- activations to smem
-// xs[(n * nb + b) * 36 + j]: fp32 activation j of chunk b of token n; slots 32..33
-// hold per-chunk constants: Q2/Q3_32: C = sum x_j 2^(23-p_j), X = sum x_j;
+// xs[(n * nb + b) * 36 + j]: pre-scaled activation x_j 2^(23-p_j) of chunk b of
+// token n; slots 32..33 hold per-chunk constants: Q2/Q3_32: C = sum x_j 2^(23-p_j),
+// X = sum x_j;
 // Q3_S256: C'lo, C'hi = sum over the half of x_j (2^(23-p_j) + 4)  (the +4 folds
 // the min -4*S of the sub-block into the constant).  Run by the consumer threads.
 template <int FMT>
-__device__ void stage_activations(const uint16_t* __restrict__ src, size_t tok_stride, int ntok, int K, float* xs) {
+__device__ void stage_activations(const uint16_t* src, size_t tok_stride, int ntok, int K, float* xs,
+                                  int first = 0, int nthreads = kConsumers, bool coherent = false) {
     const int nb = K / 32;
-    for (int idx = threadIdx.x; idx < ntok * nb; idx += kConsumers) {
+    for (int idx = (int)threadIdx.x - first; idx < ntok * nb; idx += nthreads) {
         const int n = idx / nb, b = idx - n * nb;
         const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)n * tok_stride + 32 * b);
         float v[32];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint4 w = p[q];
+            const uint4 w = coherent ? __ldcg(p + q) : __ldg(p + q);
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -284,41 +348,60 @@ __device__ void stage_activations(const uint16_t* __restrict__ src, size_t tok_s
             }
         }
         float* dst = xs + (size_t)idx * kXStride;
+        float vp[32];
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-        double c0 = 0.0, c1 = 0.0;
+        for (int j = 0; j < 32; ++j) vp[j] = v[j] * (float)(1u << (23 - code_pos<FMT>(j)));   // exact
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(vp[j], vp[j + 1], vp[j + 2], vp[j + 3]);
+        // constants from fp32 partial sums per magic position (few terms each),
+        // combined in double: sum_j x_j 2^(23-p_j) (+ 4 x_j for Q3_S256)
+        float part[2][10];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int c = 0; c < 10; ++c) part[h][c] = 0.f;
+        float xs0 = 0.f, xs1 = 0.f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const double base = (double)(1u << (23 - code_pos<FMT>(j)));
-            if constexpr (FMT == MOE_Q3_S256) {
-                const double c = (double)v[j] * (base + 4.0);
-                if (j < 16) c0 += c; else c1 += c;
-            } else {
-                c0 += (double)v[j] * base;
-                c1 += (double)v[j];
-            }
+            const int c = code_pos<FMT>(j) - 13;       // 0..9
+            const int h = (FMT == MOE_Q3_S256 && j >= 16) ? 1 : 0;
+            part[h][c] += v[j];
+            if (j < 16) xs0 += v[j]; else xs1 += v[j];
+        }
+        double c0 = 0.0, c1 = 0.0;
+#pragma unroll
+        for (int c = 0; c < 10; ++c) {
+            c0 += (double)part[0][c] * (double)(1u << (10 - c));
+            c1 += (double)part[1][c] * (double)(1u << (10 - c));
+        }
+        if constexpr (FMT == MOE_Q3_S256) {
+            c0 += 4.0 * (double)xs0;
+            c1 += 4.0 * (double)xs1;
+        } else {
+            c1 = (double)xs0 + (double)xs1;
         }
         dst[32] = (float)c0;
         dst[33] = (float)c1;
     }
 }
 
-// ---------------------------------------------------------------- one chunk, four rows
+// ---------------------------------------------------------------- one chunk, R rows
 // cw[r]: the chunk's code words of row r; sa/sb: Q2/Q3_32 (s, m), Q3_S256 (S_lo, S_hi).
 // xc[t]: the chunk's activations of the t-th served token.
-template <int FMT, int NT>
-MOE_DEVINL void chunk4(const uint32_t (&cw)[4][3], const float (&sa)[4], const float (&sb)[4],
-                       const float* const (&xc)[NT], float (&res)[4][NT]) {
+template <int FMT, int NT, int R>
+MOE_DEVINL void chunk_rows(const uint32_t (&cw)[R][3], const float (&sa)[R], const float (&sb)[R],
+                           const float* const (&xc)[NT], float (&res)[R][NT]) {
     constexpr int H = (FMT == MOE_Q3_S256) ? 2 : 1;
-    float2 acc[4][NT][H];
+    const uint32_t one = opaque_one();
+    float2 acc[R][NT][H];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
             for (int h = 0; h < H; ++h) acc[r][t][h] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int sc = 0; sc < 4; ++sc) {
+    static_for<0, 4>([&](auto SC) {
+        constexpr int sc = decltype(SC)::value;
         float xv[NT][8];
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -327,25 +410,25 @@ MOE_DEVINL void chunk4(const uint32_t (&cw)[4][3], const float (&sa)[4], const f
             xv[t][0] = a.x; xv[t][1] = a.y; xv[t][2] = a.z; xv[t][3] = a.w;
             xv[t][4] = b.x; xv[t][5] = b.y; xv[t][6] = b.z; xv[t][7] = b.w;
         }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                const int code = 8 * sc + i;
-                const float2 f = make_float2(code_f<FMT>(cw[r], code), code_f<FMT>(cw[r], code + 1));
-                const int h = (H == 2 && code >= 16) ? 1 : 0;
+        static_for<0, R>([&](auto RR) {
+            constexpr int r = decltype(RR)::value;
+            static_for<0, 4>([&](auto II) {
+                constexpr int i = 2 * decltype(II)::value;
+                constexpr int code = 8 * sc + i;
+                constexpr int h = (H == 2 && code >= 16) ? 1 : 0;
+                const float2 f = make_float2(code_c<FMT, code>(cw[r], one), code_c<FMT, code + 1>(cw[r], one));
 #pragma unroll
                 for (int t = 0; t < NT; ++t)
                     acc[r][t][h] = ffma2(make_float2(xv[t][i], xv[t][i + 1]), f, acc[r][t][h]);
-            }
-        }
-    }
+            });
+        });
+    });
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
         const float c0 = xc[t][32];
         const float c1 = xc[t][33];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < R; ++r) {
             if constexpr (H == 2) {
                 res[r][t] = __fmaf_rn(sa[r], (acc[r][t][0].x + acc[r][t][0].y) - c0, res[r][t]);
                 res[r][t] = __fmaf_rn(sb[r], (acc[r][t][1].x + acc[r][t][1].y) - c1, res[r][t]);
@@ -364,15 +447,15 @@ MOE_DEVINL void smem_chunk(const uint8_t* cbase, const uint8_t* mbase, const uin
     if constexpr (FMT == MOE_Q2_32) {
         const uint2 c = *reinterpret_cast<const uint2*>(cbase + (size_t)row * Geo<FMT>::code_row(K) + b * 8);
         w[0] = c.x; w[1] = c.y; w[2] = 0;
-        const uint32_t sm = *reinterpret_cast<const uint32_t*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + b * 4);
-        sa = f16_bits_to_f32(sm & 0xffffu);
-        sb = f16_bits_to_f32(sm >> 16);
+        const float2 sm = __half22float2(*reinterpret_cast<const __half2*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + b * 4));
+        sa = sm.x;
+        sb = sm.y;
     } else if constexpr (FMT == MOE_Q3_32) {
         const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)row * Geo<FMT>::code_row(K) + b * 12);
         w[0] = p[0]; w[1] = p[1]; w[2] = p[2];
-        const uint32_t sm = *reinterpret_cast<const uint32_t*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + b * 4);
-        sa = f16_bits_to_f32(sm & 0xffffu);
-        sb = f16_bits_to_f32(sm >> 16);
+        const float2 sm = __half22float2(*reinterpret_cast<const __half2*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + b * 4));
+        sa = sm.x;
+        sb = sm.y;
     } else {
         const int sbk = b >> 3, j = b & 7;
         const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)row * Geo<FMT>::code_row(K) + b * 12);
@@ -402,11 +485,13 @@ MOE_DEVINL void issue_rows(const Planes& pl, int row0, int nrows, int K, uint8_t
 
 // ---------------------------------------------------------------- gate | up
 // Item = (owner u, features [f0, f0 + rf)); staged as gate rows then up rows.
+// One feature (its gate row and up row) per warp-group pass; the chunk data of
+// the next chunk is read from shared memory while the current one is computed.
 template <int FMT, int NT>
-__device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int f0, const uint8_t* stage,
+__device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int f0, int rf, const uint8_t* stage,
                             const float* xs) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = prm.P.D, F = prm.P.F, rf = prm.rf;
+    const int D = prm.P.D, F = prm.P.F;
     const int nb = D / 32;
     const int lpr = min(32, nb & -nb);
     const int G = 32 / lpr, group = lane / lpr, gl = lane % lpr;
@@ -418,111 +503,55 @@ __device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int 
     const uint8_t* uc = stage + half;
     const uint8_t* um = uc + cr * rf;
     const uint8_t* ud = uc + (cr + mr) * rf;
-    for (int q = warp * G + group; q < rf / 2; q += kConsumerWarps * G) {
-        const int fl = 2 * q;   // local feature
-        float res[4][NT];
+    const float* xt[NT];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+    for (int t = 0; t < NT; ++t) xt[t] = xs + (size_t)o.tok[t] * nb * kXStride;
+    for (int fl = warp * G + group; fl < rf; fl += kConsumerWarps * G) {   // local feature
+        float res[2][NT];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int t = 0; t < NT; ++t) res[r][t] = 0.f;
+        uint32_t cw[2][3];
+        float sa[2], sb[2];
+        smem_chunk<FMT>(gc, gm, gd, fl, D, gl, cw[0], sa[0], sb[0]);
+        smem_chunk<FMT>(uc, um, ud, fl, D, gl, cw[1], sa[1], sb[1]);
         for (int b = gl; b < nb; b += lpr) {
-            uint32_t cw[4][3];
-            float sa[4], sb[4];
-            smem_chunk<FMT>(gc, gm, gd, fl, D, b, cw[0], sa[0], sb[0]);
-            smem_chunk<FMT>(gc, gm, gd, fl + 1, D, b, cw[1], sa[1], sb[1]);
-            smem_chunk<FMT>(uc, um, ud, fl, D, b, cw[2], sa[2], sb[2]);
-            smem_chunk<FMT>(uc, um, ud, fl + 1, D, b, cw[3], sa[3], sb[3]);
+            uint32_t ncw[2][3];
+            float nsa[2], nsb[2];
+            const int bn = b + lpr < nb ? b + lpr : b;
+            smem_chunk<FMT>(gc, gm, gd, fl, D, bn, ncw[0], nsa[0], nsb[0]);
+            smem_chunk<FMT>(uc, um, ud, fl, D, bn, ncw[1], nsa[1], nsb[1]);
             const float* xc[NT];
 #pragma unroll
-            for (int t = 0; t < NT; ++t) xc[t] = xs + ((size_t)o.tok[t] * nb + b) * kXStride;
-            chunk4<FMT, NT>(cw, sa, sb, xc, res);
+            for (int t = 0; t < NT; ++t) xc[t] = xt[t] + (size_t)b * kXStride;
+            chunk_rows<FMT, NT, 2>(cw, sa, sb, xc, res);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                cw[r][0] = ncw[r][0]; cw[r][1] = ncw[r][1]; cw[r][2] = ncw[r][2];
+                sa[r] = nsa[r]; sb[r] = nsb[r];
+            }
         }
         for (int off = lpr >> 1; off >= 1; off >>= 1)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int t = 0; t < NT; ++t) res[r][t] += __shfl_xor_sync(0xffffffffu, res[r][t], off);
         if (gl == 0) {
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const uint16_t h0 = f32_to_bf16_rne(silu_f(res[0][t]) * res[2][t]);
-                const uint16_t h1 = f32_to_bf16_rne(silu_f(res[1][t]) * res[3][t]);
-                *reinterpret_cast<uint32_t*>(prm.hbuf + ((size_t)u * kDecodeMaxT + t) * F + f0 + fl) =
-                    (uint32_t)h0 | ((uint32_t)h1 << 16);
-            }
+            for (int t = 0; t < NT; ++t)
+                prm.hbuf[((size_t)u * kDecodeMaxT + t) * F + f0 + fl] = f32_to_bf16_rne(silu_f(res[0][t]) * res[1][t]);
         }
-    }
-}
-
-template <int FMT, int NTMAX>
-__global__ void __launch_bounds__(kThreads, 1) decode_gateup_kernel(DecodeParams prm) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ Shared sh;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = prm.P.D, F = prm.P.F, rf = prm.rf, NS = prm.ns_gu;
-    const int nb = D / 32;
-    const size_t xs_bytes = ((size_t)prm.T * nb * kXStride * 4 + 127) / 128 * 128;
-    float* xs = reinterpret_cast<float*>(smem);
-    uint8_t* stages = smem + xs_bytes;
-    const uint32_t item_bytes = 2u * Geo<FMT>::row_bytes(D) * rf;
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kConsumerWarps); }
-        fence_mbar_init();
-    }
-    pdl_wait();                      // ids come from the router
-    if (warp == 0) resolve_owners(prm, sh, blockIdx.x == 0);
-    __syncthreads();
-    pdl_launch_dependents();         // the down kernel may start its prologue
-    const int nfb = F / rf;
-    const int n_items = sh.n_owners * nfb;
-    if (warp == kConsumerWarps) {    // producer: round-robin items
-        if (lane == 0) {
-            int j = 0;
-            for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++j) {
-                const int s = j % NS;
-                if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) break;
-                const int u = i / nfb, f0 = (i % nfb) * rf;
-                const int slot = sh.owners[u].slot;
-                uint8_t* dst = stages + (size_t)s * item_bytes;
-                mbar_arrive_expect_tx(&sh.full[s], item_bytes);
-                issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 0), f0, rf, D, dst, &sh.full[s]);
-                issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 1), f0, rf, D, dst + item_bytes / 2, &sh.full[s]);
-            }
-        }
-        return;
-    }
-    stage_activations<FMT>(prm.x, D, prm.T, D, xs);
-    consumer_sync();
-    int j = 0;
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++j) {
-        const int s = j % NS;
-        if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) return;
-        const int u = i / nfb, f0 = (i % nfb) * rf;
-        const Owner& o = sh.owners[u];
-        const uint8_t* st = stages + (size_t)s * item_bytes;
-        if constexpr (NTMAX == 1) {
-            gateup_item<FMT, 1>(prm, o, u, f0, st, xs);
-        } else {
-            switch (o.ntok) {
-                case 1: gateup_item<FMT, 1>(prm, o, u, f0, st, xs); break;
-                case 2: gateup_item<FMT, 2>(prm, o, u, f0, st, xs); break;
-                case 3: gateup_item<FMT, 3>(prm, o, u, f0, st, xs); break;
-                default: gateup_item<FMT, 4>(prm, o, u, f0, st, xs); break;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[s]);
     }
 }
 
 // ---------------------------------------------------------------- down
-// Item = (owner u, rows [d0, d0 + rd)) of Wd.  Items are split in contiguous
-// ranges per CTA so that consecutive items mostly share the owner (h is
-// re-staged only when the owner changes).
+// Item = (owner u, rows [d0, d0 + rd)) of Wd; two rows per warp-group pass.
 template <int FMT, int NT>
-__device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, const uint8_t* stage, const float* hs) {
+__device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int rd, const uint8_t* stage,
+                          const float* hs) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = prm.P.D, F = prm.P.F, k = prm.k, rd = prm.rd;
+    const int D = prm.P.D, F = prm.P.F, k = prm.k;
     const int nb = F / 32;
     const int lpr = min(32, nb & -nb);
     const int G = 32 / lpr, group = lane / lpr, gl = lane % lpr;
@@ -530,108 +559,208 @@ __device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, const
     const uint8_t* dc = stage;
     const uint8_t* dm = stage + cr * rd;
     const uint8_t* dd = stage + (cr + mr) * rd;
-    for (int q = warp * G + group; q < rd / 4; q += kConsumerWarps * G) {
-        const int rl = 4 * q;
-        float res[4][NT];
+    for (int q = warp * G + group; q < rd / 2; q += kConsumerWarps * G) {
+        const int rl = 2 * q;
+        float res[2][NT];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int t = 0; t < NT; ++t) res[r][t] = 0.f;
-        for (int b = gl; b < nb; b += lpr) {
-            uint32_t cw[4][3];
-            float sa[4], sb[4];
+        uint32_t cw[2][3];
+        float sa[2], sb[2];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, b, cw[r], sa[r], sb[r]);
+        for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, gl, cw[r], sa[r], sb[r]);
+        for (int b = gl; b < nb; b += lpr) {
+            uint32_t ncw[2][3];
+            float nsa[2], nsb[2];
+            const int bn = b + lpr < nb ? b + lpr : b;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, bn, ncw[r], nsa[r], nsb[r]);
             const float* xc[NT];
 #pragma unroll
             for (int t = 0; t < NT; ++t) xc[t] = hs + ((size_t)t * nb + b) * kXStride;
-            chunk4<FMT, NT>(cw, sa, sb, xc, res);
+            chunk_rows<FMT, NT, 2>(cw, sa, sb, xc, res);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                cw[r][0] = ncw[r][0]; cw[r][1] = ncw[r][1]; cw[r][2] = ncw[r][2];
+                sa[r] = nsa[r]; sb[r] = nsb[r];
+            }
         }
         for (int off = lpr >> 1; off >= 1; off >>= 1)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int t = 0; t < NT; ++t) res[r][t] += __shfl_xor_sync(0xffffffffu, res[r][t], off);
         if (gl == 0) {
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const float4 v = make_float4(res[0][t], res[1][t], res[2][t], res[3][t]);
+                const float2 v = make_float2(res[0][t], res[1][t]);
                 uint32_t m = o.rmask[t];
                 while (m) {
                     const int r = __ffs(m) - 1;
                     m &= m - 1;
-                    *reinterpret_cast<float4*>(prm.yrows + ((size_t)o.tok[t] * (k + 1) + r) * D + d0 + rl) = v;
+                    *reinterpret_cast<float2*>(prm.yrows + ((size_t)o.tok[t] * (k + 1) + r) * D + d0 + rl) = v;
                 }
             }
         }
     }
 }
 
+MOE_DEVINL void red_release_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------- the fused kernel
+// One persistent CTA per SM.  Each CTA takes its gate|up items (round-robin),
+// then a contiguous range of down items, through one ring of stages.  A
+// down item of owner u waits until every gate|up item of u has published its
+// h (a per-owner item counter in ws, advanced by each CTA once its whole gate|up
+// range is done); the down weights stream in meanwhile.  The last CTA to finish
+// resets the counters, so every completed call leaves them zero.
 template <int FMT, int NTMAX>
-__global__ void __launch_bounds__(kThreads, 1) decode_down_kernel(DecodeParams prm) {
+__global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams prm) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ Shared sh;
+    __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = prm.P.D, F = prm.P.F, rd = prm.rd, NS = prm.ns_dn;
-    const int nb = F / 32;
-    const size_t hs_bytes = ((size_t)kDecodeMaxT * nb * kXStride * 4 + 127) / 128 * 128;
-    float* hs = reinterpret_cast<float*>(smem);
-    uint8_t* stages = smem + hs_bytes;
-    const uint32_t item_bytes = (uint32_t)Geo<FMT>::row_bytes(F) * rd;
+    const int D = prm.P.D, F = prm.P.F, rf = prm.rf, rd = prm.rd, NS = prm.ns_gu;
+    const int nbx = D / 32, nbh = F / 32;
+    const size_t xs_bytes = ((size_t)prm.T * nbx * kXStride * 4 + 127) / 128 * 128;
+    const size_t hs_bytes = ((size_t)kDecodeMaxT * nbh * kXStride * 4 + 127) / 128 * 128;
+    float* xs = reinterpret_cast<float*>(smem);
+    float* hs = reinterpret_cast<float*>(smem + xs_bytes);
+    uint8_t* stages = smem + xs_bytes + hs_bytes;
+    const uint32_t gu_bytes = 2u * Geo<FMT>::row_bytes(D) * rf;
+    const uint32_t dn_bytes = (uint32_t)Geo<FMT>::row_bytes(F) * rd;
+    const uint32_t stage_bytes = gu_bytes > dn_bytes ? gu_bytes : dn_bytes;
+    const int nfb = F / rf, nrb = D / rd;
+    uint32_t* done = prm.done;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kConsumerWarps); }
         fence_mbar_init();
-        sh.cur_owner = -1;
+        abort_flag = 0;
     }
-    // ids and the slot table were complete before the gate|up kernel passed its
-    // own dependency wait, which precedes the launch of this grid: the owners can
-    // be resolved and the down weights prefetched before waiting for h.
-    if (warp == 0) resolve_owners(prm, sh, false);
+    stage_table(prm, sh);
     __syncthreads();
-    const int nrb = D / rd;
-    const int n_items = sh.n_owners * nrb;
-    const int per = (n_items + gridDim.x - 1) / gridDim.x;
-    const int i0 = blockIdx.x * per, i1 = min(n_items, i0 + per);
-    if (warp == kConsumerWarps) {
+    pdl_wait();                      // ids come from the router
+    if (warp == 0) {
+        resolve_owners(prm, sh, blockIdx.x == 0);
+    } else if (warp < kConsumerWarps) {
+        stage_activations<FMT>(prm.x, D, prm.T, D, xs, 32, kConsumers - 32);
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+    // gate|up items round-robin over the CTAs (x is staged for every token);
+    // down items in equal-count contiguous ranges (h is re-staged per owner)
+    const int n_g = items_of(sh.n_owners, nfb), n_d = items_of(sh.n_owners, nrb);
+    const int ng = n_g > (int)blockIdx.x ? (n_g - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int per_d = (n_d + gridDim.x - 1) / gridDim.x;
+    const int d0r = min(n_d, (int)blockIdx.x * per_d), d1r = min(n_d, d0r + per_d);
+    if (warp == kConsumerWarps) {    // producer: gate|up items, then down items
         if (lane == 0) {
-            for (int i = i0, j = 0; i < i1; ++i, ++j) {
+            const int total = ng + (d1r - d0r);
+            for (int j = 0; j < total; ++j) {
                 const int s = j % NS;
                 if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) break;
-                const int u = i / nrb, d0 = (i % nrb) * rd;
-                mbar_arrive_expect_tx(&sh.full[s], item_bytes);
-                issue_rows<FMT>(planes_of<FMT>(prm.P, sh.owners[u].slot, 2), d0, rd, F, stages + (size_t)s * item_bytes,
-                                &sh.full[s]);
+                if (abort_flag) break;
+                uint8_t* dst = stages + (size_t)s * stage_bytes;
+                if (j < ng) {
+                    const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
+                    const int slot = sh.owners[ip.u].slot;
+                    const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * ip.nrows;
+                    mbar_arrive_expect_tx(&sh.full[s], 2 * half);
+                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 0), ip.row0, ip.nrows, D, dst, &sh.full[s]);
+                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 1), ip.row0, ip.nrows, D, dst + half, &sh.full[s]);
+                } else {
+                    const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
+                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)Geo<FMT>::row_bytes(F) * ip.nrows);
+                    issue_rows<FMT>(planes_of<FMT>(prm.P, sh.owners[ip.u].slot, 2), ip.row0, ip.nrows, F, dst, &sh.full[s]);
+                }
             }
         }
-        return;
+    } else {
+        int j = 0;
+        bool ok = true;
+        for (; j < ng && ok; ++j) {
+            const int s = j % NS;
+            if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) { ok = false; break; }
+            const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
+            const int u = ip.u, f0 = ip.row0;
+            const Owner& o = sh.owners[u];
+            const uint8_t* st = stages + (size_t)s * stage_bytes;
+            if constexpr (NTMAX == 1) {
+                gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs);
+            } else {
+                switch (o.ntok) {
+                    case 1: gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs); break;
+                    case 2: gateup_item<FMT, 2>(prm, o, u, f0, ip.nrows, st, xs); break;
+                    case 3: gateup_item<FMT, 3>(prm, o, u, f0, ip.nrows, st, xs); break;
+                    default: gateup_item<FMT, 4>(prm, o, u, f0, ip.nrows, st, xs); break;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.empty[s]);
+        }
+        // publish this CTA's h once for its whole gate|up range: every writer
+        // fences its own stores, then one thread adds the item counts per owner
+        __threadfence();
+        consumer_sync();
+        if (threadIdx.x == 0) {
+            for (int jj = 0; jj < ng; ++jj) atomicAdd(done + item_pos(blockIdx.x + jj * gridDim.x, nfb, rf).u, 1u);
+        }
+        int cur = -1;
+        for (int i = d0r; i < d1r && ok; ++i, ++j) {
+            const int s = j % NS;
+            const ItemPos ip = item_pos(i, nrb, rd);
+            const int u = ip.u, r0 = ip.row0;
+            const Owner& o = sh.owners[u];
+            if (u != cur) {
+                consumer_sync();
+                if (threadIdx.x == 0) {
+                    const uint32_t target = (uint32_t)(u == 0 ? 2 * nfb : nfb);   // items of owner u
+                    uint32_t polls = 0;
+                    while (ld_acquire(done + u) < target) {
+                        if (++polls > kMaxPolls) { atomicOr(prm.err, kErrTimeout); abort_flag = 1; break; }
+                        __nanosleep(64);
+                    }
+                }
+                consumer_sync();
+                if (abort_flag) { ok = false; break; }
+                stage_activations<FMT>(prm.hbuf + (size_t)u * kDecodeMaxT * F, F, o.ntok, F, hs, 0, kConsumers, true);
+                consumer_sync();
+                cur = u;
+            }
+            if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) { ok = false; break; }
+            const uint8_t* st = stages + (size_t)s * stage_bytes;
+            if constexpr (NTMAX == 1) {
+                down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hs);
+            } else {
+                switch (o.ntok) {
+                    case 1: down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hs); break;
+                    case 2: down_item<FMT, 2>(prm, o, r0, ip.nrows, st, hs); break;
+                    case 3: down_item<FMT, 3>(prm, o, r0, ip.nrows, st, hs); break;
+                    default: down_item<FMT, 4>(prm, o, r0, ip.nrows, st, hs); break;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.empty[s]);
+        }
     }
-    pdl_wait();                      // h comes from the gate|up kernel
-    pdl_launch_dependents();
-    int cur = -1;
-    for (int i = i0, j = 0; i < i1; ++i, ++j) {
-        const int s = j % NS;
-        const int u = i / nrb, d0 = (i % nrb) * rd;
-        const Owner& o = sh.owners[u];
-        if (u != cur) {
-            consumer_sync();
-            stage_activations<FMT>(prm.hbuf + (size_t)u * kDecodeMaxT * F, F, o.ntok, F, hs);
-            consumer_sync();
-            cur = u;
+    // last CTA out resets the per-owner counters for the next call
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const uint32_t ticket = atomicAdd(done + kMaxPairs, 1u);
+        if (ticket == gridDim.x - 1) {
+            for (int u = 0; u < kMaxPairs; ++u) done[u] = 0u;
+            __threadfence();
+            done[kMaxPairs] = 0u;
         }
-        if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) return;
-        const uint8_t* st = stages + (size_t)s * item_bytes;
-        if constexpr (NTMAX == 1) {
-            down_item<FMT, 1>(prm, o, d0, st, hs);
-        } else {
-            switch (o.ntok) {
-                case 1: down_item<FMT, 1>(prm, o, d0, st, hs); break;
-                case 2: down_item<FMT, 2>(prm, o, d0, st, hs); break;
-                case 3: down_item<FMT, 3>(prm, o, d0, st, hs); break;
-                default: down_item<FMT, 4>(prm, o, d0, st, hs); break;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[s]);
     }
 }
 
@@ -649,39 +778,48 @@ int num_sms() {
 template <int FMT, int NTMAX>
 moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
     const int T = prm.T, D = prm.P.D, F = prm.P.F;
-    // gate|up: features per item and stages so that x + stages fit the budget
     const size_t xs_bytes = ((size_t)T * (D / 32) * kXStride * 4 + 127) / 128 * 128;
-    int rf = 16;
-    while (rf > 2 && xs_bytes + 2 * 2 * (size_t)Geo<FMT>::row_bytes(D) * rf > 150 * 1024) rf /= 2;
-    prm.rf = rf;
-    prm.ns_gu = 2;
-    const size_t smem1 = xs_bytes + (size_t)prm.ns_gu * 2 * Geo<FMT>::row_bytes(D) * rf;
-    // down: rows per item and stages within ~100 KB (co-resident with gate|up)
     const size_t hs_bytes = ((size_t)kDecodeMaxT * (F / 32) * kXStride * 4 + 127) / 128 * 128;
-    int rd = 128;
-    while (rd > 16 && hs_bytes + 3 * (size_t)Geo<FMT>::row_bytes(F) * rd > 100 * 1024) rd /= 2;
+    // gate|up items of rf features, down items of rd rows, one ring of up to 4
+    // stages (~3-4 items in flight per SM cover the copy latency)
+    int rf = 16, rd = 128;
+    const size_t budget = 212 * 1024;
+    auto stage_of = [&](int rf_, int rd_) {
+        const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf_, b = (size_t)Geo<FMT>::row_bytes(F) * rd_;
+        return a > b ? a : b;
+    };
+    while (rf > 2 && xs_bytes + hs_bytes + 2 * stage_of(rf, rd) > budget) rf /= 2;
+    while (rd > 16 && (size_t)Geo<FMT>::row_bytes(F) * rd > 2 * (size_t)Geo<FMT>::row_bytes(D) * rf) rd /= 2;
+    int ns = 4;
+    while (ns > 2 && xs_bytes + hs_bytes + ns * stage_of(rf, rd) > budget) --ns;
+    prm.rf = rf;
     prm.rd = rd;
-    prm.ns_dn = 3;
-    const size_t smem2 = hs_bytes + (size_t)prm.ns_dn * Geo<FMT>::row_bytes(F) * rd;
-    if (smem1 > kSmemBudget || smem2 > kSmemBudget || F % rf || D % rd) return MOE_ERR_UNSUPPORTED;
+    prm.ns_gu = prm.ns_dn = ns;
+    const size_t smem = xs_bytes + hs_bytes + ns * stage_of(rf, rd);
+    if (smem > kSmemBudget || F % rf || D % rd || rf < 2 || rd < 2) return MOE_ERR_UNSUPPORTED;
+    // every bulk copy (full and half items) must be a multiple of 16 bytes
+    auto ok16 = [](int K, int n) {
+        return ((size_t)Geo<FMT>::code_row(K) * n) % 16 == 0 && ((size_t)Geo<FMT>::meta_row(K) * n) % 16 == 0 &&
+               ((size_t)Geo<FMT>::d_row(K) * n) % 16 == 0;
+    };
+    if (!ok16(D, rf) || !ok16(D, rf / 2) || !ok16(F, rd) || !ok16(F, rd / 2)) return MOE_ERR_UNSUPPORTED;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaFuncSetAttribute(decode_gateup_kernel<FMT, NTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
-        cudaFuncSetAttribute(decode_down_kernel<FMT, NTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
+        cudaFuncSetAttribute(decode_ffn_kernel<FMT, NTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
         attr_done = true;
     }
-    const int grid = num_sms();
-    cudaError_t e = launch_pdl(decode_gateup_kernel<FMT, NTMAX>, dim3(grid), dim3(kThreads), smem1, s, prm);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_pdl(decode_down_kernel<FMT, NTMAX>, dim3(grid), dim3(kThreads), smem2, s, prm);
+    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NTMAX>, dim3(num_sms()), dim3(kThreads), smem, s, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
 
+// ws layout: [0,4) reserved, [4,8) device error word, [64, 64 + 4*(kMaxPairs+1))
+// completion counters (zero before the first call; every completed call leaves
+// them zero), [1024, ...) h buffer.
 size_t decode_workspace_bytes(int T, int D, int F, int k) {
     (void)D; (void)T; (void)k;
-    return 256 + (size_t)kMaxPairs * kDecodeMaxT * F * sizeof(uint16_t);
+    return 1024 + (size_t)kMaxPairs * kDecodeMaxT * F * sizeof(uint16_t);
 }
 
 moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
@@ -700,7 +838,8 @@ moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, i
     prm.miss_list = miss_list;
     prm.miss_count = miss_count;
     prm.err = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
-    prm.hbuf = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 256);
+    prm.done = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 64);
+    prm.hbuf = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 1024);
     const bool one = (T == 1);
     switch (P.fmt) {
         case MOE_Q2_32: return one ? launch_fmt<MOE_Q2_32, 1>(prm, s) : launch_fmt<MOE_Q2_32, 4>(prm, s);

@@ -59,33 +59,51 @@ __device__ __forceinline__ bool cand_better(float va, int ea, float vb, int eb) 
     return va > vb || (va == vb && ea < eb);
 }
 
-// One warp selects the top-k of one token's E logits (E <= 1024) and writes
-// ids and gates.  Each lane keeps the best of its own E/32 values; every
-// round takes the warp's best and only the winning lane rescans.  Gates are
-// formed in double from the selected fp32 logits.
-__device__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
-                          float* __restrict__ gates) {
-    const int lane = threadIdx.x & 31;
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = (e < E) ? __ldcg(lrow + e) : -INFINITY;
+// Compare-exchange for a descending order by (value, then lower id).
+__device__ __forceinline__ void cex(float& va, int& ea, float& vb, int& eb) {
+    if (cand_better(vb, eb, va, ea)) {
+        const float tv = va; va = vb; vb = tv;
+        const int te = ea; ea = eb; eb = te;
     }
-    uint32_t taken = 0;
+}
+
+// One warp selects the top-k of one token's E logits (E <= 32 * NV) and
+// writes ids and gates.  Each lane sorts its NV values once (a bitonic network
+// in registers); each of the k rounds then takes the warp's best lane head and
+// the winning lane shifts its list.  Gates are formed in double from the
+// selected fp32 logits.
+template <int NV>
+__device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
+                            float* __restrict__ gates) {
+    const int lane = threadIdx.x & 31;
+    float v[NV];
+    int e[NV];
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-        if (lane + 32 * i >= E) taken |= 1u << i;
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+    for (int i = 0; i < NV; ++i) {
+        e[i] = lane + 32 * i;
+        v[i] = (e[i] < E) ? __ldcg(lrow + e[i]) : -INFINITY;
+        if (e[i] >= E) e[i] = 0x7fffffff;
+    }
+    // bitonic sort, descending
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-        if (!(taken >> i & 1u) && cand_better(v[i], lane + 32 * i, bv, be)) { bv = v[i]; be = lane + 32 * i; }
+    for (int kk = 2; kk <= NV; kk <<= 1) {
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    if ((i & kk) == 0) cex(v[i], e[i], v[l], e[l]);
+                    else cex(v[l], e[l], v[i], e[i]);
+                }
+            }
+        }
+    }
     float my_v = 0.f, l0 = 0.f;
     int my_e = 0;
     for (int r = 0; r < k; ++r) {
-        float wv = bv;
-        int we = be;
+        float wv = v[0];
+        int we = e[0];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
@@ -94,13 +112,11 @@ __device__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t*
         }
         if (r == 0) l0 = wv;
         if (lane == r) { my_v = wv; my_e = we; }
-        if ((we & 31) == lane) {
-            taken |= 1u << (we >> 5);
-            bv = -INFINITY;
-            be = 0x7fffffff;
+        if (e[0] == we) {                       // this lane supplied the winner: pop its head
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (!(taken >> i & 1u) && cand_better(v[i], lane + 32 * i, bv, be)) { bv = v[i]; be = lane + 32 * i; }
+            for (int i = 0; i + 1 < NV; ++i) { v[i] = v[i + 1]; e[i] = e[i + 1]; }
+            v[NV - 1] = -INFINITY;
+            e[NV - 1] = 0x7fffffff;
         }
     }
     const double ex = (lane < k) ? exp((double)my_v - (double)l0) : 0.0;
@@ -111,6 +127,12 @@ __device__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t*
         ids[lane] = my_e;
         gates[lane] = (float)(ex / z);
     }
+}
+
+__device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
+                                          float* __restrict__ gates) {
+    if (E <= 512) topk_warp_n<16>(lrow, E, k, ids, gates);
+    else topk_warp_n<32>(lrow, E, k, ids, gates);
 }
 
 // Decode route (T <= 4): one warp per expert computes its logits for all T

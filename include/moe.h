@@ -158,8 +158,13 @@ moe_status moe_route_topk(const uint16_t* x, int T, int D, const uint16_t* Wr,
  *          then rank order (wiselychen report §2: misses go to the CPU, which
  *          computes them in place; here they are returned to the caller)
  *   miss_count   int32 [1] out
- *   ws     scratch of moe_workspace_size bytes, 256-byte aligned, contents
- *          need not be initialised.
+ *   ws     scratch of moe_workspace_size bytes, 256-byte aligned, distinct
+ *          from the ws given to moe_route_topk.  Its first 1024 bytes must be
+ *          zero before the first call with this buffer (zero it once at
+ *          allocation); every completed call leaves them zero.  Calls sharing
+ *          one ws must not overlap on the device.  Word 1 (bytes 4..7) is the
+ *          device error word: nonzero after a bounded device-side wait gave up
+ *          (then re-zero the first 1024 bytes before reuse).
  * Per expert (reading; the pages do not give the FFN form):
  *   h = bf16( silu(Wg x) * (Wu x) ),  y = Wd h,  fp32 accumulation.
  * Missed experts are not computed.
