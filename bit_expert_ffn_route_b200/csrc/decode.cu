@@ -723,9 +723,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                 consumer_sync();
                 if (threadIdx.x == 0) {
                     const uint32_t target = (uint32_t)(u == 0 ? 2 * nfb : nfb);   // items of owner u
-                    uint32_t polls = 0;
+                    const uint64_t t0 = globaltimer_ns();
                     while (ld_acquire(done + u) < target) {
-                        if (++polls > kMaxPolls) { atomicOr(prm.err, kErrTimeout); abort_flag = 1; break; }
+                        if (*reinterpret_cast<volatile uint32_t*>(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
+                            atomicOr(prm.err, kErrTimeout);
+                            abort_flag = 1;
+                            break;
+                        }
                         __nanosleep(64);
                     }
                 }

@@ -12,10 +12,16 @@ namespace moe {
 
 // Device error word values (written into the workspace; 0 = ok).
 constexpr uint32_t kErrTimeout = 1u;
-// Bounded waits: give up after this many polls (well above any legitimate wait).
-constexpr uint32_t kMaxPolls = 1u << 26;
+// Bounded waits give up after this long (far above any legitimate wait).
+constexpr uint64_t kWaitLimitNs = 500ull * 1000 * 1000;
+constexpr uint32_t kMaxPolls = 1u << 24;
 
 MOE_DEVINL uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+MOE_DEVINL uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
 
 MOE_DEVINL void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -40,12 +46,20 @@ MOE_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false (and sets *err) if the phase never completes.
+// Bounded wait: returns false, and sets *err, if the phase does not complete
+// within kWaitLimitNs; returns false at once if another CTA already set *err.
 MOE_DEVINL bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    if (err) atomicOr(err, kErrTimeout);
-    return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (err && *reinterpret_cast<volatile uint32_t*>(err)) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (err) atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
 }
 
 // Bulk copy global -> shared, completing `bytes` of transaction on `bar`.
