@@ -241,3 +241,43 @@ size_t route_workspace_bytes(int T, int D, int E, int k) {
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------- no-allocation entry point
+// Scratch for moe_route_topk_static: a 256-byte header (word 0 = the block
+// counter of the last-block top-k) followed by room for the logits of up to
+// kStaticMaxT tokens x kStaticMaxE experts.  Every GPU that loads this library
+// holds it until the process exits.
+namespace {
+constexpr int kStaticMaxT = 4;
+constexpr int kStaticMaxE = 1024;
+constexpr size_t kStaticScratchBytes = 256 + (size_t)kStaticMaxT * kStaticMaxE * sizeof(float);
+static __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
+constexpr int kMaxDevices = 64;
+static void* g_scratch_ptr[kMaxDevices];
+}  // namespace
+
+extern "C" moe_status moe_route_topk_static(const uint16_t* x, int T, int D, const uint16_t* Wr,
+                                             const float* bias, int E, int k, int32_t* ids, float* gates,
+                                             float* logits, moe_stream_t stream) {
+    if (T < 0 || D <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (D % 256 || D > 8192 || k > moe::kMaxTopK || E < k) return MOE_ERR_UNSUPPORTED;
+    if (T > kStaticMaxT || E > kStaticMaxE) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
+    if (T == 0) return MOE_OK;
+    if (!x || !Wr || !ids || !gates) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)x % 16) || ((uintptr_t)Wr % 16) || (logits && ((uintptr_t)logits % 16))) return MOE_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    if (!g_scratch_ptr[dev]) {
+        // host code only holds a stand-in for the array: ask the runtime for the
+        // device address once per device, with that device current
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+        g_scratch_ptr[dev] = p;
+    }
+    void* ws = g_scratch_ptr[dev];
+    cudaStream_t s = (cudaStream_t)stream;
+    // the counter must start at zero (a call that did not complete may have left it set)
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return moe::launch_route(x, T, D, Wr, bias, E, k, ids, gates, logits, ws, s);
+}
+

@@ -23,7 +23,7 @@ MOE_Q2_32, MOE_Q3_32, MOE_Q3_S256 = 0, 1, 2
 
 EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_size", "moe_workspace_size",
            "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
-           "moe_status_string"]
+           "moe_status_string", "moe_route_topk_static"]
 
 
 class MoeError(RuntimeError):
@@ -67,6 +67,8 @@ def lib():
         L.moe_combine.argtypes = [P, P, i, i, i, P, P, P, P]
         L.moe_dequantize.restype = i
         L.moe_dequantize.argtypes = [ctypes.POINTER(moe_pool), i, i, P, P]
+        L.moe_route_topk_static.restype = i
+        L.moe_route_topk_static.argtypes = [P, i, i, P, P, i, i, P, P, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [i]
         _lib = L
@@ -123,6 +125,15 @@ def moe_route_topk(x, Wr, bias, k, ids, gates, ws, logits=None, stream=None):
     st = lib().moe_route_topk(_p(x), T, D, _p(Wr), _p(bias), E, k, _p(ids), _p(gates), _p(logits),
                               _p(ws), ws.numel(), _stream(stream))
     _check("moe_route_topk", st)
+
+
+def moe_route_topk_static(x, Wr, bias, k, ids, gates, logits=None, stream=None):
+    """moe_route_topk with library-owned static scratch (T <= 4, E <= 1024)."""
+    T, D = x.shape
+    E = Wr.shape[0]
+    st = lib().moe_route_topk_static(_p(x), T, D, _p(Wr), _p(bias), E, k, _p(ids), _p(gates), _p(logits),
+                                     _stream(stream))
+    _check("moe_route_topk_static", st)
 
 
 def moe_expert_forward(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_list, miss_count, ws, stream=None):

@@ -145,6 +145,26 @@ moe_status moe_route_topk(const uint16_t* x, int T, int D, const uint16_t* Wr,
                           float* logits, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_route_topk without a workspace argument, for callers that cannot
+ * allocate device memory themselves: code running under a host framework that
+ * owns all device memory through a fixed, pre-sized arena, or code that must
+ * not call cudaMalloc on its path (e.g. while a CUDA stream is being captured).
+ * The pages describe no such call; it is an addition of this library.
+ *   Same arguments and results as moe_route_topk (decode path only).
+ *   Scratch: a library-owned static device array of 16,640 bytes per GPU, held
+ *   until the process exits; sizes beyond it (T > 4 or E > 1024) return
+ *   MOE_ERR_UNSUPPORTED.  Nothing is allocated or freed.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  Every call resets the array's counter with an async memset on
+ *   `stream`.  All calls on a device share the array: calls that overlap on the
+ *   GPU (different streams) race and must be serialised by the caller.
+ */
+moe_status moe_route_topk_static(const uint16_t* x, int T, int D, const uint16_t* Wr,
+                                 const float* bias, int E, int k, int32_t* ids, float* gates,
+                                 float* logits, moe_stream_t stream);
+
+/*
  * Slot lookup, miss list and expert FFNs.
  *   slot_table int32 [E]: expert id -> slot, -1 = not resident.  Any entry
  *          outside [0, n_slots) is treated as a miss.
