@@ -1,7 +1,7 @@
 // prefill.cu — expert pass for chunks of many tokens (T > 4): a deterministic
 // tokens-by-expert permute, then two grouped GEMMs on the 5th-generation tensor
-// cores (tcgen05, accumulators in tensor memory) whose weight operand is
-// dequantised from the 2-/3-bit blocks into shared memory on the fly.
+// cores (tcgen05) whose weight operand is dequantised from the 2-/3-bit blocks
+// on the fly, straight into tensor memory.
 //
 // The pages: prefill runs in chunks, with expert transfers overlapped with GPU
 // compute (greenbean-ai "Strata 如何讓 12GB 顯卡跑 Qwen3.8-Flash-Next" §三);
@@ -11,11 +11,27 @@
 // Rows.  Every resident (token, rank) pair and every token's shared-expert
 // evaluation is one row; rows are grouped by expert (routed experts in id
 // order, tokens ascending within an expert), then the T shared rows.
-//   GEMM 1 (gate|up): per tile of 128 features x up to 256 rows of one group,
-//     acc_g = Wg x, acc_u = Wu x in TMEM; epilogue h = bf16(silu(acc_g) * acc_u)
-//   GEMM 2 (down): per tile of 128 outputs x up to 256 rows, acc = Wd h;
+//   GEMM 1 (gate|up): per tile of 64 features x up to 128 rows of one group,
+//     one M = 128 accumulator holds Wg x (lanes 0..63) and Wu x (lanes
+//     64..127) in TMEM; epilogue h = bf16(silu(Wg x) * (Wu x))
+//   GEMM 2 (down): per tile of 128 outputs x up to 128 rows, acc = Wd h;
 //     epilogue y = bf16(acc) into the expert_out rows
-// Both are "swap-AB": the weights are the M = 128 operand, the rows are N.
+// Both are "swap-AB": the weights are the M = 128 operand (A, in tensor
+// memory), the rows are N (B, in shared memory).
+//
+// Operand type.  The MMAs run kind::f16 with fp16 A and B.  Weights are
+// dequantised with packed fp16 arithmetic, which rounds once (Q2_32 / Q3_32:
+// fma(s, q, m); Q3_S256: fp16(d (sc - 32)) (q - 4), two roundings), i.e. to
+// within one fp16 ulp of the exact weight — finer than a bf16 weight.  The bf16
+// activations convert to fp16 exactly inside the fp16 range; an activation
+// of magnitude >= 65520 (x or h) sets kErrRange in the error word.
+//
+// K order.  Inside every group of 16 consecutive K indices the operands use
+// the order (0, 8, 1, 9, ..., 7, 15): one 32-bit word of A then holds the
+// weight pair (i, i + 8), which the block formats deliver in the same word at
+// the same bit offset of both halves.  x (gate|up) is staged into that order by
+// to_f16p_kernel and h (down) is written in it by the gate|up epilogue.
+#include <cuda.h>            // CUtensorMap types; the encoder is fetched at run time
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -25,16 +41,22 @@
 namespace moe {
 namespace {
 
+constexpr uint32_t kErrRange = 2u;     // error word: an activation outside the fp16 range
+
 constexpr int kChunk = 256;            // tokens per plan chunk
 constexpr int kMaxE = 1024;
-constexpr int kTileM = 128;
-constexpr int kTileN = 256;            // max rows per tile
-constexpr int kTileK = 64;             // one 128-byte swizzle atom of bf16
-constexpr int kStages = 3;
-constexpr int kDqWarps = 8;            // dequant + epilogue warps
-constexpr int kThreads = (kDqWarps + 2) * 32;   // + B gather warp + MMA warp
-constexpr int kGatherWarp = kDqWarps;
-constexpr int kMmaWarp = kDqWarps + 1;
+constexpr int kTileM = 128;            // weight rows per tile (MMA M)
+constexpr int kN1 = 128;               // max rows per gate|up tile
+constexpr int kN2 = 128;               // max rows per down tile
+constexpr int kGateRows = 64;          // gate|up tile: 64 gate + the same 64 up features
+constexpr int kKStep = 64;             // K per row-operand stage: one 128-byte swizzle atom of fp16
+constexpr int kRoundK = 128;           // K per dequant round (two k-steps)
+constexpr int kDqWarps = 16;           // 4 per TMEM lane quadrant
+constexpr int kEpiWarps = 4;
+constexpr int kTmaWarp = kDqWarps + kEpiWarps;
+constexpr int kGatherWarp = kTmaWarp + 1;
+constexpr int kMmaWarp = kGatherWarp + 1;
+constexpr int kGemmThreads = (kMmaWarp + 1) * 32;
 
 // ---------------------------------------------------------------- workspace
 struct PrefillWs {
@@ -44,29 +66,37 @@ struct PrefillWs {
     int4* tiles1;         // (group row0, rows, m0, slot)
     int4* tiles2;
     int32_t* perm;        // [rows] token of each row
-    uint16_t* h;          // [rows][F] bf16
+    uint16_t* x16;        // [T][x16_stride(D)] fp16, K-permuted
+    uint16_t* h;          // [rows][F] fp16, K-permuted
     uint32_t* err;
 };
 
 inline size_t align256(size_t n) { return (n + 255) / 256 * 256; }
+// Row stride (elements) of the fp16 copy of x: padded by 128 bytes so that the
+// same K slice of different rows does not fall on one L2 set.
+inline int x16_stride(int D) { return D + 64; }
 
 struct WsSizes {
-    size_t hist, miss, meta, t1, t2, perm, h, total;
+    size_t hist, miss, meta, t1, t2, perm, x16, h, total;
+    size_t max_t1, max_t2;
 };
 
 inline WsSizes ws_sizes(int T, int D, int F, int E, int k) {
     const int nchunk = (T + kChunk - 1) / kChunk;
     const size_t rows = (size_t)T * (k + 1);
-    const size_t ntiles = rows / kTileN + (size_t)E + 2;   // bound on sum over groups of ceil(n/256)
     WsSizes s;
+    // bound on sum over groups of ceil(n / N): rows / N + (number of groups)
+    s.max_t1 = (rows / kN1 + (size_t)E + 2) * (F / kGateRows);
+    s.max_t2 = (rows / kN2 + (size_t)E + 2) * (D / kTileM);
     s.hist = align256((size_t)nchunk * E * 4);
     s.miss = align256((size_t)nchunk * 4);
     s.meta = 256;
-    s.t1 = align256(ntiles * (F / kTileM) * sizeof(int4));
-    s.t2 = align256(ntiles * (D / kTileM) * sizeof(int4));
+    s.t1 = align256(s.max_t1 * sizeof(int4));
+    s.t2 = align256(s.max_t2 * sizeof(int4));
     s.perm = align256(rows * 4);
+    s.x16 = align256((size_t)T * x16_stride(D) * 2);
     s.h = align256(rows * F * 2);
-    s.total = 1024 + s.hist + s.miss + s.meta + s.t1 + s.t2 + s.perm + s.h;
+    s.total = 1024 + s.hist + s.miss + s.meta + s.t1 + s.t2 + s.perm + s.x16 + s.h;
     return s;
 }
 
@@ -82,6 +112,7 @@ inline PrefillWs carve(void* ws, int T, int D, int F, int E, int k) {
     w.tiles1 = reinterpret_cast<int4*>(p); p += s.t1;
     w.tiles2 = reinterpret_cast<int4*>(p); p += s.t2;
     w.perm = reinterpret_cast<int32_t*>(p); p += s.perm;
+    w.x16 = reinterpret_cast<uint16_t*>(p); p += s.x16;
     w.h = reinterpret_cast<uint16_t*>(p);
     return w;
 }
@@ -148,6 +179,7 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
     __shared__ int tot[kMaxE];
     __shared__ int off[kMaxE + 1];
     __shared__ int t1off[kMaxE + 2];
+    __shared__ int t2off[kMaxE + 2];
     pdl_wait();
     const int nchunk = (a.T + kChunk - 1) / kChunk;
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
@@ -165,16 +197,19 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
         for (int c = 0; c < nchunk; ++c) { const int v = a.w.miss_hist[c]; a.w.miss_hist[c] = m; m += v; }
         a.miss_count[0] = m;
         a.w.meta[0] = run;
-        // tile counts per group (routed groups in id order, then the shared group)
-        int nt = 0;
+        // row tiles per group (routed groups in id order, then the shared group)
+        int n1 = 0, n2 = 0;
         for (int e = 0; e <= a.E; ++e) {
-            t1off[e] = nt;
+            t1off[e] = n1;
+            t2off[e] = n2;
             const int n = e < a.E ? tot[e] : a.T;
-            nt += (n + kTileN - 1) / kTileN;
+            n1 += (n + kN1 - 1) / kN1;
+            n2 += (n + kN2 - 1) / kN2;
         }
-        t1off[a.E + 1] = nt;
-        a.w.meta[1] = nt * (a.F / kTileM);
-        a.w.meta[2] = nt * (a.D / kTileM);
+        t1off[a.E + 1] = n1;
+        t2off[a.E + 1] = n2;
+        a.w.meta[1] = n1 * (a.F / kGateRows);
+        a.w.meta[2] = n2 * (a.D / kTileM);
     }
     __syncthreads();
     // per-chunk base rows of every expert
@@ -186,17 +221,21 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
             run += v;
         }
     }
-    // tile lists: group e (or the shared group), n-tile, m-tile
-    const int mt1 = a.F / kTileM, mt2 = a.D / kTileM;
+    // tile lists: group, row tile, then weight-row tile (the fastest index)
+    const int mt1 = a.F / kGateRows, mt2 = a.D / kTileM;
     for (int g = threadIdx.x; g <= a.E; g += blockDim.x) {
         const int n = g < a.E ? tot[g] : a.T;
         const int row0 = g < a.E ? off[g] : off[a.E];
         const int slot = g < a.E ? (n > 0 ? plan_slot(a, g) : -1) : a.shared_slot;
-        const int first = t1off[g], cnt = t1off[g + 1] - first;
-        for (int j = 0; j < cnt; ++j) {
-            const int r0 = row0 + j * kTileN, rows = min(kTileN, n - j * kTileN);
-            for (int m = 0; m < mt1; ++m) a.w.tiles1[(size_t)(first + j) * mt1 + m] = make_int4(r0, rows, m * kTileM, slot);
-            for (int m = 0; m < mt2; ++m) a.w.tiles2[(size_t)(first + j) * mt2 + m] = make_int4(r0, rows, m * kTileM, slot);
+        for (int j = 0; j < t1off[g + 1] - t1off[g]; ++j) {
+            const int r0 = row0 + j * kN1, rows = min(kN1, n - j * kN1);
+            for (int m = 0; m < mt1; ++m)
+                a.w.tiles1[(size_t)(t1off[g] + j) * mt1 + m] = make_int4(r0, rows, m * kGateRows, slot);
+        }
+        for (int j = 0; j < t2off[g + 1] - t2off[g]; ++j) {
+            const int r0 = row0 + j * kN2, rows = min(kN2, n - j * kN2);
+            for (int m = 0; m < mt2; ++m)
+                a.w.tiles2[(size_t)(t2off[g] + j) * mt2 + m] = make_int4(r0, rows, m * kTileM, slot);
         }
     }
 }
@@ -248,7 +287,40 @@ __global__ void __launch_bounds__(kChunk) plan_scatter_kernel(PlanArgs a) {
     a.rowmap[(size_t)t * (k + 1) + k] = S + t;
 }
 
-// ---------------------------------------------------------------- tcgen05 helpers
+// ---------------------------------------------------------------- x -> fp16, K-permuted
+MOE_DEVINL uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+MOE_DEVINL uint32_t bf16_half(uint32_t w, int hi) { return hi ? (w & 0xffff0000u) : (w << 16); }
+
+// One thread per 16-element group: out word i = (x[i], x[i + 8]) in fp16.
+__global__ void __launch_bounds__(256) to_f16p_kernel(const uint16_t* __restrict__ x, size_t ngroups, int row_groups,
+                                                      int out_stride, uint16_t* __restrict__ x16, uint32_t* err) {
+    pdl_wait();
+    bool bad = false;
+    for (size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x; gi < ngroups; gi += (size_t)gridDim.x * blockDim.x) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(x) + 2 * gi);
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(x) + 2 * gi + 1);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float lo = __uint_as_float(bf16_half(aw[i >> 1], i & 1));
+            const float hi = __uint_as_float(bf16_half(bw[i >> 1], i & 1));
+            bad |= !(fabsf(lo) < 65520.f) || !(fabsf(hi) < 65520.f);
+            o[i] = pack_f16x2(lo, hi);
+        }
+        const size_t t = gi / row_groups, gc = gi % row_groups;
+        uint4* dst = reinterpret_cast<uint4*>(x16 + t * out_stride + gc * 16);
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    if (bad) atomicOr(err, kErrRange);
+}
+
+// ---------------------------------------------------------------- tcgen05 / TMA helpers
 MOE_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr & 0x3ffffu) >> 4);        // start address
@@ -258,15 +330,16 @@ MOE_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
     d |= (uint64_t)2 << 61;                           // 128-byte swizzle
     return d;
 }
-// kind::f16, A = B = bf16, D = f32, both K-major, M = 128.
-MOE_DEVINL uint32_t instr_desc(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+// kind::f16, A = B = fp16, D = f32, A and B K-major, M = 128.
+MOE_DEVINL uint32_t instr_desc_f16(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
 }
-MOE_DEVINL void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[tmem] * B[smem]^T
+MOE_DEVINL void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 MOE_DEVINL void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -274,280 +347,544 @@ MOE_DEVINL void mma_commit(uint64_t* bar) {
 }
 MOE_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 MOE_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-MOE_DEVINL void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-    uint32_t r[8];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+MOE_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
 }
-MOE_DEVINL void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+MOE_DEVINL void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+MOE_DEVINL void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
 }
-MOE_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+MOE_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// L2 policies: the weight stream is read once (evict first); the activation
+// rows are re-read by every weight tile of their group (evict last).
+MOE_DEVINL uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+MOE_DEVINL uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+MOE_DEVINL void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+        "%3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+MOE_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+        "%3}], [%4], %5;" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// Four rows (y0..y3) of a 2D tensor whose box is one row high, stacked in
+// shared memory at the box pitch.
+MOE_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2, int y3, uint64_t* bar,
+                            uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+// Bounded wait that does not give up early on the error word: used to drain
+// copies and MMAs still in flight before the CTA exits.
+MOE_DEVINL void mbar_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+}
+
+// AND of `v` over the epilogue warps (named barrier 1): they leave their loop
+// together, so none is left waiting at a named barrier.
+MOE_DEVINL bool epilogue_all(bool v, int nthreads_const_128) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(nthreads_const_128)
+        : "memory");
+    return r != 0;
+}
 
 // Byte offset of the 16-byte chunk c of row r in a K-major 128B-swizzled tile.
 MOE_DEVINL uint32_t sw128(int r, int c) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)); }
 
-MOE_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
+// ---------------------------------------------------------------- dequantisation to fp16 pairs
+// fp16 "magic" numbers 2^(10-b): OR-ing a code field that sits at bit b of a
+// half into one gives 2^(10-b) + code exactly; subtracting it back gives the
+// code (exact small integers).
+struct Magic {
+    uint32_t m1024, m256, m128, m64, m16, m8, m4;      // f16x2, both halves
+    uint32_t s1028, s132, s20, s12;                     // magic + 4 (the Q3_S256 code centre)
+};
+MOE_DEVINL uint32_t opaque_u32(uint32_t v) {
     uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
+    return r;
+}
+MOE_DEVINL Magic make_magic() {
+    Magic m;
+    m.m1024 = opaque_u32(0x64006400u);
+    m.m256 = opaque_u32(0x5C005C00u);
+    m.m128 = opaque_u32(0x58005800u);
+    m.m64 = opaque_u32(0x54005400u);
+    m.m16 = opaque_u32(0x4C004C00u);
+    m.m8 = opaque_u32(0x48004800u);
+    m.m4 = opaque_u32(0x44004400u);
+    m.s1028 = opaque_u32(0x64046404u);
+    m.s132 = opaque_u32(0x58205820u);
+    m.s20 = opaque_u32(0x4D004D00u);
+    m.s12 = opaque_u32(0x4A004A00u);
+    return m;
+}
+template <uint32_t MASK>
+MOE_DEVINL uint32_t field_or(uint32_t w, uint32_t magic) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "n"(MASK), "r"(magic));   // (w & MASK) | magic
+    return r;
+}
+MOE_DEVINL uint32_t hsub2u(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+MOE_DEVINL uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+MOE_DEVINL uint32_t hmul2u(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 
-// ---------------------------------------------------------------- dequantisation
-// Exact weights w = fmaf(s, q, m) (Q2_32 / Q3_32) or d (sc - 32)(q - 4)
-// (Q3_S256) for 32 consecutive codes, then rounded to bf16 (nearest even).
-// Codes are taken from their words with the same bit-field logic as the
-// format definition: bit stream position nbits * j.
-template <int NB>
-MOE_DEVINL int field(const uint32_t* w, int j) {
-    const int bit = NB * j, wi = bit >> 5, sh = bit & 31;
-    const uint32_t lo = w[wi];
-    const uint32_t hi = (sh + NB > 32) ? w[wi + 1] : 0u;
-    return (int)(__funnelshift_r(lo, hi, sh) & ((1u << NB) - 1u));
+// Q2_32, one 16-weight group: word w holds code i at bits [2i, 2i+2).
+// out[i] = (w_i, w_{i+8}) = fma(s, q, m) in fp16.
+MOE_DEVINL void dq_q2_group(uint32_t w, uint32_t s2, uint32_t m2, const Magic& M, uint32_t* out) {
+    const uint32_t w10 = w >> 10;
+    out[0] = hfma2u(s2, hsub2u(field_or<0x00030003u>(w, M.m1024), M.m1024), m2);
+    out[1] = hfma2u(s2, hsub2u(field_or<0x000C000Cu>(w, M.m256), M.m256), m2);
+    out[2] = hfma2u(s2, hsub2u(field_or<0x00300030u>(w, M.m64), M.m64), m2);
+    out[3] = hfma2u(s2, hsub2u(field_or<0x00C000C0u>(w, M.m16), M.m16), m2);
+    out[4] = hfma2u(s2, hsub2u(field_or<0x03000300u>(w, M.m4), M.m4), m2);
+    out[5] = hfma2u(s2, hsub2u(field_or<0x00030003u>(w10, M.m1024), M.m1024), m2);
+    out[6] = hfma2u(s2, hsub2u(field_or<0x000C000Cu>(w10, M.m256), M.m256), m2);
+    out[7] = hfma2u(s2, hsub2u(field_or<0x00300030u>(w10, M.m64), M.m64), m2);
 }
 
-template <int FMT>
-struct Dq {
-    static constexpr int kCodeChunk = (FMT == MOE_Q2_32) ? 8 : 12;   // code bytes per 32 weights
-    static constexpr int kBlock = (FMT == MOE_Q3_S256) ? 256 : 32;
-    static constexpr int kBlockCode = (FMT == MOE_Q2_32) ? 8 : (FMT == MOE_Q3_32 ? 12 : 96);
-};
-
-// Dequantise 32 weights (chunk cb of row `row`, K weights per row) of plane pl
-// into 16 packed bf16 pairs.
-template <int FMT>
-MOE_DEVINL void dequant32(const uint8_t* cplane, const uint8_t* mplane, const uint8_t* dplane, int row, int K, int cb,
-                          uint32_t (&out)[16]) {
-    uint32_t w[3];
-    float wv[32];
-    if constexpr (FMT == MOE_Q3_S256) {
-        const int nsb = K / 256, sb = cb >> 3, j = cb & 7;
-        const size_t blk = (size_t)row * nsb + sb;
-        const uint8_t* p = cplane + blk * 96 + j * 12;
-        w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
-        w[1] = __ldg(reinterpret_cast<const uint32_t*>(p + 4));
-        w[2] = __ldg(reinterpret_cast<const uint32_t*>(p + 8));
-        const uint32_t* scp = reinterpret_cast<const uint32_t*>(mplane + blk * 12);
-        uint32_t sw[3] = {__ldg(scp), __ldg(scp + 1), __ldg(scp + 2)};
-        const float d = f16_bits_to_f32(__ldg(reinterpret_cast<const uint16_t*>(dplane) + blk));
-        const int s0 = field<6>(sw, 2 * j), s1 = field<6>(sw, 2 * j + 1);
-        const float S0 = d * (float)(s0 - 32), S1 = d * (float)(s1 - 32);   // exact
-#pragma unroll
-        for (int i = 0; i < 32; ++i) wv[i] = (i < 16 ? S0 : S1) * (float)(field<3>(w, i) - 4);   // exact
-    } else {
-        const size_t blk = (size_t)row * (K / 32) + cb;
-        const uint8_t* p = cplane + blk * Dq<FMT>::kCodeChunk;
-        if constexpr (FMT == MOE_Q2_32) {
-            const uint2 c = __ldg(reinterpret_cast<const uint2*>(p));
-            w[0] = c.x; w[1] = c.y; w[2] = 0;
-        } else {
-            w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
-            w[1] = __ldg(reinterpret_cast<const uint32_t*>(p + 4));
-            w[2] = __ldg(reinterpret_cast<const uint32_t*>(p + 8));
-        }
-        const float2 sm = __half22float2(*reinterpret_cast<const __half2*>(mplane + blk * 4));
-        constexpr int NB = (FMT == MOE_Q2_32) ? 2 : 3;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) wv[i] = __fmaf_rn(sm.x, (float)field<NB>(w, i), sm.y);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) out[i] = pack_bf16x2(wv[2 * i], wv[2 * i + 1]);
+// 3-bit codes of one 16-weight group, given P = (stream bits [0,16) | [24,40))
+// and P2 = (bits [8,24) | [32,48)) of the group's 48-bit stream: code i of the
+// low half (code i + 8 of the high half) sits at bit 3i of P for i <= 4 and at
+// bit 3i - 8 of P2 for i >= 5.  q[i] = the code pair, minus 4 when CENTRED.
+template <bool CENTRED>
+MOE_DEVINL void q3_codes(uint32_t P, uint32_t P2, const Magic& M, uint32_t* q) {
+    const uint32_t P9 = P >> 9, P10 = P2 >> 10;
+    q[0] = hsub2u(field_or<0x00070007u>(P, M.m1024), CENTRED ? M.s1028 : M.m1024);
+    q[1] = hsub2u(field_or<0x00380038u>(P, M.m128), CENTRED ? M.s132 : M.m128);
+    q[2] = hsub2u(field_or<0x01C001C0u>(P, M.m16), CENTRED ? M.s20 : M.m16);
+    q[3] = hsub2u(field_or<0x00070007u>(P9, M.m1024), CENTRED ? M.s1028 : M.m1024);
+    q[4] = hsub2u(field_or<0x00380038u>(P9, M.m128), CENTRED ? M.s132 : M.m128);
+    q[5] = hsub2u(field_or<0x03800380u>(P2, M.m8), CENTRED ? M.s12 : M.m8);
+    q[6] = hsub2u(field_or<0x00070007u>(P10, M.m1024), CENTRED ? M.s1028 : M.m1024);
+    q[7] = hsub2u(field_or<0x00380038u>(P10, M.m128), CENTRED ? M.s132 : M.m128);
 }
 
-template <int FMT>
-struct PlanesP {
-    const uint8_t* c;
-    const uint8_t* m;
-    const uint8_t* d;
-};
-template <int FMT>
-MOE_DEVINL PlanesP<FMT> pplanes(const PoolView& P, int slot, int mat) {
-    const size_t blocks = (size_t)P.D * P.F / Dq<FMT>::kBlock;
-    PlanesP<FMT> pl;
-    pl.c = P.codes + (size_t)slot * P.stride_c + (size_t)mat * blocks * Dq<FMT>::kBlockCode;
-    const uint8_t* meta = P.scales + (size_t)slot * P.stride_s;
-    if constexpr (FMT == MOE_Q3_S256) {
-        pl.m = meta + (size_t)mat * blocks * 12;
-        pl.d = meta + 3 * blocks * 12 + (size_t)mat * blocks * 2;
-    } else {
-        pl.m = meta + (size_t)mat * blocks * 4;
-        pl.d = nullptr;
-    }
-    return pl;
+// One 32-weight block (12 code bytes = words c0, c1, c2) of a 3-bit format:
+// group 0 = stream bytes 0..5, group 1 = bytes 6..11.
+template <bool CENTRED>
+MOE_DEVINL void q3_block_codes(uint32_t c0, uint32_t c1, uint32_t c2, const Magic& M, uint32_t* q) {
+    q3_codes<CENTRED>(__byte_perm(c0, c1, 0x4310), __byte_perm(c0, c1, 0x5421), M, q);
+    q3_codes<CENTRED>(__byte_perm(c1, c2, 0x6532), __byte_perm(c1, c2, 0x7643), M, q + 8);
 }
 
 // ---------------------------------------------------------------- grouped GEMM
-struct GemmArgs {
-    PoolView P;
+struct GemmParams {
     const int4* tiles;
     const int32_t* n_tiles;      // device count
-    const uint16_t* src;         // MODE 1: x [T][D]; MODE 2: h [rows][F]
+    const uint16_t* src;         // MODE 1: x16 [T][x16_stride(D)]; MODE 2: h [rows][F]
     const int32_t* perm;         // MODE 1: token of each row
-    uint16_t* dst;               // MODE 1: h [rows][F]; MODE 2: y rows [rows][D]
+    uint16_t* dst;               // MODE 1: h [rows][F] fp16; MODE 2: y rows [rows][D] bf16
+    const uint8_t* scales;       // Q3_S256: the pool's scale base (sub-scales, d)
+    size_t stride_s;
+    int D, F;
     uint32_t* err;
 };
 
-// MODE 1: gate|up (two accumulators, K = D, SwiGLU epilogue into h).
-// MODE 2: down (one accumulator, K = F, epilogue into the y rows).
+template <int FMT>
+struct GemmFmt {
+    static constexpr int kCb = FMT == MOE_Q2_32 ? 8 : 12;                  // code bytes per 32 weights
+    static constexpr int kRb = 4 * kCb;                                    // code bytes per row per round
+    static constexpr bool kTmaScales = FMT != MOE_Q3_S256;
+    static constexpr uint32_t kStageBytes = 128 * kRb + (kTmaScales ? 128 * 16 : 0);
+};
+
+constexpr int kNmax = 128;                 // rows per tile (MMA N <= 128)
+constexpr int kAccCols = 128;              // one accumulator: 128 lanes x N fp32 columns
+constexpr int kAccBufs = 2;                // double-buffered accumulators
+constexpr int kABufs = 4;                  // dequantised A round buffers, one per warp group
+constexpr int kABufCols = 2 * 32;          // a round: 2 k-steps x 32 columns (64 fp16 per lane)
+constexpr int kACol0 = kAccBufs * kAccCols;
+constexpr uint32_t kBStepBytes = (uint32_t)kNmax * kKStep * 2;     // one k-step of the row operand
+constexpr uint32_t kBStageBytes = 2 * kBStepBytes;                  // a round: two k-steps
+constexpr int kCodeStages8 = 8;
+constexpr uint32_t kCodeStage8Bytes = 8192;
+constexpr uint32_t kGemmSmem = kCodeStages8 * kCodeStage8Bytes + kABufs * kBStageBytes;
+static_assert(kACol0 + kABufs * kABufCols == 512, "TMEM columns");
+
+// Warp roles: 0..15 dequantise (warp w owns TMEM lanes 32 (w % 4) ..; the four
+// warps of a lane quadrant take rounds in turn), 16..19 epilogue, 20 TMA for
+// the code tiles, 21 row-operand gather, 22 MMA issue.
+// The A operand of a tile has 128 rows: MODE 1 rows 0..63 are the gate
+// features m0..m0+63 and rows 64..127 the same up features, so one M = 128
+// accumulator holds both halves of the SwiGLU; MODE 2 rows are 128 outputs.
+// TMEM columns: two accumulators [0, 256), then four A round buffers.
 template <int FMT, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) expert_gemm_kernel(GemmArgs g) {
-    constexpr int NMAT = (MODE == 1) ? 2 : 1;
-    constexpr uint32_t kA = kTileM * kTileK * 2;            // 16 KB per weight matrix
-    constexpr uint32_t kB = kTileN * kTileK * 2;            // 32 KB
-    constexpr uint32_t kStage = NMAT * kA + kB;
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_scales,
+                       const __grid_constant__ CUtensorMap map_rows, GemmParams g) {
+    using Fm = GemmFmt<FMT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ uint64_t full_a[kStages], full_b[kStages], empty[kStages], done_bar;
+    __shared__ uint64_t full_c[kCodeStages8], empty_c[kCodeStages8];
+    // round slot i (= round % 4): its TMEM A buffer and its row-operand stage are
+    // filled by full_a[i] / full_b[i] and released together by round_empty[i]
+    __shared__ uint64_t full_a[kABufs], full_b[kABufs], round_empty[kABufs];
+    __shared__ uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain_bar;
     __shared__ uint32_t tmem_base;
-    __shared__ int rows_idx[kTileN];
-    // 1024-byte alignment of the swizzled tiles
+    __shared__ int rows_idx[kNmax];
+    __shared__ float gate_x[kGateRows][17];        // epilogue: gate values handed to the up lanes
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* code_ring = smem;
+    uint8_t* b_ring = smem + kCodeStages8 * kCodeStage8Bytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    pdl_wait();
-    const int tile = blockIdx.x;
-    if (tile >= __ldg(g.n_tiles)) return;
-    if (*reinterpret_cast<volatile uint32_t*>(g.err)) return;   // an earlier CTA gave up
-    const int4 td = __ldg(g.tiles + tile);
-    const int row0 = td.x, nrows = td.y, m0 = td.z, slot = td.w;
-    const int npad = (nrows + 15) & ~15;
-    const int D = g.P.D, F = g.P.F;
-    const int K = (MODE == 1) ? D : F;
-    const int KT = K / kTileK;
+    const int D = g.D, F = g.F;
+    const int K = MODE == 1 ? D : F;
+    const int R = K / kRoundK;                  // dequant rounds per tile
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full_a[s], kDqWarps);
-            mbar_init(&full_b[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kCodeStages8; ++s) {
+            mbar_init(&full_c[s], 1);
+            mbar_init(&empty_c[s], 4);
         }
-        mbar_init(&done_bar, 1);
+        for (int s = 0; s < kABufs; ++s) {
+            mbar_init(&full_a[s], 4);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&round_empty[s], 1);
+        }
+        for (int s = 0; s < kAccBufs; ++s) {
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], kEpiWarps);
+        }
+        mbar_init(&drain_bar, 1);
         fence_mbar_init();
     }
     if (warp == kMmaWarp) {
-        const uint32_t ncols = (MODE == 1) ? 512u : 256u;
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base)),
-                     "r"(ncols)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&tmem_base))
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    const int tix = (int)threadIdx.x;
-    if (tix < kTileN) rows_idx[tix] = tix < nrows ? ((MODE == 1) ? __ldg(g.perm + row0 + tix) : row0 + tix) : -1;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
-    if (warp < kDqWarps) {
-        // ---------------- producers of the weight tiles
-        const PlanesP<FMT> pl0 = pplanes<FMT>(g.P, slot, MODE == 1 ? 0 : 2);
-        const PlanesP<FMT> pl1 = pplanes<FMT>(g.P, slot, 1);
-        // 256 threads: MODE 1 -> thread = (matrix, row), 64 weights each per stage;
-        //              MODE 2 -> thread = (row, half), 32 weights each per stage.
-        const int tid = threadIdx.x;
-        for (int j = 0; j < KT; ++j) {
-            const int s = j % kStages;
-            if (j >= kStages && !mbar_wait(&empty[s], ((j / kStages) - 1) & 1, g.err)) break;
-            uint8_t* a_base = smem + (size_t)s * kStage;
-            if constexpr (MODE == 1) {
-                const int mat = tid >> 7, r = tid & 127;
-                const PlanesP<FMT>& pl = mat ? pl1 : pl0;
-                uint8_t* at = a_base + mat * kA;
+    pdl_wait();
+    const int n_tiles = __ldg(g.n_tiles);
+    const bool dead = *reinterpret_cast<volatile uint32_t*>(g.err) != 0;   // an earlier kernel gave up
+    const int first = blockIdx.x, step = gridDim.x;
+
+    if (!dead && warp < kDqWarps) {
+        // ---------------- dequantisation into TMEM
+        const int q = warp & 3, par = warp >> 2;
+        const int r = 32 * q + lane;
+        const Magic Mg = make_magic();
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+        int li = 0;
+        bool ok = true;
+        for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
+            const int4 td = __ldg(g.tiles + tile);
+            const int m0 = td.z, slot = td.w;
+            for (int rr = 0; rr < R; ++rr) {
+                const int gr = li * R + rr;
+                if ((gr & 3) != par) continue;
+                const int st = gr % kCodeStages8;
+                if (!mbar_wait(&full_c[st], (gr / kCodeStages8) & 1, g.err)) { ok = false; break; }
+                const uint8_t* cs = code_ring + st * kCodeStage8Bytes;
+                // codes of this row for the round's 4 blocks, and the (s, m) words
+                uint32_t cw[3 * 4];
+                uint32_t sw[4] = {0, 0, 0, 0};
+                if constexpr (FMT == MOE_Q2_32) {
+                    const uint8_t* row = cs + r * 32;
+                    const uint32_t x = (uint32_t)((r >> 2) & 1);     // 32-byte TMA swizzle
+                    const uint4 a = *reinterpret_cast<const uint4*>(row + ((0u ^ x) << 4));
+                    const uint4 b = *reinterpret_cast<const uint4*>(row + ((1u ^ x) << 4));
+                    cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
+                    cw[4] = b.x; cw[5] = b.y; cw[6] = b.z; cw[7] = b.w;
+                } else {
+                    const uint8_t* row = cs + r * 48;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[16];
-                    dequant32<FMT>(pl.c, pl.m, pl.d, m0 + r, K, 2 * j + half, pk);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(at + sw128(r, half * 4 + c)) =
-                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                    for (int i = 0; i < 3; ++i) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * i);
+                        cw[4 * i] = a.x; cw[4 * i + 1] = a.y; cw[4 * i + 2] = a.z; cw[4 * i + 3] = a.w;
+                    }
                 }
-            } else {
-                const int r = tid >> 1, half = tid & 1;
-                uint32_t pk[16];
-                dequant32<FMT>(pl0.c, pl0.m, pl0.d, m0 + r, K, 2 * j + half, pk);
+                if constexpr (Fm::kTmaScales) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(cs + 128 * Fm::kRb + r * 16);
+                    sw[0] = a.x; sw[1] = a.y; sw[2] = a.z; sw[3] = a.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty_c[st]);
+                // Q3_S256: the super-block's sub-scales and d, straight from global memory
+                float sd = 0.f;
+                uint32_t sub0 = 0, sub1 = 0, sub2 = 0;
+                if constexpr (FMT == MOE_Q3_S256) {
+                    const int pm = MODE == 1 ? (r >> 6) : 2;                   // plane: gate, up, down
+                    const int wrow = m0 + (MODE == 1 ? (r & 63) : r);
+                    const size_t blocks = (size_t)D * F / 256;                 // super-blocks per plane
+                    const size_t sb = (size_t)wrow * (K / 256) + (size_t)(rr >> 1);
+                    const uint8_t* base = g.scales + (size_t)slot * g.stride_s;
+                    const uint8_t* sp = base + (size_t)pm * blocks * 12 + sb * 12;
+                    sub0 = __ldg(reinterpret_cast<const uint32_t*>(sp));
+                    sub1 = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
+                    sub2 = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
+                    sd = f16_bits_to_f32(__ldg(reinterpret_cast<const uint16_t*>(base + 3 * blocks * 12) + pm * blocks + sb));
+                }
+                const int buf = par, use = gr >> 2;
+                const uint32_t col0 = (uint32_t)(kACol0 + buf * kABufCols);
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    *reinterpret_cast<uint4*>(a_base + sw128(r, half * 4 + c)) =
-                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                for (int b = 0; b < 4; ++b) {
+                    uint32_t o[16];
+                    if constexpr (FMT == MOE_Q2_32) {
+                        const uint32_t s2 = __byte_perm(sw[b], 0, 0x1010), m2 = __byte_perm(sw[b], 0, 0x3232);
+                        dq_q2_group(cw[2 * b], s2, m2, Mg, o);
+                        dq_q2_group(cw[2 * b + 1], s2, m2, Mg, o + 8);
+                    } else if constexpr (FMT == MOE_Q3_32) {
+                        const uint32_t s2 = __byte_perm(sw[b], 0, 0x1010), m2 = __byte_perm(sw[b], 0, 0x3232);
+                        q3_block_codes<false>(cw[3 * b], cw[3 * b + 1], cw[3 * b + 2], Mg, o);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = hfma2u(s2, o[i], m2);
+                    } else {
+                        // sub-blocks 2c and 2c + 1 of the super-block, c = 32-weight chunk (0..7)
+                        const int c = 4 * (rr & 1) + b;
+                        const uint64_t lo = ((uint64_t)sub1 << 32) | sub0, hi = ((uint64_t)sub2 << 32) | sub1;
+                        const uint32_t bits = c < 4 ? (uint32_t)(lo >> (12 * c)) : (uint32_t)(hi >> (12 * c - 32));
+                        const float S0 = sd * (float)((int)(bits & 63u) - 32);
+                        const float S1 = sd * (float)((int)((bits >> 6) & 63u) - 32);
+                        const uint32_t S0h = pack_f16x2(S0, S0), S1h = pack_f16x2(S1, S1);
+                        q3_block_codes<true>(cw[3 * b], cw[3 * b + 1], cw[3 * b + 2], Mg, o);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = hmul2u(i < 8 ? S0h : S1h, o[i]);
+                    }
+                    if (b == 0 && use > 0) {
+                        if (!mbar_wait(&round_empty[buf], (use - 1) & 1, g.err)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    // block b -> k-step b / 2, columns (b % 2) * 16 of the step's 32
+                    tmem_st16(lane_addr + col0 + (uint32_t)((b >> 1) * 32 + (b & 1) * 16), o);
+                }
+                if (!ok) break;
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_a[buf]);
             }
-            fence_proxy_async();     // make the generic-proxy stores visible to the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_a[s]);
         }
+    } else if (!dead && warp < kTmaWarp) {
         // ---------------- epilogue: TMEM -> registers -> global
-        if (mbar_wait(&done_bar, 0, g.err)) {
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
+        int li = 0;
+        bool range_bad = false, ok = true;
+        for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
+            const int4 td = __ldg(g.tiles + tile);
+            const int row0 = td.x, nrows = td.y, m0 = td.z;
+            const int npad = (nrows + 15) & ~15;
+            const int ab = li & 1;
+            bool got = mbar_wait(&acc_full[ab], (li >> 1) & 1, g.err);
+            if constexpr (MODE == 1) got = epilogue_all(got, kEpiWarps * 32);
+            if (!got) { ok = false; break; }
             tc_fence_after();
-            const int q = warp & 3;                      // TMEM lane quadrant
-            const int r = q * 32 + lane;                 // tile row = feature / output index
-            const int c_lo = (warp >> 2) * (npad / 2), c_hi = c_lo + npad / 2;
-            for (int c = c_lo; c < c_hi; c += 8) {
-                const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c;
-                float v0[8];
-                tmem_ld8(ta, v0);
+            const uint32_t acc = lane_addr + (uint32_t)(ab * kAccCols);
+            for (int c = 0; c < npad; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(acc + (uint32_t)c, v);
+                tmem_ld_wait();
                 if constexpr (MODE == 1) {
-                    float v1[8];
-                    tmem_ld8(ta + 256, v1);
+                    // lanes 0..63 hold gate, 64..127 up of the same features
+                    if (q < 2) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int n = c + i;
-                        if (n < nrows) {
-                            const float gte = v0[i], up = v1[i];
-                            const float hv = gte / (1.0f + expf(-gte)) * up;
-                            g.dst[(size_t)(row0 + n) * F + m0 + r] = f32_to_bf16_rne(hv);
+                        for (int i = 0; i < 16; ++i) gate_x[r][i] = __uint_as_float(v[i]);
+                    }
+                    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+                    if (q >= 2) {
+                        const int f = m0 + (r - 64);
+                        const int fpos = (f & ~15) | ((f & 7) << 1) | ((f >> 3) & 1);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int n = c + i;
+                            if (n < nrows) {
+                                const float gte = gate_x[r - 64][i], up = __uint_as_float(v[i]);
+                                const float hv = gte / (1.0f + expf(-gte)) * up;
+                                const float hb = bf16_bits_to_f32(f32_to_bf16_rne(hv));   // h is a bf16 value
+                                range_bad |= !(fabsf(hb) < 65520.f);
+                                g.dst[(size_t)(row0 + n) * F + fpos] = __half_as_ushort(__float2half_rn(hb));
+                            }
                         }
                     }
+                    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
+                    for (int i = 0; i < 16; ++i) {
                         const int n = c + i;
-                        if (n < nrows) g.dst[(size_t)(row0 + n) * D + m0 + r] = f32_to_bf16_rne(v0[i]);
+                        if (n < nrows) g.dst[(size_t)(row0 + n) * D + m0 + r] = f32_to_bf16_rne(__uint_as_float(v[i]));
                     }
                 }
             }
-        }
-    } else if (warp == kGatherWarp) {
-        // ---------------- gather of the row operand (K-major, 128B swizzle) with cp.async
-        for (int j = 0; j < KT; ++j) {
-            const int s = j % kStages;
-            if (j >= kStages && !mbar_wait(&empty[s], ((j / kStages) - 1) & 1, g.err)) break;
-            const uint32_t b_base = smem_u32(smem + (size_t)s * kStage + NMAT * kA);
-            const size_t stride = (size_t)K;
-            for (int i = lane; i < npad * 8; i += 32) {
-                const int n = i >> 3, c = i & 7;
-                const int src_row = rows_idx[n] >= 0 ? rows_idx[n] : rows_idx[0];   // pad rows repeat row 0
-                cp_async16(b_base + sw128(n, c), g.src + (size_t)src_row * stride + (size_t)j * kTileK + c * 8);
-            }
-            cp_async_wait_all();
-            fence_proxy_async();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&full_b[s]);
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
         }
-    } else if (warp == kMmaWarp) {
-        // ---------------- single-thread MMA issue
+        if (range_bad) atomicOr(g.err, kErrRange);
+    } else if (!dead && warp == kTmaWarp) {
+        // ---------------- TMA loads of the code (and scale) tiles, one stage per round
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(npad);
+            const uint64_t pol = l2_evict_first();
+            int li = 0, issued = 0;
             bool ok = true;
-            for (int j = 0; j < KT && ok; ++j) {
-                const int s = j % kStages;
-                ok = mbar_wait(&full_a[s], (j / kStages) & 1, g.err) && mbar_wait(&full_b[s], (j / kStages) & 1, g.err);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t a_addr = smem_u32(smem + (size_t)s * kStage);
-                const uint32_t b_addr = a_addr + NMAT * kA;
+            for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
+                const int4 td = __ldg(g.tiles + tile);
+                const int m0 = td.z, slot = td.w;
+                for (int rr = 0; rr < R; ++rr) {
+                    const int gr = li * R + rr;
+                    const int st = gr % kCodeStages8;
+                    if (gr >= kCodeStages8 && !mbar_wait(&empty_c[st], ((gr / kCodeStages8) - 1) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* cs = code_ring + st * kCodeStage8Bytes;
+                    mbar_arrive_expect_tx(&full_c[st], Fm::kStageBytes);
+                    if constexpr (MODE == 1) {
+                        // gate rows m0.. into rows 0..63, up rows F + m0.. into rows 64..127
 #pragma unroll
-                for (int kk = 0; kk < kTileK / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
-                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                    mma_bf16(tmem, smem_desc_sw128(a_addr + kk * 32), bd, idesc, acc);
-                    if constexpr (MODE == 1) mma_bf16(tmem + 256, smem_desc_sw128(a_addr + kA + kk * 32), bd, idesc, acc);
+                        for (int m = 0; m < 2; ++m) {
+                            const int y = m * F + m0;
+                            tma_load_3d(smem_u32(cs + m * 64 * Fm::kRb), &map_codes, rr * Fm::kRb, y, slot, &full_c[st],
+                                        pol);
+                            if constexpr (Fm::kTmaScales)
+                                tma_load_3d(smem_u32(cs + 128 * Fm::kRb + m * 64 * 16), &map_scales, rr * 16, y, slot,
+                                            &full_c[st], pol);
+                        }
+                    } else {
+                        tma_load_3d(smem_u32(cs), &map_codes, rr * Fm::kRb, m0, slot, &full_c[st], pol);
+                        if constexpr (Fm::kTmaScales)
+                            tma_load_3d(smem_u32(cs + 128 * Fm::kRb), &map_scales, rr * 16, m0, slot, &full_c[st], pol);
+                    }
+                    issued = gr + 1;
                 }
-                mma_commit(&empty[s]);     // frees the stage once these MMAs completed
             }
-            mma_commit(&done_bar);         // all MMAs of the tile
+            // every issued stage completes before the CTA exits
+            for (int j = issued - kCodeStages8; j < issued; ++j)
+                if (j >= 0) mbar_drain(&full_c[j % kCodeStages8], (j / kCodeStages8) & 1);
+        }
+        __syncwarp();
+    } else if (!dead && warp == kGatherWarp) {
+        // ---------------- row operand (K-major, 128B swizzle) by TMA: gate|up gathers the
+        // rows' tokens four at a time; down reads its contiguous rows in 16-row boxes
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_last();
+            bool ok = true;
+            int issued = 0;
+            for (int tile = first, h = 0; tile < n_tiles && ok; tile += step) {
+                const int4 td = __ldg(g.tiles + tile);
+                const int row0 = td.x, nrows = td.y;
+                const int npad = (nrows + 15) & ~15;
+                if constexpr (MODE == 1)
+                    for (int n = 0; n < npad; ++n) rows_idx[n] = __ldg(g.perm + row0 + (n < nrows ? n : 0));
+                for (int rr = 0; rr < R; ++rr, ++h) {
+                    const int st = h & 3;
+                    if (h >= kABufs && !mbar_wait(&round_empty[st], ((h >> 2) - 1) & 1, g.err)) { ok = false; break; }
+                    const uint32_t b_base = smem_u32(b_ring + st * kBStageBytes);
+                    mbar_arrive_expect_tx(&full_b[st], 2u * (uint32_t)npad * kKStep * 2);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int x = (2 * rr + j) * kKStep;
+                        const uint32_t dst = b_base + j * kBStepBytes;
+                        if constexpr (MODE == 1) {
+                            for (int n = 0; n < npad; n += 4)
+                                tma_gather4(dst + n * 128, &map_rows, x, rows_idx[n], rows_idx[n + 1], rows_idx[n + 2],
+                                            rows_idx[n + 3], &full_b[st], pol);
+                        } else {
+                            for (int n = 0; n < npad; n += 16)
+                                tma_load_2d(dst + n * 128, &map_rows, x, row0 + n, &full_b[st], pol);
+                        }
+                    }
+                    issued = h + 1;
+                }
+            }
+            // every issued stage completes before the CTA exits
+            for (int j = issued - kABufs; j < issued; ++j)
+                if (j >= 0) mbar_drain(&full_b[j & 3], (j >> 2) & 1);
+        }
+        __syncwarp();
+    } else if (!dead && warp == kMmaWarp) {
+        // ---------------- single-thread MMA issue: per round, 2 k-steps x 4 MMAs of K = 16
+        if (lane == 0) {
+            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(b_ring));
+            int li = 0;
+            bool ok = true, issued = false;
+            for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
+                const int4 td = __ldg(g.tiles + tile);
+                const int npad = (td.y + 15) & ~15;
+                const uint32_t idesc = instr_desc_f16(npad);
+                const int ab = li & 1;
+                if (li >= kAccBufs) {
+                    if (!mbar_wait(&acc_empty[ab], ((li >> 1) - 1) & 1, g.err)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                const uint32_t d_tmem = tmem + (uint32_t)(ab * kAccCols);
+                for (int rr = 0; rr < R; ++rr) {
+                    const int gr = li * R + rr;
+                    const int buf = gr & 3;
+                    if (!mbar_wait(&full_a[buf], (gr >> 2) & 1, g.err) || !mbar_wait(&full_b[buf], (gr >> 2) & 1, g.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // descriptor start addresses advance in 16-byte units
+                    const uint64_t bd = bdesc0 + (uint64_t)((buf * kBStageBytes) >> 4);
+                    const uint32_t at = tmem + (uint32_t)(kACol0 + buf * kABufCols);
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int kk = 0; kk < kKStep / 16; ++kk)
+                            mma_ts(d_tmem, at + (uint32_t)(j * 32 + kk * 8), bd + (uint64_t)((j * kBStepBytes + kk * 32) >> 4),
+                                   idesc, (rr > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    issued = true;
+                    mma_commit(&round_empty[buf]);     // frees the round's A buffer and row stage
+                }
+                if (ok) mma_commit(&acc_full[ab]);
+            }
+            if (issued) {                              // every MMA completes before TMEM is released
+                mma_commit(&drain_bar);
+                mbar_drain(&drain_bar, 0);
+            }
         }
         __syncwarp();
     }
@@ -555,30 +892,116 @@ __global__ void __launch_bounds__(kThreads, 1) expert_gemm_kernel(GemmArgs g) {
     __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after();
-        const uint32_t ncols = (MODE == 1) ? 512u : 256u;
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
     }
 }
 
-template <int FMT>
-moe_status launch_gemms(const PoolView& P, const PrefillWs& w, const uint16_t* x, uint16_t* yrows, int max_t1,
-                        int max_t2, cudaStream_t s) {
-    const size_t smem1 = (size_t)kStages * (2 * kTileM * kTileK * 2 + kTileN * kTileK * 2) + 1024;
-    const size_t smem2 = (size_t)kStages * (kTileM * kTileK * 2 + kTileN * kTileK * 2) + 1024;
+// ---------------------------------------------------------------- host: tensor maps and launches
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// A byte tensor [slots][rows][row_bytes] (slot stride given), boxes of
+// box_x bytes x box_y rows.
+bool byte_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint64_t slots,
+              uint64_t slot_stride, uint32_t box_x, uint32_t box_y, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {row_bytes, rows, slots};
+    const cuuint64_t strides[2] = {row_bytes, slot_stride};
+    const cuuint32_t box[3] = {box_x, box_y, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int gemm_num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+// The row operand: fp16 [rows][stride] (K used) with boxes of 64 x box_rows, 128B swizzle.
+bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t stride, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {K, rows};
+    const cuuint64_t strides[1] = {stride * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kKStep, box_rows};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, int MODE>
+moe_status launch_gemm(const PoolView& P, const GemmParams& prm, uint64_t src_rows, int max_tiles, cudaStream_t s) {
+    using Fm = GemmFmt<FMT>;
+    const int D = P.D, F = P.F;
+    const int Kg = MODE == 1 ? D : F;                 // K of the matrix set
+    const uint64_t rows = MODE == 1 ? 2 * (uint64_t)F : (uint64_t)D;
+    const uint64_t code_row = (uint64_t)Kg / 32 * Fm::kCb;
+    const uint8_t* codes = P.codes + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * Fm::kCb));
+    CUtensorMap mc, ms;
+    const uint32_t box_y = MODE == 1 ? kGateRows : kTileM;   // gate|up: two 64-row boxes per round
+    const CUtensorMapSwizzle csw = FMT == MOE_Q2_32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (!byte_map(&mc, codes, code_row, rows, (uint64_t)P.n_slots, P.stride_c, (uint32_t)Fm::kRb, box_y, csw))
+        return MOE_ERR_CUDA;
+    if constexpr (Fm::kTmaScales) {
+        const uint64_t scale_row = (uint64_t)Kg / 32 * 4;
+        const uint8_t* scales = P.scales + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * 4));
+        if (!byte_map(&ms, scales, scale_row, rows, (uint64_t)P.n_slots, P.stride_s, 16, box_y,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return MOE_ERR_CUDA;
+    } else {
+        ms = mc;
+    }
+    CUtensorMap mr;   // gate|up: x16 rows gathered one at a time; down: h in 16-row boxes
+    const uint64_t stride = MODE == 1 ? (uint64_t)x16_stride(D) : (uint64_t)F;
+    if (!row_map(&mr, prm.src, (uint64_t)Kg, stride, src_rows, MODE == 1 ? 1u : 16u)) return MOE_ERR_CUDA;
+    const size_t smem = kGemmSmem + 1024;
     static bool attr = false;
     if (!attr) {
-        cudaFuncSetAttribute(expert_gemm_kernel<FMT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
-        cudaFuncSetAttribute(expert_gemm_kernel<FMT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+        if (cudaFuncSetAttribute(expert_gemm_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
         attr = true;
     }
-    GemmArgs a1;
-    a1.P = P; a1.tiles = w.tiles1; a1.n_tiles = w.meta + 1; a1.src = x; a1.perm = w.perm; a1.dst = w.h; a1.err = w.err;
-    cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, 1>, dim3(max_t1), dim3(kThreads), smem1, s, a1);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    GemmArgs a2;
-    a2.P = P; a2.tiles = w.tiles2; a2.n_tiles = w.meta + 2; a2.src = w.h; a2.perm = nullptr; a2.dst = yrows; a2.err = w.err;
-    e = launch_pdl(expert_gemm_kernel<FMT, 2>, dim3(max_t2), dim3(kThreads), smem2, s, a2);
+    const int grid = max_tiles < gemm_num_sms() ? (max_tiles > 0 ? max_tiles : 1) : gemm_num_sms();
+    const cudaError_t e =
+        launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms, mr, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <int FMT>
+moe_status launch_gemms(const PoolView& P, const PrefillWs& w, uint16_t* yrows, const WsSizes& sz, int T, int k,
+                        cudaStream_t s) {
+    GemmParams a1;
+    a1.tiles = w.tiles1; a1.n_tiles = w.meta + 1; a1.src = w.x16; a1.perm = w.perm; a1.dst = w.h;
+    a1.scales = P.scales; a1.stride_s = P.stride_s; a1.D = P.D; a1.F = P.F; a1.err = w.err;
+    moe_status st = launch_gemm<FMT, 1>(P, a1, (uint64_t)T, (int)sz.max_t1, s);
+    if (st != MOE_OK) return st;
+    GemmParams a2 = a1;
+    a2.tiles = w.tiles2; a2.n_tiles = w.meta + 2; a2.src = w.h; a2.perm = nullptr; a2.dst = yrows;
+    return launch_gemm<FMT, 2>(P, a2, (uint64_t)T * (k + 1), (int)sz.max_t2, s);
 }
 
 }  // namespace
@@ -588,7 +1011,8 @@ size_t prefill_workspace_bytes(int T, int D, int F, int E, int k) { return ws_si
 moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
                                   const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
                                   int32_t* miss_count, void* ws, cudaStream_t s) {
-    if (P.F % kTileM || P.D % kTileM || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    if (P.F % kRoundK || P.D % kRoundK || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    if (!encode_tiled()) return MOE_ERR_CUDA;
     const PrefillWs w = carve(ws, T, P.D, P.F, E, k);
     PlanArgs a;
     a.ids = ids; a.slot_table = slot_table; a.T = T; a.k = k; a.E = E; a.n_slots = P.n_slots;
@@ -597,19 +1021,24 @@ moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, 
     a.miss_list = miss_list;
     a.miss_count = miss_count;
     const int nchunk = (T + kChunk - 1) / kChunk;
-    cudaError_t e = launch_pdl(plan_count_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
+    const size_t ngroups = (size_t)T * P.D / 16;
+    const size_t cblocks = (ngroups + 255) / 256;
+    const int cgrid = (int)(cblocks < 1184 ? (cblocks > 0 ? cblocks : 1) : 1184);
+    cudaError_t e = launch_pdl(to_f16p_kernel, dim3(cgrid), dim3(256), 0, s, x, ngroups, P.D / 16, x16_stride(P.D),
+                               w.x16, w.err);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = launch_pdl(plan_count_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_pdl(plan_scan_kernel, dim3(1), dim3(1024), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_pdl(plan_scatter_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const WsSizes sz = ws_sizes(T, P.D, P.F, E, k);
-    const int max_t1 = (int)(sz.t1 / sizeof(int4)), max_t2 = (int)(sz.t2 / sizeof(int4));
     uint16_t* yrows = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T, k));
     switch (P.fmt) {
-        case MOE_Q2_32: return launch_gemms<MOE_Q2_32>(P, w, x, yrows, max_t1, max_t2, s);
-        case MOE_Q3_32: return launch_gemms<MOE_Q3_32>(P, w, x, yrows, max_t1, max_t2, s);
-        default: return launch_gemms<MOE_Q3_S256>(P, w, x, yrows, max_t1, max_t2, s);
+        case MOE_Q2_32: return launch_gemms<MOE_Q2_32>(P, w, yrows, sz, T, k, s);
+        case MOE_Q3_32: return launch_gemms<MOE_Q3_32>(P, w, yrows, sz, T, k, s);
+        default: return launch_gemms<MOE_Q3_S256>(P, w, yrows, sz, T, k, s);
     }
 }
 

@@ -1,7 +1,7 @@
 """GPU parity of the prefill path (T > 4: permute + tcgen05 grouped GEMMs)
 against the CPU oracle, through the C ABI.  Bars as for the decode path:
 routing ids and miss lists bit-exact; outputs within relative L2 1e-2 per token
-(bf16 weights and bf16 y rows on this path, fp32 accumulation)."""
+(fp16 tensor-core operands and bf16 y rows on this path, fp32 accumulation)."""
 import numpy as np
 import pytest
 import torch
@@ -36,6 +36,7 @@ def _check(wl, x, sample=None, residual=None):
     ref = oracle_layer(wl.pool, L, wl.cfg.k, xs, residual_bits=None if residual is None else u16(residual)[idx],
                        n_threads=16)
     assert np.array_equal(layer.ids.cpu().numpy()[idx], ref.ids)
+    assert int(layer.ws[4:8].view(torch.int32).item()) == 0     # device error word
     err = rel_l2_per_token(u16(out)[idx], ref.out)
     assert err.max() <= TOL_OUT, err
     if sample is None:
