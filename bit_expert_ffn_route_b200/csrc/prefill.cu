@@ -29,8 +29,10 @@
 // K order.  Inside every group of 16 consecutive K indices the operands use
 // the order (0, 8, 1, 9, ..., 7, 15): one 32-bit word of A then holds the
 // weight pair (i, i + 8), which the block formats deliver in the same word at
-// the same bit offset of both halves.  x (gate|up) is staged into that order by
-// to_f16p_kernel and h (down) is written in it by the gate|up epilogue.
+// the same bit offset of both halves.  The rows of x are gathered into group
+// order and converted (gather_f16p_kernel), so that both GEMMs read their row
+// operand as contiguous 2D TMA boxes; h (down) is written in that order by the
+// gate|up epilogue.
 #include <cuda.h>            // CUtensorMap types; the encoder is fetched at run time
 #include <cuda_fp16.h>
 
@@ -66,18 +68,15 @@ struct PrefillWs {
     int4* tiles1;         // (group row0, rows, m0, slot)
     int4* tiles2;
     int32_t* perm;        // [rows] token of each row
-    uint16_t* x16;        // [T][x16_stride(D)] fp16, K-permuted
+    uint16_t* xg;         // [rows][D] fp16, K-permuted: x of each row's token
     uint16_t* h;          // [rows][F] fp16, K-permuted
     uint32_t* err;
 };
 
 inline size_t align256(size_t n) { return (n + 255) / 256 * 256; }
-// Row stride (elements) of the fp16 copy of x: padded by 128 bytes so that the
-// same K slice of different rows does not fall on one L2 set.
-inline int x16_stride(int D) { return D + 64; }
 
 struct WsSizes {
-    size_t hist, miss, meta, t1, t2, perm, x16, h, total;
+    size_t hist, miss, meta, t1, t2, perm, xg, h, total;
     size_t max_t1, max_t2;
 };
 
@@ -94,9 +93,9 @@ inline WsSizes ws_sizes(int T, int D, int F, int E, int k) {
     s.t1 = align256(s.max_t1 * sizeof(int4));
     s.t2 = align256(s.max_t2 * sizeof(int4));
     s.perm = align256(rows * 4);
-    s.x16 = align256((size_t)T * x16_stride(D) * 2);
+    s.xg = align256(rows * D * 2);
     s.h = align256(rows * F * 2);
-    s.total = 1024 + s.hist + s.miss + s.meta + s.t1 + s.t2 + s.perm + s.x16 + s.h;
+    s.total = 1024 + s.hist + s.miss + s.meta + s.t1 + s.t2 + s.perm + s.xg + s.h;
     return s;
 }
 
@@ -112,7 +111,7 @@ inline PrefillWs carve(void* ws, int T, int D, int F, int E, int k) {
     w.tiles1 = reinterpret_cast<int4*>(p); p += s.t1;
     w.tiles2 = reinterpret_cast<int4*>(p); p += s.t2;
     w.perm = reinterpret_cast<int32_t*>(p); p += s.perm;
-    w.x16 = reinterpret_cast<uint16_t*>(p); p += s.x16;
+    w.xg = reinterpret_cast<uint16_t*>(p); p += s.xg;
     w.h = reinterpret_cast<uint16_t*>(p);
     return w;
 }
@@ -287,7 +286,7 @@ __global__ void __launch_bounds__(kChunk) plan_scatter_kernel(PlanArgs a) {
     a.rowmap[(size_t)t * (k + 1) + k] = S + t;
 }
 
-// ---------------------------------------------------------------- x -> fp16, K-permuted
+// ---------------------------------------------------------------- x rows -> fp16, group order, K-permuted
 MOE_DEVINL uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -295,14 +294,19 @@ MOE_DEVINL uint32_t pack_f16x2(float lo, float hi) {
 }
 MOE_DEVINL uint32_t bf16_half(uint32_t w, int hi) { return hi ? (w & 0xffff0000u) : (w << 16); }
 
-// One thread per 16-element group: out word i = (x[i], x[i + 8]) in fp16.
-__global__ void __launch_bounds__(256) to_f16p_kernel(const uint16_t* __restrict__ x, size_t ngroups, int row_groups,
-                                                      int out_stride, uint16_t* __restrict__ x16, uint32_t* err) {
+// xg[row] = x[perm[row]] in fp16 and K order: one thread per 16-element group,
+// out word i = (x[i], x[i + 8]).  Rows: the routed rows, then the T shared rows.
+__global__ void __launch_bounds__(256) gather_f16p_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+                                                          const int32_t* __restrict__ meta, int T, int D,
+                                                          uint16_t* __restrict__ xg, uint32_t* err) {
     pdl_wait();
+    const int row_groups = D / 16;
+    const size_t ngroups = (size_t)(__ldg(meta) + T) * row_groups;
     bool bad = false;
     for (size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x; gi < ngroups; gi += (size_t)gridDim.x * blockDim.x) {
-        const uint4 a = __ldg(reinterpret_cast<const uint4*>(x) + 2 * gi);
-        const uint4 b = __ldg(reinterpret_cast<const uint4*>(x) + 2 * gi + 1);
+        const size_t row = gi / row_groups, gc = gi % row_groups;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)__ldg(perm + row) * D + gc * 16);
+        const uint4 a = __ldg(src), b = __ldg(src + 1);
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
         uint32_t o[8];
 #pragma unroll
@@ -312,8 +316,7 @@ __global__ void __launch_bounds__(256) to_f16p_kernel(const uint16_t* __restrict
             bad |= !(fabsf(lo) < 65520.f) || !(fabsf(hi) < 65520.f);
             o[i] = pack_f16x2(lo, hi);
         }
-        const size_t t = gi / row_groups, gc = gi % row_groups;
-        uint4* dst = reinterpret_cast<uint4*>(x16 + t * out_stride + gc * 16);
+        uint4* dst = reinterpret_cast<uint4*>(xg + row * D + gc * 16);
         dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
         dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
@@ -389,16 +392,6 @@ MOE_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, 
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
         "%3}], [%4], %5;" ::"r"(dst),
         "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
-}
-// Four rows (y0..y3) of a 2D tensor whose box is one row high, stacked in
-// shared memory at the box pitch.
-MOE_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2, int y3, uint64_t* bar,
-                            uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
-        "[%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
-        "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
 }
 // Bounded wait that does not give up early on the error word: used to drain
@@ -517,12 +510,11 @@ MOE_DEVINL void q3_block_codes(uint32_t c0, uint32_t c1, uint32_t c2, const Magi
 struct GemmParams {
     const int4* tiles;
     const int32_t* n_tiles;      // device count
-    const uint16_t* src;         // MODE 1: x16 [T][x16_stride(D)]; MODE 2: h [rows][F]
-    const int32_t* perm;         // MODE 1: token of each row
     uint16_t* dst;               // MODE 1: h [rows][F] fp16; MODE 2: y rows [rows][D] bf16
     const uint8_t* scales;       // Q3_S256: the pool's scale base (sub-scales, d)
     size_t stride_s;
     int D, F;
+    int rps;                     // dequant rounds per code stage (4, 2 or 1: K / 128 is a multiple)
     uint32_t* err;
 };
 
@@ -531,8 +523,14 @@ struct GemmFmt {
     static constexpr int kCb = FMT == MOE_Q2_32 ? 8 : 12;                  // code bytes per 32 weights
     static constexpr int kRb = 4 * kCb;                                    // code bytes per row per round
     static constexpr bool kTmaScales = FMT != MOE_Q3_S256;
-    static constexpr uint32_t kStageBytes = 128 * kRb + (kTmaScales ? 128 * 16 : 0);
 };
+
+// 16-byte chunk c of row r in a TMA tile of `pitch`-byte rows (32, 64 or 128:
+// the swizzle of that width; other pitches are not swizzled).
+MOE_DEVINL uint32_t swz_chunk(int r, int c, int pitch) {
+    const int sw = (pitch == 32 || pitch == 64 || pitch == 128) ? ((r * pitch) >> 7) & (pitch / 16 - 1) : 0;
+    return (uint32_t)(r * pitch + ((c ^ sw) << 4));
+}
 
 constexpr int kNmax = 128;                 // rows per tile (MMA N <= 128)
 constexpr int kAccCols = 128;              // one accumulator: 128 lanes x N fp32 columns
@@ -542,14 +540,14 @@ constexpr int kABufCols = 2 * 32;          // a round: 2 k-steps x 32 columns (6
 constexpr int kACol0 = kAccBufs * kAccCols;
 constexpr uint32_t kBStepBytes = (uint32_t)kNmax * kKStep * 2;     // one k-step of the row operand
 constexpr uint32_t kBStageBytes = 2 * kBStepBytes;                  // a round: two k-steps
-constexpr int kCodeStages8 = 8;
-constexpr uint32_t kCodeStage8Bytes = 8192;
-constexpr uint32_t kGemmSmem = kCodeStages8 * kCodeStage8Bytes + kABufs * kBStageBytes;
+constexpr int kCodeSlots = 2;             // code stages of up to 4 rounds (K = 512)
+constexpr uint32_t kCodeSlotBytes = 32768;
+constexpr uint32_t kGemmSmem = kCodeSlots * kCodeSlotBytes + kABufs * kBStageBytes;
 static_assert(kACol0 + kABufs * kABufCols == 512, "TMEM columns");
 
 // Warp roles: 0..15 dequantise (warp w owns TMEM lanes 32 (w % 4) ..; the four
 // warps of a lane quadrant take rounds in turn), 16..19 epilogue, 20 TMA for
-// the code tiles, 21 row-operand gather, 22 MMA issue.
+// the code tiles (one stage per rps rounds), 21 TMA for the row operand, 22 MMA issue.
 // The A operand of a tile has 128 rows: MODE 1 rows 0..63 are the gate
 // features m0..m0+63 and rows 64..127 the same up features, so one M = 128
 // accumulator holds both halves of the SwiGLU; MODE 2 rows are 128 outputs.
@@ -557,30 +555,33 @@ static_assert(kACol0 + kABufs * kABufCols == 512, "TMEM columns");
 template <int FMT, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_scales,
-                       const __grid_constant__ CUtensorMap map_rows, GemmParams g) {
+                       const __grid_constant__ CUtensorMap rows128, const __grid_constant__ CUtensorMap rows64,
+                       const __grid_constant__ CUtensorMap rows32, const __grid_constant__ CUtensorMap rows16,
+                       GemmParams g) {
     using Fm = GemmFmt<FMT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    __shared__ uint64_t full_c[kCodeStages8], empty_c[kCodeStages8];
+    __shared__ uint64_t full_c[kCodeSlots], empty_c[kCodeSlots];
     // round slot i (= round % 4): its TMEM A buffer and its row-operand stage are
     // filled by full_a[i] / full_b[i] and released together by round_empty[i]
     __shared__ uint64_t full_a[kABufs], full_b[kABufs], round_empty[kABufs];
     __shared__ uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain_bar;
     __shared__ uint32_t tmem_base;
-    __shared__ int rows_idx[kNmax];
     __shared__ float gate_x[kGateRows][17];        // epilogue: gate values handed to the up lanes
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* code_ring = smem;
-    uint8_t* b_ring = smem + kCodeStages8 * kCodeStage8Bytes;
+    uint8_t* b_ring = smem + kCodeSlots * kCodeSlotBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = g.D, F = g.F;
     const int K = MODE == 1 ? D : F;
     const int R = K / kRoundK;                  // dequant rounds per tile
+    const int rps = g.rps;                      // rounds per code stage
+    const int CP = rps * Fm::kRb, SP = rps * 16;  // code / scale bytes per row of a code stage
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kCodeStages8; ++s) {
+        for (int s = 0; s < kCodeSlots; ++s) {
             mbar_init(&full_c[s], 1);
-            mbar_init(&empty_c[s], 4);
+            mbar_init(&empty_c[s], 4 * rps);    // the 4 quadrant warps of each of its rounds
         }
         for (int s = 0; s < kABufs; ++s) {
             mbar_init(&full_a[s], 4);
@@ -623,33 +624,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int rr = 0; rr < R; ++rr) {
                 const int gr = li * R + rr;
                 if ((gr & 3) != par) continue;
-                const int st = gr % kCodeStages8;
-                if (!mbar_wait(&full_c[st], (gr / kCodeStages8) & 1, g.err)) { ok = false; break; }
-                const uint8_t* cs = code_ring + st * kCodeStage8Bytes;
-                // codes of this row for the round's 4 blocks, and the (s, m) words
+                const int cst = gr / rps, sub = gr % rps, cslot = cst & 1;
+                if (!mbar_wait(&full_c[cslot], (cst >> 1) & 1, g.err)) { ok = false; break; }
+                const uint8_t* cs = code_ring + cslot * kCodeSlotBytes;
+                // codes of this row for the round's 4 blocks (bytes sub * kRb .. of the
+                // stage row), and the (s, m) words
                 uint32_t cw[3 * 4];
                 uint32_t sw[4] = {0, 0, 0, 0};
-                if constexpr (FMT == MOE_Q2_32) {
-                    const uint8_t* row = cs + r * 32;
-                    const uint32_t x = (uint32_t)((r >> 2) & 1);     // 32-byte TMA swizzle
-                    const uint4 a = *reinterpret_cast<const uint4*>(row + ((0u ^ x) << 4));
-                    const uint4 b = *reinterpret_cast<const uint4*>(row + ((1u ^ x) << 4));
-                    cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
-                    cw[4] = b.x; cw[5] = b.y; cw[6] = b.z; cw[7] = b.w;
-                } else {
-                    const uint8_t* row = cs + r * 48;
 #pragma unroll
-                    for (int i = 0; i < 3; ++i) {
-                        const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * i);
-                        cw[4 * i] = a.x; cw[4 * i + 1] = a.y; cw[4 * i + 2] = a.z; cw[4 * i + 3] = a.w;
-                    }
+                for (int i = 0; i < Fm::kRb / 16; ++i) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(cs + swz_chunk(r, sub * (Fm::kRb / 16) + i, CP));
+                    cw[4 * i] = a.x; cw[4 * i + 1] = a.y; cw[4 * i + 2] = a.z; cw[4 * i + 3] = a.w;
                 }
                 if constexpr (Fm::kTmaScales) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(cs + 128 * Fm::kRb + r * 16);
+                    const uint4 a = *reinterpret_cast<const uint4*>(cs + 128 * CP + swz_chunk(r, sub, SP));
                     sw[0] = a.x; sw[1] = a.y; sw[2] = a.z; sw[3] = a.w;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty_c[st]);
+                if (lane == 0) mbar_arrive(&empty_c[cslot]);
                 // Q3_S256: the super-block's sub-scales and d, straight from global memory
                 float sd = 0.f;
                 uint32_t sub0 = 0, sub1 = 0, sub2 = 0;
@@ -763,60 +755,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (range_bad) atomicOr(g.err, kErrRange);
     } else if (!dead && warp == kTmaWarp) {
-        // ---------------- TMA loads of the code (and scale) tiles, one stage per round
+        // ---------------- TMA loads of the code (and scale) tiles, one stage per rps rounds
         if (lane == 0) {
             const uint64_t pol = l2_evict_first();
+            const uint32_t bytes = 128u * CP + (Fm::kTmaScales ? 128u * SP : 0u);
             int li = 0, issued = 0;
             bool ok = true;
             for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
                 const int4 td = __ldg(g.tiles + tile);
-                const int m0 = td.z, slot = td.w;
-                for (int rr = 0; rr < R; ++rr) {
-                    const int gr = li * R + rr;
-                    const int st = gr % kCodeStages8;
-                    if (gr >= kCodeStages8 && !mbar_wait(&empty_c[st], ((gr / kCodeStages8) - 1) & 1, g.err)) {
+                const int m0 = td.z, slot_id = td.w;
+                for (int c = 0; c < R / rps; ++c) {
+                    const int cst = li * (R / rps) + c, slot = cst & 1;
+                    if (cst >= kCodeSlots && !mbar_wait(&empty_c[slot], ((cst >> 1) - 1) & 1, g.err)) {
                         ok = false;
                         break;
                     }
-                    uint8_t* cs = code_ring + st * kCodeStage8Bytes;
-                    mbar_arrive_expect_tx(&full_c[st], Fm::kStageBytes);
+                    uint8_t* cs = code_ring + slot * kCodeSlotBytes;
+                    mbar_arrive_expect_tx(&full_c[slot], bytes);
                     if constexpr (MODE == 1) {
                         // gate rows m0.. into rows 0..63, up rows F + m0.. into rows 64..127
 #pragma unroll
                         for (int m = 0; m < 2; ++m) {
                             const int y = m * F + m0;
-                            tma_load_3d(smem_u32(cs + m * 64 * Fm::kRb), &map_codes, rr * Fm::kRb, y, slot, &full_c[st],
-                                        pol);
+                            tma_load_3d(smem_u32(cs + m * 64 * CP), &map_codes, c * CP, y, slot_id, &full_c[slot], pol);
                             if constexpr (Fm::kTmaScales)
-                                tma_load_3d(smem_u32(cs + 128 * Fm::kRb + m * 64 * 16), &map_scales, rr * 16, y, slot,
-                                            &full_c[st], pol);
+                                tma_load_3d(smem_u32(cs + 128 * CP + m * 64 * SP), &map_scales, c * SP, y, slot_id,
+                                            &full_c[slot], pol);
                         }
                     } else {
-                        tma_load_3d(smem_u32(cs), &map_codes, rr * Fm::kRb, m0, slot, &full_c[st], pol);
+                        tma_load_3d(smem_u32(cs), &map_codes, c * CP, m0, slot_id, &full_c[slot], pol);
                         if constexpr (Fm::kTmaScales)
-                            tma_load_3d(smem_u32(cs + 128 * Fm::kRb), &map_scales, rr * 16, m0, slot, &full_c[st], pol);
+                            tma_load_3d(smem_u32(cs + 128 * CP), &map_scales, c * SP, m0, slot_id, &full_c[slot], pol);
                     }
-                    issued = gr + 1;
+                    issued = cst + 1;
                 }
             }
             // every issued stage completes before the CTA exits
-            for (int j = issued - kCodeStages8; j < issued; ++j)
-                if (j >= 0) mbar_drain(&full_c[j % kCodeStages8], (j / kCodeStages8) & 1);
+            for (int j = issued - kCodeSlots; j < issued; ++j)
+                if (j >= 0) mbar_drain(&full_c[j & 1], (j >> 1) & 1);
         }
         __syncwarp();
     } else if (!dead && warp == kGatherWarp) {
-        // ---------------- row operand (K-major, 128B swizzle) by TMA: gate|up gathers the
-        // rows' tokens four at a time; down reads its contiguous rows in 16-row boxes
+        // ---------------- row operand (K-major, 128B swizzle) by TMA: the tile's rows are
+        // contiguous (group order), read as boxes of 128 / 64 / 32 / 16 rows
         if (lane == 0) {
             const uint64_t pol = l2_evict_last();
             bool ok = true;
             int issued = 0;
             for (int tile = first, h = 0; tile < n_tiles && ok; tile += step) {
                 const int4 td = __ldg(g.tiles + tile);
-                const int row0 = td.x, nrows = td.y;
-                const int npad = (nrows + 15) & ~15;
-                if constexpr (MODE == 1)
-                    for (int n = 0; n < npad; ++n) rows_idx[n] = __ldg(g.perm + row0 + (n < nrows ? n : 0));
+                const int row0 = td.x, npad = (td.y + 15) & ~15;
                 for (int rr = 0; rr < R; ++rr, ++h) {
                     const int st = h & 3;
                     if (h >= kABufs && !mbar_wait(&round_empty[st], ((h >> 2) - 1) & 1, g.err)) { ok = false; break; }
@@ -826,13 +814,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     for (int j = 0; j < 2; ++j) {
                         const int x = (2 * rr + j) * kKStep;
                         const uint32_t dst = b_base + j * kBStepBytes;
-                        if constexpr (MODE == 1) {
-                            for (int n = 0; n < npad; n += 4)
-                                tma_gather4(dst + n * 128, &map_rows, x, rows_idx[n], rows_idx[n + 1], rows_idx[n + 2],
-                                            rows_idx[n + 3], &full_b[st], pol);
-                        } else {
-                            for (int n = 0; n < npad; n += 16)
-                                tma_load_2d(dst + n * 128, &map_rows, x, row0 + n, &full_b[st], pol);
+                        for (int n = 0; n < npad;) {
+                            const int left = npad - n;
+                            const CUtensorMap* m = left >= 128 ? &rows128 : left >= 64 ? &rows64 : left >= 32 ? &rows32 : &rows16;
+                            const int nb = left >= 128 ? 128 : left >= 64 ? 64 : left >= 32 ? 32 : 16;
+                            tma_load_2d(dst + n * 128, m, x, row0 + n, &full_b[st], pol);
+                            n += nb;
                         }
                     }
                     issued = h + 1;
@@ -939,12 +926,12 @@ int gemm_num_sms() {
     return n;
 }
 
-// The row operand: fp16 [rows][stride] (K used) with boxes of 64 x box_rows, 128B swizzle.
-bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t stride, uint64_t rows, uint32_t box_rows) {
+// The row operand: fp16 [rows][K] with boxes of 64 x box_rows, 128B swizzle.
+bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[2] = {K, rows};
-    const cuuint64_t strides[1] = {stride * 2};
+    const cuuint64_t strides[1] = {K * 2};
     const cuuint32_t box[2] = {(cuuint32_t)kKStep, box_rows};
     const cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
@@ -952,8 +939,14 @@ bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t stride, uint
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+CUtensorMapSwizzle swizzle_for(uint32_t pitch) {
+    return pitch == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : pitch == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : pitch == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
+}
+
 template <int FMT, int MODE>
-moe_status launch_gemm(const PoolView& P, const GemmParams& prm, uint64_t src_rows, int max_tiles, cudaStream_t s) {
+moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, uint64_t src_rows, int max_tiles,
+                       cudaStream_t s) {
     using Fm = GemmFmt<FMT>;
     const int D = P.D, F = P.F;
     const int Kg = MODE == 1 ? D : F;                 // K of the matrix set
@@ -961,22 +954,24 @@ moe_status launch_gemm(const PoolView& P, const GemmParams& prm, uint64_t src_ro
     const uint64_t code_row = (uint64_t)Kg / 32 * Fm::kCb;
     const uint8_t* codes = P.codes + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * Fm::kCb));
     CUtensorMap mc, ms;
-    const uint32_t box_y = MODE == 1 ? kGateRows : kTileM;   // gate|up: two 64-row boxes per round
-    const CUtensorMapSwizzle csw = FMT == MOE_Q2_32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
-    if (!byte_map(&mc, codes, code_row, rows, (uint64_t)P.n_slots, P.stride_c, (uint32_t)Fm::kRb, box_y, csw))
+    const int R = Kg / kRoundK;
+    prm.rps = R % 4 == 0 ? 4 : (R % 2 == 0 ? 2 : 1);
+    const uint32_t cp = (uint32_t)(prm.rps * Fm::kRb), sp = (uint32_t)(prm.rps * 16);
+    const uint32_t box_y = MODE == 1 ? kGateRows : kTileM;   // gate|up: two 64-row boxes per stage
+    if (!byte_map(&mc, codes, code_row, rows, (uint64_t)P.n_slots, P.stride_c, cp, box_y, swizzle_for(cp)))
         return MOE_ERR_CUDA;
     if constexpr (Fm::kTmaScales) {
         const uint64_t scale_row = (uint64_t)Kg / 32 * 4;
         const uint8_t* scales = P.scales + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * 4));
-        if (!byte_map(&ms, scales, scale_row, rows, (uint64_t)P.n_slots, P.stride_s, 16, box_y,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+        if (!byte_map(&ms, scales, scale_row, rows, (uint64_t)P.n_slots, P.stride_s, sp, box_y, swizzle_for(sp)))
             return MOE_ERR_CUDA;
     } else {
         ms = mc;
     }
-    CUtensorMap mr;   // gate|up: x16 rows gathered one at a time; down: h in 16-row boxes
-    const uint64_t stride = MODE == 1 ? (uint64_t)x16_stride(D) : (uint64_t)F;
-    if (!row_map(&mr, prm.src, (uint64_t)Kg, stride, src_rows, MODE == 1 ? 1u : 16u)) return MOE_ERR_CUDA;
+    CUtensorMap r128, r64, r32, r16;
+    if (!row_map(&r128, src, (uint64_t)Kg, src_rows, 128) || !row_map(&r64, src, (uint64_t)Kg, src_rows, 64) ||
+        !row_map(&r32, src, (uint64_t)Kg, src_rows, 32) || !row_map(&r16, src, (uint64_t)Kg, src_rows, 16))
+        return MOE_ERR_CUDA;
     const size_t smem = kGemmSmem + 1024;
     static bool attr = false;
     if (!attr) {
@@ -986,8 +981,8 @@ moe_status launch_gemm(const PoolView& P, const GemmParams& prm, uint64_t src_ro
         attr = true;
     }
     const int grid = max_tiles < gemm_num_sms() ? (max_tiles > 0 ? max_tiles : 1) : gemm_num_sms();
-    const cudaError_t e =
-        launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms, mr, prm);
+    const cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms,
+                                     r128, r64, r32, r16, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -995,13 +990,14 @@ template <int FMT>
 moe_status launch_gemms(const PoolView& P, const PrefillWs& w, uint16_t* yrows, const WsSizes& sz, int T, int k,
                         cudaStream_t s) {
     GemmParams a1;
-    a1.tiles = w.tiles1; a1.n_tiles = w.meta + 1; a1.src = w.x16; a1.perm = w.perm; a1.dst = w.h;
+    a1.tiles = w.tiles1; a1.n_tiles = w.meta + 1; a1.dst = w.h;
     a1.scales = P.scales; a1.stride_s = P.stride_s; a1.D = P.D; a1.F = P.F; a1.err = w.err;
-    moe_status st = launch_gemm<FMT, 1>(P, a1, (uint64_t)T, (int)sz.max_t1, s);
+    const uint64_t rows = (uint64_t)T * (k + 1);
+    moe_status st = launch_gemm<FMT, 1>(P, a1, w.xg, rows, (int)sz.max_t1, s);
     if (st != MOE_OK) return st;
     GemmParams a2 = a1;
-    a2.tiles = w.tiles2; a2.n_tiles = w.meta + 2; a2.src = w.h; a2.perm = nullptr; a2.dst = yrows;
-    return launch_gemm<FMT, 2>(P, a2, (uint64_t)T * (k + 1), (int)sz.max_t2, s);
+    a2.tiles = w.tiles2; a2.n_tiles = w.meta + 2; a2.dst = yrows;
+    return launch_gemm<FMT, 2>(P, a2, w.h, rows, (int)sz.max_t2, s);
 }
 
 }  // namespace
@@ -1021,17 +1017,15 @@ moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, 
     a.miss_list = miss_list;
     a.miss_count = miss_count;
     const int nchunk = (T + kChunk - 1) / kChunk;
-    const size_t ngroups = (size_t)T * P.D / 16;
-    const size_t cblocks = (ngroups + 255) / 256;
-    const int cgrid = (int)(cblocks < 1184 ? (cblocks > 0 ? cblocks : 1) : 1184);
-    cudaError_t e = launch_pdl(to_f16p_kernel, dim3(cgrid), dim3(256), 0, s, x, ngroups, P.D / 16, x16_stride(P.D),
-                               w.x16, w.err);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_pdl(plan_count_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
+    cudaError_t e = launch_pdl(plan_count_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_pdl(plan_scan_kernel, dim3(1), dim3(1024), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_pdl(plan_scatter_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    const size_t gblocks = ((size_t)T * (k + 1) * (P.D / 16) + 255) / 256;
+    e = launch_pdl(gather_f16p_kernel, dim3((unsigned)(gblocks < 2368 ? gblocks : 2368)), dim3(256), 0, s, x, w.perm,
+                   w.meta, T, P.D, w.xg, w.err);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const WsSizes sz = ws_sizes(T, P.D, P.F, E, k);
     uint16_t* yrows = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T, k));
