@@ -30,6 +30,9 @@ struct PoolView {
 moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, const float* bias, int E,
                         int k, int32_t* ids, float* gates, float* logits, void* ws, cudaStream_t s);
 size_t route_workspace_bytes(int T, int D, int E, int k);
+moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t* Wr, const float* bias, int E, int k,
+                                int32_t* ids, float* gates, float* logits, float* wnorm, uint32_t* err,
+                                cudaStream_t s);
 
 moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x,
                                  int T, const int32_t* ids, int k, void* expert_out, int32_t* miss_list,

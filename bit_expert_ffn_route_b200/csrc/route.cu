@@ -7,133 +7,10 @@
 // then + bias) is what makes the selected ids reproducible bit for bit.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "route_warp.cuh"
 #include "sync.cuh"
 
 namespace moe {
-
-// Canonical logits of expert e for NT tokens whose bf16 rows are xrow[t]
-// (shared or global memory).  Lane L accumulates elements 256c + 8L + j.
-template <int NT>
-__device__ __forceinline__ void canon_logits_warp(const uint16_t* const (&xrow)[NT], int nt, int D,
-                                                  const uint16_t* __restrict__ Wr, const float* __restrict__ bias,
-                                                  int E, int e, float* __restrict__ lout /* + t*E */) {
-    const int lane = threadIdx.x & 31;
-    float acc[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
-    const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
-    const int nc = D >> 8;
-#pragma unroll 6
-    for (int c = 0; c < nc; ++c) {
-        const uint4 w = ld_nc_u128(wrow + 256 * c);
-        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            if (t < nt) {
-                const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow[t] + 256 * c + 8 * lane);
-                const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {   // element j = 2q (low half), 2q+1 (high half)
-                    acc[t] = __fmaf_rn(bf16lo(xv[q]), bf16lo(wv[q]), acc[t]);
-                    acc[t] = __fmaf_rn(bf16hi(xv[q]), bf16hi(wv[q]), acc[t]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1)
-            acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
-    }
-    if (lane == 0) {
-        const float b = bias ? bias[e] : 0.0f;
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-            if (t < nt) lout[(size_t)t * E + e] = bias ? __fadd_rn(acc[t], b) : acc[t];
-    }
-}
-
-// "a before b": larger logit, then lower id.
-__device__ __forceinline__ bool cand_better(float va, int ea, float vb, int eb) {
-    return va > vb || (va == vb && ea < eb);
-}
-
-// Compare-exchange for a descending order by (value, then lower id).
-__device__ __forceinline__ void cex(float& va, int& ea, float& vb, int& eb) {
-    if (cand_better(vb, eb, va, ea)) {
-        const float tv = va; va = vb; vb = tv;
-        const int te = ea; ea = eb; eb = te;
-    }
-}
-
-// One warp selects the top-k of one token's E logits (E <= 32 * NV) and
-// writes ids and gates.  Each lane sorts its NV values once (a bitonic network
-// in registers); each of the k rounds then takes the warp's best lane head and
-// the winning lane shifts its list.  Gates are formed in double from the
-// selected fp32 logits.
-template <int NV>
-__device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
-                            float* __restrict__ gates) {
-    const int lane = threadIdx.x & 31;
-    float v[NV];
-    int e[NV];
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        e[i] = lane + 32 * i;
-        v[i] = (e[i] < E) ? __ldcg(lrow + e[i]) : -INFINITY;
-        if (e[i] >= E) e[i] = 0x7fffffff;
-    }
-    // bitonic sort, descending
-#pragma unroll
-    for (int kk = 2; kk <= NV; kk <<= 1) {
-#pragma unroll
-        for (int j = kk >> 1; j > 0; j >>= 1) {
-#pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                const int l = i ^ j;
-                if (l > i) {
-                    if ((i & kk) == 0) cex(v[i], e[i], v[l], e[l]);
-                    else cex(v[l], e[l], v[i], e[i]);
-                }
-            }
-        }
-    }
-    float my_v = 0.f, l0 = 0.f;
-    int my_e = 0;
-    for (int r = 0; r < k; ++r) {
-        float wv = v[0];
-        int we = e[0];
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, we, off);
-            if (cand_better(ov, oe, wv, we)) { wv = ov; we = oe; }
-        }
-        if (r == 0) l0 = wv;
-        if (lane == r) { my_v = wv; my_e = we; }
-        if (e[0] == we) {                       // this lane supplied the winner: pop its head
-#pragma unroll
-            for (int i = 0; i + 1 < NV; ++i) { v[i] = v[i + 1]; e[i] = e[i + 1]; }
-            v[NV - 1] = -INFINITY;
-            e[NV - 1] = 0x7fffffff;
-        }
-    }
-    const double ex = (lane < k) ? exp((double)my_v - (double)l0) : 0.0;
-    double z = ex;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-    if (lane < k) {
-        ids[lane] = my_e;
-        gates[lane] = (float)(ex / z);
-    }
-}
-
-__device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
-                                          float* __restrict__ gates) {
-    if (E <= 512) topk_warp_n<16>(lrow, E, k, ids, gates);
-    else topk_warp_n<32>(lrow, E, k, ids, gates);
-}
 
 // Decode route (T <= 4): one warp per expert computes its logits for all T
 // tokens, then the last block to finish selects every token's top-k.  The
@@ -168,29 +45,6 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
     if (!last) return;
     __threadfence();
     if (warp < T) topk_warp(logits + (size_t)warp * E, E, k, ids + (size_t)warp * k, gates + (size_t)warp * k);
-}
-
-// Prefill route, canonical path: grid (E/8, T/4).
-__global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t* __restrict__ x, int T, int D,
-                                                           const uint16_t* __restrict__ Wr,
-                                                           const float* __restrict__ bias, int E,
-                                                           float* __restrict__ logits) {
-    pdl_wait();
-    const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int t0 = blockIdx.y * 4;
-    if (e < E) {
-        const uint16_t* xr[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) xr[t] = x + (size_t)min(t0 + t, T - 1) * D;
-        canon_logits_warp<4>(xr, min(4, T - t0), D, Wr, bias, E, e, logits + (size_t)t0 * E);
-    }
-}
-
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                   int32_t* __restrict__ ids, float* __restrict__ gates) {
-    pdl_wait();
-    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (t < T) topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, gates + (size_t)t * k);
 }
 
 int route_num_sms() {
@@ -229,15 +83,19 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
         return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
     (void)route_num_sms;
-    e = launch_pdl(route_logits_kernel, dim3((E + 7) / 8, (T + 3) / 4), dim3(256), 0, s, x, T, D, Wr, bias, E, lg);
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = launch_pdl(topk_kernel, dim3((T + 7) / 8), dim3(256), 0, s, (const float*)lg, T, E, k, ids, gates);
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    // prefill: tensor-core logits, then canonical logits of each token's candidates
+    float* wnorm = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256 +
+                                            ((size_t)T * E * sizeof(float) + 255) / 256 * 256);
+    uint32_t* err = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
+    return launch_route_prefill(x, T, D, Wr, bias, E, k, ids, gates, lg, wnorm, err, s);
 }
 
+// ws: [0,4) decode block counter, [4,8) device error word, [256, ...) logits
+// scratch [T][E] fp32 (used when the caller passes no logits buffer), then the
+// expert norms of the prefill router.
 size_t route_workspace_bytes(int T, int D, int E, int k) {
     (void)D; (void)k;
-    return 256 + (size_t)T * E * sizeof(float);
+    return 256 + ((size_t)T * E * sizeof(float) + 255) / 256 * 256 + ((size_t)E * sizeof(float) + 255) / 256 * 256;
 }
 
 }  // namespace moe

@@ -1,0 +1,165 @@
+// route_warp.cuh — warp-level router pieces shared by the decode and prefill
+// routers: logits in the canonical fp32 order and the top-k selection.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Canonical logits of expert e for NT tokens whose bf16 rows are xrow[t]
+// (shared or global memory).  Lane L accumulates elements 256c + 8L + j.
+template <int NT>
+__device__ __forceinline__ void canon_logits_warp(const uint16_t* const (&xrow)[NT], int nt, int D,
+                                                  const uint16_t* __restrict__ Wr, const float* __restrict__ bias,
+                                                  int E, int e, float* __restrict__ lout /* + t*E */) {
+    const int lane = threadIdx.x & 31;
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
+    const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
+    const int nc = D >> 8;
+#pragma unroll 6
+    for (int c = 0; c < nc; ++c) {
+        const uint4 w = ld_nc_u128(wrow + 256 * c);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            if (t < nt) {
+                const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow[t] + 256 * c + 8 * lane);
+                const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {   // element j = 2q (low half), 2q+1 (high half)
+                    acc[t] = __fmaf_rn(bf16lo(xv[q]), bf16lo(wv[q]), acc[t]);
+                    acc[t] = __fmaf_rn(bf16hi(xv[q]), bf16hi(wv[q]), acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+            acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
+    }
+    if (lane == 0) {
+        const float b = bias ? bias[e] : 0.0f;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            if (t < nt) lout[(size_t)t * E + e] = bias ? __fadd_rn(acc[t], b) : acc[t];
+    }
+}
+
+// "a before b": larger logit, then lower id.
+__device__ __forceinline__ bool cand_better(float va, int ea, float vb, int eb) {
+    return va > vb || (va == vb && ea < eb);
+}
+
+// Compare-exchange for a descending order by (value, then lower id).
+__device__ __forceinline__ void cex(float& va, int& ea, float& vb, int& eb) {
+    if (cand_better(vb, eb, va, ea)) {
+        const float tv = va; va = vb; vb = tv;
+        const int te = ea; ea = eb; eb = te;
+    }
+}
+
+// One warp selects the top-k of one token's E logits (E <= 32 * NV) and
+// writes ids and gates.  Each lane sorts its NV values once (a bitonic network
+// in registers); each of the k rounds then takes the warp's best lane head and
+// the winning lane shifts its list.  Gates are formed in double from the
+// selected fp32 logits.
+template <int NV, bool SHARED = false>
+__device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
+                            float* __restrict__ gates) {
+    const int lane = threadIdx.x & 31;
+    float v[NV];
+    int e[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        e[i] = lane + 32 * i;
+        v[i] = (e[i] < E) ? (SHARED ? lrow[e[i]] : __ldcg(lrow + e[i])) : -INFINITY;
+        if (e[i] >= E) e[i] = 0x7fffffff;
+    }
+    // bitonic sort, descending
+#pragma unroll
+    for (int kk = 2; kk <= NV; kk <<= 1) {
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    if ((i & kk) == 0) cex(v[i], e[i], v[l], e[l]);
+                    else cex(v[l], e[l], v[i], e[i]);
+                }
+            }
+        }
+    }
+    float my_v = 0.f, l0 = 0.f;
+    int my_e = 0;
+    for (int r = 0; r < k; ++r) {
+        float wv = v[0];
+        int we = e[0];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, we, off);
+            if (cand_better(ov, oe, wv, we)) { wv = ov; we = oe; }
+        }
+        if (r == 0) l0 = wv;
+        if (lane == r) { my_v = wv; my_e = we; }
+        if (e[0] == we) {                       // this lane supplied the winner: pop its head
+#pragma unroll
+            for (int i = 0; i + 1 < NV; ++i) { v[i] = v[i + 1]; e[i] = e[i + 1]; }
+            v[NV - 1] = -INFINITY;
+            e[NV - 1] = 0x7fffffff;
+        }
+    }
+    const double ex = (lane < k) ? exp((double)my_v - (double)l0) : 0.0;
+    double z = ex;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    if (lane < k) {
+        ids[lane] = my_e;
+        gates[lane] = (float)(ex / z);
+    }
+}
+
+__device__ __forceinline__ void topk_warp(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
+                                          float* __restrict__ gates) {
+    if (E <= 512) topk_warp_n<16>(lrow, E, k, ids, gates);
+    else topk_warp_n<32>(lrow, E, k, ids, gates);
+}
+
+// Canonical logit (+ bias) of expert e for one token (bf16 row xrow), every
+// lane returning the value: the same order as canon_logits_warp.
+__device__ __forceinline__ float canon_logit_one(const uint16_t* __restrict__ xrow, int D,
+                                                 const uint16_t* __restrict__ Wr, const float* __restrict__ bias,
+                                                 int e) {
+    const int lane = threadIdx.x & 31;
+    float acc = 0.0f;
+    const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
+    const int nc = D >> 8;
+    for (int c = 0; c < nc; ++c) {
+        const uint4 w = ld_nc_u128(wrow + 256 * c);
+        const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow + 256 * c + 8 * lane);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc = __fmaf_rn(bf16lo(xv[q]), bf16lo(wv[q]), acc);
+            acc = __fmaf_rn(bf16hi(xv[q]), bf16hi(wv[q]), acc);
+        }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+    return bias ? __fadd_rn(acc, __ldg(bias + e)) : acc;
+}
+
+// Top-k of a row of logits held in shared memory.
+__device__ __forceinline__ void topk_row_warp(const float* lrow, int E, int k, int32_t* __restrict__ ids,
+                                              float* __restrict__ gates) {
+    if (E <= 512) topk_warp_n<16, true>(lrow, E, k, ids, gates);
+    else topk_warp_n<32, true>(lrow, E, k, ids, gates);
+}
+
+}  // namespace moe

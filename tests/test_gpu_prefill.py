@@ -7,7 +7,8 @@ import pytest
 import torch
 
 from bit_expert_ffn_route_b200 import configs, moe, synth
-from tests.harness import oracle_layer, rel_l2_per_token, u16
+import oracle
+from tests.harness import f64, oracle_layer, rel_l2_per_token, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +37,10 @@ def _check(wl, x, sample=None, residual=None):
     ref = oracle_layer(wl.pool, L, wl.cfg.k, xs, residual_bits=None if residual is None else u16(residual)[idx],
                        n_threads=16)
     assert np.array_equal(layer.ids.cpu().numpy()[idx], ref.ids)
+    g = layer.gates.cpu().numpy()[idx].astype(np.float64)
+    assert np.all(np.abs(g - ref.gates) <= 1e-6 * np.abs(ref.gates) + 1e-12)
     assert int(layer.ws[4:8].view(torch.int32).item()) == 0     # device error word
+    assert int(layer.route_ws[4:8].view(torch.int32).item()) == 0
     err = rel_l2_per_token(u16(out)[idx], ref.out)
     assert err.max() <= TOL_OUT, err
     if sample is None:
@@ -97,3 +101,27 @@ def test_prefill_config_2048_tokens():
     loads = np.bincount(ids.ravel(), minlength=cfg.E)
     print(f"prefill loads: max {loads.max()}, zero-load experts {(loads == 0).sum()}, worst rel L2 {err.max():.2e}")
     assert loads.max() >= 200
+
+
+def test_prefill_router_logits_bound_and_canonical_selection():
+    """Prefill router: tensor-core logits within 2^-12 |x|_2 |Wr_e|_2 of the
+    canonical ones; ids and gates from the canonical logits of the candidates,
+    so they match the oracle exactly (ids) / within 1e-6 (gates)."""
+    cfg = configs.CONFIGS["prefill"]
+    wl = configs.build(cfg, device="cuda", T=192)
+    L = wl.layers[0]
+    layer = moe.Layer(wl.pool, L.shared_slot, L.slot_table, L.Wr, L.bias, cfg.k, 192)
+    moe.moe_route_topk(wl.x, L.Wr, L.bias, cfg.k, layer.ids, layer.gates, layer.route_ws, logits=layer.logits)
+    torch.cuda.synchronize()
+    xb, wb = u16(wl.x), u16(L.Wr)
+    ref_l = oracle.router_logits(xb, wb, L.bias.cpu().numpy())
+    ref_ids, ref_g = oracle.topk_gates(ref_l, cfg.k)
+    assert np.array_equal(layer.ids.cpu().numpy(), ref_ids)
+    g = layer.gates.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(g - ref_g) <= 1e-6 * np.abs(ref_g) + 1e-12)
+    xn = np.linalg.norm(f64(xb), axis=1)
+    wn = np.linalg.norm(f64(wb), axis=1)
+    bound = 2.0 ** -12 * np.outer(xn, wn)
+    dev = np.abs(layer.logits.cpu().numpy().astype(np.float64) - ref_l.astype(np.float64))
+    assert np.all(dev <= bound), float((dev / bound).max())
+    assert int(layer.route_ws[4:8].view(torch.int32).item()) == 0
