@@ -393,13 +393,18 @@ MOE_DEVINL void chunk_rows(const uint32_t (&cw)[R][3], const float (&sa)[R], con
                            const float* const (&xc)[NT], float (&res)[R][NT]) {
     constexpr int H = (FMT == MOE_Q3_S256) ? 2 : 1;
     const uint32_t one = opaque_one();
-    float2 acc[R][NT][H];
+    // NC independent accumulator chains per (row, token, half) (even and odd code
+    // pairs when few tokens leave registers to spare): shorter FMA dependency chains
+    constexpr int NC = NT <= 2 ? 2 : 1;
+    float2 acc[R][NT][H][NC];
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int h = 0; h < H; ++h) acc[r][t][h] = make_float2(0.f, 0.f);
+            for (int h = 0; h < H; ++h)
+#pragma unroll
+                for (int c = 0; c < NC; ++c) acc[r][t][h][c] = make_float2(0.f, 0.f);
     static_for<0, 4>([&](auto SC) {
         constexpr int sc = decltype(SC)::value;
         float xv[NT][8];
@@ -416,10 +421,11 @@ MOE_DEVINL void chunk_rows(const uint32_t (&cw)[R][3], const float (&sa)[R], con
                 constexpr int i = 2 * decltype(II)::value;
                 constexpr int code = 8 * sc + i;
                 constexpr int h = (H == 2 && code >= 16) ? 1 : 0;
+                constexpr int c2 = decltype(II)::value % NC;
                 const float2 f = make_float2(code_c<FMT, code>(cw[r], one), code_c<FMT, code + 1>(cw[r], one));
 #pragma unroll
                 for (int t = 0; t < NT; ++t)
-                    acc[r][t][h] = ffma2(make_float2(xv[t][i], xv[t][i + 1]), f, acc[r][t][h]);
+                    acc[r][t][h][c2] = ffma2(make_float2(xv[t][i], xv[t][i + 1]), f, acc[r][t][h][c2]);
             });
         });
     });
@@ -429,11 +435,17 @@ MOE_DEVINL void chunk_rows(const uint32_t (&cw)[R][3], const float (&sa)[R], con
         const float c1 = xc[t][33];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
+            float sum[H];
+#pragma unroll
+            for (int h = 0; h < H; ++h) {
+                sum[h] = acc[r][t][h][0].x + acc[r][t][h][0].y;
+                if constexpr (NC == 2) sum[h] += acc[r][t][h][1].x + acc[r][t][h][1].y;
+            }
             if constexpr (H == 2) {
-                res[r][t] = __fmaf_rn(sa[r], (acc[r][t][0].x + acc[r][t][0].y) - c0, res[r][t]);
-                res[r][t] = __fmaf_rn(sb[r], (acc[r][t][1].x + acc[r][t][1].y) - c1, res[r][t]);
+                res[r][t] = __fmaf_rn(sa[r], sum[0] - c0, res[r][t]);
+                res[r][t] = __fmaf_rn(sb[r], sum[1] - c1, res[r][t]);
             } else {
-                res[r][t] = __fmaf_rn(sa[r], (acc[r][t][0].x + acc[r][t][0].y) - c0, __fmaf_rn(sb[r], c1, res[r][t]));
+                res[r][t] = __fmaf_rn(sa[r], sum[0] - c0, __fmaf_rn(sb[r], c1, res[r][t]));
             }
         }
     }

@@ -49,69 +49,55 @@ __device__ __forceinline__ void canon_logits_warp(const uint16_t* const (&xrow)[
     }
 }
 
-// "a before b": larger logit, then lower id.
-__device__ __forceinline__ bool cand_better(float va, int ea, float vb, int eb) {
-    return va > vb || (va == vb && ea < eb);
-}
-
-// Compare-exchange for a descending order by (value, then lower id).
-__device__ __forceinline__ void cex(float& va, int& ea, float& vb, int& eb) {
-    if (cand_better(vb, eb, va, ea)) {
-        const float tv = va; va = vb; vb = tv;
-        const int te = ea; ea = eb; eb = te;
-    }
+// Order-preserving map of a float to an unsigned key (larger float, larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 // One warp selects the top-k of one token's E logits (E <= 32 * NV) and
-// writes ids and gates.  Each lane sorts its NV values once (a bitonic network
-// in registers); each of the k rounds then takes the warp's best lane head and
-// the winning lane shifts its list.  Gates are formed in double from the
+// writes ids and gates.  Each lane keeps its NV values and its best one; each
+// of the k rounds takes the warp's best (a warp max of the value keys, then
+// the lowest id among the lanes holding that key), and only the winning lane
+// removes it and rescans its values.  Gates are formed in double from the
 // selected fp32 logits.
 template <int NV, bool SHARED = false>
 __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
                             float* __restrict__ gates) {
     const int lane = threadIdx.x & 31;
     float v[NV];
-    int e[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-        e[i] = lane + 32 * i;
-        v[i] = (e[i] < E) ? (SHARED ? lrow[e[i]] : __ldcg(lrow + e[i])) : -INFINITY;
-        if (e[i] >= E) e[i] = 0x7fffffff;
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? (SHARED ? lrow[e] : __ldcg(lrow + e)) : -INFINITY;
     }
-    // bitonic sort, descending
+    // the lane's best: larger value, then lower id (= lower i for one lane)
+    auto rescan = [&](float& bv, int& be) {
+        bv = v[0];
+        int bi = 0;
 #pragma unroll
-    for (int kk = 2; kk <= NV; kk <<= 1) {
-#pragma unroll
-        for (int j = kk >> 1; j > 0; j >>= 1) {
-#pragma unroll
-            for (int i = 0; i < NV; ++i) {
-                const int l = i ^ j;
-                if (l > i) {
-                    if ((i & kk) == 0) cex(v[i], e[i], v[l], e[l]);
-                    else cex(v[l], e[l], v[i], e[i]);
-                }
-            }
-        }
-    }
+        for (int i = 1; i < NV; ++i)
+            if (v[i] > bv) { bv = v[i]; bi = i; }
+        be = (lane + 32 * bi < E) ? lane + 32 * bi : 0x7fffffff;
+    };
+    float bv;
+    int be;
+    rescan(bv, be);
     float my_v = 0.f, l0 = 0.f;
     int my_e = 0;
     for (int r = 0; r < k; ++r) {
-        float wv = v[0];
-        int we = e[0];
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, wv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, we, off);
-            if (cand_better(ov, oe, wv, we)) { wv = ov; we = oe; }
-        }
+        const uint32_t mykey = float_key(bv);
+        const uint32_t wkey = __reduce_max_sync(0xffffffffu, mykey);
+        const int we = (int)__reduce_min_sync(0xffffffffu, mykey == wkey ? (uint32_t)be : 0xffffffffu);
+        const float wv = __shfl_sync(0xffffffffu, bv, we & 31);
         if (r == 0) l0 = wv;
         if (lane == r) { my_v = wv; my_e = we; }
-        if (e[0] == we) {                       // this lane supplied the winner: pop its head
+        if (be == we) {                         // this lane supplied the winner: remove it
+            const int wi = (we - lane) >> 5;
 #pragma unroll
-            for (int i = 0; i + 1 < NV; ++i) { v[i] = v[i + 1]; e[i] = e[i + 1]; }
-            v[NV - 1] = -INFINITY;
-            e[NV - 1] = 0x7fffffff;
+            for (int i = 0; i < NV; ++i)
+                if (i == wi) v[i] = -INFINITY;
+            rescan(bv, be);
         }
     }
     const double ex = (lane < k) ? exp((double)my_v - (double)l0) : 0.0;
