@@ -271,7 +271,7 @@ def run_ours(args, ws_, rank, local):
                    "parallelism": f"replicas x{ws_}"},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": T * D * 2,
                 "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": (3 if T <= 4 else 8) * K,
+        "gpu_launches": (3 if T <= 4 else 10) * K,
         "roofline": roofline,
         "hit_rate": round(float(np.mean(hits)), 4), "u_hit_mean": round(float(np.mean(u_hit)), 2),
         "step_alg_bytes": round(float(np.mean(step_bytes))),
