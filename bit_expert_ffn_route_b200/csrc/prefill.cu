@@ -562,8 +562,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_c[kCodeSlots], empty_c[kCodeSlots];
     // round slot i (= round % 4): its TMEM A buffer and its row-operand stage are
-    // filled by full_a[i] / full_b[i] and released together by round_empty[i]
-    __shared__ uint64_t full_a[kABufs], full_b[kABufs], round_empty[kABufs];
+    // filled under round_full[i] (the 4 dequant warps of the round arrive, the
+    // row-operand TMA arrives with its byte count) and released by round_empty[i]
+    __shared__ uint64_t round_full[kABufs], round_empty[kABufs];
     __shared__ uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain_bar;
     __shared__ uint32_t tmem_base;
     __shared__ float gate_x[kGateRows][17];        // epilogue: gate values handed to the up lanes
@@ -584,8 +585,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&empty_c[s], 4 * rps);    // the 4 quadrant warps of each of its rounds
         }
         for (int s = 0; s < kABufs; ++s) {
-            mbar_init(&full_a[s], 4);
-            mbar_init(&full_b[s], 1);
+            mbar_init(&round_full[s], 5);
             mbar_init(&round_empty[s], 1);
         }
         for (int s = 0; s < kAccBufs; ++s) {
@@ -694,7 +694,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full_a[buf]);
+                if (lane == 0) mbar_arrive(&round_full[buf]);
             }
         }
     } else if (!dead && warp < kTmaWarp) {
@@ -809,7 +809,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int st = h & 3;
                     if (h >= kABufs && !mbar_wait(&round_empty[st], ((h >> 2) - 1) & 1, g.err)) { ok = false; break; }
                     const uint32_t b_base = smem_u32(b_ring + st * kBStageBytes);
-                    mbar_arrive_expect_tx(&full_b[st], 2u * (uint32_t)npad * kKStep * 2);
+                    mbar_arrive_expect_tx(&round_full[st], 2u * (uint32_t)npad * kKStep * 2);
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const int x = (2 * rr + j) * kKStep;
@@ -818,7 +818,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             const int left = npad - n;
                             const CUtensorMap* m = left >= 128 ? &rows128 : left >= 64 ? &rows64 : left >= 32 ? &rows32 : &rows16;
                             const int nb = left >= 128 ? 128 : left >= 64 ? 64 : left >= 32 ? 32 : 16;
-                            tma_load_2d(dst + n * 128, m, x, row0 + n, &full_b[st], pol);
+                            tma_load_2d(dst + n * 128, m, x, row0 + n, &round_full[st], pol);
                             n += nb;
                         }
                     }
@@ -827,7 +827,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             // every issued stage completes before the CTA exits
             for (int j = issued - kABufs; j < issued; ++j)
-                if (j >= 0) mbar_drain(&full_b[j & 3], (j >> 2) & 1);
+                if (j >= 0) mbar_drain(&round_full[j & 3], (j >> 2) & 1);
         }
         __syncwarp();
     } else if (!dead && warp == kMmaWarp) {
@@ -849,10 +849,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int rr = 0; rr < R; ++rr) {
                     const int gr = li * R + rr;
                     const int buf = gr & 3;
-                    if (!mbar_wait(&full_a[buf], (gr >> 2) & 1, g.err) || !mbar_wait(&full_b[buf], (gr >> 2) & 1, g.err)) {
-                        ok = false;
-                        break;
-                    }
+                    if (!mbar_wait(&round_full[buf], (gr >> 2) & 1, g.err)) { ok = false; break; }
                     tc_fence_after();
                     // descriptor start addresses advance in 16-byte units
                     const uint64_t bd = bdesc0 + (uint64_t)((buf * kBStageBytes) >> 4);
