@@ -15,6 +15,7 @@ Per-kernel durations come from external event nodes inside the same graph.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -43,6 +44,24 @@ def _peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
     return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _traffic(kind):
+    """DRAM bytes per launch from the committed ncu capture of this kernel, or
+    None when the kernel's sources changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            e = json.load(f)[kind]
+        h = hashlib.sha256()
+        for src in e["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != e["sha256"]:
+            return None, None
+        return int(e["bytes_per_launch"]), e["covers"]
+    except (OSError, KeyError, ValueError):
+        return None, None
 
 
 class ClockSampler:
@@ -210,17 +229,18 @@ def run_ours(args, ws_, rank, local):
     fwd_avg_ms = float(np.mean(fwd_ms))
     fwd_alg = float(np.mean([fwd_bytes[i % R] for i in range(G)]))
     fwd_fl = float(np.mean([fwd_flops[i % R] for i in range(G)]))
+    traffic, traffic_covers = _traffic("decode" if T <= 4 else "prefill")
     if T <= 4:
         achieved = fwd_alg / (fwd_avg_ms / 1e3) / 1e9
         roofline = {"kernel": "moe_expert_forward (decode_ffn_kernel: gate|up + down dequant-GEMV)", "bound": "hbm",
                     "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                    "traffic": None, "peak_kind": f"{peak_kind} copy bandwidth",
+                    "traffic": traffic, "traffic_covers": traffic_covers, "peak_kind": f"{peak_kind} copy bandwidth",
                     "algorithmic_bytes_per_launch": round(fwd_alg), "avg_launch_us": round(fwd_avg_ms * 1e3, 3)}
     else:
         achieved = fwd_fl / (fwd_avg_ms / 1e3) / 1e12
         roofline = {"kernel": "moe_expert_forward (plan + tcgen05 gate|up and down grouped GEMMs)", "bound": "tensor",
                     "achieved": round(achieved, 1), "peak": tf_sus, "unit": "TFLOP/s", "frac": round(achieved / tf_sus, 4),
-                    "traffic": None, "peak_kind": f"{peak_kind} bf16 sustained (burst {tf})",
+                    "traffic": traffic, "traffic_covers": traffic_covers, "peak_kind": f"{peak_kind} bf16 sustained (burst {tf})",
                     "algorithmic_flops_per_launch": round(fwd_fl), "avg_launch_us": round(fwd_avg_ms * 1e3, 3)}
 
     # end to end through the public API: pinned host input -> device, the three
