@@ -39,6 +39,8 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kTeams = 2;                        // consumer teams, alternating items
+constexpr int kTeamWarps = kConsumerWarps / kTeams;
 constexpr int kThreads = kConsumers + 32;        // + one producer warp
 constexpr int kXStride = 36;                     // floats per 32-weight chunk: 32 x + 4 constants
 constexpr int kMaxPairs = kDecodeMaxT * kMaxTopK + 1;
@@ -138,7 +140,14 @@ MOE_DEVINL int code_pos(int i) {
 
 MOE_DEVINL float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-MOE_DEVINL void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
+MOE_DEVINL void team_sync(int team) { asm volatile("bar.sync %0, %1;" ::"r"(2 + team), "n"(kTeamWarps * 32) : "memory"); }
+// A team barrier that also returns whether v held on every thread of the team.
+MOE_DEVINL bool team_all(int team, bool v) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)v), "r"(2 + team), "n"(kTeamWarps * 32) : "memory");
+    return r != 0;
+}
 
 // ---------------------------------------------------------------- format geometry
 template <int FMT>
@@ -212,6 +221,7 @@ struct Shared {
     int slot_of[kMaxPairs];
     int table[kMaxE];          // the slot table, staged before the dependency wait
     int n_owners;
+    int abort[kTeams];         // set by a consumer team that stopped on an error
 };
 
 // The slot table is an input of the layer, not produced by the router: stage it
@@ -495,18 +505,44 @@ MOE_DEVINL void issue_rows(const Planes& pl, int row0, int nrows, int K, uint8_t
     if constexpr (FMT == MOE_Q3_S256) bulk_g2s(dst + (cr + mr) * nrows, pl.d + (size_t)row0 * dr, dr * nrows, bar);
 }
 
+// ---------------------------------------------------------------- item geometry
+// The consumers form two teams of eight warps; a team takes every other item
+// of the ring, so that one team's per-item tail (reduction, stores, barrier
+// waits) overlaps the other team's inner loops.  Within an item a warp is cut
+// into G groups of lpr lanes; a group owns one unit (a gate|up feature or a
+// pair of down rows) and its lanes split the unit's nb chunks, nb / lpr each.
+// G grows (lpr shrinks) until the team's 8*G groups cover the item's units
+// in one pass, which keeps every warp busy and the shuffle reductions short.
+// Lane gl of group g takes chunk gl + lpr * ((it + g) mod (nb / lpr)) at
+// iteration it: the groups of one warp start on different chunks, so their
+// code, scale and activation reads fall in different shared-memory banks.
+struct Split { int lpr, G, nit; };
+MOE_DEVINL Split split_for(int units, int nb) {
+    const int want = units / kTeamWarps;      // groups per warp for one pass
+    int gp = 1;                               // largest power of two <= want, at most 8
+    while (gp < 8 && 2 * gp <= want) gp *= 2;
+    int lpr = 32 / gp;
+    const int pow2nb = nb & -nb;              // lpr must divide nb
+    if (lpr > pow2nb) lpr = pow2nb;
+    Split sp;
+    sp.lpr = lpr;
+    sp.G = 32 / lpr;
+    sp.nit = nb / lpr;
+    return sp;
+}
+
 // ---------------------------------------------------------------- gate | up
 // Item = (owner u, features [f0, f0 + rf)); staged as gate rows then up rows.
-// One feature (its gate row and up row) per warp-group pass; the chunk data of
-// the next chunk is read from shared memory while the current one is computed.
+// A group computes one feature: its gate row and its up row, chunk by chunk,
+// the next chunk's codes read from shared memory while this one is computed.
 template <int FMT, int NT>
 __device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int f0, int rf, const uint8_t* stage,
-                            const float* xs) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                            const float* xs, int wt) {
+    const int lane = threadIdx.x & 31;
     const int D = prm.P.D, F = prm.P.F;
     const int nb = D / 32;
-    const int lpr = min(32, nb & -nb);
-    const int G = 32 / lpr, group = lane / lpr, gl = lane % lpr;
+    const Split sp = split_for(rf, nb);
+    const int lpr = sp.lpr, G = sp.G, nit = sp.nit, group = lane / lpr, gl = lane % lpr;
     const uint32_t cr = Geo<FMT>::code_row(D), mr = Geo<FMT>::meta_row(D);
     const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * rf;   // gate rows then up rows
     const uint8_t* gc = stage;
@@ -518,20 +554,26 @@ __device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int 
     const float* xt[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) xt[t] = xs + (size_t)o.tok[t] * nb * kXStride;
-    for (int fl = warp * G + group; fl < rf; fl += kConsumerWarps * G) {   // local feature
+    for (int base = wt * G; base < rf; base += kTeamWarps * G) {
+        const int fq = base + group;
+        const bool act = fq < rf;
+        const int fl = act ? fq : rf - 1;      // idle groups recompute a valid feature, unstored
         float res[2][NT];
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int t = 0; t < NT; ++t) res[r][t] = 0.f;
+        int c = group % nit;
+        int b = gl + lpr * c;
         uint32_t cw[2][3];
         float sa[2], sb[2];
-        smem_chunk<FMT>(gc, gm, gd, fl, D, gl, cw[0], sa[0], sb[0]);
-        smem_chunk<FMT>(uc, um, ud, fl, D, gl, cw[1], sa[1], sb[1]);
-        for (int b = gl; b < nb; b += lpr) {
+        smem_chunk<FMT>(gc, gm, gd, fl, D, b, cw[0], sa[0], sb[0]);
+        smem_chunk<FMT>(uc, um, ud, fl, D, b, cw[1], sa[1], sb[1]);
+        for (int it = 0; it < nit; ++it) {
+            c = c + 1 == nit ? 0 : c + 1;
+            const int bn = gl + lpr * c;       // next chunk (wraps to the first on the last pass: unused)
             uint32_t ncw[2][3];
             float nsa[2], nsb[2];
-            const int bn = b + lpr < nb ? b + lpr : b;
             smem_chunk<FMT>(gc, gm, gd, fl, D, bn, ncw[0], nsa[0], nsb[0]);
             smem_chunk<FMT>(uc, um, ud, fl, D, bn, ncw[1], nsa[1], nsb[1]);
             const float* xc[NT];
@@ -543,13 +585,14 @@ __device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int 
                 cw[r][0] = ncw[r][0]; cw[r][1] = ncw[r][1]; cw[r][2] = ncw[r][2];
                 sa[r] = nsa[r]; sb[r] = nsb[r];
             }
+            b = bn;
         }
         for (int off = lpr >> 1; off >= 1; off >>= 1)
 #pragma unroll
             for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int t = 0; t < NT; ++t) res[r][t] += __shfl_xor_sync(0xffffffffu, res[r][t], off);
-        if (gl == 0) {
+        if (act && gl == 0) {
 #pragma unroll
             for (int t = 0; t < NT; ++t)
                 prm.hbuf[((size_t)u * kDecodeMaxT + t) * F + f0 + fl] = f32_to_bf16_rne(silu_f(res[0][t]) * res[1][t]);
@@ -558,34 +601,40 @@ __device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int 
 }
 
 // ---------------------------------------------------------------- down
-// Item = (owner u, rows [d0, d0 + rd)) of Wd; two rows per warp-group pass.
+// Item = (owner u, rows [d0, d0 + rd)) of Wd; a group computes two rows.
 template <int FMT, int NT>
 __device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int rd, const uint8_t* stage,
-                          const float* hs) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                          const float* hs, int wt) {
+    const int lane = threadIdx.x & 31;
     const int D = prm.P.D, F = prm.P.F, k = prm.k;
     const int nb = F / 32;
-    const int lpr = min(32, nb & -nb);
-    const int G = 32 / lpr, group = lane / lpr, gl = lane % lpr;
+    const int pairs = rd / 2;
+    const Split sp = split_for(pairs, nb);
+    const int lpr = sp.lpr, G = sp.G, nit = sp.nit, group = lane / lpr, gl = lane % lpr;
     const uint32_t cr = Geo<FMT>::code_row(F), mr = Geo<FMT>::meta_row(F);
     const uint8_t* dc = stage;
     const uint8_t* dm = stage + cr * rd;
     const uint8_t* dd = stage + (cr + mr) * rd;
-    for (int q = warp * G + group; q < rd / 2; q += kConsumerWarps * G) {
-        const int rl = 2 * q;
+    for (int base = wt * G; base < pairs; base += kTeamWarps * G) {
+        const int qq = base + group;
+        const bool act = qq < pairs;
+        const int rl = 2 * (act ? qq : pairs - 1);
         float res[2][NT];
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
             for (int t = 0; t < NT; ++t) res[r][t] = 0.f;
+        int c = group % nit;
+        int b = gl + lpr * c;
         uint32_t cw[2][3];
         float sa[2], sb[2];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, gl, cw[r], sa[r], sb[r]);
-        for (int b = gl; b < nb; b += lpr) {
+        for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, b, cw[r], sa[r], sb[r]);
+        for (int it = 0; it < nit; ++it) {
+            c = c + 1 == nit ? 0 : c + 1;
+            const int bn = gl + lpr * c;
             uint32_t ncw[2][3];
             float nsa[2], nsb[2];
-            const int bn = b + lpr < nb ? b + lpr : b;
 #pragma unroll
             for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, bn, ncw[r], nsa[r], nsb[r]);
             const float* xc[NT];
@@ -597,13 +646,14 @@ __device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int r
                 cw[r][0] = ncw[r][0]; cw[r][1] = ncw[r][1]; cw[r][2] = ncw[r][2];
                 sa[r] = nsa[r]; sb[r] = nsb[r];
             }
+            b = bn;
         }
         for (int off = lpr >> 1; off >= 1; off >>= 1)
 #pragma unroll
             for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int t = 0; t < NT; ++t) res[r][t] += __shfl_xor_sync(0xffffffffu, res[r][t], off);
-        if (gl == 0) {
+        if (act && gl == 0) {
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const float2 v = make_float2(res[0][t], res[1][t]);
@@ -638,12 +688,12 @@ template <int FMT, int NTMAX>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams prm) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ Shared sh;
-    __shared__ int abort_flag;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = prm.P.D, F = prm.P.F, rf = prm.rf, rd = prm.rd, NS = prm.ns_gu;
     const int nbx = D / 32, nbh = F / 32;
     const size_t xs_bytes = ((size_t)prm.T * nbx * kXStride * 4 + 127) / 128 * 128;
-    const size_t hs_bytes = ((size_t)kDecodeMaxT * nbh * kXStride * 4 + 127) / 128 * 128;
+    const size_t hs_floats = ((size_t)kDecodeMaxT * nbh * kXStride + 31) / 32 * 32;   // one per team
+    const size_t hs_bytes = kTeams * hs_floats * 4;
     float* xs = reinterpret_cast<float*>(smem);
     float* hs = reinterpret_cast<float*>(smem + xs_bytes);
     uint8_t* stages = smem + xs_bytes + hs_bytes;
@@ -653,9 +703,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     const int nfb = F / rf, nrb = D / rd;
     uint32_t* done = prm.done;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kConsumerWarps); }
+        for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kTeamWarps); }
         fence_mbar_init();
-        abort_flag = 0;
+        for (int tm = 0; tm < kTeams; ++tm) sh.abort[tm] = 0;
     }
     stage_table(prm, sh);
     __syncthreads();
@@ -679,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
             for (int j = 0; j < total; ++j) {
                 const int s = j % NS;
                 if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) break;
-                if (abort_flag) break;
+                if (*reinterpret_cast<volatile int*>(&sh.abort[0]) | *reinterpret_cast<volatile int*>(&sh.abort[1])) break;
                 uint8_t* dst = stages + (size_t)s * stage_bytes;
                 if (j < ng) {
                     const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
@@ -696,76 +746,86 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
             }
         }
     } else {
-        int j = 0;
+        // consumer teams: team tm takes items j = tm, tm + 2, ... of the ring
+        const int team = warp / kTeamWarps, wt = warp % kTeamWarps;
+        const int tl = (int)threadIdx.x - team * kTeamWarps * 32;
+        float* hst = hs + (size_t)team * hs_floats;
         bool ok = true;
-        for (; j < ng && ok; ++j) {
-            const int s = j % NS;
-            if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) { ok = false; break; }
-            const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
-            const int u = ip.u, f0 = ip.row0;
-            const Owner& o = sh.owners[u];
-            const uint8_t* st = stages + (size_t)s * stage_bytes;
-            if constexpr (NTMAX == 1) {
-                gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs);
-            } else {
-                switch (o.ntok) {
-                    case 1: gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs); break;
-                    case 2: gateup_item<FMT, 2>(prm, o, u, f0, ip.nrows, st, xs); break;
-                    case 3: gateup_item<FMT, 3>(prm, o, u, f0, ip.nrows, st, xs); break;
-                    default: gateup_item<FMT, 4>(prm, o, u, f0, ip.nrows, st, xs); break;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.empty[s]);
-        }
-        // publish this CTA's h once for its whole gate|up range: every writer
-        // fences its own stores, then one thread adds the item counts per owner
-        __threadfence();
-        consumer_sync();
-        if (threadIdx.x == 0) {
-            for (int jj = 0; jj < ng; ++jj) atomicAdd(done + item_pos(blockIdx.x + jj * gridDim.x, nfb, rf).u, 1u);
-        }
         int cur = -1;
-        for (int i = d0r; i < d1r && ok; ++i, ++j) {
+        const int total = ng + (d1r - d0r);
+        for (int j = team; j < total; j += kTeams) {
             const int s = j % NS;
-            const ItemPos ip = item_pos(i, nrb, rd);
-            const int u = ip.u, r0 = ip.row0;
-            const Owner& o = sh.owners[u];
-            if (u != cur) {
-                consumer_sync();
-                if (threadIdx.x == 0) {
-                    const uint32_t target = (uint32_t)(u == 0 ? 2 * nfb : nfb);   // items of owner u
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire(done + u) < target) {
-                        if (*reinterpret_cast<volatile uint32_t*>(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
-                            atomicOr(prm.err, kErrTimeout);
-                            abort_flag = 1;
-                            break;
+            const uint8_t* st = stages + (size_t)s * stage_bytes;
+            if (j < ng) {
+                bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
+                const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
+                const int u = ip.u, f0 = ip.row0;
+                const Owner& o = sh.owners[u];
+                if (got) {
+                    if constexpr (NTMAX == 1) {
+                        gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs, wt);
+                    } else {
+                        switch (o.ntok) {
+                            case 1: gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
+                            case 2: gateup_item<FMT, 2>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
+                            case 3: gateup_item<FMT, 3>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
+                            default: gateup_item<FMT, 4>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
                         }
-                        __nanosleep(64);
                     }
                 }
-                consumer_sync();
-                if (abort_flag) { ok = false; break; }
-                stage_activations<FMT>(prm.hbuf + (size_t)u * kDecodeMaxT * F, F, o.ntok, F, hs, 0, kConsumers, true);
-                consumer_sync();
-                cur = u;
-            }
-            if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) { ok = false; break; }
-            const uint8_t* st = stages + (size_t)s * stage_bytes;
-            if constexpr (NTMAX == 1) {
-                down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hs);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.empty[s]);
+                // the team's h stores of this item are done (and the verdict is
+                // the team's, so every thread leaves the loop together): publish
+                ok = team_all(team, got);
+                if (!ok) break;
+                if (tl == 0) red_release_add(done + u, 1u);
             } else {
-                switch (o.ntok) {
-                    case 1: down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hs); break;
-                    case 2: down_item<FMT, 2>(prm, o, r0, ip.nrows, st, hs); break;
-                    case 3: down_item<FMT, 3>(prm, o, r0, ip.nrows, st, hs); break;
-                    default: down_item<FMT, 4>(prm, o, r0, ip.nrows, st, hs); break;
+                const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
+                const int u = ip.u, r0 = ip.row0;
+                const Owner& o = sh.owners[u];
+                if (u != cur) {
+                    team_sync(team);                    // the team is done reading hst
+                    bool waited = true;
+                    if (tl == 0) {
+                        const uint32_t target = (uint32_t)(u == 0 ? 2 * nfb : nfb);   // items of owner u
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire(done + u) < target) {
+                            if (*reinterpret_cast<volatile uint32_t*>(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
+                                atomicOr(prm.err, kErrTimeout);
+                                waited = false;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                    ok = team_all(team, waited);
+                    if (!ok) break;
+                    stage_activations<FMT>(prm.hbuf + (size_t)u * kDecodeMaxT * F, F, o.ntok, F, hst,
+                                           team * kTeamWarps * 32, kTeamWarps * 32, true);
+                    team_sync(team);
+                    cur = u;
                 }
+                const bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
+                if (got) {
+                    if constexpr (NTMAX == 1) {
+                        down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hst, wt);
+                    } else {
+                        switch (o.ntok) {
+                            case 1: down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hst, wt); break;
+                            case 2: down_item<FMT, 2>(prm, o, r0, ip.nrows, st, hst, wt); break;
+                            case 3: down_item<FMT, 3>(prm, o, r0, ip.nrows, st, hst, wt); break;
+                            default: down_item<FMT, 4>(prm, o, r0, ip.nrows, st, hst, wt); break;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.empty[s]);
+                ok = team_all(team, got);
+                if (!ok) break;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.empty[s]);
         }
+        if (!ok && tl == 0) sh.abort[team] = 1;
     }
     // last CTA out resets the per-owner counters for the next call
     __syncthreads();
@@ -795,11 +855,11 @@ template <int FMT, int NTMAX>
 moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
     const int T = prm.T, D = prm.P.D, F = prm.P.F;
     const size_t xs_bytes = ((size_t)T * (D / 32) * kXStride * 4 + 127) / 128 * 128;
-    const size_t hs_bytes = ((size_t)kDecodeMaxT * (F / 32) * kXStride * 4 + 127) / 128 * 128;
+    const size_t hs_bytes = kTeams * (((size_t)kDecodeMaxT * (F / 32) * kXStride + 31) / 32 * 32) * 4;
     // gate|up items of rf features, down items of rd rows, one ring of up to 4
     // stages (~3-4 items in flight per SM cover the copy latency)
     int rf = 16, rd = 128;
-    const size_t budget = 212 * 1024;
+    const size_t budget = 216 * 1024;
     auto stage_of = [&](int rf_, int rd_) {
         const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf_, b = (size_t)Geo<FMT>::row_bytes(F) * rd_;
         return a > b ? a : b;
