@@ -26,20 +26,27 @@ __global__ void __launch_bounds__(256) combine_f32_kernel(const int32_t* __restr
     const int t = blockIdx.y;
     const int d = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (d >= D) return;
-    // all row indices and gates first, then all rows: two round trips in total
+    // The decode path writes the row of (t, r) at index t*(k+1) + r (the row
+    // map holds that index for a hit, -1 for a miss) and the shared row at
+    // t*(k+1) + k: load those rows together with the map and the gates (one
+    // round trip); a map entry pointing elsewhere is followed with a second load.
     int row[kMaxTopK];
     float g[kMaxTopK];
-#pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r) row[r] = (r < k) ? __ldg(rowmap + t * (k + 1) + r) : -1;
-#pragma unroll
-    for (int r = 0; r < kMaxTopK; ++r) g[r] = (r < k) ? __ldg(gates + t * k + r) : 0.f;
-    const int srow = __ldg(rowmap + t * (k + 1) + k);
     float4 y[kMaxTopK];
 #pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r) {
+        row[r] = (r < k) ? __ldg(rowmap + t * (k + 1) + r) : -1;
+        g[r] = (r < k) ? __ldg(gates + t * k + r) : 0.f;
+        y[r] = (r < k) ? __ldg(reinterpret_cast<const float4*>(rows + (size_t)(t * (k + 1) + r) * D + d))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int srow = __ldg(rowmap + t * (k + 1) + k);
+    float4 ys = __ldg(reinterpret_cast<const float4*>(rows + (size_t)(t * (k + 1) + k) * D + d));
+#pragma unroll
     for (int r = 0; r < kMaxTopK; ++r)
-        y[r] = (row[r] >= 0) ? __ldg(reinterpret_cast<const float4*>(rows + (size_t)row[r] * D + d))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 ys = __ldg(reinterpret_cast<const float4*>(rows + (size_t)srow * D + d));
+        if (row[r] >= 0 && row[r] != t * (k + 1) + r)
+            y[r] = __ldg(reinterpret_cast<const float4*>(rows + (size_t)row[r] * D + d));
+    if (srow != t * (k + 1) + k) ys = __ldg(reinterpret_cast<const float4*>(rows + (size_t)srow * D + d));
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int r = 0; r < kMaxTopK; ++r) {

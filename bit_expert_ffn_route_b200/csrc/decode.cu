@@ -41,7 +41,9 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kTeams = 2;                        // consumer teams, alternating items
 constexpr int kTeamWarps = kConsumerWarps / kTeams;
-constexpr int kThreads = kConsumers + 32;        // + one producer warp
+constexpr int kProducerWarp = kConsumerWarps;    // bulk copies into the stage ring
+constexpr int kPublisherWarp = kConsumerWarps + 1; // releases finished gate|up items to other CTAs
+constexpr int kThreads = kConsumers + 64;
 constexpr int kXStride = 36;                     // floats per 32-weight chunk: 32 x + 4 constants
 constexpr int kMaxPairs = kDecodeMaxT * kMaxTopK + 1;
 constexpr int kMaxStages = 8;
@@ -222,6 +224,7 @@ struct Shared {
     int table[kMaxE];          // the slot table, staged before the dependency wait
     int n_owners;
     int abort[kTeams];         // set by a consumer team that stopped on an error
+    uint32_t team_items[kTeams];   // gate|up items finished by each team (release.cta by its leader)
 };
 
 // The slot table is an input of the layer, not produced by the router: stage it
@@ -668,9 +671,59 @@ __device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int r
     }
 }
 
-MOE_DEVINL void red_release_add(uint32_t* p, uint32_t v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+MOE_DEVINL void st_release_cta(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v) : "memory");
 }
+MOE_DEVINL uint32_t ld_acquire_cta(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared.u32 %0, [%1];" : "=r"(v) : "r"((uint32_t)__cvta_generic_to_shared(p)) : "memory");
+    return v;
+}
+MOE_DEVINL void red_relaxed_add(uint32_t* p, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+MOE_DEVINL void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Down items are split into contiguous per-CTA ranges of equal estimated cost.
+// An item of n rows of an owner serving nt tokens costs n * (4 + 3 (nt - 1))
+// (a row served to four tokens measured about three times one served to one).
+struct DownCost {
+    int items;     // items of the owner
+    int cost;      // cost of one item
+};
+MOE_DEVINL DownCost down_cost(const Shared& sh, int u, int nrb, int rd) {
+    DownCost c;
+    const int nt = sh.owners[u].ntok;
+    c.items = u == 0 ? 2 * nrb : nrb;
+    c.cost = (u == 0 ? rd / 2 : rd) * (4 + 3 * (nt - 1));
+    return c;
+}
+// Index (in item_pos order) of the first down item whose cumulative cost
+// start is >= pos.
+MOE_DEVINL int down_item_at(const Shared& sh, long long pos, int nrb, int rd) {
+    long long base = 0;
+    int idx = 0;
+    for (int u = 0; u < sh.n_owners; ++u) {
+        const DownCost c = down_cost(sh, u, nrb, rd);
+        const long long end = base + (long long)c.items * c.cost;
+        if (end > pos) {
+            const long long m = pos <= base ? 0 : (pos - base + c.cost - 1) / c.cost;
+            return idx + (int)(m < c.items ? m : c.items);
+        }
+        base = end;
+        idx += c.items;
+    }
+    return idx;
+}
+MOE_DEVINL long long down_total_cost(const Shared& sh, int nrb, int rd) {
+    long long t = 0;
+    for (int u = 0; u < sh.n_owners; ++u) {
+        const DownCost c = down_cost(sh, u, nrb, rd);
+        t += (long long)c.items * c.cost;
+    }
+    return t;
+}
+
 MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -679,11 +732,13 @@ MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
 
 // ---------------------------------------------------------------- the fused kernel
 // One persistent CTA per SM.  Each CTA takes its gate|up items (round-robin),
-// then a contiguous range of down items, through one ring of stages.  A
-// down item of owner u waits until every gate|up item of u has published its
-// h (a per-owner item counter in ws, advanced by each CTA once its whole gate|up
-// range is done); the down weights stream in meanwhile.  The last CTA to finish
-// resets the counters, so every completed call leaves them zero.
+// then a contiguous range of down items (equal estimated cost per CTA),
+// through one ring of stages.  A down item of owner u waits until every
+// gate|up item of u has published its h: a per-owner item counter in ws,
+// advanced by a publisher warp that releases each finished item at gpu scope,
+// off the computing warps' path.  The down weights stream in meanwhile.  The
+// last CTA to finish resets the counters, so every completed call leaves them
+// zero.
 template <int FMT, int NTMAX>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams prm) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -705,25 +760,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kTeamWarps); }
         fence_mbar_init();
-        for (int tm = 0; tm < kTeams; ++tm) sh.abort[tm] = 0;
+        for (int tm = 0; tm < kTeams; ++tm) { sh.abort[tm] = 0; sh.team_items[tm] = 0; }
     }
     stage_table(prm, sh);
     __syncthreads();
     pdl_wait();                      // ids come from the router
+    // warp 0 resolves the owners and releases the producer and publisher
+    // (barrier 1) while the other consumers stage x; the consumers meet at
+    // barrier 4 before computing
     if (warp == 0) {
         resolve_owners(prm, sh, blockIdx.x == 0);
+        asm volatile("bar.arrive 1, 96;" ::: "memory");
+        asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
     } else if (warp < kConsumerWarps) {
         stage_activations<FMT>(prm.x, D, prm.T, D, xs, 32, kConsumers - 32);
+        asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
+    } else {
+        asm volatile("bar.sync 1, 96;" ::: "memory");
     }
-    __syncthreads();
     pdl_launch_dependents();
     // gate|up items round-robin over the CTAs (x is staged for every token);
-    // down items in equal-count contiguous ranges (h is re-staged per owner)
-    const int n_g = items_of(sh.n_owners, nfb), n_d = items_of(sh.n_owners, nrb);
+    // down items in contiguous ranges of equal cost (h is re-staged per owner)
+    const int n_g = items_of(sh.n_owners, nfb);
     const int ng = n_g > (int)blockIdx.x ? (n_g - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const int per_d = (n_d + gridDim.x - 1) / gridDim.x;
-    const int d0r = min(n_d, (int)blockIdx.x * per_d), d1r = min(n_d, d0r + per_d);
-    if (warp == kConsumerWarps) {    // producer: gate|up items, then down items
+    const long long dcost = down_total_cost(sh, nrb, rd);
+    const int d0r = down_item_at(sh, dcost * (long long)blockIdx.x / gridDim.x + (dcost * (long long)blockIdx.x % gridDim.x != 0), nrb, rd);
+    const int d1r = down_item_at(sh, dcost * (long long)(blockIdx.x + 1) / gridDim.x + (dcost * (long long)(blockIdx.x + 1) % gridDim.x != 0), nrb, rd);
+    if (warp == kPublisherWarp) {    // publisher: release finished gate|up items, in each team's order
+        if (lane == 0) {
+            uint32_t pub[kTeams] = {0u, 0u};
+            const uint32_t want[kTeams] = {(uint32_t)((ng + 1) / 2), (uint32_t)(ng / 2)};
+            const uint64_t t0 = globaltimer_ns();
+            while (pub[0] < want[0] || pub[1] < want[1]) {
+                const uint32_t c0 = ld_acquire_cta(&sh.team_items[0]), c1 = ld_acquire_cta(&sh.team_items[1]);
+                if (c0 > pub[0] || c1 > pub[1]) {
+                    fence_acq_rel_gpu();             // with the relaxed adds below: one release per batch
+                    const uint32_t c[kTeams] = {c0, c1};
+                    for (int tm = 0; tm < kTeams; ++tm)
+                        for (uint32_t n = pub[tm]; n < c[tm]; ++n) {
+                            const int j = tm + kTeams * (int)n;
+                            red_relaxed_add(done + item_pos(blockIdx.x + j * gridDim.x, nfb, rf).u, 1u);
+                        }
+                    pub[0] = c0;
+                    pub[1] = c1;
+                } else {
+                    if (*reinterpret_cast<volatile uint32_t*>(prm.err) ||
+                        *reinterpret_cast<volatile int*>(&sh.abort[0]) || *reinterpret_cast<volatile int*>(&sh.abort[1]))
+                        break;
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        atomicOr(prm.err, kErrTimeout);
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
+        }
+    } else if (warp == kProducerWarp) {    // producer: gate|up items, then down items
         if (lane == 0) {
             const int total = ng + (d1r - d0r);
             for (int j = 0; j < total; ++j) {
@@ -752,6 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         float* hst = hs + (size_t)team * hs_floats;
         bool ok = true;
         int cur = -1;
+        uint32_t gu_done = 0;
         const int total = ng + (d1r - d0r);
         for (int j = team; j < total; j += kTeams) {
             const int s = j % NS;
@@ -779,7 +872,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                 // the team's, so every thread leaves the loop together): publish
                 ok = team_all(team, got);
                 if (!ok) break;
-                if (tl == 0) red_release_add(done + u, 1u);
+                ++gu_done;
+                if (tl == 0) st_release_cta(&sh.team_items[team], gu_done);
             } else {
                 const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
                 const int u = ip.u, r0 = ip.row0;
@@ -828,13 +922,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         if (!ok && tl == 0) sh.abort[team] = 1;
     }
     // last CTA out resets the per-owner counters for the next call
+    // (acq_rel ticket: this CTA's counter updates, ordered before it by the
+    // barrier, precede the reset; the last CTA sees every other CTA's)
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        const uint32_t ticket = atomicAdd(done + kMaxPairs, 1u);
+        uint32_t ticket;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(ticket) : "l"(done + kMaxPairs) : "memory");
         if (ticket == gridDim.x - 1) {
             for (int u = 0; u < kMaxPairs; ++u) done[u] = 0u;
-            __threadfence();
             done[kMaxPairs] = 0u;
         }
     }

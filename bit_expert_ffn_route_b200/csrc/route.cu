@@ -15,35 +15,66 @@ namespace moe {
 // Decode route (T <= 4): one warp per expert computes its logits for all T
 // tokens, then the last block to finish selects every token's top-k.  The
 // block counter lives in ws and wraps back to zero on every completed launch.
-// Wr rows are prefetched into L2 before waiting on the producer of x.
+// Wr is not produced by the preceding kernel: each warp loads its expert's
+// row (up to kWrPre 256-element spans into registers, the rest prefetched into
+// L2) before waiting on the producer of x.  x is staged once per block as
+// fp32 in shared memory.
+constexpr int kWrPre = 12;
 template <int NT>
 __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __restrict__ x, int T, int D,
                                                            const uint16_t* __restrict__ Wr,
                                                            const float* __restrict__ bias, int E, int k,
                                                            float* __restrict__ logits, int32_t* __restrict__ ids,
                                                            float* __restrict__ gates, unsigned int* counter) {
-    extern __shared__ __align__(16) uint16_t xsm[];
+    extern __shared__ __align__(16) float xsf[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 4 + warp;
-    if (e < E && lane == 0) prefetch_l2(Wr + (size_t)e * D, (uint32_t)D * 2);
+    const int nc = D >> 8;
+    uint4 wpre[kWrPre];
+    if (e < E) {
+        const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
+#pragma unroll
+        for (int c = 0; c < kWrPre; ++c) wpre[c] = c < nc ? ld_nc_u128(wrow + 256 * c) : make_uint4(0, 0, 0, 0);
+        if (nc > kWrPre && lane == 0)
+            prefetch_l2(Wr + (size_t)e * D + 256 * kWrPre, (uint32_t)(D - 256 * kWrPre) * 2);
+    }
     pdl_wait();
-    for (int i = threadIdx.x; i < T * D / 8; i += blockDim.x)
-        reinterpret_cast<uint4*>(xsm)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
+    // stage x: every load of a batch is in flight before the first store
+    constexpr int kBatch = 8;
+    const int n16 = T * D / 8;
+    for (int i0 = 0; i0 < n16; i0 += kBatch * 128) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int i = i0 + q * 128 + (int)threadIdx.x;
+            v[q] = i < n16 ? __ldg(reinterpret_cast<const uint4*>(x) + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int i = i0 + q * 128 + (int)threadIdx.x;
+            if (i < n16) {
+                const int t = (8 * i) / D, d = 8 * i - t * D;
+                float* dst = xsf + (size_t)t * D + canon_stage_pos(d);
+                *reinterpret_cast<float4*>(dst) = make_float4(bf16lo(v[q].x), bf16hi(v[q].x), bf16lo(v[q].y), bf16hi(v[q].y));
+                *reinterpret_cast<float4*>(dst + 128) = make_float4(bf16lo(v[q].z), bf16hi(v[q].z), bf16lo(v[q].w), bf16hi(v[q].w));
+            }
+        }
+    }
     __syncthreads();
     pdl_launch_dependents();
-    if (e < E) {
-        const uint16_t* xr[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) xr[t] = xsm + (size_t)t * D;
-        canon_logits_warp<NT>(xr, T, D, Wr, bias, E, e, logits);
-    }
+    if (e < E) canon_logits_warp_staged<NT, kWrPre>(xsf, T, D, wpre, Wr, bias, E, e, logits);
+    // the last block to arrive selects: one acq_rel ticket per block (release:
+    // the block's logits, ordered before it by the barrier; acquire: every
+    // other block's logits for the last one)
     __shared__ bool last;
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) last = (atomicInc(counter, gridDim.x - 1) == gridDim.x - 1);
+    if (threadIdx.x == 0) {
+        unsigned int prev;
+        asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(prev) : "l"(counter), "r"(gridDim.x - 1) : "memory");
+        last = (prev == gridDim.x - 1);
+    }
     __syncthreads();
     if (!last) return;
-    __threadfence();
     if (warp < T) topk_warp(logits + (size_t)warp * E, E, k, ids + (size_t)warp * k, gates + (size_t)warp * k);
 }
 
@@ -65,13 +96,13 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
     cudaError_t e;
     if (T <= kDecodeMaxT) {
         const dim3 grid((E + 3) / 4), block(128);
-        const size_t smem = (size_t)T * D * sizeof(uint16_t);
+        const size_t smem = (size_t)T * D * sizeof(float);
         static bool attr = false;
         if (!attr) {
-            cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
             attr = true;
         }
         switch (T) {

@@ -49,6 +49,71 @@ __device__ __forceinline__ void canon_logits_warp(const uint16_t* const (&xrow)[
     }
 }
 
+// Position of element d of a token row in the fp32 staging layout of the
+// decode router: within each 256-element span, elements j = 0..3 of lane L's
+// eight sit at 4L + j and elements j = 4..7 at 128 + 4L + (j - 4), so each of a
+// lane's two 16-byte reads is one contiguous 512-byte sweep of the warp.
+__device__ __forceinline__ int canon_stage_pos(int d) {
+    const int c = d >> 8, L = (d >> 3) & 31, j = d & 7;
+    return (c << 8) + ((j >> 2) << 7) + (L << 2) + (j & 3);
+}
+
+// canon_logits_warp for token rows staged in shared memory as fp32 (exact
+// copies of the bf16 values) in the canon_stage_pos layout; the expert's Wr
+// row comes in as wpre[c] for c < NPRE (loaded by the caller, possibly before
+// waiting on the producer of x) and from global memory beyond.
+template <int NT, int NPRE>
+__device__ __forceinline__ void canon_logits_warp_staged(const float* __restrict__ xs /* [NT][D] */, int nt, int D,
+                                                         const uint4 (&wpre)[NPRE], const uint16_t* __restrict__ Wr,
+                                                         const float* __restrict__ bias, int E, int e,
+                                                         float* __restrict__ lout /* + t*E */) {
+    const int lane = threadIdx.x & 31;
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
+    const int nc = D >> 8;
+    auto span = [&](const uint4& w, int c) {
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        float wf[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { wf[2 * q] = bf16lo(wv[q]); wf[2 * q + 1] = bf16hi(wv[q]); }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            if (t < nt) {
+                const float* xr = xs + (size_t)t * D + 256 * c + 4 * lane;
+                const float4 a = *reinterpret_cast<const float4*>(xr);
+                const float4 b = *reinterpret_cast<const float4*>(xr + 128);
+                acc[t] = __fmaf_rn(a.x, wf[0], acc[t]);
+                acc[t] = __fmaf_rn(a.y, wf[1], acc[t]);
+                acc[t] = __fmaf_rn(a.z, wf[2], acc[t]);
+                acc[t] = __fmaf_rn(a.w, wf[3], acc[t]);
+                acc[t] = __fmaf_rn(b.x, wf[4], acc[t]);
+                acc[t] = __fmaf_rn(b.y, wf[5], acc[t]);
+                acc[t] = __fmaf_rn(b.z, wf[6], acc[t]);
+                acc[t] = __fmaf_rn(b.w, wf[7], acc[t]);
+            }
+        }
+    };
+#pragma unroll
+    for (int c = 0; c < NPRE; ++c)
+        if (c < nc) span(wpre[c], c);
+    const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
+#pragma unroll 4
+    for (int c = NPRE; c < nc; ++c) span(ld_nc_u128(wrow + 256 * c), c);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+            acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
+    }
+    if (lane == 0) {
+        const float b = bias ? bias[e] : 0.0f;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            if (t < nt) lout[(size_t)t * E + e] = bias ? __fadd_rn(acc[t], b) : acc[t];
+    }
+}
+
 // Order-preserving map of a float to an unsigned key (larger float, larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -71,14 +136,22 @@ __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_
         const int e = lane + 32 * i;
         v[i] = (e < E) ? (SHARED ? lrow[e] : __ldcg(lrow + e)) : -INFINITY;
     }
-    // the lane's best: larger value, then lower id (= lower i for one lane)
+    // the lane's best: larger value, then lower id (= lower i for one lane),
+    // by a pairwise tree (depth log2 NV): each pair keeps its left member
+    // unless the right one is strictly larger, and the left member always
+    // covers the lower indices, so equal values resolve to the lowest index
     auto rescan = [&](float& bv, int& be) {
-        bv = v[0];
-        int bi = 0;
+        float tv[NV];
+        int ti[NV];
 #pragma unroll
-        for (int i = 1; i < NV; ++i)
-            if (v[i] > bv) { bv = v[i]; bi = i; }
-        be = (lane + 32 * bi < E) ? lane + 32 * bi : 0x7fffffff;
+        for (int i = 0; i < NV; ++i) { tv[i] = v[i]; ti[i] = i; }
+#pragma unroll
+        for (int st = 1; st < NV; st *= 2)
+#pragma unroll
+            for (int i = 0; i + st < NV; i += 2 * st)
+                if (tv[i + st] > tv[i]) { tv[i] = tv[i + st]; ti[i] = ti[i + st]; }
+        bv = tv[0];
+        be = (lane + 32 * ti[0] < E) ? lane + 32 * ti[0] : 0x7fffffff;
     };
     float bv;
     int be;
