@@ -15,32 +15,32 @@ namespace moe {
 // Decode route (T <= 4): one warp per expert computes its logits for all T
 // tokens, then the last block to finish selects every token's top-k.  The
 // block counter lives in ws and wraps back to zero on every completed launch.
-// Wr is not produced by the preceding kernel: each warp loads its expert's
-// row (up to kWrPre 256-element spans into registers, the rest prefetched into
-// L2) before waiting on the producer of x.  x is staged once per block as
-// fp32 in shared memory.
-constexpr int kWrPre = 12;
+// Wr is not produced by the preceding kernel: one bulk copy brings the block's
+// four expert rows into shared memory before waiting on the producer of x.
+// x is staged once per block as fp32 in shared memory.
 template <int NT>
 __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __restrict__ x, int T, int D,
                                                            const uint16_t* __restrict__ Wr,
                                                            const float* __restrict__ bias, int E, int k,
                                                            float* __restrict__ logits, int32_t* __restrict__ ids,
-                                                           float* __restrict__ gates, unsigned int* counter) {
-    extern __shared__ __align__(16) float xsf[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 4 + warp;
-    const int nc = D >> 8;
-    uint4 wpre[kWrPre];
-    if (e < E) {
-        const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
-#pragma unroll
-        for (int c = 0; c < kWrPre; ++c) wpre[c] = c < nc ? ld_nc_u128(wrow + 256 * c) : make_uint4(0, 0, 0, 0);
-        if (nc > kWrPre && lane == 0)
-            prefetch_l2(Wr + (size_t)e * D + 256 * kWrPre, (uint32_t)(D - 256 * kWrPre) * 2);
+                                                           float* __restrict__ gates, unsigned int* counter,
+                                                           uint32_t* err) {
+    extern __shared__ __align__(128) uint8_t rsm[];
+    float* xsf = reinterpret_cast<float*>(rsm);                                // [T][D], canon_stage_pos order
+    uint16_t* wsm = reinterpret_cast<uint16_t*>(rsm + (size_t)T * D * 4);      // the block's Wr rows [4][D]
+    __shared__ uint64_t wbar;
+    const int warp = threadIdx.x >> 5;
+    const int e0 = blockIdx.x * 4, e = e0 + warp;
+    if (threadIdx.x == 0) {
+        mbar_init(&wbar, 1);
+        fence_mbar_init();
+        const uint32_t bytes = (uint32_t)min(4, E - e0) * (uint32_t)D * 2u;
+        mbar_arrive_expect_tx(&wbar, bytes);
+        bulk_g2s(wsm, Wr + (size_t)e0 * D, bytes, &wbar);
     }
     pdl_wait();
     // stage x: every load of a batch is in flight before the first store
-    constexpr int kBatch = 8;
+    constexpr int kBatch = 16;
     const int n16 = T * D / 8;
     for (int i0 = 0; i0 < n16; i0 += kBatch * 128) {
         uint4 v[kBatch];
@@ -62,7 +62,8 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
     }
     __syncthreads();
     pdl_launch_dependents();
-    if (e < E) canon_logits_warp_staged<NT, kWrPre>(xsf, T, D, wpre, Wr, bias, E, e, logits);
+    const bool have_w = mbar_wait(&wbar, 0, err);
+    if (e < E && have_w) canon_logits_warp_staged<NT>(xsf, T, D, wsm + (size_t)warp * D, bias, E, e, logits);
     // the last block to arrive selects: one acq_rel ticket per block (release:
     // the block's logits, ordered before it by the barrier; acquire: every
     // other block's logits for the last one)
@@ -92,24 +93,25 @@ int route_num_sms() {
 moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, const float* bias, int E,
                         int k, int32_t* ids, float* gates, float* logits, void* ws, cudaStream_t s) {
     unsigned int* counter = reinterpret_cast<unsigned int*>(ws);
+    uint32_t* rerr = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
     float* lg = logits ? logits : reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256);
     cudaError_t e;
     if (T <= kDecodeMaxT) {
         const dim3 grid((E + 3) / 4), block(128);
-        const size_t smem = (size_t)T * D * sizeof(float);
+        const size_t smem = (size_t)T * D * sizeof(float) + (size_t)4 * D * sizeof(uint16_t);
         static bool attr = false;
         if (!attr) {
-            cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
+            cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
             attr = true;
         }
         switch (T) {
-            case 1: e = launch_pdl(route_decode_kernel<1>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter); break;
-            case 2: e = launch_pdl(route_decode_kernel<2>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter); break;
-            case 3: e = launch_pdl(route_decode_kernel<3>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter); break;
-            default: e = launch_pdl(route_decode_kernel<4>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter); break;
+            case 1: e = launch_pdl(route_decode_kernel<1>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            case 2: e = launch_pdl(route_decode_kernel<2>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            case 3: e = launch_pdl(route_decode_kernel<3>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            default: e = launch_pdl(route_decode_kernel<4>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
         }
         return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
