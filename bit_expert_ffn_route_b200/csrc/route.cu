@@ -16,7 +16,8 @@ namespace moe {
 // tokens, then the last block to finish selects every token's top-k.  The
 // block counter lives in ws and wraps back to zero on every completed launch.
 // Wr is not produced by the preceding kernel: one bulk copy brings the block's
-// four expert rows into shared memory before waiting on the producer of x.
+// four expert rows into shared memory, and each warp loads its expert's bias,
+// before waiting on the producer of x.
 // x is staged once per block as fp32 in shared memory.
 template <int NT>
 __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __restrict__ x, int T, int D,
@@ -38,6 +39,7 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
         mbar_arrive_expect_tx(&wbar, bytes);
         bulk_g2s(wsm, Wr + (size_t)e0 * D, bytes, &wbar);
     }
+    const float bias_e = (bias && e < E) ? __ldg(bias + e) : 0.0f;   // a weight too: load it now
     pdl_wait();
     // stage x: every load of a batch is in flight before the first store
     constexpr int kBatch = 16;
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
     __syncthreads();
     pdl_launch_dependents();
     const bool have_w = mbar_wait(&wbar, 0, err);
-    if (e < E && have_w) canon_logits_warp_staged<NT>(xsf, T, D, wsm + (size_t)warp * D, bias, E, e, logits);
+    if (e < E && have_w) canon_logits_warp_staged<NT>(xsf, T, D, wsm + (size_t)warp * D, bias != nullptr, bias_e, E, e, logits);
     // the last block to arrive selects: one acq_rel ticket per block (release:
     // the block's logits, ordered before it by the barrier; acquire: every
     // other block's logits for the last one)

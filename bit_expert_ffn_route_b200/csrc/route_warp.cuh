@@ -59,20 +59,21 @@ __device__ __forceinline__ int canon_stage_pos(int d) {
 }
 
 // canon_logits_warp for token rows staged in shared memory as fp32 (exact
-// copies of the bf16 values) in the canon_stage_pos layout; the expert's Wr
-// row comes in as wpre[c] for c < NPRE (loaded by the caller, possibly before
-// waiting on the producer of x) and from global memory beyond.
-template <int NT, int NPRE>
+// copies of the bf16 values) in the canon_stage_pos layout, with the expert's
+// Wr row in shared memory too, and the expert's bias (if any) in a register.
+template <int NT>
 __device__ __forceinline__ void canon_logits_warp_staged(const float* __restrict__ xs /* [NT][D] */, int nt, int D,
-                                                         const uint4 (&wpre)[NPRE], const uint16_t* __restrict__ Wr,
-                                                         const float* __restrict__ bias, int E, int e,
+                                                         const uint16_t* __restrict__ wrow_s, bool has_bias,
+                                                         float bias_e, int E, int e,
                                                          float* __restrict__ lout /* + t*E */) {
     const int lane = threadIdx.x & 31;
     float acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
     const int nc = D >> 8;
-    auto span = [&](const uint4& w, int c) {
+#pragma unroll 2
+    for (int c = 0; c < nc; ++c) {
+        const uint4 w = *reinterpret_cast<const uint4*>(wrow_s + 256 * c + 8 * lane);
         const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
         float wf[8];
 #pragma unroll
@@ -93,13 +94,7 @@ __device__ __forceinline__ void canon_logits_warp_staged(const float* __restrict
                 acc[t] = __fmaf_rn(b.w, wf[7], acc[t]);
             }
         }
-    };
-#pragma unroll
-    for (int c = 0; c < NPRE; ++c)
-        if (c < nc) span(wpre[c], c);
-    const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
-#pragma unroll 4
-    for (int c = NPRE; c < nc; ++c) span(ld_nc_u128(wrow + 256 * c), c);
+    }
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
 #pragma unroll
@@ -107,10 +102,9 @@ __device__ __forceinline__ void canon_logits_warp_staged(const float* __restrict
             acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
     }
     if (lane == 0) {
-        const float b = bias ? bias[e] : 0.0f;
 #pragma unroll
         for (int t = 0; t < NT; ++t)
-            if (t < nt) lout[(size_t)t * E + e] = bias ? __fadd_rn(acc[t], b) : acc[t];
+            if (t < nt) lout[(size_t)t * E + e] = has_bias ? __fadd_rn(acc[t], bias_e) : acc[t];
     }
 }
 
@@ -120,65 +114,106 @@ __device__ __forceinline__ uint32_t float_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Selection key of (logit, id): larger logit first, equal logits lower id
+// first, as one unsigned 64-bit order (-0.0 is taken as +0.0 before keying).
+__device__ __forceinline__ uint64_t sel_key(float v, int id) {
+    return ((uint64_t)float_key(v) << 32) | (uint64_t)(~(uint32_t)id);
+}
+__device__ __forceinline__ float key_value(uint64_t key) {
+    const uint32_t h = (uint32_t)(key >> 32);
+    return __uint_as_float((h & 0x80000000u) ? (h & 0x7fffffffu) : ~h);
+}
+__device__ __forceinline__ int key_id(uint64_t key) { return (int)(~(uint32_t)key); }
+
 // One warp selects the top-k of one token's E logits (E <= 32 * NV) and
-// writes ids and gates.  Each lane keeps its NV values and its best one; each
-// of the k rounds takes the warp's best (a warp max of the value keys, then
-// the lowest id among the lanes holding that key), and only the winning lane
-// removes it and rescans its values.  Gates are formed in double from the
-// selected fp32 logits.
+// writes ids and gates.  Each lane holds NV logits (ids lane + 32 i).
+// Fast path: the k-th largest of the 32 lane maxima is a threshold that at
+// least k logits reach, so the top-k lie among the logits at or above it;
+// when those candidates fit one per lane, each candidate's rank among them
+// is counted directly.  Otherwise k tournament rounds (warp max of the
+// lanes' best keys; the winning lane drops it and rescans).  Gates are formed
+// in double from the selected fp32 logits.
 template <int NV, bool SHARED = false>
 __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_t* __restrict__ ids,
                             float* __restrict__ gates) {
-    const int lane = threadIdx.x & 31;
-    float v[NV];
+    __shared__ uint64_t s_keys[8][32];   // per warp: lane maxima, then the candidates
+    __shared__ uint64_t s_sel[8][32];    // per warp: the selected keys by rank
+    const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) & 7;
+    uint64_t key[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? (SHARED ? lrow[e] : __ldcg(lrow + e)) : -INFINITY;
+        const float raw = (e < E) ? (SHARED ? lrow[e] : __ldcg(lrow + e)) : -INFINITY;
+        key[i] = sel_key(__fadd_rn(raw, 0.0f), e < E ? e : 0x7fffffff);
     }
-    // the lane's best: larger value, then lower id (= lower i for one lane),
-    // by a pairwise tree (depth log2 NV): each pair keeps its left member
-    // unless the right one is strictly larger, and the left member always
-    // covers the lower indices, so equal values resolve to the lowest index
-    auto rescan = [&](float& bv, int& be) {
-        float tv[NV];
-        int ti[NV];
+    // the lane's best key, by a pairwise tree
+    auto lane_best = [&]() {
+        uint64_t t[NV];
 #pragma unroll
-        for (int i = 0; i < NV; ++i) { tv[i] = v[i]; ti[i] = i; }
+        for (int i = 0; i < NV; ++i) t[i] = key[i];
 #pragma unroll
         for (int st = 1; st < NV; st *= 2)
 #pragma unroll
-            for (int i = 0; i + st < NV; i += 2 * st)
-                if (tv[i + st] > tv[i]) { tv[i] = tv[i + st]; ti[i] = ti[i + st]; }
-        bv = tv[0];
-        be = (lane + 32 * ti[0] < E) ? lane + 32 * ti[0] : 0x7fffffff;
+            for (int i = 0; i + st < NV; i += 2 * st) t[i] = t[i + st] > t[i] ? t[i + st] : t[i];
+        return t[0];
     };
-    float bv;
-    int be;
-    rescan(bv, be);
-    float my_v = 0.f, l0 = 0.f;
-    int my_e = 0;
-    for (int r = 0; r < k; ++r) {
-        const uint32_t mykey = float_key(bv);
-        const uint32_t wkey = __reduce_max_sync(0xffffffffu, mykey);
-        const int we = (int)__reduce_min_sync(0xffffffffu, mykey == wkey ? (uint32_t)be : 0xffffffffu);
-        const float wv = __shfl_sync(0xffffffffu, bv, we & 31);
-        if (r == 0) l0 = wv;
-        if (lane == r) { my_v = wv; my_e = we; }
-        if (be == we) {                         // this lane supplied the winner: remove it
-            const int wi = (we - lane) >> 5;
+    uint64_t best = lane_best();
+    s_keys[w][lane] = best;
+    __syncwarp();
+    int above = 0;                           // lane maxima larger than this lane's
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) above += s_keys[w][i] > best;
+    const uint32_t at_k = __ballot_sync(0xffffffffu, above == k - 1);   // keys are distinct: one lane
+    const uint64_t tau = __shfl_sync(0xffffffffu, best, __ffs(at_k) - 1);
+    int cnt = 0;
 #pragma unroll
-            for (int i = 0; i < NV; ++i)
-                if (i == wi) v[i] = -INFINITY;
-            rescan(bv, be);
+    for (int i = 0; i < NV; ++i) cnt += key[i] >= tau;
+    const int total = (int)__reduce_add_sync(0xffffffffu, (uint32_t)cnt);
+    uint64_t my = 0;
+    if (total <= 32) {
+        int pos = cnt;                       // inclusive scan of the counts
+#pragma unroll
+        for (int off = 1; off < 32; off *= 2) {
+            const int o = __shfl_up_sync(0xffffffffu, pos, off);
+            if (lane >= off) pos += o;
+        }
+        pos -= cnt;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+            if (key[i] >= tau) s_keys[w][pos++] = key[i];
+        __syncwarp();
+        if (lane < total) {
+            const uint64_t c = s_keys[w][lane];
+            int rank = 0;
+            for (int i = 0; i < total; ++i) rank += s_keys[w][i] > c;
+            if (rank < k) s_sel[w][rank] = c;
+        }
+        __syncwarp();
+        if (lane < k) my = s_sel[w][lane];
+        __syncwarp();
+    } else {
+        for (int r = 0; r < k; ++r) {
+            const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
+            const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
+            const uint64_t wk = ((uint64_t)hi << 32) | lo;
+            if (lane == r) my = wk;
+            if (best == wk) {                // this lane supplied the winner: drop it
+#pragma unroll
+                for (int i = 0; i < NV; ++i)
+                    if (key[i] == wk) key[i] = 0;
+                best = lane_best();
+            }
         }
     }
+    const float my_v = key_value(my);
+    const float l0 = __shfl_sync(0xffffffffu, my_v, 0);
     const double ex = (lane < k) ? exp((double)my_v - (double)l0) : 0.0;
     double z = ex;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     if (lane < k) {
-        ids[lane] = my_e;
+        ids[lane] = key_id(my);
         gates[lane] = (float)(ex / z);
     }
 }

@@ -35,6 +35,13 @@
  *  - T == 0 is valid and launches nothing (miss_count is still zeroed).
  *  - Path: T <= 4 is the decode path (1 token + up to 3 draft tokens);
  *    T > 4 is the prefill path.  Both compute the same function.
+ *  - Kernels are launched with programmatic dependent launch: each may start
+ *    while the previous kernel on the stream is finishing, and waits for it
+ *    before reading the activations, ids, gates or expert_out it may have
+ *    produced.  The layer's constants (Wr, bias, slot_table and the pool) may
+ *    be read before that wait, to overlap their fetch with the previous kernel:
+ *    they must not be written by the kernel launched immediately before the
+ *    call (any earlier kernel, copy or event in between is fine).
  */
 #ifndef MOE_H
 #define MOE_H
