@@ -224,6 +224,8 @@ struct Shared {
     int table[kMaxE];          // the slot table, staged before the dependency wait
     int n_owners;
     int abort[kTeams];         // set by a consumer team that stopped on an error
+    int d_range[2];            // this CTA's down items [d_range[0], d_range[1])
+    uint64_t range_bar;        // completes once d_range is written
     uint32_t team_items[kTeams];   // gate|up items finished by each team (release.cta by its leader)
 };
 
@@ -684,44 +686,89 @@ MOE_DEVINL void red_relaxed_add(uint32_t* p, uint32_t v) {
 }
 MOE_DEVINL void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
-// Down items are split into contiguous per-CTA ranges of equal estimated cost.
-// An item of n rows of an owner serving nt tokens costs n * (4 + 3 (nt - 1))
-// (a row served to four tokens measured about three times one served to one).
-struct DownCost {
-    int items;     // items of the owner
-    int cost;      // cost of one item
-};
-MOE_DEVINL DownCost down_cost(const Shared& sh, int u, int nrb, int rd) {
-    DownCost c;
-    const int nt = sh.owners[u].ntok;
-    c.items = u == 0 ? 2 * nrb : nrb;
-    c.cost = (u == 0 ? rd / 2 : rd) * (4 + 3 * (nt - 1));
-    return c;
+// Work is balanced by an estimated cost: an item of n weights of an owner
+// serving nt tokens costs n / 128 * (4 + 3 (nt - 1)) (a weight served to four
+// tokens measured about three times one served to one).  Gate|up items go
+// round-robin over the CTAs; each CTA then takes a contiguous range of down
+// items such that its gate|up and down costs together approach the average.
+MOE_DEVINL int cost_weight(const Shared& sh, int u) { return 4 + 3 * (sh.owners[u].ntok - 1); }
+MOE_DEVINL long long warp_sum_ll(long long v) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
 }
-// Index (in item_pos order) of the first down item whose cumulative cost
-// start is >= pos.
-MOE_DEVINL int down_item_at(const Shared& sh, long long pos, int nrb, int rd) {
-    long long base = 0;
-    int idx = 0;
-    for (int u = 0; u < sh.n_owners; ++u) {
-        const DownCost c = down_cost(sh, u, nrb, rd);
-        const long long end = base + (long long)c.items * c.cost;
-        if (end > pos) {
-            const long long m = pos <= base ? 0 : (pos - base + c.cost - 1) / c.cost;
-            return idx + (int)(m < c.items ? m : c.items);
+MOE_DEVINL long long warp_incl_scan_ll(long long v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off *= 2) {
+        const long long o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+    }
+    return v;
+}
+// One warp computes this CTA's down range [d0, d1) (item_pos order).  Owner u
+// has gate|up items from index nfb*(u+1) (owner 0: 0, with 2*nfb half items)
+// and down items from nrb*(u+1) (owner 0: 0, 2*nrb half items); gate|up item i
+// runs on CTA i mod G.  The cumulative down cost before CTA b is its share of
+// all work less the gate|up work of CTAs 0 .. b-1, clamped to [0, total down
+// cost]: any such sequence from 0 to the total covers every item (a decrease
+// only makes two neighbouring ranges overlap, and an overlapped item is
+// computed twice with identical results).
+MOE_DEVINL void down_range_warp(const Shared& sh, int b, int G, int nfb, int rf, int D, int nrb, int rd, int F,
+                                int& d0, int& d1) {
+    const int lane = threadIdx.x & 31, n = sh.n_owners;
+    auto below = [&](int m, int cb) {          // #{i < m : i mod G < cb}
+        const unsigned q = (unsigned)m / (unsigned)G, r = (unsigned)m % (unsigned)G;
+        return (long long)q * cb + (long long)(r < (unsigned)cb ? r : (unsigned)cb);
+    };
+    long long gu_all = 0, gu_b0 = 0, gu_b1 = 0, dn_part[2] = {0, 0};
+    int dcost[2] = {1, 1}, ditems[2] = {0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int u = lane + 32 * h;
+        if (u < n) {
+            const int w = cost_weight(sh, u);
+            const int gi = u == 0 ? 2 * nfb : nfb, gs = u == 0 ? 0 : nfb * (u + 1);
+            const long long gc = 2ll * (u == 0 ? rf / 2 : rf) * D / 128 * w;
+            gu_all += gc * gi;
+            gu_b0 += gc * (below(gs + gi, b) - below(gs, b));
+            gu_b1 += gc * (below(gs + gi, b + 1) - below(gs, b + 1));
+            ditems[h] = u == 0 ? 2 * nrb : nrb;
+            dcost[h] = (u == 0 ? rd / 2 : rd) * F / 128 * w;
+            dn_part[h] = (long long)dcost[h] * ditems[h];
         }
-        base = end;
-        idx += c.items;
     }
-    return idx;
-}
-MOE_DEVINL long long down_total_cost(const Shared& sh, int nrb, int rd) {
-    long long t = 0;
-    for (int u = 0; u < sh.n_owners; ++u) {
-        const DownCost c = down_cost(sh, u, nrb, rd);
-        t += (long long)c.items * c.cost;
-    }
-    return t;
+    gu_all = warp_sum_ll(gu_all);
+    gu_b0 = warp_sum_ll(gu_b0);
+    gu_b1 = warp_sum_ll(gu_b1);
+    // exclusive prefix of the down costs over owners 0 .. n-1
+    const long long in0 = warp_incl_scan_ll(dn_part[0]);
+    const long long tot0 = __shfl_sync(0xffffffffu, in0, 31);
+    const long long in1 = warp_incl_scan_ll(dn_part[1]) + tot0;
+    const long long dn_all = __shfl_sync(0xffffffffu, in1, 31);
+    const long long base[2] = {in0 - dn_part[0], in1 - dn_part[1]};
+    const long long all = gu_all + dn_all;
+    auto start = [&](int cb, long long gub) -> long long {
+        if (cb <= 0) return 0;
+        if (cb >= G) return dn_all;
+        const long long ds = (all * cb + G - 1) / G - gub;
+        return ds < 0 ? 0 : (ds > dn_all ? dn_all : ds);
+    };
+    auto item_at = [&](long long pos) -> int {
+        int idx = -1;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int u = lane + 32 * h;
+            if (u < n && pos >= base[h] && pos < base[h] + dn_part[h]) {
+                const int m = (int)((pos - base[h] + dcost[h] - 1) / dcost[h]);
+                idx = (u == 0 ? 0 : nrb * (u + 1)) + (m < ditems[h] ? m : ditems[h]);
+            }
+        }
+        const uint32_t hit = __ballot_sync(0xffffffffu, idx >= 0);
+        return hit ? __shfl_sync(0xffffffffu, idx, __ffs(hit) - 1) : (n == 0 ? 0 : nrb * (n + 1));
+    };
+    d0 = item_at(start(b, gu_b0));
+    d1 = item_at(start(b + 1, gu_b1));
 }
 
 MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
@@ -732,7 +779,7 @@ MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
 
 // ---------------------------------------------------------------- the fused kernel
 // One persistent CTA per SM.  Each CTA takes its gate|up items (round-robin),
-// then a contiguous range of down items (equal estimated cost per CTA),
+// then a contiguous range of down items (balancing the estimated cost of both),
 // through one ring of stages.  A down item of owner u waits until every
 // gate|up item of u has published its h: a per-owner item counter in ws,
 // advanced by a publisher warp that releases each finished item at gpu scope,
@@ -759,6 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     uint32_t* done = prm.done;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kTeamWarps); }
+        mbar_init(&sh.range_bar, 1);
         fence_mbar_init();
         for (int tm = 0; tm < kTeams; ++tm) { sh.abort[tm] = 0; sh.team_items[tm] = 0; }
     }
@@ -783,10 +831,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     // down items in contiguous ranges of equal cost (h is re-staged per owner)
     const int n_g = items_of(sh.n_owners, nfb);
     const int ng = n_g > (int)blockIdx.x ? (n_g - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    const long long dcost = down_total_cost(sh, nrb, rd);
-    const int d0r = down_item_at(sh, dcost * (long long)blockIdx.x / gridDim.x + (dcost * (long long)blockIdx.x % gridDim.x != 0), nrb, rd);
-    const int d1r = down_item_at(sh, dcost * (long long)(blockIdx.x + 1) / gridDim.x + (dcost * (long long)(blockIdx.x + 1) % gridDim.x != 0), nrb, rd);
-    if (warp == kPublisherWarp) {    // publisher: release finished gate|up items, in each team's order
+    // the down range is computed by the publisher warp, off the producer's path;
+    // the others wait for it only when they reach their first down item
+    int d0r = 0, d1r = 0;
+    bool have_range = false;
+    auto get_range = [&]() -> bool {
+        if (!have_range) {
+            if (!mbar_wait(&sh.range_bar, 0, prm.err)) return false;
+            d0r = sh.d_range[0];
+            d1r = sh.d_range[1];
+            have_range = true;
+        }
+        return true;
+    };
+    if (warp == kPublisherWarp) {    // publisher: the down range, then release finished gate|up items
+        {
+            int r0, r1;
+            down_range_warp(sh, (int)blockIdx.x, (int)gridDim.x, nfb, rf, D, nrb, rd, F, r0, r1);
+            if (lane == 0) {
+                sh.d_range[0] = r0;
+                sh.d_range[1] = r1;
+                mbar_arrive(&sh.range_bar);
+            }
+        }
         if (lane == 0) {
             uint32_t pub[kTeams] = {0u, 0u};
             const uint32_t want[kTeams] = {(uint32_t)((ng + 1) / 2), (uint32_t)(ng / 2)};
@@ -817,8 +884,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         }
     } else if (warp == kProducerWarp) {    // producer: gate|up items, then down items
         if (lane == 0) {
-            const int total = ng + (d1r - d0r);
-            for (int j = 0; j < total; ++j) {
+            for (int j = 0;; ++j) {
+                if (j >= ng && !get_range()) break;
+                if (j >= ng + (d1r - d0r)) break;
                 const int s = j % NS;
                 if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) break;
                 if (*reinterpret_cast<volatile int*>(&sh.abort[0]) | *reinterpret_cast<volatile int*>(&sh.abort[1])) break;
@@ -845,8 +913,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         bool ok = true;
         int cur = -1;
         uint32_t gu_done = 0;
-        const int total = ng + (d1r - d0r);
-        for (int j = team; j < total; j += kTeams) {
+        for (int j = team;; j += kTeams) {
+            if (j >= ng) {
+                ok = team_all(team, get_range());     // the same verdict on every thread of the team
+                if (!ok) break;
+                if (j >= ng + (d1r - d0r)) break;
+            }
             const int s = j % NS;
             const uint8_t* st = stages + (size_t)s * stage_bytes;
             if (j < ng) {
