@@ -6,49 +6,6 @@
 
 namespace moe {
 
-// Canonical logits of expert e for NT tokens whose bf16 rows are xrow[t]
-// (shared or global memory).  Lane L accumulates elements 256c + 8L + j.
-template <int NT>
-__device__ __forceinline__ void canon_logits_warp(const uint16_t* const (&xrow)[NT], int nt, int D,
-                                                  const uint16_t* __restrict__ Wr, const float* __restrict__ bias,
-                                                  int E, int e, float* __restrict__ lout /* + t*E */) {
-    const int lane = threadIdx.x & 31;
-    float acc[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
-    const uint16_t* wrow = Wr + (size_t)e * D + 8 * lane;
-    const int nc = D >> 8;
-#pragma unroll 6
-    for (int c = 0; c < nc; ++c) {
-        const uint4 w = ld_nc_u128(wrow + 256 * c);
-        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            if (t < nt) {
-                const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow[t] + 256 * c + 8 * lane);
-                const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {   // element j = 2q (low half), 2q+1 (high half)
-                    acc[t] = __fmaf_rn(bf16lo(xv[q]), bf16lo(wv[q]), acc[t]);
-                    acc[t] = __fmaf_rn(bf16hi(xv[q]), bf16hi(wv[q]), acc[t]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1)
-            acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
-    }
-    if (lane == 0) {
-        const float b = bias ? bias[e] : 0.0f;
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-            if (t < nt) lout[(size_t)t * E + e] = bias ? __fadd_rn(acc[t], b) : acc[t];
-    }
-}
-
 // Position of element d of a token row in the fp32 staging layout of the
 // decode router: within each 256-element span, elements j = 0..3 of lane L's
 // eight sit at 4L + j and elements j = 4..7 at 128 + 4L + (j - 4), so each of a
@@ -58,9 +15,11 @@ __device__ __forceinline__ int canon_stage_pos(int d) {
     return (c << 8) + ((j >> 2) << 7) + (L << 2) + (j & 3);
 }
 
-// canon_logits_warp for token rows staged in shared memory as fp32 (exact
-// copies of the bf16 values) in the canon_stage_pos layout, with the expert's
-// Wr row in shared memory too, and the expert's bias (if any) in a register.
+// Canonical logits of expert e for NT tokens: lane L accumulates elements
+// 256c + 8L + j (c ascending), then the xor butterfly, then + bias.  The token
+// rows are staged in shared memory as fp32 (exact copies of the bf16 values)
+// in the canon_stage_pos layout, the expert's Wr row is in shared memory too,
+// and its bias (if any) in a register.
 template <int NT>
 __device__ __forceinline__ void canon_logits_warp_staged(const float* __restrict__ xs /* [NT][D] */, int nt, int D,
                                                          const uint16_t* __restrict__ wrow_s, bool has_bias,
