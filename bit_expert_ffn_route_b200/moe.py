@@ -11,6 +11,7 @@ import ctypes
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 from . import synth
@@ -23,7 +24,7 @@ MOE_Q2_32, MOE_Q3_32, MOE_Q3_S256 = 0, 1, 2
 
 EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_size", "moe_workspace_size",
            "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
-           "moe_status_string", "moe_route_topk_static"]
+           "moe_status_string", "moe_route_topk_static", "moe_expert_hist", "moe_cache_plan", "moe_slot_fill"]
 
 
 class MoeError(RuntimeError):
@@ -69,6 +70,12 @@ def lib():
         L.moe_dequantize.argtypes = [ctypes.POINTER(moe_pool), i, i, P, P]
         L.moe_route_topk_static.restype = i
         L.moe_route_topk_static.argtypes = [P, i, i, P, P, i, i, P, P, P, P]
+        L.moe_expert_hist.restype = i
+        L.moe_expert_hist.argtypes = [P, i, i, i, P, P]
+        L.moe_cache_plan.restype = i
+        L.moe_cache_plan.argtypes = [P, i, P, P, i, ctypes.c_float, i, P, P]
+        L.moe_slot_fill.restype = i
+        L.moe_slot_fill.argtypes = [ctypes.POINTER(moe_pool), i, P, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [i]
         _lib = L
@@ -153,6 +160,41 @@ def moe_combine(expert_out, gates, T, D, k, out, miss_partial=None, residual=Non
 
 def moe_dequantize(pool: moe_pool, slot, matrix, out, stream=None):
     _check("moe_dequantize", lib().moe_dequantize(ctypes.byref(pool), slot, matrix, _p(out), _stream(stream)))
+
+
+def moe_expert_hist(ids, E, counts, stream=None):
+    """counts[e] += occurrences of e in ids (int32 [T][k], device); counts uint32 [E], device."""
+    T, k = ids.shape
+    _check("moe_expert_hist", lib().moe_expert_hist(_p(ids), T, k, E, _p(counts), _stream(stream)))
+
+
+def moe_cache_plan(score, slot_table, slots, hysteresis=1.0, max_moves=None):
+    """Host plan of admissions/evictions.  score float32 [E], slot_table int32 [E],
+    slots int32 [n] (numpy).  Returns (moves int32 [n_moves][3] as (slot, evict,
+    admit), new_slot_table int32 [E])."""
+    score = np.ascontiguousarray(score, np.float32)
+    table = np.ascontiguousarray(slot_table, np.int32)
+    slots = np.ascontiguousarray(slots, np.int32)
+    E = score.shape[0]
+    if table.shape != (E,):
+        raise ValueError("slot_table must have E entries")
+    m = len(slots) if max_moves is None else int(max_moves)
+    moves = np.zeros((max(m, 1), 3), np.int32)
+    new_table = np.empty(E, np.int32)
+    n = lib().moe_cache_plan(score.ctypes.data, E, table.ctypes.data, slots.ctypes.data if len(slots) else None,
+                             len(slots), float(hysteresis), m, moves.ctypes.data, new_table.ctypes.data)
+    if n < 0:
+        raise MoeError("moe_cache_plan", n)
+    return moves[:n].copy(), new_table
+
+
+def moe_slot_fill(pool: moe_pool, slot, host_codes, host_scales, stream=None):
+    """Copy one expert's packed weights (host uint8 tensors, pinned for overlap) into a pool slot."""
+    for t in (host_codes, host_scales):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host_codes / host_scales must be contiguous host tensors")
+    _check("moe_slot_fill", lib().moe_slot_fill(ctypes.byref(pool), int(slot), ctypes.c_void_p(host_codes.data_ptr()),
+                                                ctypes.c_void_p(host_scales.data_ptr()), _stream(stream)))
 
 
 class Layer:

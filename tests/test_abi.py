@@ -1,4 +1,4 @@
-"""The C-ABI library loads and exports every symbol include/moe.h declares;
+"""The C-ABI library loads and exports every symbol include/*.h declares;
 size queries and argument checks behave as documented (no GPU needed: these
 calls return before touching the device)."""
 import ctypes
@@ -20,9 +20,13 @@ def L():
 
 
 def declared_functions():
-    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
-    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", txt)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", txt))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
