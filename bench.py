@@ -121,6 +121,16 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(value: float, ws: int, device) -> float:
+    """The largest of every rank's value (each rank calls it at the same point;
+    with one rank, the value itself)."""
+    if ws <= 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _graph_of(fn, n_steps, stream):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -219,10 +229,7 @@ def run_ours(args, ws_, rank, local):
         torch.distributed.barrier()
     ms = t0.elapsed_time(t1)
     fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(G)]
-    if ws_ > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, ws_, dev)
     ms_per_step = ms / K
     value = ws_ * T * K / (ms / 1e3)
     hbm, tf, tf_sus, peak_kind = _peaks()
@@ -274,10 +281,7 @@ def run_ours(args, ws_, rank, local):
         e1.record(stream)
     torch.cuda.synchronize()
     ems = e0.elapsed_time(e1)
-    if ws_ > 1:
-        tt = torch.tensor([ems], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ems = float(tt.item())
+    ems = max_over_ranks(ems, ws_, dev)
     e2e_value = ws_ * T * Ke / (ems / 1e3)
 
     line = {
