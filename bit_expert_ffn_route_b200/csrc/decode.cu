@@ -53,34 +53,9 @@ constexpr int kSmemBudget = 220 * 1024;
 // Q2_32: code j of a 32-bit word sits at bits [2j, 2j+2).  Shifting the word by
 // 21, 11, 1 or -9 places codes {0}, {1..5}, {6..10}, {11..15} at mantissa bits 13..21.
 MOE_DEVINL int q2_pos(int j) { return j == 0 ? 21 : (j <= 5 ? 2 * j + 11 : (j <= 10 ? 2 * j + 1 : 2 * j - 9)); }
-MOE_DEVINL float q2_code(const uint32_t* w, int i) {
-    const uint32_t word = w[i >> 4];
-    const int j = i & 15;
-    const uint32_t src = j == 0 ? (word << 21) : (j <= 5 ? (word << 11) : (j <= 10 ? (word << 1) : (word >> 9)));
-    const int p = q2_pos(j);
-    return __uint_as_float((src & (3u << p)) | 0x3f800000u);
-}
 // Q3 (32 codes in 3 words, code i at stream bits [3i, 3i+3)): groups of three
 // codes are moved to bits 14..22, so code i sits at bit 14 + 3*(i % 3).
 MOE_DEVINL int q3_pos(int i) { return 14 + 3 * (i % 3); }
-MOE_DEVINL float q3_code(const uint32_t* w, int i) {
-    uint32_t src;
-    switch (i / 3) {
-        case 0: src = w[0] << 14; break;
-        case 1: src = w[0] << 5; break;
-        case 2: src = w[0] >> 4; break;
-        case 3: src = __funnelshift_r(w[0], w[1], 13); break;
-        case 4: src = w[1] << 10; break;
-        case 5: src = w[1] << 1; break;
-        case 6: src = w[1] >> 8; break;
-        case 7: src = __funnelshift_r(w[1], w[2], 17); break;
-        case 8: src = w[2] << 6; break;
-        case 9: src = w[2] >> 3; break;
-        default: src = w[2] >> 12; break;
-    }
-    const int p = q3_pos(i);
-    return __uint_as_float((src & (7u << p)) | 0x3f800000u);
-}
 // Compile-time loop: f(std::integral_constant<int, I>) for I in [B, E).
 template <int B, int E, typename Fn>
 MOE_DEVINL void static_for(Fn&& fn) {
