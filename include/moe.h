@@ -136,7 +136,8 @@ size_t moe_expert_out_size(int T, int D, int k);
  *          (reading: softmax restricted to the selected experts; sums to 1)
  *   logits fp32 [T][E] out, or NULL.  Decode path: the canonical-order
  *          values below.  Prefill path: tensor-core values within the bound
- *          |l - canonical| <= 2^-18 * D * |x_t|_2 * |Wr_e|_2.
+ *          |l - canonical| <= 2^-12 * |x_t|_2 * |Wr_e|_2 (D <= 8192); the ids
+ *          and gates always come from the canonical values.
  *   ws     device scratch of moe_route_workspace_size bytes, 256-byte
  *          aligned.  Its first 4 bytes must be zero before the first call
  *          with this buffer (e.g. zero it once at allocation); every completed
