@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "once.cuh"
 #include "sync.cuh"
 
 namespace moe {
@@ -1021,11 +1022,12 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
                ((size_t)Geo<FMT>::d_row(K) * n) % 16 == 0;
     };
     if (!ok16(D, rf) || !ok16(D, rf / 2) || !ok16(F, rd) || !ok16(F, rd / 2)) return MOE_ERR_UNSUPPORTED;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaFuncSetAttribute(decode_ffn_kernel<FMT, NTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
-        attr_done = true;
-    }
+    static std::atomic<uint64_t> attr_done{0};
+    if (!once_per_device(attr_done, [] {
+            return cudaFuncSetAttribute(decode_ffn_kernel<FMT, NTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kSmemBudget) == cudaSuccess;
+        }))
+        return MOE_ERR_CUDA;
     cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NTMAX>, dim3(num_sms()), dim3(kThreads), smem, s, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

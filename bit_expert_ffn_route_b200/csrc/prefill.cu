@@ -38,6 +38,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "once.cuh"
 #include "sync.cuh"
 
 namespace moe {
@@ -970,13 +971,12 @@ moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, u
         !row_map(&r32, src, (uint64_t)Kg, src_rows, 32) || !row_map(&r16, src, (uint64_t)Kg, src_rows, 16))
         return MOE_ERR_CUDA;
     const size_t smem = kGemmSmem + 1024;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(expert_gemm_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (!once_per_device(attr, [&] {
+            return cudaFuncSetAttribute(expert_gemm_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)smem) == cudaSuccess;
+        }))
+        return MOE_ERR_CUDA;
     const int grid = max_tiles < gemm_num_sms() ? (max_tiles > 0 ? max_tiles : 1) : gemm_num_sms();
     const cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms,
                                      r128, r64, r32, r16, prm);

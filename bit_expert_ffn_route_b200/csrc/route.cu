@@ -7,6 +7,7 @@
 // then + bias) is what makes the selected ids reproducible bit for bit.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "once.cuh"
 #include "route_warp.cuh"
 #include "sync.cuh"
 
@@ -101,14 +102,15 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
     if (T <= kDecodeMaxT) {
         const dim3 grid((E + 3) / 4), block(128);
         const size_t smem = (size_t)T * D * sizeof(float) + (size_t)4 * D * sizeof(uint16_t);
-        static bool attr = false;
-        if (!attr) {
-            cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
-            cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 192 * 1024);
-            attr = true;
-        }
+        static std::atomic<uint64_t> attr{0};
+        if (!once_per_device(attr, [] {
+                const int b = 192 * 1024;
+                return cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess;
+            }))
+            return MOE_ERR_CUDA;
         switch (T) {
             case 1: e = launch_pdl(route_decode_kernel<1>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
             case 2: e = launch_pdl(route_decode_kernel<2>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;

@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "once.cuh"
 #include "route_warp.cuh"
 #include "sync.cuh"
 
@@ -307,12 +308,12 @@ moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t*
     CUtensorMap mx, mw;
     if (!bf16_rows_map(&mx, x, D, T) || !bf16_rows_map(&mw, Wr, D, E)) return MOE_ERR_CUDA;
     const size_t smem = kRStages * kRStageBytes + 1024;
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (!once_per_device(attr, [&] {
+            return cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
+                   cudaSuccess;
+        }))
+        return MOE_ERR_CUDA;
     cudaError_t e = launch_pdl(wnorm_kernel, dim3((E + 7) / 8), dim3(256), 0, s, Wr, D, E, wnorm);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_pdl(router_tc_kernel, dim3((E + kRN - 1) / kRN, (T + kRM - 1) / kRM), dim3(kRThreads), smem, s, mx, mw,
