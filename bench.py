@@ -20,6 +20,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -70,7 +71,10 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # raw samples: a scratch file (the summary goes into the JSON line);
+        # MOE_BENCH_CLOCKS_DIR keeps them somewhere else
+        out_dir = os.environ.get("MOE_BENCH_CLOCKS_DIR", tempfile.gettempdir())
+        self.path = os.path.join(out_dir, f"moe_bench_clocks_rank{index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
