@@ -114,3 +114,21 @@ def test_combine_and_dequant_argument_errors(L):
     assert L.moe_combine(None, None, 0, 3072, 10, None, None, None, None) == moe.MOE_OK
     assert L.moe_dequantize(ctypes.byref(_pool()), 4, 0, f, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_dequantize(ctypes.byref(_pool()), 0, 3, f, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_cache_call_argument_errors(L):
+    f = _fake()
+    # popularity count: shape / pointer errors, and T == 0 launches nothing
+    assert L.moe_expert_hist(f, 4, 0, 512, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_hist(f, 4, 10, 0, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_hist(None, 4, 10, 512, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_hist(f, 4, 10, 512, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_hist(None, 0, 10, 512, None, None) == moe.MOE_OK
+    # slot fill: bad pool, slot or host pointers are refused before any copy
+    fill = lambda pool, slot=0, hc=f, hs=f: L.moe_slot_fill(ctypes.byref(pool), slot, hc, hs, None)
+    assert fill(_pool(fmt=5)) == moe.MOE_ERR_INVALID_ARG
+    assert fill(_pool(), slot=4) == moe.MOE_ERR_INVALID_ARG
+    assert fill(_pool(), slot=-1) == moe.MOE_ERR_INVALID_ARG
+    assert fill(_pool(), hc=None) == moe.MOE_ERR_INVALID_ARG
+    assert fill(_pool(stride_c=256)) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_slot_fill(None, 0, f, f, None) == moe.MOE_ERR_INVALID_ARG
