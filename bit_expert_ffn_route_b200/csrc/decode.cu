@@ -692,16 +692,20 @@ MOE_DEVINL long long warp_incl_scan_ll(long long v) {
 // computed twice with identical results).
 MOE_DEVINL void down_range_warp(const Shared& sh, int b, int G, int nfb, int rf, int D, int nrb, int rd, int F,
                                 int& d0, int& d1) {
+    constexpr int H = (kMaxPairs + 31) / 32;   // owners per lane: u = lane + 32 h
     const int lane = threadIdx.x & 31, n = sh.n_owners;
     auto below = [&](int m, int cb) {          // #{i < m : i mod G < cb}
         const unsigned q = (unsigned)m / (unsigned)G, r = (unsigned)m % (unsigned)G;
         return (long long)q * cb + (long long)(r < (unsigned)cb ? r : (unsigned)cb);
     };
-    long long gu_all = 0, gu_b0 = 0, gu_b1 = 0, dn_part[2] = {0, 0};
-    int dcost[2] = {1, 1}, ditems[2] = {0, 0};
+    long long gu_all = 0, gu_b0 = 0, gu_b1 = 0, dn_part[H];
+    int dcost[H], ditems[H];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < H; ++h) {
         const int u = lane + 32 * h;
+        dn_part[h] = 0;
+        dcost[h] = 1;
+        ditems[h] = 0;
         if (u < n) {
             const int w = cost_weight(sh, u);
             const int gi = u == 0 ? 2 * nfb : nfb, gs = u == 0 ? 0 : nfb * (u + 1);
@@ -717,12 +721,15 @@ MOE_DEVINL void down_range_warp(const Shared& sh, int b, int G, int nfb, int rf,
     gu_all = warp_sum_ll(gu_all);
     gu_b0 = warp_sum_ll(gu_b0);
     gu_b1 = warp_sum_ll(gu_b1);
-    // exclusive prefix of the down costs over owners 0 .. n-1
-    const long long in0 = warp_incl_scan_ll(dn_part[0]);
-    const long long tot0 = __shfl_sync(0xffffffffu, in0, 31);
-    const long long in1 = warp_incl_scan_ll(dn_part[1]) + tot0;
-    const long long dn_all = __shfl_sync(0xffffffffu, in1, 31);
-    const long long base[2] = {in0 - dn_part[0], in1 - dn_part[1]};
+    // exclusive prefix of the down costs over owners 0 .. n-1, 32 owners a pass
+    long long base[H], carry = 0;
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        const long long in = warp_incl_scan_ll(dn_part[h]) + carry;
+        base[h] = in - dn_part[h];
+        carry = __shfl_sync(0xffffffffu, in, 31);
+    }
+    const long long dn_all = carry;
     const long long all = gu_all + dn_all;
     auto start = [&](int cb, long long gub) -> long long {
         if (cb <= 0) return 0;
@@ -733,7 +740,7 @@ MOE_DEVINL void down_range_warp(const Shared& sh, int b, int G, int nfb, int rf,
     auto item_at = [&](long long pos) -> int {
         int idx = -1;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < H; ++h) {
             const int u = lane + 32 * h;
             if (u < n && pos >= base[h] && pos < base[h] + dn_part[h]) {
                 const int m = (int)((pos - base[h] + dcost[h] - 1) / dcost[h]);

@@ -168,3 +168,24 @@ def test_decode48_chain_per_layer():
     hit_rate = hits / (48 * cfg.k)
     print(f"decode48: hit rate {hit_rate:.3f}, worst rel L2 {worst:.2e}")
     assert 0.85 < hit_rate <= 1.0
+
+
+def test_decode_65_owners():
+    """T = 4, k = 16, every selected expert distinct and resident: the shared
+    expert plus 64 routed owners, the most the decode path serves."""
+    cfg = configs.Config("edge65", 1, 256, 128, 128, 16, 4, synth.Q2_32, None, None, None, seed=3)
+    wl = configs.build(cfg, device="cuda")
+    L = wl.layers[0]
+    # token t prefers experts 16t .. 16t+15 (strictly decreasing logits, no ties)
+    Wr = torch.zeros(cfg.E, cfg.D, dtype=torch.float32)
+    for t in range(cfg.T):
+        for j in range(16):
+            Wr[16 * t + j, t] = 1.0 - j / 64.0
+    L.Wr = Wr.to(torch.bfloat16).cuda()
+    x = torch.zeros(cfg.T, cfg.D, dtype=torch.float32)
+    for t in range(cfg.T):
+        x[t, t] = 4.0
+    x[:, cfg.T:] = 0.01 * torch.randn(cfg.T, cfg.D - cfg.T, generator=torch.Generator().manual_seed(5))
+    x = x.to(torch.bfloat16).cuda()
+    layer, ref, err = _check_layer(wl, x, k=16)
+    assert len(np.unique(ref.ids)) == 64 and int(layer.miss_count.item()) == 0
