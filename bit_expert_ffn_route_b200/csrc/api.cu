@@ -7,6 +7,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "moe.h"
+#include "sync.cuh"
 
 using namespace moe;
 
@@ -89,6 +90,7 @@ const char* moe_status_string(moe_status s) {
         case MOE_ERR_WORKSPACE: return "workspace too small";
         case MOE_ERR_CUDA: return "CUDA error";
         case MOE_ERR_TIMEOUT: return "device wait timed out";
+        case MOE_ERR_RANGE: return "activation outside the fp16 range";
     }
     return "unknown status";
 }
@@ -146,6 +148,26 @@ moe_status moe_dequantize(const moe_pool* pool, int slot, int matrix, float* out
     if (st != MOE_OK) return st;
     if (slot < 0 || slot >= v.n_slots || matrix < 0 || matrix > 2 || !out) return MOE_ERR_INVALID_ARG;
     return launch_dequantize(v, slot, matrix, out, (cudaStream_t)stream);
+}
+
+moe_status moe_workspace_status(const void* ws, moe_stream_t stream) {
+    if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&word, static_cast<const char*>(ws) + 4, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (word & kErrTimeout) return MOE_ERR_TIMEOUT;
+    if (word & kErrRange) return MOE_ERR_RANGE;
+    return MOE_OK;
+}
+
+moe_status moe_debug_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t limit_us, void* ws,
+                               moe_stream_t stream) {
+    if (!flag || !ws || !aligned(flag, 4) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    if (limit_us == 0 || limit_us > 1000000u) return MOE_ERR_INVALID_ARG;
+    return launch_wait_flag(flag, expect, limit_us, reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 4),
+                            (cudaStream_t)stream);
 }
 
 }  // extern "C"

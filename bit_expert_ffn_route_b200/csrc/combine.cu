@@ -1,5 +1,4 @@
-// combine.cu — gate-weighted combine of the expert outputs (and the test-only
-// dequantiser).
+// combine.cu — gate-weighted combine of the expert outputs.
 //
 //   out[t] = bf16( sum_{r<k, hit} g[t,r] * y[t,r] + y_shared[t] (+ miss_partial[t]) (+ residual[t]) )
 //
@@ -123,49 +122,6 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const int32_t* __rest
     *reinterpret_cast<uint4*>(out + (size_t)t * D + d) = o;
 }
 
-// Test hook: one thread per block of one row; exact fp32 weights.
-__global__ void dequant_kernel(PoolView P, int slot, int mat, float* __restrict__ out) {
-    const int rows = (mat == 2) ? P.D : P.F;
-    const int K = (mat == 2) ? P.F : P.D;
-    const int bw = (P.fmt == MOE_Q3_S256) ? 256 : 32;
-    const int nbk = K / bw;
-    const size_t blocks = (size_t)P.D * P.F / bw;
-    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= rows * nbk) return;
-    const int row = idx / nbk, b = idx % nbk;
-    const uint8_t* codes = P.codes + (size_t)slot * P.stride_c;
-    const uint8_t* meta = P.scales + (size_t)slot * P.stride_s;
-    float* o = out + (size_t)row * K + (size_t)b * bw;
-    if (P.fmt == MOE_Q3_S256) {
-        const uint8_t* c = codes + ((size_t)mat * blocks + (size_t)row * nbk + b) * 96;
-        const uint8_t* sc = meta + ((size_t)mat * blocks + (size_t)row * nbk + b) * 12;
-        const uint16_t dbits = *reinterpret_cast<const uint16_t*>(meta + 3 * blocks * 12 +
-                                                                 ((size_t)mat * blocks + (size_t)row * nbk + b) * 2);
-        const float d = f16_bits_to_f32(dbits);
-        for (int i = 0; i < 256; ++i) {
-            const int bit = 3 * i;
-            const uint32_t two = (uint32_t)c[bit >> 3] | ((uint32_t)((bit >> 3) + 1 < 96 ? c[(bit >> 3) + 1] : 0) << 8);
-            const int q = (two >> (bit & 7)) & 7;
-            const int sbit = 6 * (i >> 4);
-            const uint32_t stwo = (uint32_t)sc[sbit >> 3] | ((uint32_t)((sbit >> 3) + 1 < 12 ? sc[(sbit >> 3) + 1] : 0) << 8);
-            const int s6 = (stwo >> (sbit & 7)) & 63;
-            o[i] = d * (float)((s6 - 32) * (q - 4));   // integer product first: exact, +0.0 for q == 4
-        }
-    } else {
-        const int nbits = (P.fmt == MOE_Q2_32) ? 2 : 3;
-        const int cb = (P.fmt == MOE_Q2_32) ? 8 : 12;
-        const uint8_t* c = codes + ((size_t)mat * blocks + (size_t)row * nbk + b) * cb;
-        const uint32_t sm = *reinterpret_cast<const uint32_t*>(meta + ((size_t)mat * blocks + (size_t)row * nbk + b) * 4);
-        const float s = f16_bits_to_f32(sm & 0xffffu), m = f16_bits_to_f32(sm >> 16);
-        for (int j = 0; j < 32; ++j) {
-            const int bit = nbits * j;
-            const uint32_t two = (uint32_t)c[bit >> 3] | ((uint32_t)((bit >> 3) + 1 < cb ? c[(bit >> 3) + 1] : 0) << 8);
-            const int q = (two >> (bit & 7)) & ((1 << nbits) - 1);
-            o[j] = __fmaf_rn(s, (float)q, m);
-        }
-    }
-}
-
 }  // namespace
 
 moe_status launch_combine(const void* expert_out, const float* gates, int T, int D, int k,
@@ -181,15 +137,6 @@ moe_status launch_combine(const void* expert_out, const float* gates, int T, int
                        reinterpret_cast<const uint16_t*>(rows), gates, T, D, k, miss_partial, residual, out);
     }
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
-}
-
-moe_status launch_dequantize(const PoolView& P, int slot, int matrix, float* out, cudaStream_t s) {
-    const int rows = (matrix == 2) ? P.D : P.F;
-    const int K = (matrix == 2) ? P.F : P.D;
-    const int bw = (P.fmt == MOE_Q3_S256) ? 256 : 32;
-    const int n = rows * (K / bw);
-    dequant_kernel<<<(n + 127) / 128, 128, 0, s>>>(P, slot, matrix, out);
-    return last_launch_status();
 }
 
 }  // namespace moe

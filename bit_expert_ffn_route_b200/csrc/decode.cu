@@ -796,6 +796,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     stage_table(prm, sh);
     __syncthreads();
     pdl_wait();                      // ids come from the router
+    // a call on a workspace whose timeout bit is set does no work (every CTA
+    // still takes its ticket below, so the counters are left zero); one read,
+    // shared by the whole CTA, so that every warp takes the same branch
+    __shared__ int dead;
+    if (threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
+    __syncthreads();
+    if (!dead) {
     // warp 0 resolves the owners and releases the producer and publisher
     // (barrier 1) while the other consumers stage x; the consumers meet at
     // barrier 4 before computing
@@ -854,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                     pub[0] = c0;
                     pub[1] = c1;
                 } else {
-                    if (*reinterpret_cast<volatile uint32_t*>(prm.err) ||
+                    if (timed_out(prm.err) ||
                         *reinterpret_cast<volatile int*>(&sh.abort[0]) || *reinterpret_cast<volatile int*>(&sh.abort[1]))
                         break;
                     if (globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -940,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                         const uint32_t target = (uint32_t)(u == 0 ? 2 * nfb : nfb);   // items of owner u
                         const uint64_t t0 = globaltimer_ns();
                         while (ld_acquire(done + u) < target) {
-                            if (*reinterpret_cast<volatile uint32_t*>(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
+                            if (timed_out(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
                                 atomicOr(prm.err, kErrTimeout);
                                 waited = false;
                                 break;
@@ -976,6 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         }
         if (!ok && tl == 0) sh.abort[team] = 1;
     }
+    }   // !dead
     // last CTA out resets the per-owner counters for the next call
     // (acq_rel ticket: this CTA's counter updates, ordered before it by the
     // barrier, precede the reset; the last CTA sees every other CTA's)
@@ -988,17 +996,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
             done[kMaxPairs] = 0u;
         }
     }
-}
-
-int num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
 }
 
 template <int FMT, int NTMAX>
@@ -1035,7 +1032,7 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
                                         kSmemBudget) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
-    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NTMAX>, dim3(num_sms()), dim3(kThreads), smem, s, prm);
+    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NTMAX>, dim3(device_sm_count()), dim3(kThreads), smem, s, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -48,5 +48,6 @@ moe_status launch_combine(const void* expert_out, const float* gates, int T, int
                           const float* miss_partial, const uint16_t* residual, uint16_t* out, cudaStream_t s);
 
 moe_status launch_dequantize(const PoolView& P, int slot, int matrix, float* out, cudaStream_t s);
+moe_status launch_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t limit_us, uint32_t* err, cudaStream_t s);
 
 }  // namespace moe

@@ -26,4 +26,24 @@ bool once_per_device(std::atomic<uint64_t>& done, Fn&& fn) {
     return true;
 }
 
+// SM count of the current device, looked up once per device (148 if the
+// query fails).
+inline int device_sm_count() {
+    static std::atomic<int> counts[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    auto query = [dev] {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        return n;
+    };
+    if (dev < 0 || dev >= 64) return query();
+    int n = counts[dev].load(std::memory_order_relaxed);
+    if (!n) {
+        n = query();
+        counts[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
 }  // namespace moe

@@ -44,8 +44,6 @@
 namespace moe {
 namespace {
 
-constexpr uint32_t kErrRange = 2u;     // error word: an activation outside the fp16 range
-
 constexpr int kChunk = 256;            // tokens per plan chunk
 constexpr int kMaxE = 1024;
 constexpr int kTileM = 128;            // weight rows per tile (MMA M)
@@ -395,14 +393,6 @@ MOE_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, 
         "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
 }
-// Bounded wait that does not give up early on the error word: used to drain
-// copies and MMAs still in flight before the CTA exits.
-MOE_DEVINL void mbar_drain(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
-
 // AND of `v` over the epilogue warps (named barrier 1): they leave their loop
 // together, so none is left waiting at a named barrier.
 MOE_DEVINL bool epilogue_all(bool v, int nthreads_const_128) {
@@ -608,7 +598,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     pdl_wait();
     const int n_tiles = __ldg(g.n_tiles);
-    const bool dead = *reinterpret_cast<volatile uint32_t*>(g.err) != 0;   // an earlier kernel gave up
+    __shared__ int dead_s;                      // an earlier kernel gave up: one read for the CTA
+    if (threadIdx.x == 0) dead_s = timed_out(g.err) ? 1 : 0;
+    __syncthreads();
+    const bool dead = dead_s != 0;
     const int first = blockIdx.x, step = gridDim.x;
 
     if (!dead && warp < kDqWarps) {
@@ -913,17 +906,6 @@ bool byte_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int gemm_num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 // The row operand: fp16 [rows][K] with boxes of 64 x box_rows, 128B swizzle.
 bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
     EncodeTiledFn fn = encode_tiled();
@@ -977,7 +959,7 @@ moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, u
                                         (int)smem) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
-    const int grid = max_tiles < gemm_num_sms() ? (max_tiles > 0 ? max_tiles : 1) : gemm_num_sms();
+    const int grid = max_tiles < device_sm_count() ? (max_tiles > 0 ? max_tiles : 1) : device_sm_count();
     const cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms,
                                      r128, r64, r32, r16, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
     __syncthreads();
     pdl_launch_dependents();
     const bool have_w = mbar_wait(&wbar, 0, err);
+    if (!have_w && threadIdx.x == 0) mbar_drain(&wbar, 0);   // the copy lands before the CTA moves on
     if (e < E && have_w) canon_logits_warp_staged<NT>(xsf, T, D, wsm + (size_t)warp * D, bias != nullptr, bias_e, E, e, logits);
     // the last block to arrive selects: one acq_rel ticket per block (release:
     // the block's logits, ordered before it by the barrier; acquire: every
@@ -79,18 +80,11 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
     }
     __syncthreads();
     if (!last) return;
-    if (warp < T) topk_warp(logits + (size_t)warp * E, E, k, ids + (size_t)warp * k, gates + (size_t)warp * k);
-}
-
-int route_num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    if (timed_out(err)) {            // some block gave up: no selection from incomplete logits
+        for (int i = threadIdx.x; i < T * k; i += blockDim.x) { ids[i] = -1; gates[i] = 0.f; }
+        return;
     }
-    return n;
+    if (warp < T) topk_warp(logits + (size_t)warp * E, E, k, ids + (size_t)warp * k, gates + (size_t)warp * k);
 }
 
 moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, const float* bias, int E,
@@ -119,7 +113,6 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
         }
         return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
-    (void)route_num_sms;
     // prefill: tensor-core logits, then canonical logits of each token's candidates
     float* wnorm = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256 +
                                             ((size_t)T * E * sizeof(float) + 255) / 256 * 256);
@@ -139,7 +132,7 @@ size_t route_workspace_bytes(int T, int D, int E, int k) {
 
 // ---------------------------------------------------------------- no-allocation entry point
 // Scratch for moe_route_topk_static: a 256-byte header (word 0 = the block
-// counter of the last-block top-k) followed by room for the logits of up to
+// counter of the last-block top-k, word 1 = the device error word) followed by room for the logits of up to
 // kStaticMaxT tokens x kStaticMaxE experts.  Every GPU that loads this library
 // holds it until the process exits.
 namespace {
@@ -171,8 +164,9 @@ extern "C" moe_status moe_route_topk_static(const uint16_t* x, int T, int D, con
     }
     void* ws = g_scratch_ptr[dev];
     cudaStream_t s = (cudaStream_t)stream;
-    // the counter must start at zero (a call that did not complete may have left it set)
-    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ERR_CUDA;
+    // the block counter and the device error word start at zero on every call
+    // (a call that did not complete may have left either set)
+    if (cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
     return moe::launch_route(x, T, D, Wr, bias, E, k, ids, gates, logits, ws, s);
 }
 

@@ -51,11 +51,6 @@ MOE_DEVINL void r_tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uin
         "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
 }
-MOE_DEVINL void r_drain(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
 
 // Logits of a 128-token x 128-expert tile: TMA streams x and Wr tiles, one
 // thread issues tcgen05 MMAs into a TMEM accumulator, four warps add the bias
@@ -99,7 +94,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 issued = j + 1;
             }
             for (int j = issued - kRStages; j < issued; ++j)
-                if (j >= 0) r_drain(&full[j % kRStages], (j / kRStages) & 1);
+                if (j >= 0) mbar_drain(&full[j % kRStages], (j / kRStages) & 1);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -127,7 +122,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                                  smem_u32(&done))
                              : "memory");
-            r_drain(&done, 0);
+            mbar_drain(&done, 0);
         }
         __syncwarp();
     } else {
@@ -201,12 +196,17 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
                                                                        const float* __restrict__ bias, int E, int k,
                                                                        const float* __restrict__ approx,
                                                                        const float* __restrict__ wn,
-                                                                       int32_t* __restrict__ ids, float* __restrict__ gates) {
+                                                                       int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                                       const uint32_t* err) {
     extern __shared__ float rows[];          // [kSelWarps][E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kSelWarps + warp;
     pdl_wait();
     if (t >= T) return;
+    if (timed_out(err)) {            // the logits kernel gave up: no selection from incomplete logits
+        if (lane < k) { ids[(size_t)t * k + lane] = -1; gates[(size_t)t * k + lane] = 0.f; }
+        return;
+    }
     float* row = rows + (size_t)warp * E;
     const float* ar = approx + (size_t)t * E;
     const uint16_t* xr = x + (size_t)t * D;
@@ -321,7 +321,7 @@ moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t*
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const size_t sel_smem = (size_t)kSelWarps * E * sizeof(float);
     e = launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), sel_smem, s, x,
-                   T, D, Wr, bias, E, k, (const float*)logits, (const float*)wnorm, ids, gates);
+                   T, D, Wr, bias, E, k, (const float*)logits, (const float*)wnorm, ids, gates, (const uint32_t*)err);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

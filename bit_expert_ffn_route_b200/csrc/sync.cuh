@@ -10,8 +10,14 @@
 
 namespace moe {
 
-// Device error word values (written into the workspace; 0 = ok).
+// Device error word bits (word 1 of a workspace; 0 = ok).
+//   kErrTimeout: a bounded wait gave up; the call's outputs are not valid, and
+//                every later call on the same workspace gives up at its first
+//                wait until the word is cleared.
+//   kErrRange  : a prefill activation (x or h) outside the fp16 range; the rows
+//                of those tokens are not valid, the others are.
 constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrRange = 2u;
 // Bounded waits give up after this long (far above any legitimate wait).
 constexpr uint64_t kWaitLimitNs = 500ull * 1000 * 1000;
 constexpr uint32_t kMaxPolls = 1u << 24;
@@ -46,20 +52,32 @@ MOE_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false, and sets *err, if the phase does not complete
-// within kWaitLimitNs; returns false at once if another CTA already set *err.
+MOE_DEVINL bool timed_out(const uint32_t* err) {
+    return err && (*reinterpret_cast<const volatile uint32_t*>(err) & kErrTimeout);
+}
+// Bounded wait: returns false, and sets the timeout bit of *err, if the phase
+// does not complete within kWaitLimitNs; returns false as soon as it finds the
+// timeout bit already set (another CTA or an earlier kernel gave up).
 MOE_DEVINL bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (err && *reinterpret_cast<volatile uint32_t*>(err)) return false;
+        if (timed_out(err)) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             if (err) atomicOr(err, kErrTimeout);
             return false;
         }
     }
+}
+
+// Bounded wait that does not give up early on the error word: used to let
+// copies and MMAs still in flight land before the CTA exits.
+MOE_DEVINL void mbar_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return;
 }
 
 // Bulk copy global -> shared, completing `bytes` of transaction on `bar`.

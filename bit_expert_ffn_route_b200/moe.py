@@ -19,12 +19,14 @@ from . import synth
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_RANGE = \
+    0, -1, -2, -3, -4, -5, -6
 MOE_Q2_32, MOE_Q3_32, MOE_Q3_S256 = 0, 1, 2
 
 EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_size", "moe_workspace_size",
            "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
-           "moe_status_string", "moe_route_topk_static", "moe_expert_hist", "moe_cache_plan", "moe_slot_fill"]
+           "moe_status_string", "moe_route_topk_static", "moe_expert_hist", "moe_cache_plan", "moe_slot_fill",
+           "moe_workspace_status", "moe_debug_wait_flag"]
 
 
 class MoeError(RuntimeError):
@@ -76,6 +78,10 @@ def lib():
         L.moe_cache_plan.argtypes = [P, i, P, P, i, ctypes.c_float, i, P, P]
         L.moe_slot_fill.restype = i
         L.moe_slot_fill.argtypes = [ctypes.POINTER(moe_pool), i, P, P, P]
+        L.moe_workspace_status.restype = i
+        L.moe_workspace_status.argtypes = [P, P]
+        L.moe_debug_wait_flag.restype = i
+        L.moe_debug_wait_flag.argtypes = [P, ctypes.c_uint32, ctypes.c_uint32, P, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [i]
         _lib = L
@@ -156,6 +162,17 @@ def moe_combine(expert_out, gates, T, D, k, out, miss_partial=None, residual=Non
     st = lib().moe_combine(_p(expert_out), _p(gates), T, D, k, _p(miss_partial), _p(residual), _p(out),
                            _stream(stream))
     _check("moe_combine", st)
+
+
+def moe_workspace_status(ws, stream=None) -> int:
+    """The device error word of a workspace as a status code (synchronises the stream)."""
+    return int(lib().moe_workspace_status(_p(ws), _stream(stream)))
+
+
+def moe_debug_wait_flag(flag, expect, limit_us, ws, stream=None):
+    """Test hook: a bounded device wait for flag[0] == expect (flag: int32/uint32 device tensor)."""
+    _check("moe_debug_wait_flag", lib().moe_debug_wait_flag(_p(flag), int(expect), int(limit_us), _p(ws),
+                                                            _stream(stream)))
 
 
 def moe_dequantize(pool: moe_pool, slot, matrix, out, stream=None):

@@ -25,7 +25,8 @@
  *  - Pointers named x, Wr, ids, gates, logits, slot_table, expert_out,
  *    miss_list, miss_count, miss_partial, residual, out, ws and the pool's
  *    codes/scales are DEVICE pointers; the caller allocates and owns them.
- *    The library never allocates, frees or synchronises.
+ *    The library never allocates or frees, and synchronises only in
+ *    moe_workspace_status.
  *  - bf16 and fp16 values are passed as uint16_t bit patterns.
  *  - Calls are asynchronous on `stream` (NULL = legacy default stream).
  *    Argument and shape errors are returned synchronously and launch nothing;
@@ -62,7 +63,8 @@ typedef enum moe_status {
     MOE_ERR_UNSUPPORTED = -2,   /* shape outside the limits below */
     MOE_ERR_WORKSPACE = -3,     /* ws / expert_out smaller than the size query */
     MOE_ERR_CUDA = -4,          /* a CUDA call or launch failed */
-    MOE_ERR_TIMEOUT = -5        /* a bounded device-side wait gave up */
+    MOE_ERR_TIMEOUT = -5,       /* a bounded device-side wait gave up (moe_workspace_status) */
+    MOE_ERR_RANGE = -6          /* a prefill activation outside the fp16 range (moe_workspace_status) */
 } moe_status;
 
 /*
@@ -139,10 +141,14 @@ size_t moe_expert_out_size(int T, int D, int k);
  *          |l - canonical| <= 2^-12 * |x_t|_2 * |Wr_e|_2 (D <= 8192); the ids
  *          and gates always come from the canonical values.
  *   ws     device scratch of moe_route_workspace_size bytes, 256-byte
- *          aligned.  Its first 4 bytes must be zero before the first call
+ *          aligned.  Its first 8 bytes must be zero before the first call
  *          with this buffer (e.g. zero it once at allocation); every completed
  *          call leaves them zero.  Calls sharing one ws must not overlap on
- *          the device.
+ *          the device.  Bytes 4..7 are the device error word: if a bounded
+ *          device wait gave up (bit 0, MOE_ERR_TIMEOUT from
+ *          moe_workspace_status), that call writes ids = -1 and gates = 0 for
+ *          every token, and every later call on the same ws does the same
+ *          until the caller zeroes the 8 bytes again.
  * The selection and the gates use logits in a canonical fp32 order: 32
  * partial sums, lane L accumulating fmaf over elements 256c + 8L + j (c
  * ascending, j = 0..7), then added pairwise (L with L+16, then +8, +4, +2,
@@ -155,8 +161,8 @@ moe_status moe_route_topk(const uint16_t* x, int T, int D, const uint16_t* Wr,
 /*
  * moe_route_topk without a workspace argument, for callers that cannot
  * allocate device memory themselves: code running under a host framework that
- * owns all device memory through a fixed, pre-sized arena, or code that must
- * not call cudaMalloc on its path (e.g. while a CUDA stream is being captured).
+ * owns all device memory through a fixed, pre-sized arena and hands out no
+ * scratch, or code that must not call cudaMalloc on its path.
  * The pages describe no such call; it is an addition of this library.
  *   Same arguments and results as moe_route_topk (decode path only).
  *   Scratch: a library-owned static device array of 16,640 bytes per GPU, held
@@ -164,9 +170,11 @@ moe_status moe_route_topk(const uint16_t* x, int T, int D, const uint16_t* Wr,
  *   MOE_ERR_UNSUPPORTED.  Nothing is allocated or freed.
  *   The first call on a device looks up the array's device address (once per
  *   device, with that device current); make that first call before any stream
- *   capture.  Every call resets the array's counter with an async memset on
- *   `stream`.  All calls on a device share the array: calls that overlap on the
- *   GPU (different streams) race and must be serialised by the caller.
+ *   capture.  Every call clears the array's block counter and device error
+ *   word (8 bytes) with an async memset on `stream`; a call whose bounded
+ *   device wait gave up writes ids = -1 and gates = 0.  All calls on a device
+ *   share the array, which keeps the last call's logits: calls that overlap
+ *   on the GPU (different streams) race and must be serialised by the caller.
  */
 moe_status moe_route_topk_static(const uint16_t* x, int T, int D, const uint16_t* Wr,
                                  const float* bias, int E, int k, int32_t* ids, float* gates,
@@ -191,11 +199,26 @@ moe_status moe_route_topk_static(const uint16_t* x, int T, int D, const uint16_t
  *          zero before the first call with this buffer (zero it once at
  *          allocation); every completed call leaves them zero.  Calls sharing
  *          one ws must not overlap on the device.  Word 1 (bytes 4..7) is the
- *          device error word: nonzero after a bounded device-side wait gave up
- *          (then re-zero the first 1024 bytes before reuse).
+ *          device error word, read with moe_workspace_status:
+ *            bit 0 (MOE_ERR_TIMEOUT): a bounded device wait gave up; the
+ *              call's outputs are not valid, and every later call on this ws
+ *              does no work until the caller zeroes its first 1024 bytes;
+ *            bit 1 (MOE_ERR_RANGE, prefill path only): some x or h value has
+ *              magnitude >= 65520, which the fp16 tensor-core operands cannot
+ *              hold; the output rows of those tokens are not valid, the other
+ *              rows are, and later calls are not affected (the bit stays set
+ *              until the caller clears it).
  * Per expert (reading; the pages do not give the FFN form):
  *   h = bf16( silu(Wg x) * (Wu x) ),  y = Wd h,  fp32 accumulation.
  * Missed experts are not computed.
+ * Operand precision.  Decode path (T <= 4): the inner products consume the
+ * codes directly, s * sum(q x) + m * sum(x) in fp32, without forming weights.
+ * Prefill path (T > 4): the tensor cores take fp16 operands.  Each weight is
+ * formed in fp16 arithmetic: Q2_32/Q3_32 fp16(s*q + m) (one rounding);
+ * Q3_S256 fp16( fp16(d*(sc-32)) * (q-4) ) (two roundings); x and h (bf16
+ * values) convert to fp16 exactly when their magnitude is below 65520.
+ * Outputs of both paths are within the relative L2 bound of 1e-2 per token of
+ * the exact-weight result.
  */
 moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, int E,
                               const uint16_t* x, int T, const int32_t* ids, int k,
@@ -225,6 +248,24 @@ moe_status moe_combine(const void* expert_out, const float* gates, int T, int D,
  */
 moe_status moe_dequantize(const moe_pool* pool, int slot, int matrix, float* out,
                           moe_stream_t stream);
+
+/*
+ * Device error word of a workspace (moe_route_topk's or moe_expert_forward's
+ * ws): MOE_OK, MOE_ERR_TIMEOUT (bit 0) or MOE_ERR_RANGE (bit 1).  Unlike every
+ * other call, this one synchronises `stream` (it waits for the work queued
+ * on it) to read the word.
+ */
+moe_status moe_workspace_status(const void* ws, moe_stream_t stream);
+
+/*
+ * Test hook for the device error word: one device thread polls *flag (device
+ * memory) until it equals `expect` or limit_us microseconds (1..1,000,000)
+ * have passed; on the limit it sets bit 0 of ws's error word, as a bounded
+ * wait of the expert pass does.  Returns at once on the device if that bit is
+ * already set.
+ */
+moe_status moe_debug_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t limit_us, void* ws,
+                               moe_stream_t stream);
 
 /* Static text for a status code. */
 const char* moe_status_string(moe_status s);

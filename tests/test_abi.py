@@ -54,7 +54,7 @@ def test_size_queries(L):
 
 
 def test_status_strings(L):
-    for s in (0, -1, -2, -3, -4, -5):
+    for s in (0, -1, -2, -3, -4, -5, -6):
         assert L.moe_status_string(s)
 
 
@@ -132,3 +132,13 @@ def test_cache_call_argument_errors(L):
     assert fill(_pool(), hc=None) == moe.MOE_ERR_INVALID_ARG
     assert fill(_pool(stride_c=256)) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_slot_fill(None, 0, f, f, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_status_query_and_wait_hook_argument_errors(L):
+    f = _fake()
+    assert L.moe_workspace_status(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_status(_fake((1 << 20) + 16), None) == moe.MOE_ERR_INVALID_ARG   # not 256-aligned
+    assert L.moe_debug_wait_flag(None, 1, 1000, f, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_debug_wait_flag(f, 1, 1000, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_debug_wait_flag(f, 1, 0, f, None) == moe.MOE_ERR_INVALID_ARG             # no limit
+    assert L.moe_debug_wait_flag(f, 1, 2000000, f, None) == moe.MOE_ERR_INVALID_ARG       # above 1 s

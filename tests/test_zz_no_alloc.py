@@ -7,12 +7,15 @@ static device array instead of a caller-provided workspace.
 The test calls it through the C ABI twice in a row and checks each result
 against the workspace-taking moe_route_topk on the same inputs: expert ids and
 logits identical, gates within the 1e-6 relative tolerance the other GPU tests
-use.  It also checks that sizes beyond the static array are refused."""
+use.  It also checks ragged shapes against the CPU oracle directly, and that
+sizes beyond the static array are refused."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from bit_expert_ffn_route_b200 import configs, moe, synth
+from tests.harness import u16
 
 pytestmark = pytest.mark.gpu
 
@@ -55,3 +58,23 @@ def test_static_router_refuses_sizes_beyond_its_array():
     with pytest.raises(moe.MoeError) as e:
         moe.moe_route_topk_static(x[:4], Wr2, None, 10, ids[:4], gates[:4])
     assert e.value.status == moe.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 18, 4), (3, 18, 4), (2, 1024, 16)])
+def test_static_router_ragged_shapes_match_oracle(T, E, k):
+    D = 256
+    x = synth.hidden(T, D, seed=11, stream=T, device="cuda")
+    Wr = synth.router_weight(E, D, seed=11, layer=E, device="cuda")
+    bias = synth.zipf_bias(E, 1.1, 0.5, seed=11).cuda()
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gates = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    for call in range(2):
+        moe.moe_route_topk_static(x, Wr, bias, k, ids, gates, logits=logits)
+        torch.cuda.synchronize()
+        want_l = oracle.router_logits(u16(x), u16(Wr), bias.cpu().numpy())
+        want_ids, want_g = oracle.topk_gates(want_l, k)
+        assert np.array_equal(logits.cpu().numpy().view(np.uint32), want_l.view(np.uint32)), call
+        assert np.array_equal(ids.cpu().numpy(), want_ids), call
+        g = gates.double().cpu().numpy()
+        assert np.all(np.abs(g - want_g) <= TOL_GATE * np.abs(want_g)), call
