@@ -47,9 +47,9 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 EXTRA = ["prefill", "decode48", "prefill48"]
-# kernels per layer and step: decode route 1, expert pass 1, combine 1; prefill
-# route 3 (norms, tensor-core logits, selection), expert pass 6 (3 plan,
-# gather, 2 GEMMs), combine 1
+# kernels per layer and step: decode (T <= 4) route 1, expert pass 1, combine 1;
+# prefill route 3 (norms, tensor-core logits, selection), expert pass 6 (3
+# plan, gather, 2 GEMMs), combine 1
 LAUNCHES = {"decode": 3, "prefill": 10}
 
 
@@ -329,6 +329,42 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     return res
 
 
+# ---------------------------------------------------------------- small verify batches
+def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 16, 64), K=64):
+    """The decode layer's shapes at other batch sizes (MTP draft verification):
+    per-step time and tokens/s of the three calls, and which expert-pass path
+    ran (decode: T <= 8, tensor-core GEMV; prefill: T > 8, grouped GEMMs)."""
+    cfg = configs.CONFIGS["decode"]
+    wl = configs.build(cfg, device=dev, T=max(Ts))
+    L0 = wl.layers[0]
+    R = 8
+    pools = [wl.pool] + [synth.PoolData(wl.pool.fmt, cfg.D, cfg.F, wl.pool.n_slots, wl.pool.codes.clone(),
+                                        wl.pool.scales.clone(), wl.pool.stride_codes, wl.pool.stride_scales)
+                         for _ in range(R - 1)]
+    stream = torch.cuda.Stream(device=dev)
+    out = {}
+    for T in Ts:
+        layers = [moe.Layer(pools[r], L0.shared_slot, L0.slot_table, L0.Wr, L0.bias, cfg.k, T, device=dev)
+                  for r in range(R)]
+        xs = [synth.hidden(T, cfg.D, cfg.seed, stream=600 + r, device=dev) for r in range(R)]
+
+        def step(i):
+            layers[i % R](xs[i % R], stream=stream)
+
+        G = _divisor_at_most(K, 64)
+        graph = _graph_of(step, G, stream)
+        with torch.cuda.stream(stream):
+            graph.replay()
+        ms, _ = _timed_replays(graph, K // G, stream, ws_, dev, local, clocks=False)
+        out[str(T)] = {"ms_per_step": round(ms / K, 5), "tokens_per_s": round(ws_ * T * K / (ms / 1e3), 1),
+                       "expert_pass": "decode" if T <= 8 else "prefill",
+                       "router": "canonical CUDA-core" if T <= 4 else "tensor-core + canonical recheck"}
+        del layers, xs, graph
+    del pools, wl
+    return {"workload": "decode layer shapes (D=3072, F=512, E=512, top-10+1, Q2_32, 320/512 resident), "
+                        "T tokens per step, 8 rotating pool replicas", "by_T": out}
+
+
 # ---------------------------------------------------------------- 48-layer chains
 class ChainBuffers:
     """One set of buffers shared by every layer of a chain (the calls of a step
@@ -561,6 +597,9 @@ def run_ours(args, ws_, rank, local):
             line[name] = fn(name, k_, max(w_, 1), ws_, dev, local, args, cpu)
             gc.collect()
             torch.cuda.empty_cache()
+        line["small_batches"] = bench_small_batches(ws_, dev, local, args)
+        gc.collect()
+        torch.cuda.empty_cache()
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -50,6 +50,13 @@ moe_status check_pool(const moe_pool* pool, PoolView& v) {
     return MOE_OK;
 }
 
+// A failed launch also leaves its (non-sticky) error as the runtime's last
+// error; the status reports it, so clear it for the caller's next CUDA call.
+moe_status reported(moe_status st) {
+    if (st == MOE_ERR_CUDA) (void)cudaGetLastError();
+    return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -105,7 +112,7 @@ moe_status moe_route_topk(const uint16_t* x, int T, int D, const uint16_t* Wr, c
     if (!aligned(x, 16) || !aligned(Wr, 16) || !aligned(ws, 256) || (logits && !aligned(logits, 16)))
         return MOE_ERR_INVALID_ARG;
     if (ws_bytes < route_workspace_bytes(T, D, E, k)) return MOE_ERR_WORKSPACE;
-    return launch_route(x, T, D, Wr, bias, E, k, ids, gates, logits, ws, (cudaStream_t)stream);
+    return reported(launch_route(x, T, D, Wr, bias, E, k, ids, gates, logits, ws, (cudaStream_t)stream));
 }
 
 moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, int E, const uint16_t* x, int T,
@@ -124,10 +131,10 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
     if (expert_out_bytes_ < expert_out_bytes(T, v.D, k)) return MOE_ERR_WORKSPACE;
     if (ws_bytes < moe_workspace_size(T, v.D, v.F, E, k, v.fmt)) return MOE_ERR_WORKSPACE;
     if (T <= kDecodeMaxT)
-        return launch_decode_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
-                                     (cudaStream_t)stream);
-    return launch_prefill_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
-                                  (cudaStream_t)stream);
+        return reported(launch_decode_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
+                                              (cudaStream_t)stream));
+    return reported(launch_prefill_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
+                                           (cudaStream_t)stream));
 }
 
 moe_status moe_combine(const void* expert_out, const float* gates, int T, int D, int k, const float* miss_partial,
@@ -139,7 +146,7 @@ moe_status moe_combine(const void* expert_out, const float* gates, int T, int D,
     if (!aligned(expert_out, 256) || !aligned(out, 16) || (residual && !aligned(residual, 16)) ||
         (miss_partial && !aligned(miss_partial, 16)))
         return MOE_ERR_INVALID_ARG;
-    return launch_combine(expert_out, gates, T, D, k, miss_partial, residual, out, (cudaStream_t)stream);
+    return reported(launch_combine(expert_out, gates, T, D, k, miss_partial, residual, out, (cudaStream_t)stream));
 }
 
 moe_status moe_dequantize(const moe_pool* pool, int slot, int matrix, float* out, moe_stream_t stream) {
@@ -147,7 +154,7 @@ moe_status moe_dequantize(const moe_pool* pool, int slot, int matrix, float* out
     moe_status st = check_pool(pool, v);
     if (st != MOE_OK) return st;
     if (slot < 0 || slot >= v.n_slots || matrix < 0 || matrix > 2 || !out) return MOE_ERR_INVALID_ARG;
-    return launch_dequantize(v, slot, matrix, out, (cudaStream_t)stream);
+    return reported(launch_dequantize(v, slot, matrix, out, (cudaStream_t)stream));
 }
 
 moe_status moe_workspace_status(const void* ws, moe_stream_t stream) {
@@ -166,8 +173,25 @@ moe_status moe_debug_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t l
                                moe_stream_t stream) {
     if (!flag || !ws || !aligned(flag, 4) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
     if (limit_us == 0 || limit_us > 1000000u) return MOE_ERR_INVALID_ARG;
-    return launch_wait_flag(flag, expect, limit_us, reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 4),
-                            (cudaStream_t)stream);
+    return reported(launch_wait_flag(flag, expect, limit_us, reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 4),
+                                     (cudaStream_t)stream));
+}
+
+size_t moe_debug_operand_workspace_size(int d_model, int d_ff) {
+    if (d_model <= 0 || d_ff <= 0) return 0;
+    return prefill_operand_dump_ws_bytes(d_model, d_ff);
+}
+
+moe_status moe_debug_prefill_operand(const moe_pool* pool, int gemm, int slot, int m0, uint32_t* dump, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream) {
+    PoolView v;
+    moe_status st = check_pool(pool, v);
+    if (st != MOE_OK) return st;
+    if (gemm != 1 && gemm != 2) return MOE_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= v.n_slots || !dump || !ws || !aligned(ws, 256) || !aligned(dump, 4)) return MOE_ERR_INVALID_ARG;
+    if (m0 < 0 || (gemm == 1 ? (m0 % 64 || m0 >= v.F) : (m0 % 128 || m0 >= v.D))) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < prefill_operand_dump_ws_bytes(v.D, v.F)) return MOE_ERR_WORKSPACE;
+    return reported(launch_prefill_operand_dump(v, gemm, slot, m0, dump, ws, (cudaStream_t)stream));
 }
 
 }  // extern "C"

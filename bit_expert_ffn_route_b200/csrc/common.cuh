@@ -12,7 +12,13 @@
 namespace moe {
 
 constexpr int kMaxTopK = 16;
-constexpr int kDecodeMaxT = 4;   // T <= 4: decode path
+constexpr int kDecodeMaxT = 8;        // T <= 8: decode expert pass (tensor-core GEMV over bulk-copied codes)
+// The router computes logits on CUDA cores in the canonical order for T <= 8
+// tokens when x (fp32) and four rows of Wr fit in its shared memory
+// ((4 T + 8) D bytes <= kRouteDecodeSmem); otherwise on the tensor cores, with
+// each token's candidates recomputed in the canonical order.
+constexpr int kRouteDecodeMaxT = 8;
+constexpr size_t kRouteDecodeSmem = 192 * 1024;
 
 MOE_DEVINL float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 MOE_DEVINL float bf16lo(uint32_t packed) { return __uint_as_float(packed << 16); }

@@ -1,4 +1,4 @@
-// decode.cu — expert pass for 1-4 tokens (one token plus MTP drafts):
+// decode.cu — expert pass for 1-8 tokens (one token plus MTP drafts):
 // expert-cache slot lookup with a miss list, then a grouped dequant-GEMV that
 // streams the packed codes of every selected resident expert from HBM once.
 //
@@ -19,18 +19,29 @@
 // (TMA), completing on mbarriers; sixteen consumer warps compute from shared
 // memory.  Programmatic dependent launch overlaps its prologue with the router.
 //
-// Inner product without dequantising each weight: for a block with scale s
-// and min m, sum_j (s q_j + m) x_j = s * sum_j q_j x_j + m * sum_j x_j.  Each
-// code, left at mantissa bit p_j of its word, is OR-ed into 1.0f (one logic op
-// per code, one shared constant): f_j = 1 + q_j 2^(p_j - 23), exactly.  The
-// staged activations are pre-scaled, x'_j = x_j 2^(23 - p_j) (exact), so that
-// sum_j x'_j f_j = sum_j x'_j + sum_j q_j x_j, the first sum being a per-block
-// constant of the token computed once.
+// Arithmetic: warp-level tensor-core MMAs (mma.sync m16n8k16, fp16 operands,
+// fp32 accumulation).  A = 16 weight rows x 16 K, dequantised in registers to
+// fp16 (dequant.cuh: each weight the exact weight rounded once to fp16);
+// B = 16 K x 8 token columns holding the (up to eight) tokens; columns past T
+// are zero.  Every owner is evaluated for all tokens of
+// the batch (the tensor cores have the columns to spare) and only the outputs
+// of the tokens that selected it are kept, so the cost per weight does not
+// depend on how many tokens share an expert.
+//
+// K order.  Within every 128-K unit U of a row, lane c of a lane quad handles
+// the 32-weight block 4U + c; step (i, j) (i = half of the block, j = 0..3)
+// gives its A registers the weight pairs (j, j + 8) and (j + 4, j + 12) of
+// half i, which one word of codes yields without moving bits (dequant.cuh).
+// The MMA's K index 2c + e (e = 0, 1) of step (i, j) is weight
+// 128U + 32c + 16i + j + 8e, and 2c + 8 + e is 128U + 32c + 16i + j + 4 + 8e.
+// Activations (x, and h for the down projection) are stored in fp16 in that
+// order ("fragment order"), so a lane's B registers are one 8-byte load.
 #include <cuda_fp16.h>
 
 #include <type_traits>
 
 #include "common.cuh"
+#include "dequant.cuh"
 #include "kernels.cuh"
 #include "once.cuh"
 #include "sync.cuh"
@@ -40,101 +51,29 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kTeams = 2;                        // consumer teams, alternating items
+constexpr int kTeams = 2;                          // consumer teams, alternating items
 constexpr int kTeamWarps = kConsumerWarps / kTeams;
-constexpr int kProducerWarp = kConsumerWarps;    // bulk copies into the stage ring
+constexpr int kProducerWarp = kConsumerWarps;      // bulk copies into the stage ring
 constexpr int kPublisherWarp = kConsumerWarps + 1; // releases finished gate|up items to other CTAs
 constexpr int kThreads = kConsumers + 64;
-constexpr int kXStride = 36;                     // floats per 32-weight chunk: 32 x + 4 constants
+constexpr int kUnitK = 128;
 constexpr int kMaxPairs = kDecodeMaxT * kMaxTopK + 1;
 constexpr int kMaxStages = 8;
-constexpr int kSmemBudget = 220 * 1024;
-
-// ---------------------------------------------------------------- code decode
-// Q2_32: code j of a 32-bit word sits at bits [2j, 2j+2).  Shifting the word by
-// 21, 11, 1 or -9 places codes {0}, {1..5}, {6..10}, {11..15} at mantissa bits 13..21.
-MOE_DEVINL int q2_pos(int j) { return j == 0 ? 21 : (j <= 5 ? 2 * j + 11 : (j <= 10 ? 2 * j + 1 : 2 * j - 9)); }
-// Q3 (32 codes in 3 words, code i at stream bits [3i, 3i+3)): groups of three
-// codes are moved to bits 14..22, so code i sits at bit 14 + 3*(i % 3).
-MOE_DEVINL int q3_pos(int i) { return 14 + 3 * (i % 3); }
-// Compile-time loop: f(std::integral_constant<int, I>) for I in [B, E).
-template <int B, int E, typename Fn>
-MOE_DEVINL void static_for(Fn&& fn) {
-    if constexpr (B < E) {
-        fn(std::integral_constant<int, B>{});
-        static_for<B + 1, E>(fn);
-    }
-}
-
-// 1.0f as a register operand the compiler cannot fold: `(src & mask) | one`
-// must stay one 3-input logic op (lop3 encodes a single immediate, so two
-// immediates would cost two logic ops per code on the half-rate ALU pipe).
-MOE_DEVINL uint32_t opaque_one() {
-    uint32_t v;
-    asm volatile("mov.b32 %0, 0x3f800000;" : "=r"(v));
-    return v;
-}
-template <uint32_t MASK>
-MOE_DEVINL float and_or(uint32_t src, uint32_t one) {
-    uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(src), "n"(MASK), "r"(one));   // (a & b) | c
-    return __uint_as_float(r);
-}
-
-// Code I of a chunk as 1 + q 2^(p-23), with I a compile-time constant so that
-// the shift and mask are immediates.
-template <int FMT, int I>
-MOE_DEVINL float code_c(const uint32_t* w, uint32_t one) {
-    if constexpr (FMT == MOE_Q2_32) {
-        constexpr int j = I & 15;
-        constexpr int sh = j == 0 ? 21 : (j <= 5 ? 11 : (j <= 10 ? 1 : -9));
-        constexpr int p = j == 0 ? 21 : (j <= 5 ? 2 * j + 11 : (j <= 10 ? 2 * j + 1 : 2 * j - 9));
-        const uint32_t word = w[I >> 4];
-        const uint32_t src = sh >= 0 ? (word << (sh >= 0 ? sh : 0)) : (word >> (sh < 0 ? -sh : 0));
-        return and_or<(3u << p)>(src, one);
-    } else {
-        constexpr int g = I / 3;
-        constexpr int p = 14 + 3 * (I % 3);
-        uint32_t src;
-        if constexpr (g == 0) src = w[0] << 14;
-        else if constexpr (g == 1) src = w[0] << 5;
-        else if constexpr (g == 2) src = w[0] >> 4;
-        else if constexpr (g == 3) src = __funnelshift_r(w[0], w[1], 13);
-        else if constexpr (g == 4) src = w[1] << 10;
-        else if constexpr (g == 5) src = w[1] << 1;
-        else if constexpr (g == 6) src = w[1] >> 8;
-        else if constexpr (g == 7) src = __funnelshift_r(w[1], w[2], 17);
-        else if constexpr (g == 8) src = w[2] << 6;
-        else if constexpr (g == 9) src = w[2] >> 3;
-        else src = w[2] >> 12;
-        return and_or<(7u << p)>(src, one);
-    }
-}
-template <int FMT>
-MOE_DEVINL int code_pos(int i) {
-    if constexpr (FMT == MOE_Q2_32) return q2_pos(i & 15);
-    else return q3_pos(i);
-}
-
-MOE_DEVINL float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-
-MOE_DEVINL void team_sync(int team) { asm volatile("bar.sync %0, %1;" ::"r"(2 + team), "n"(kTeamWarps * 32) : "memory"); }
-// A team barrier that also returns whether v held on every thread of the team.
-MOE_DEVINL bool team_all(int team, bool v) {
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r) : "r"((uint32_t)v), "r"(2 + team), "n"(kTeamWarps * 32) : "memory");
-    return r != 0;
-}
+constexpr int kMaxTiles = 2;                       // gate|up 16-row tiles per item (rf <= 16)
+// one warp's partial sums of a gate|up item: tiles x (16 rows x NSLOT tokens)
+template <int NSLOT>
+constexpr int red_floats() { return kMaxTiles * 16 * NSLOT; }
+constexpr int kSmemBudget = 220 * 1024;            // dynamic shared memory, at most (see smem_budget)
+constexpr int kMaxE = 1024;
 
 // ---------------------------------------------------------------- format geometry
 template <int FMT>
 struct Geo {
-    static constexpr int kCodeBytes = (FMT == MOE_Q2_32) ? 8 : 12;   // per 32-weight chunk
     static constexpr int kBlock = (FMT == MOE_Q3_S256) ? 256 : 32;
     static constexpr int kBlockCode = (FMT == MOE_Q2_32) ? 8 : (FMT == MOE_Q3_32 ? 12 : 96);
+    static constexpr int kCb = (FMT == MOE_Q2_32) ? 8 : 12;    // code bytes per 32 weights
     // bytes of one matrix row with K weights, per region
-    static constexpr int code_row(int K) { return K / 32 * kCodeBytes; }
+    static constexpr int code_row(int K) { return K / 32 * kCb; }
     static constexpr int meta_row(int K) { return (FMT == MOE_Q3_S256) ? K / 256 * 12 : K / 32 * 4; }
     static constexpr int d_row(int K) { return (FMT == MOE_Q3_S256) ? K / 256 * 2 : 0; }
     static constexpr int row_bytes(int K) { return code_row(K) + meta_row(K) + d_row(K); }
@@ -165,9 +104,7 @@ MOE_DEVINL Planes planes_of(const PoolView& P, int slot, int mat) {
 // ---------------------------------------------------------------- work resolution
 struct Owner {
     int slot;
-    int ntok;
-    int tok[kDecodeMaxT];
-    uint32_t rmask[kDecodeMaxT];   // ranks of the token served by this expert
+    uint32_t rmask[kDecodeMaxT];   // ranks of token t served by this expert (0: token not served)
 };
 
 struct DecodeParams {
@@ -182,15 +119,13 @@ struct DecodeParams {
     float* yrows;          // [T*(k+1)][D]
     int32_t* miss_list;
     int32_t* miss_count;
-    uint16_t* hbuf;        // [kMaxPairs][4][F]
+    uint16_t* hfrag;       // [kMaxPairs][F * NSLOT] fp16, fragment order
     uint32_t* err;
     uint32_t* done;        // [kMaxPairs + 1]: per-owner gate|up completion counters + CTA ticket
-    int rf;                // gate|up: features per item
-    int rd;                // down: rows per item
-    int ns_gu, ns_dn;      // pipeline stages
+    int rf;                // gate|up: features per item (8 or 16)
+    int rd;                // down: rows per item (multiple of 16)
+    int ns;                // pipeline stages
 };
-
-constexpr int kMaxE = 1024;
 
 struct Shared {
     uint64_t full[kMaxStages];
@@ -202,7 +137,7 @@ struct Shared {
     int abort[kTeams];         // set by a consumer team that stopped on an error
     int d_range[2];            // this CTA's down items [d_range[0], d_range[1])
     uint64_t range_bar;        // completes once d_range is written
-    uint32_t team_items[kTeams];   // gate|up items finished by each team (release.cta by its leader)
+    uint32_t team_items[kTeams];   // gate|up items finished by each team (release.cta by its reducer)
 };
 
 // The slot table is an input of the layer, not produced by the router: stage it
@@ -214,19 +149,16 @@ __device__ void stage_table(const DecodeParams& prm, Shared& sh) {
     }
 }
 
-// Work items.  Owner 0 (the shared expert, which serves every token and so
-// costs about twice as much per row) is cut into half-size items, so that
-// equal item counts are roughly equal work:
-//   gate|up: 2*nfb shared items of rf/2 features, then nfb items of rf per owner
-//   down   : 2*nrb shared items of rd/2 rows,     then nrb items of rd per owner
-struct ItemPos { int u, row0, nrows; };
+// Work items: owner u's gate|up items are nfb = F / rf blocks of rf features,
+// its down items nrb = D / rd blocks of rd output rows; item i of a phase
+// belongs to owner i / per_owner.
+struct ItemPos { int u, row0; };
 MOE_DEVINL ItemPos item_pos(int i, int per_owner, int rows) {
     ItemPos p;
-    if (i < 2 * per_owner) { p.u = 0; p.nrows = rows / 2; p.row0 = i * p.nrows; }
-    else { const int r = i - 2 * per_owner; p.u = 1 + r / per_owner; p.nrows = rows; p.row0 = (r % per_owner) * rows; }
+    p.u = i / per_owner;
+    p.row0 = (i - p.u * per_owner) * rows;
     return p;
 }
-MOE_DEVINL int items_of(int n_owners, int per_owner) { return 2 * per_owner + (n_owners - 1) * per_owner; }
 
 MOE_DEVINL int lookup_slot(const DecodeParams& prm, const Shared& sh, int e) {
     return (e >= 0 && e < prm.E) ? sh.table[e] : -1;
@@ -234,244 +166,268 @@ MOE_DEVINL int lookup_slot(const DecodeParams& prm, const Shared& sh, int e) {
 
 // One warp: resolve every pair's slot and the owners — owner 0 is the shared
 // expert, then the first pair of each distinct resident slot in pair order —
-// and, with `book`, the row map, miss list and miss count.
+// and, with `book`, the row map, miss list and miss count.  Lane L handles
+// pairs L + 32h (h = 0..3; T * k <= 128).
 __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, bool book) {
+    constexpr int H = (kMaxPairs - 1 + 31) / 32;
     const int lane = threadIdx.x & 31;
-    const int T = prm.T, k = prm.k, n = T * k;   // n <= 64
-    const int e0 = lane < n ? __ldg(prm.ids + lane) : -1;
-    const int e1 = lane + 32 < n ? __ldg(prm.ids + lane + 32) : -1;
-    const int s0 = lane < n ? lookup_slot(prm, sh, e0) : -1;
-    const int s1 = lane + 32 < n ? lookup_slot(prm, sh, e1) : -1;
-    if (lane < n) sh.slot_of[lane] = s0;
-    if (lane + 32 < n) sh.slot_of[lane + 32] = s1;
-    const uint32_t miss0 = __ballot_sync(0xffffffffu, lane < n && s0 < 0);
-    const uint32_t miss1 = __ballot_sync(0xffffffffu, lane + 32 < n && s1 < 0);
+    const int T = prm.T, k = prm.k, n = T * k;   // n <= 128
     const uint32_t below = (1u << lane) - 1u;
+    int e[H], s[H];
+    uint32_t missb[H];
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        const int p = lane + 32 * h;
+        e[h] = p < n ? __ldg(prm.ids + p) : -1;
+        s[h] = p < n ? lookup_slot(prm, sh, e[h]) : -1;
+        if (p < n) sh.slot_of[p] = s[h];
+        missb[h] = __ballot_sync(0xffffffffu, p < n && s[h] < 0);
+    }
     if (book) {
-        if (lane < n) {
-            const int t = lane / k, r = lane % k;
-            prm.rowmap[t * (k + 1) + r] = s0 >= 0 ? t * (k + 1) + r : -1;
-            if (s0 < 0) {
-                const int pos = __popc(miss0 & below);
-                prm.miss_list[3 * pos + 0] = t; prm.miss_list[3 * pos + 1] = r; prm.miss_list[3 * pos + 2] = e0;
+        int base = 0;
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+            const int p = lane + 32 * h;
+            if (p < n) {
+                const int t = p / k, r = p % k;
+                prm.rowmap[t * (k + 1) + r] = s[h] >= 0 ? t * (k + 1) + r : -1;
+                if (s[h] < 0) {
+                    const int pos = base + __popc(missb[h] & below);
+                    prm.miss_list[3 * pos + 0] = t; prm.miss_list[3 * pos + 1] = r; prm.miss_list[3 * pos + 2] = e[h];
+                }
             }
-        }
-        if (lane + 32 < n) {
-            const int q = lane + 32, t = q / k, r = q % k;
-            prm.rowmap[t * (k + 1) + r] = s1 >= 0 ? t * (k + 1) + r : -1;
-            if (s1 < 0) {
-                const int pos = __popc(miss0) + __popc(miss1 & below);
-                prm.miss_list[3 * pos + 0] = t; prm.miss_list[3 * pos + 1] = r; prm.miss_list[3 * pos + 2] = e1;
-            }
+            base += __popc(missb[h]);
         }
         if (lane < T) prm.rowmap[lane * (k + 1) + k] = lane * (k + 1) + k;
-        if (lane == 0) prm.miss_count[0] = __popc(miss0) + __popc(miss1);
+        if (lane == 0) prm.miss_count[0] = base;
     }
     __syncwarp();
-    // lane handles pairs p = lane (h = 0) and p = lane + 32 (h = 1)
-    uint32_t rm0[kDecodeMaxT] = {0, 0, 0, 0}, rm1[kDecodeMaxT] = {0, 0, 0, 0};
-    bool own0 = lane < n && s0 >= 0, own1 = lane + 32 < n && s1 >= 0;
-    uint64_t eq0 = 0, eq1 = 0;                 // pairs q with the same slot
-#pragma unroll 8
-    for (int q = 0; q < n; ++q) {
+    // eq[h]: the pairs q with the same slot as pair lane + 32h (bits of 2 words)
+    uint64_t eq[H][2];
+    bool own[H];
+#pragma unroll
+    for (int h = 0; h < H; ++h) { eq[h][0] = eq[h][1] = 0; }
+    for (int q = 0; q < n && q < 64; ++q) {
         const int sq = sh.slot_of[q];
-        if (sq == s0) eq0 |= 1ull << q;
-        if (sq == s1) eq1 |= 1ull << q;
-    }
-    if (own0 && (eq0 & ((1ull << lane) - 1ull))) own0 = false;
-    if (own1 && (eq1 & ((1ull << (lane + 32)) - 1ull))) own1 = false;
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxT; ++t) {
-        if (t < T) {
-            rm0[t] = (uint32_t)(eq0 >> (t * k)) & ((1u << k) - 1u);
-            rm1[t] = (uint32_t)(eq1 >> (t * k)) & ((1u << k) - 1u);
+        for (int h = 0; h < H; ++h)
+            if (sq == s[h]) eq[h][0] |= 1ull << q;
+    }
+    for (int q = 64; q < n; ++q) {
+        const int sq = sh.slot_of[q];
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+            if (sq == s[h]) eq[h][1] |= 1ull << (q - 64);
+    }
+    uint32_t ownb[H];
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        const int p = lane + 32 * h;
+        bool o = p < n && s[h] >= 0;
+        if (o) {   // an earlier pair with the same slot owns it
+            const uint64_t lo = p >= 64 ? eq[h][0] : (eq[h][0] & ((1ull << p) - 1ull));
+            const uint64_t hi = p >= 64 ? (eq[h][1] & ((1ull << (p - 64)) - 1ull)) : 0ull;
+            if (lo | hi) o = false;
         }
+        own[h] = o;
+        ownb[h] = __ballot_sync(0xffffffffu, o);
     }
-    const uint32_t b0 = __ballot_sync(0xffffffffu, own0);
-    const uint32_t b1 = __ballot_sync(0xffffffffu, own1);
+    int base = 1;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const bool own = h == 0 ? own0 : own1;
-        if (own) {
-            const int idx = h == 0 ? 1 + __popc(b0 & below) : 1 + __popc(b0) + __popc(b1 & below);
-            Owner& o = sh.owners[idx];
-            int nt = 0;
+    for (int h = 0; h < H; ++h) {
+        if (own[h]) {
+            Owner& o = sh.owners[base + __popc(ownb[h] & below)];
 #pragma unroll
             for (int t = 0; t < kDecodeMaxT; ++t) {
-                const uint32_t m = h == 0 ? rm0[t] : rm1[t];
-                if (t < T && m) { o.tok[nt] = t; o.rmask[nt] = m; ++nt; }
+                uint32_t m = 0;
+                if (t < T) {
+                    const int b0 = t * k;                       // bits [b0, b0 + k) of the 128-bit eq
+                    uint64_t w;
+                    if (b0 >= 64) w = eq[h][1] >> (b0 - 64);
+                    else if (b0 == 0) w = eq[h][0];
+                    else w = (eq[h][0] >> b0) | (eq[h][1] << (64 - b0));
+                    m = (uint32_t)w & ((1u << k) - 1u);
+                }
+                o.rmask[t] = m;
             }
-            o.ntok = nt;
-            o.slot = h == 0 ? s0 : s1;
+            o.slot = s[h];
         }
+        base += __popc(ownb[h]);
     }
-    if (lane < T) { sh.owners[0].tok[lane] = lane; sh.owners[0].rmask[lane] = 1u << k; }
+    if (lane < kDecodeMaxT) sh.owners[0].rmask[lane] = lane < T ? 1u << k : 0u;
     if (lane == 0) {
         sh.owners[0].slot = prm.P.shared_slot;
-        sh.owners[0].ntok = T;
-        sh.n_owners = 1 + __popc(b0) + __popc(b1);
+        sh.n_owners = base;
     }
     __syncwarp();
 }
 
-// ---------------------------------------------------------------- activations to smem
-// xs[(n * nb + b) * 36 + j]: pre-scaled activation x_j 2^(23-p_j) of chunk b of
-// token n; slots 32..33 hold per-chunk constants: Q2/Q3_32: C = sum x_j 2^(23-p_j),
-// X = sum x_j;
-// Q3_S256: C'lo, C'hi = sum over the half of x_j (2^(23-p_j) + 4)  (the +4 folds
-// the min -4*S of the sub-block into the constant).  Run by the consumer threads.
-template <int FMT>
-__device__ void stage_activations(const uint16_t* src, size_t tok_stride, int ntok, int K, float* xs,
-                                  int first = 0, int nthreads = kConsumers, bool coherent = false) {
-    const int nb = K / 32;
-    for (int idx = (int)threadIdx.x - first; idx < ntok * nb; idx += nthreads) {
-        const int n = idx / nb, b = idx - n * nb;
-        const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)n * tok_stride + 32 * b);
-        float v[32];
+// ---------------------------------------------------------------- activations in fragment order
+// Byte offset of the 8-byte B-register pair of step s = (U * 2 + i) * 4 + j,
+// token column n, lane-in-quad c.
+template <int NSLOT>
+MOE_DEVINL uint32_t frag_off(int step, int n, int c) { return (uint32_t)(((step * NSLOT + n) * 4 + c) * 8); }
+
+// 16 consecutive bf16 values of one token (a half block) as fp16 in fragment
+// order: four 8-byte words (j = 0..3), each (v[j], v[j + 8]) in the low word
+// and (v[j + 4], v[j + 12]) in the high word.  Returns false if a value is
+// outside the fp16 range.
+MOE_DEVINL bool half_block_frag(const uint4 a, const uint4 b, uint2 (&out)[4]) {
+    float v[16];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint4 w = coherent ? __ldcg(p + q) : __ldg(p + q);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int q = 0; q < 8; ++q) { v[2 * q] = bf16lo(w[q]); v[2 * q + 1] = bf16hi(w[q]); }
+    bool ok = true;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                v[8 * q + 2 * h] = bf16lo(ww[h]);
-                v[8 * q + 2 * h + 1] = bf16hi(ww[h]);
-            }
-        }
-        float* dst = xs + (size_t)idx * kXStride;
-        float vp[32];
+    for (int q = 0; q < 16; ++q) ok &= fabsf(v[q]) < 65520.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) vp[j] = v[j] * (float)(1u << (23 - code_pos<FMT>(j)));   // exact
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(vp[j], vp[j + 1], vp[j + 2], vp[j + 3]);
-        // constants from fp32 partial sums per magic position (few terms each),
-        // combined in double: sum_j x_j 2^(23-p_j) (+ 4 x_j for Q3_S256)
-        float part[2][10];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int c = 0; c < 10; ++c) part[h][c] = 0.f;
-        float xs0 = 0.f, xs1 = 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int c = code_pos<FMT>(j) - 13;       // 0..9
-            const int h = (FMT == MOE_Q3_S256 && j >= 16) ? 1 : 0;
-            part[h][c] += v[j];
-            if (j < 16) xs0 += v[j]; else xs1 += v[j];
-        }
-        double c0 = 0.0, c1 = 0.0;
-#pragma unroll
-        for (int c = 0; c < 10; ++c) {
-            c0 += (double)part[0][c] * (double)(1u << (10 - c));
-            c1 += (double)part[1][c] * (double)(1u << (10 - c));
-        }
-        if constexpr (FMT == MOE_Q3_S256) {
-            c0 += 4.0 * (double)xs0;
-            c1 += 4.0 * (double)xs1;
-        } else {
-            c1 = (double)xs0 + (double)xs1;
-        }
-        dst[32] = (float)c0;
-        dst[33] = (float)c1;
-    }
+    for (int j = 0; j < 4; ++j) out[j] = make_uint2(pack_f16x2(v[j], v[j + 8]), pack_f16x2(v[j + 4], v[j + 12]));
+    return ok;
 }
 
-// ---------------------------------------------------------------- one chunk, R rows
-// cw[r]: the chunk's code words of row r; sa/sb: Q2/Q3_32 (s, m), Q3_S256 (S_lo, S_hi).
-// xc[t]: the chunk's activations of the t-th served token.
-template <int FMT, int NT, int R>
-MOE_DEVINL void chunk_rows(const uint32_t (&cw)[R][3], const float (&sa)[R], const float (&sb)[R],
-                           const float* const (&xc)[NT], float (&res)[R][NT]) {
-    constexpr int H = (FMT == MOE_Q3_S256) ? 2 : 1;
-    const uint32_t one = opaque_one();
-    // NC independent accumulator chains per (row, token, half) (even and odd code
-    // pairs when few tokens leave registers to spare): shorter FMA dependency chains
-    constexpr int NC = NT <= 2 ? 2 : 1;
-    float2 acc[R][NT][H][NC];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-#pragma unroll
-            for (int h = 0; h < H; ++h)
-#pragma unroll
-                for (int c = 0; c < NC; ++c) acc[r][t][h][c] = make_float2(0.f, 0.f);
-    static_for<0, 4>([&](auto SC) {
-        constexpr int sc = decltype(SC)::value;
-        float xv[NT][8];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const float4 a = *reinterpret_cast<const float4*>(xc[t] + 8 * sc);
-            const float4 b = *reinterpret_cast<const float4*>(xc[t] + 8 * sc + 4);
-            xv[t][0] = a.x; xv[t][1] = a.y; xv[t][2] = a.z; xv[t][3] = a.w;
-            xv[t][4] = b.x; xv[t][5] = b.y; xv[t][6] = b.z; xv[t][7] = b.w;
+// x [T][K] (bf16, global) -> xs (fp16 fragment order, NSLOT token columns;
+// columns >= T zero).  Run by `nthreads` threads starting at thread `first`.
+template <int NSLOT>
+__device__ void stage_x_frag(const uint16_t* __restrict__ x, int T, int K, uint8_t* xs, uint32_t* err, int first,
+                             int nthreads) {
+    const int nhb = K / 16;
+    bool ok = true;
+    for (int idx = (int)threadIdx.x - first; idx < NSLOT * nhb; idx += nthreads) {
+        const int n = idx / nhb, hb = idx - n * nhb;
+        uint2 o[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
+        if (n < T) {
+            const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)n * K + 16 * hb);
+            ok &= half_block_frag(__ldg(p), __ldg(p + 1), o);
         }
-        static_for<0, R>([&](auto RR) {
-            constexpr int r = decltype(RR)::value;
-            static_for<0, 4>([&](auto II) {
-                constexpr int i = 2 * decltype(II)::value;
-                constexpr int code = 8 * sc + i;
-                constexpr int h = (H == 2 && code >= 16) ? 1 : 0;
-                constexpr int c2 = decltype(II)::value % NC;
-                const float2 f = make_float2(code_c<FMT, code>(cw[r], one), code_c<FMT, code + 1>(cw[r], one));
+        // hb = U * 8 + c * 2 + i
+        const int U = hb >> 3, c = (hb >> 1) & 3, i = hb & 1;
 #pragma unroll
-                for (int t = 0; t < NT; ++t)
-                    acc[r][t][h][c2] = ffma2(make_float2(xv[t][i], xv[t][i + 1]), f, acc[r][t][h][c2]);
-            });
-        });
-    });
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        const float c0 = xc[t][32];
-        const float c1 = xc[t][33];
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-            float sum[H];
-#pragma unroll
-            for (int h = 0; h < H; ++h) {
-                sum[h] = acc[r][t][h][0].x + acc[r][t][h][0].y;
-                if constexpr (NC == 2) sum[h] += acc[r][t][h][1].x + acc[r][t][h][1].y;
-            }
-            if constexpr (H == 2) {
-                res[r][t] = __fmaf_rn(sa[r], sum[0] - c0, res[r][t]);
-                res[r][t] = __fmaf_rn(sb[r], sum[1] - c1, res[r][t]);
-            } else {
-                res[r][t] = __fmaf_rn(sa[r], sum[0] - c0, __fmaf_rn(sb[r], c1, res[r][t]));
-            }
-        }
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint2*>(xs + frag_off<NSLOT>((U * 2 + i) * 4 + j, n, c)) = o[j];
     }
+    if (!ok) atomicOr(err, kErrRange);
 }
 
-// Chunk b (32 weights along K) of local row `row` of a staged item region.
-// cbase/mbase/dbase: the region's code/meta/d bytes; K: row length.
+// Halfword index of element (kk, token n) in a fragment-order buffer.
+template <int NSLOT>
+MOE_DEVINL uint32_t frag_half_index(int kk, int n) {
+    const int U = kk >> 7, c = (kk >> 5) & 3, i = (kk >> 4) & 1, o = kk & 15;
+    const int j = o & 3, breg = (o >> 2) & 1, e = o >> 3;
+    return (uint32_t)((((U * 2 + i) * 4 + j) * NSLOT + n) * 4 + c) * 4 + (uint32_t)(breg * 2 + e);
+}
+
+// ---------------------------------------------------------------- MMA
+MOE_DEVINL void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One row's data for the 32-weight block of a lane in one 128-K unit: the
+// code words and the block scales.
 template <int FMT>
-MOE_DEVINL void smem_chunk(const uint8_t* cbase, const uint8_t* mbase, const uint8_t* dbase, int row, int K, int b,
-                           uint32_t (&w)[3], float& sa, float& sb) {
+struct RowBlock {
+    uint32_t w[3];           // code words (Q2: w[0], w[1] = halves 0, 1)
+    uint32_t sa, sb;         // Q2/Q3_32: s and m broadcast to f16x2; Q3_S256: sc - 32 of halves 0 and 1
+    uint32_t d2;             // Q3_S256: d broadcast to f16x2
+};
+
+// Load block (4U + c) of local row r of a staged region (codes | meta | d,
+// rows of K weights).
+template <int FMT>
+MOE_DEVINL void load_row_block(const uint8_t* cbase, const uint8_t* mbase, const uint8_t* dbase, int r, int K, int U,
+                               int c, RowBlock<FMT>& rb) {
+    const int blk = 4 * U + c;
     if constexpr (FMT == MOE_Q2_32) {
-        const uint2 c = *reinterpret_cast<const uint2*>(cbase + (size_t)row * Geo<FMT>::code_row(K) + b * 8);
-        w[0] = c.x; w[1] = c.y; w[2] = 0;
-        const float2 sm = __half22float2(*reinterpret_cast<const __half2*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + b * 4));
-        sa = sm.x;
-        sb = sm.y;
-    } else if constexpr (FMT == MOE_Q3_32) {
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)row * Geo<FMT>::code_row(K) + b * 12);
-        w[0] = p[0]; w[1] = p[1]; w[2] = p[2];
-        const float2 sm = __half22float2(*reinterpret_cast<const __half2*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + b * 4));
-        sa = sm.x;
-        sb = sm.y;
+        const uint2 v = *reinterpret_cast<const uint2*>(cbase + (size_t)r * Geo<FMT>::code_row(K) + blk * 8);
+        rb.w[0] = v.x; rb.w[1] = v.y; rb.w[2] = 0;
     } else {
-        const int sbk = b >> 3, j = b & 7;
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)row * Geo<FMT>::code_row(K) + b * 12);
-        w[0] = p[0]; w[1] = p[1]; w[2] = p[2];
-        const uint32_t* scp = reinterpret_cast<const uint32_t*>(mbase + (size_t)row * Geo<FMT>::meta_row(K) + sbk * 12);
-        const int bit = 12 * j, wi = bit >> 5, sh = bit & 31;
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)r * Geo<FMT>::code_row(K) + blk * 12);
+        rb.w[0] = p[0]; rb.w[1] = p[1]; rb.w[2] = p[2];
+    }
+    if constexpr (FMT != MOE_Q3_S256) {
+        const uint32_t sm = *reinterpret_cast<const uint32_t*>(mbase + (size_t)r * Geo<FMT>::meta_row(K) + blk * 4);
+        rb.sa = bcast_lo(sm);
+        rb.sb = bcast_hi(sm);
+        rb.d2 = 0;
+    } else {
+        // super-block U / 2; the block's two sub-blocks: 12 bits at bit 12 * (4 (U & 1) + c)
+        const uint32_t* scp =
+            reinterpret_cast<const uint32_t*>(mbase + (size_t)r * Geo<FMT>::meta_row(K) + (U >> 1) * 12);
+        const int cc = 4 * (U & 1) + c, bit = 12 * cc, wi = bit >> 5, sh = bit & 31;
         const uint32_t lo = scp[wi];
         const uint32_t hi = wi < 2 ? scp[wi + 1] : 0u;
         const uint32_t bits = __funnelshift_r(lo, hi, sh);
-        const float d = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(dbase + (size_t)row * Geo<FMT>::d_row(K) + sbk * 2));
-        sa = d * (float)((int)(bits & 63u) - 32);          // exact
-        sb = d * (float)((int)((bits >> 6) & 63u) - 32);
+        const uint32_t db = *reinterpret_cast<const uint16_t*>(dbase + (size_t)r * Geo<FMT>::d_row(K) + (U >> 1) * 2);
+        rb.d2 = db | (db << 16);
+        rb.sa = s256_sub(bits & 63u);
+        rb.sb = s256_sub((bits >> 6) & 63u);
     }
+}
+
+// Weight pairs (j, j + 8) and (j + 4, j + 12) of half I, the A registers of
+// step (I, J) for one row.
+template <int FMT, int I, int J>
+MOE_DEVINL void step_pairs(const RowBlock<FMT>& rb, const Magic& M, uint32_t& lo, uint32_t& hi) {
+    if constexpr (FMT == MOE_Q2_32) {
+        const uint32_t w = rb.w[I], w10 = w >> 10;
+        lo = w_sm(q2_codes<J>(w, w10, M), rb.sa, rb.sb);
+        hi = w_sm(q2_codes<J + 4>(w, w10, M), rb.sa, rb.sb);
+    } else {
+        uint32_t P, P2;
+        q3_group_words(rb.w[0], rb.w[1], rb.w[2], I, P, P2);
+        const uint32_t P9 = P >> 9, P10 = P2 >> 10;
+        if constexpr (FMT == MOE_Q3_32) {
+            lo = w_sm(q3_codes<J, false>(P, P9, P2, P10, M), rb.sa, rb.sb);
+            hi = w_sm(q3_codes<J + 4, false>(P, P9, P2, P10, M), rb.sa, rb.sb);
+        } else {
+            const uint32_t sc2 = I == 0 ? rb.sa : rb.sb;
+            lo = w_s256(q3_codes<J, true>(P, P9, P2, P10, M), sc2, rb.d2);
+            hi = w_s256(q3_codes<J + 4, true>(P, P9, P2, P10, M), sc2, rb.d2);
+        }
+    }
+}
+
+// Compile-time loop: f(std::integral_constant<int, I>) for I in [B, E).
+template <int B, int E, typename Fn>
+MOE_DEVINL void static_for(Fn&& fn) {
+    if constexpr (B < E) {
+        fn(std::integral_constant<int, B>{});
+        static_for<B + 1, E>(fn);
+    }
+}
+
+// One 128-K unit U for NT tiles: tile t's A rows g and g + 8 are local rows
+// rt[t] of region (ca, ma, da) and rbm[t] of region (cb, mb, db); B from the
+// fragment-order buffer bs.  Accumulates into acc[t].
+template <int FMT, int NT, int NSLOT>
+MOE_DEVINL void unit_mma(const uint8_t* ca, const uint8_t* ma, const uint8_t* da, const uint8_t* cb,
+                         const uint8_t* mb, const uint8_t* db, const int (&rt)[NT], const int (&rbm)[NT], int K, int U,
+                         const uint8_t* bs, const Magic& M, float (&acc)[NT][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    RowBlock<FMT> top[NT], bot[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        load_row_block<FMT>(ca, ma, da, rt[t], K, U, c, top[t]);
+        load_row_block<FMT>(cb, mb, db, rbm[t], K, U, c, bot[t]);
+    }
+    static_for<0, 8>([&](auto S) {
+        constexpr int s = decltype(S)::value, I = s >> 2, J = s & 3;
+        uint32_t b0 = 0, b1 = 0;
+        if (g < NSLOT) {
+            const uint2 bv = *reinterpret_cast<const uint2*>(bs + frag_off<NSLOT>(U * 8 + s, g, c));
+            b0 = bv.x;
+            b1 = bv.y;
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            uint32_t a[4];
+            step_pairs<FMT, I, J>(top[t], M, a[0], a[2]);
+            step_pairs<FMT, I, J>(bot[t], M, a[1], a[3]);
+            mma16816(acc[t], a, b0, b1);
+        }
+    });
 }
 
 MOE_DEVINL float silu_f(float g) { return g / (1.0f + expf(-g)); }
@@ -486,44 +442,17 @@ MOE_DEVINL void issue_rows(const Planes& pl, int row0, int nrows, int K, uint8_t
     if constexpr (FMT == MOE_Q3_S256) bulk_g2s(dst + (cr + mr) * nrows, pl.d + (size_t)row0 * dr, dr * nrows, bar);
 }
 
-// ---------------------------------------------------------------- item geometry
-// The consumers form two teams of eight warps; a team takes every other item
-// of the ring, so that one team's per-item tail (reduction, stores, barrier
-// waits) overlaps the other team's inner loops.  Within an item a warp is cut
-// into G groups of lpr lanes; a group owns one unit (a gate|up feature or a
-// pair of down rows) and its lanes split the unit's nb chunks, nb / lpr each.
-// G grows (lpr shrinks) until the team's 8*G groups cover the item's units
-// in one pass, which keeps every warp busy and the shuffle reductions short.
-// Lane gl of group g takes chunk gl + lpr * ((it + g) mod (nb / lpr)) at
-// iteration it: the groups of one warp start on different chunks, so their
-// code, scale and activation reads fall in different shared-memory banks.
-struct Split { int lpr, G, nit; };
-MOE_DEVINL Split split_for(int units, int nb) {
-    const int want = units / kTeamWarps;      // groups per warp for one pass
-    int gp = 1;                               // largest power of two <= want, at most 8
-    while (gp < 8 && 2 * gp <= want) gp *= 2;
-    int lpr = 32 / gp;
-    const int pow2nb = nb & -nb;              // lpr must divide nb
-    if (lpr > pow2nb) lpr = pow2nb;
-    Split sp;
-    sp.lpr = lpr;
-    sp.G = 32 / lpr;
-    sp.nit = nb / lpr;
-    return sp;
-}
-
 // ---------------------------------------------------------------- gate | up
-// Item = (owner u, features [f0, f0 + rf)); staged as gate rows then up rows.
-// A group computes one feature: its gate row and its up row, chunk by chunk,
-// the next chunk's codes read from shared memory while this one is computed.
-template <int FMT, int NT>
-__device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int f0, int rf, const uint8_t* stage,
-                            const float* xs, int wt) {
-    const int lane = threadIdx.x & 31;
-    const int D = prm.P.D, F = prm.P.F;
-    const int nb = D / 32;
-    const Split sp = split_for(rf, nb);
-    const int lpr = sp.lpr, G = sp.G, nit = sp.nit, group = lane / lpr, gl = lane % lpr;
+// Item = (owner u, features [f0, f0 + rf)), staged as gate rows then up rows.
+// 16-row MMA tile t: rows g = gate feature 8t + g, rows g + 8 = up feature
+// 8t + g, so the lane holding the gate value of (feature, token) also holds
+// the up value.  The eight warps of the team split K by 128-K units; their
+// partial sums meet in `red_w` (this warp's slot), and the team's warp 0 forms h.
+template <int FMT, int NT, int NSLOT>
+__device__ void gateup_partial(const DecodeParams& prm, int rf, const uint8_t* stage, const uint8_t* xs, int wt,
+                               float* red_w) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const int D = prm.P.D;
     const uint32_t cr = Geo<FMT>::code_row(D), mr = Geo<FMT>::meta_row(D);
     const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * rf;   // gate rows then up rows
     const uint8_t* gc = stage;
@@ -532,121 +461,95 @@ __device__ void gateup_item(const DecodeParams& prm, const Owner& o, int u, int 
     const uint8_t* uc = stage + half;
     const uint8_t* um = uc + cr * rf;
     const uint8_t* ud = uc + (cr + mr) * rf;
-    const float* xt[NT];
+    const Magic M = make_magic();
+    float acc[NT][4];
+    int rt[NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) xt[t] = xs + (size_t)o.tok[t] * nb * kXStride;
-    for (int base = wt * G; base < rf; base += kTeamWarps * G) {
-        const int fq = base + group;
-        const bool act = fq < rf;
-        const int fl = act ? fq : rf - 1;      // idle groups recompute a valid feature, unstored
-        float res[2][NT];
+    for (int t = 0; t < NT; ++t) {
+        rt[t] = 8 * t + g;
+        acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    }
+    for (int U = wt; U < D / kUnitK; U += kTeamWarps)
+        unit_mma<FMT, NT, NSLOT>(gc, gm, gd, uc, um, ud, rt, rt, D, U, xs, M, acc);
+    // lanes with c < NSLOT / 2 hold token columns 2c, 2c + 1 (the columns in use)
+    if (c < NSLOT / 2) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) res[r][t] = 0.f;
-        int c = group % nit;
-        int b = gl + lpr * c;
-        uint32_t cw[2][3];
-        float sa[2], sb[2];
-        smem_chunk<FMT>(gc, gm, gd, fl, D, b, cw[0], sa[0], sb[0]);
-        smem_chunk<FMT>(uc, um, ud, fl, D, b, cw[1], sa[1], sb[1]);
-        for (int it = 0; it < nit; ++it) {
-            c = c + 1 == nit ? 0 : c + 1;
-            const int bn = gl + lpr * c;       // next chunk (wraps to the first on the last pass: unused)
-            uint32_t ncw[2][3];
-            float nsa[2], nsb[2];
-            smem_chunk<FMT>(gc, gm, gd, fl, D, bn, ncw[0], nsa[0], nsb[0]);
-            smem_chunk<FMT>(uc, um, ud, fl, D, bn, ncw[1], nsa[1], nsb[1]);
-            const float* xc[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) xc[t] = xt[t] + (size_t)b * kXStride;
-            chunk_rows<FMT, NT, 2>(cw, sa, sb, xc, res);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                cw[r][0] = ncw[r][0]; cw[r][1] = ncw[r][1]; cw[r][2] = ncw[r][2];
-                sa[r] = nsa[r]; sb[r] = nsb[r];
-            }
-            b = bn;
-        }
-        for (int off = lpr >> 1; off >= 1; off >>= 1)
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int t = 0; t < NT; ++t) res[r][t] += __shfl_xor_sync(0xffffffffu, res[r][t], off);
-        if (act && gl == 0) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                prm.hbuf[((size_t)u * kDecodeMaxT + t) * F + f0 + fl] = f32_to_bf16_rne(silu_f(res[0][t]) * res[1][t]);
-        }
+        for (int t = 0; t < NT; ++t)
+            *reinterpret_cast<float4*>(red_w + (t * 8 * (NSLOT / 2) + g * (NSLOT / 2) + c) * 4) =
+                make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
     }
 }
 
-// ---------------------------------------------------------------- down
-// Item = (owner u, rows [d0, d0 + rd)) of Wd; a group computes two rows.
-template <int FMT, int NT>
-__device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int rd, const uint8_t* stage,
-                          const float* hs, int wt) {
+// The team's warp 0: sum the eight partials of every (feature, token) in warp
+// order, h = bf16(silu(gate) * up), stored as fp16 in the owner's
+// fragment-order h buffer.  Entry q = (tile, g, c) of the partials holds
+// gate and up of feature 8 tile + g for tokens 2c and 2c + 1.
+template <int NSLOT>
+__device__ void gateup_reduce(const DecodeParams& prm, int u, int f0, int rf, const float* red) {
     const int lane = threadIdx.x & 31;
+    constexpr int kC = NSLOT / 2;                 // lanes in use per row group
+    const int nq = (rf / 8) * 8 * kC;             // entries
+    const int F = prm.P.F;
+    uint16_t* hf = prm.hfrag + (size_t)u * F * NSLOT;
+    bool ok = true;
+    for (int q = lane; q < nq; q += 32) {
+        const int t = q / (8 * kC), g = (q / kC) & 7, c = q % kC;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kTeamWarps; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(red + w * red_floats<NSLOT>() + q * 4);
+            s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+        const int f = f0 + 8 * t + g;
+        const float hv0 = bf16_bits_to_f32(f32_to_bf16_rne(silu_f(s.x) * s.z));   // token 2c
+        const float hv1 = bf16_bits_to_f32(f32_to_bf16_rne(silu_f(s.y) * s.w));   // token 2c + 1
+        ok &= fabsf(hv0) < 65520.f && fabsf(hv1) < 65520.f;
+        hf[frag_half_index<NSLOT>(f, 2 * c)] = __half_as_ushort(__float2half_rn(hv0));
+        hf[frag_half_index<NSLOT>(f, 2 * c + 1)] = __half_as_ushort(__float2half_rn(hv1));
+    }
+    if (!ok) atomicOr(prm.err, kErrRange);
+}
+
+// ---------------------------------------------------------------- down
+// Item = (owner u, rows [d0, d0 + rd)) of Wd; warp wt takes the 16-row tile wt
+// over the whole K = F.
+template <int FMT, int NSLOT>
+__device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int rd, const uint8_t* stage,
+                          const uint8_t* hs, int wt) {
+    if (16 * wt >= rd) return;
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     const int D = prm.P.D, F = prm.P.F, k = prm.k;
-    const int nb = F / 32;
-    const int pairs = rd / 2;
-    const Split sp = split_for(pairs, nb);
-    const int lpr = sp.lpr, G = sp.G, nit = sp.nit, group = lane / lpr, gl = lane % lpr;
     const uint32_t cr = Geo<FMT>::code_row(F), mr = Geo<FMT>::meta_row(F);
     const uint8_t* dc = stage;
     const uint8_t* dm = stage + cr * rd;
     const uint8_t* dd = stage + (cr + mr) * rd;
-    for (int base = wt * G; base < pairs; base += kTeamWarps * G) {
-        const int qq = base + group;
-        const bool act = qq < pairs;
-        const int rl = 2 * (act ? qq : pairs - 1);
-        float res[2][NT];
+    const Magic M = make_magic();
+    float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
+    const int rt[1] = {16 * wt + g}, rbm[1] = {16 * wt + g + 8};
+    for (int U = 0; U < F / kUnitK; ++U) unit_mma<FMT, 1, NSLOT>(dc, dm, dd, dc, dm, dd, rt, rbm, F, U, hs, M, acc);
+    if (c < NSLOT / 2) {
+        const int row = d0 + 16 * wt + g;
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) res[r][t] = 0.f;
-        int c = group % nit;
-        int b = gl + lpr * c;
-        uint32_t cw[2][3];
-        float sa[2], sb[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, b, cw[r], sa[r], sb[r]);
-        for (int it = 0; it < nit; ++it) {
-            c = c + 1 == nit ? 0 : c + 1;
-            const int bn = gl + lpr * c;
-            uint32_t ncw[2][3];
-            float nsa[2], nsb[2];
-#pragma unroll
-            for (int r = 0; r < 2; ++r) smem_chunk<FMT>(dc, dm, dd, rl + r, F, bn, ncw[r], nsa[r], nsb[r]);
-            const float* xc[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) xc[t] = hs + ((size_t)t * nb + b) * kXStride;
-            chunk_rows<FMT, NT, 2>(cw, sa, sb, xc, res);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                cw[r][0] = ncw[r][0]; cw[r][1] = ncw[r][1]; cw[r][2] = ncw[r][2];
-                sa[r] = nsa[r]; sb[r] = nsb[r];
-            }
-            b = bn;
-        }
-        for (int off = lpr >> 1; off >= 1; off >>= 1)
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                for (int t = 0; t < NT; ++t) res[r][t] += __shfl_xor_sync(0xffffffffu, res[r][t], off);
-        if (act && gl == 0) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const float2 v = make_float2(res[0][t], res[1][t]);
-                uint32_t m = o.rmask[t];
-                while (m) {
-                    const int r = __ffs(m) - 1;
-                    m &= m - 1;
-                    *reinterpret_cast<float2*>(prm.yrows + ((size_t)o.tok[t] * (k + 1) + r) * D + d0 + rl) = v;
-                }
+        for (int h = 0; h < 2; ++h) {
+            uint32_t m = o.rmask[2 * c + h];
+            while (m) {
+                const int r = __ffs(m) - 1;
+                m &= m - 1;
+                float* dst = prm.yrows + ((size_t)(2 * c + h) * (k + 1) + r) * D + row;
+                dst[0] = acc[0][h];
+                dst[8] = acc[0][2 + h];
             }
         }
     }
+}
+
+MOE_DEVINL void team_sync(int team) { asm volatile("bar.sync %0, %1;" ::"r"(2 + team), "n"(kTeamWarps * 32) : "memory"); }
+// A team barrier that also returns whether v held on every thread of the team.
+MOE_DEVINL bool team_all(int team, bool v) {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"((uint32_t)v), "r"(2 + team), "n"(kTeamWarps * 32) : "memory");
+    return r != 0;
 }
 
 MOE_DEVINL void st_release_cta(uint32_t* p, uint32_t v) {
@@ -661,127 +564,60 @@ MOE_DEVINL void red_relaxed_add(uint32_t* p, uint32_t v) {
     asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 MOE_DEVINL void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
-// Work is balanced by an estimated cost: an item of n weights of an owner
-// serving nt tokens costs n / 128 * (4 + 3 (nt - 1)) (a weight served to four
-// tokens measured about three times one served to one).  Gate|up items go
-// round-robin over the CTAs; each CTA then takes a contiguous range of down
-// items such that its gate|up and down costs together approach the average.
-MOE_DEVINL int cost_weight(const Shared& sh, int u) { return 4 + 3 * (sh.owners[u].ntok - 1); }
-MOE_DEVINL long long warp_sum_ll(long long v) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
-MOE_DEVINL long long warp_incl_scan_ll(long long v) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int off = 1; off < 32; off *= 2) {
-        const long long o = __shfl_up_sync(0xffffffffu, v, off);
-        if (lane >= off) v += o;
-    }
-    return v;
-}
-// One warp computes this CTA's down range [d0, d1) (item_pos order).  Owner u
-// has gate|up items from index nfb*(u+1) (owner 0: 0, with 2*nfb half items)
-// and down items from nrb*(u+1) (owner 0: 0, 2*nrb half items); gate|up item i
-// runs on CTA i mod G.  The cumulative down cost before CTA b is its share of
-// all work less the gate|up work of CTAs 0 .. b-1, clamped to [0, total down
-// cost]: any such sequence from 0 to the total covers every item (a decrease
-// only makes two neighbouring ranges overlap, and an overlapped item is
-// computed twice with identical results).
-MOE_DEVINL void down_range_warp(const Shared& sh, int b, int G, int nfb, int rf, int D, int nrb, int rd, int F,
-                                int& d0, int& d1) {
-    constexpr int H = (kMaxPairs + 31) / 32;   // owners per lane: u = lane + 32 h
-    const int lane = threadIdx.x & 31, n = sh.n_owners;
-    auto below = [&](int m, int cb) {          // #{i < m : i mod G < cb}
-        const unsigned q = (unsigned)m / (unsigned)G, r = (unsigned)m % (unsigned)G;
-        return (long long)q * cb + (long long)(r < (unsigned)cb ? r : (unsigned)cb);
-    };
-    long long gu_all = 0, gu_b0 = 0, gu_b1 = 0, dn_part[H];
-    int dcost[H], ditems[H];
-#pragma unroll
-    for (int h = 0; h < H; ++h) {
-        const int u = lane + 32 * h;
-        dn_part[h] = 0;
-        dcost[h] = 1;
-        ditems[h] = 0;
-        if (u < n) {
-            const int w = cost_weight(sh, u);
-            const int gi = u == 0 ? 2 * nfb : nfb, gs = u == 0 ? 0 : nfb * (u + 1);
-            const long long gc = 2ll * (u == 0 ? rf / 2 : rf) * D / 128 * w;
-            gu_all += gc * gi;
-            gu_b0 += gc * (below(gs + gi, b) - below(gs, b));
-            gu_b1 += gc * (below(gs + gi, b + 1) - below(gs, b + 1));
-            ditems[h] = u == 0 ? 2 * nrb : nrb;
-            dcost[h] = (u == 0 ? rd / 2 : rd) * F / 128 * w;
-            dn_part[h] = (long long)dcost[h] * ditems[h];
-        }
-    }
-    gu_all = warp_sum_ll(gu_all);
-    gu_b0 = warp_sum_ll(gu_b0);
-    gu_b1 = warp_sum_ll(gu_b1);
-    // exclusive prefix of the down costs over owners 0 .. n-1, 32 owners a pass
-    long long base[H], carry = 0;
-#pragma unroll
-    for (int h = 0; h < H; ++h) {
-        const long long in = warp_incl_scan_ll(dn_part[h]) + carry;
-        base[h] = in - dn_part[h];
-        carry = __shfl_sync(0xffffffffu, in, 31);
-    }
-    const long long dn_all = carry;
-    const long long all = gu_all + dn_all;
-    auto start = [&](int cb, long long gub) -> long long {
-        if (cb <= 0) return 0;
-        if (cb >= G) return dn_all;
-        const long long ds = (all * cb + G - 1) / G - gub;
-        return ds < 0 ? 0 : (ds > dn_all ? dn_all : ds);
-    };
-    auto item_at = [&](long long pos) -> int {
-        int idx = -1;
-#pragma unroll
-        for (int h = 0; h < H; ++h) {
-            const int u = lane + 32 * h;
-            if (u < n && pos >= base[h] && pos < base[h] + dn_part[h]) {
-                const int m = (int)((pos - base[h] + dcost[h] - 1) / dcost[h]);
-                idx = (u == 0 ? 0 : nrb * (u + 1)) + (m < ditems[h] ? m : ditems[h]);
-            }
-        }
-        const uint32_t hit = __ballot_sync(0xffffffffu, idx >= 0);
-        return hit ? __shfl_sync(0xffffffffu, idx, __ffs(hit) - 1) : (n == 0 ? 0 : nrb * (n + 1));
-    };
-    d0 = item_at(start(b, gu_b0));
-    d1 = item_at(start(b + 1, gu_b1));
-}
-
 MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 
+// Work is balanced by weight count: gate|up item i (n_owners * nfb of them, gw
+// weights each) runs on CTA i mod G; down items cost dw weights each, and CTA b
+// takes a contiguous range of them.  The down work before CTA b is its share
+// of all work less the gate|up work of CTAs 0 .. b-1, clamped to [0, all down
+// work]; any such sequence from 0 to the total covers every item (a decrease
+// only makes two neighbouring ranges overlap, and an overlapped item is
+// computed twice with identical results).
+MOE_DEVINL void down_range(int n, int b, int G, int nfb, long long gw, int nrb, long long dw, int& d0, int& d1) {
+    const long long ng = (long long)n * nfb, nd = (long long)n * nrb;
+    auto below = [&](long long m, int cb) {    // #{i < m : i mod G < cb}
+        const long long q = m / G, r = m % G;
+        return q * cb + (r < cb ? r : (long long)cb);
+    };
+    const long long all = ng * gw + nd * dw;
+    auto start = [&](int cb) -> long long {   // first down item of CTA cb
+        if (cb <= 0) return 0;
+        if (cb >= G) return nd;
+        long long work = (all * cb + G - 1) / G - below(ng, cb) * gw;
+        if (work < 0) work = 0;
+        const long long it = (work + dw - 1) / dw;
+        return it > nd ? nd : it;
+    };
+    d0 = (int)start(b);
+    d1 = (int)start(b + 1);
+}
+
 // ---------------------------------------------------------------- the fused kernel
 // One persistent CTA per SM.  Each CTA takes its gate|up items (round-robin),
-// then a contiguous range of down items (balancing the estimated cost of both),
+// then a contiguous range of down items (balancing the weights of both),
 // through one ring of stages.  A down item of owner u waits until every
 // gate|up item of u has published its h: a per-owner item counter in ws,
 // advanced by a publisher warp that releases each finished item at gpu scope,
 // off the computing warps' path.  The down weights stream in meanwhile.  The
 // last CTA to finish resets the counters, so every completed call leaves them
 // zero.
-template <int FMT, int NTMAX>
+template <int FMT, int NSLOT>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams prm) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ Shared sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int D = prm.P.D, F = prm.P.F, rf = prm.rf, rd = prm.rd, NS = prm.ns_gu;
-    const int nbx = D / 32, nbh = F / 32;
-    const size_t xs_bytes = ((size_t)prm.T * nbx * kXStride * 4 + 127) / 128 * 128;
-    const size_t hs_floats = ((size_t)kDecodeMaxT * nbh * kXStride + 31) / 32 * 32;   // one per team
-    const size_t hs_bytes = kTeams * hs_floats * 4;
-    float* xs = reinterpret_cast<float*>(smem);
-    float* hs = reinterpret_cast<float*>(smem + xs_bytes);
-    uint8_t* stages = smem + xs_bytes + hs_bytes;
+    const int D = prm.P.D, F = prm.P.F, rf = prm.rf, rd = prm.rd, NS = prm.ns;
+    const size_t xs_bytes = (size_t)D * NSLOT * 2;
+    const size_t hs_bytes = (size_t)F * NSLOT * 2;                               // one per team
+    const size_t red_team = (size_t)2 * kTeamWarps * red_floats<NSLOT>();        // per team, double-buffered
+    uint8_t* xs = smem;
+    uint8_t* hs = smem + xs_bytes;
+    float* red = reinterpret_cast<float*>(smem + xs_bytes + kTeams * hs_bytes);
+    uint8_t* stages = smem + xs_bytes + kTeams * hs_bytes + kTeams * red_team * 4;
     const uint32_t gu_bytes = 2u * Geo<FMT>::row_bytes(D) * rf;
     const uint32_t dn_bytes = (uint32_t)Geo<FMT>::row_bytes(F) * rd;
     const uint32_t stage_bytes = gu_bytes > dn_bytes ? gu_bytes : dn_bytes;
@@ -793,15 +629,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         fence_mbar_init();
         for (int tm = 0; tm < kTeams; ++tm) { sh.abort[tm] = 0; sh.team_items[tm] = 0; }
     }
+    // a call on a workspace whose timeout bit is set does no work (every CTA
+    // still takes its ticket below, so the counters are left zero); one read,
+    // shared by the whole CTA, so that every warp takes the same branch.  The
+    // word is read before the dependency wait: only this kernel writes it, and
+    // its previous launch on the stream completed before the router that
+    // precedes this launch passed its own wait.
+    __shared__ int dead;
+    if (threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
     stage_table(prm, sh);
     __syncthreads();
     pdl_wait();                      // ids come from the router
-    // a call on a workspace whose timeout bit is set does no work (every CTA
-    // still takes its ticket below, so the counters are left zero); one read,
-    // shared by the whole CTA, so that every warp takes the same branch
-    __shared__ int dead;
-    if (threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
-    __syncthreads();
     if (!dead) {
     // warp 0 resolves the owners and releases the producer and publisher
     // (barrier 1) while the other consumers stage x; the consumers meet at
@@ -811,15 +649,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         asm volatile("bar.arrive 1, 96;" ::: "memory");
         asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
     } else if (warp < kConsumerWarps) {
-        stage_activations<FMT>(prm.x, D, prm.T, D, xs, 32, kConsumers - 32);
+        stage_x_frag<NSLOT>(prm.x, prm.T, D, xs, prm.err, 32, kConsumers - 32);
         asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
     } else {
         asm volatile("bar.sync 1, 96;" ::: "memory");
     }
     pdl_launch_dependents();
-    // gate|up items round-robin over the CTAs (x is staged for every token);
-    // down items in contiguous ranges of equal cost (h is re-staged per owner)
-    const int n_g = items_of(sh.n_owners, nfb);
+    // gate|up items round-robin over the CTAs; down items in contiguous ranges
+    const int n_g = sh.n_owners * nfb;
     const int ng = n_g > (int)blockIdx.x ? (n_g - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     // the down range is computed by the publisher warp, off the producer's path;
     // the others wait for it only when they reach their first down item
@@ -835,16 +672,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         return true;
     };
     if (warp == kPublisherWarp) {    // publisher: the down range, then release finished gate|up items
-        {
-            int r0, r1;
-            down_range_warp(sh, (int)blockIdx.x, (int)gridDim.x, nfb, rf, D, nrb, rd, F, r0, r1);
-            if (lane == 0) {
-                sh.d_range[0] = r0;
-                sh.d_range[1] = r1;
-                mbar_arrive(&sh.range_bar);
-            }
-        }
         if (lane == 0) {
+            int r0, r1;
+            down_range(sh.n_owners, (int)blockIdx.x, (int)gridDim.x, nfb, 2ll * rf * D, nrb, (long long)rd * F, r0, r1);
+            sh.d_range[0] = r0;
+            sh.d_range[1] = r1;
+            mbar_arrive(&sh.range_bar);
             uint32_t pub[kTeams] = {0u, 0u};
             const uint32_t want[kTeams] = {(uint32_t)((ng + 1) / 2), (uint32_t)(ng / 2)};
             const uint64_t t0 = globaltimer_ns();
@@ -852,9 +685,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                 const uint32_t c0 = ld_acquire_cta(&sh.team_items[0]), c1 = ld_acquire_cta(&sh.team_items[1]);
                 if (c0 > pub[0] || c1 > pub[1]) {
                     fence_acq_rel_gpu();             // with the relaxed adds below: one release per batch
-                    const uint32_t c[kTeams] = {c0, c1};
+                    const uint32_t cn[kTeams] = {c0, c1};
                     for (int tm = 0; tm < kTeams; ++tm)
-                        for (uint32_t n = pub[tm]; n < c[tm]; ++n) {
+                        for (uint32_t n = pub[tm]; n < cn[tm]; ++n) {
                             const int j = tm + kTeams * (int)n;
                             red_relaxed_add(done + item_pos(blockIdx.x + j * gridDim.x, nfb, rf).u, 1u);
                         }
@@ -884,14 +717,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                 if (j < ng) {
                     const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
                     const int slot = sh.owners[ip.u].slot;
-                    const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * ip.nrows;
+                    const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * rf;
                     mbar_arrive_expect_tx(&sh.full[s], 2 * half);
-                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 0), ip.row0, ip.nrows, D, dst, &sh.full[s]);
-                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 1), ip.row0, ip.nrows, D, dst + half, &sh.full[s]);
+                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 0), ip.row0, rf, D, dst, &sh.full[s]);
+                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 1), ip.row0, rf, D, dst + half, &sh.full[s]);
                 } else {
                     const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
-                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)Geo<FMT>::row_bytes(F) * ip.nrows);
-                    issue_rows<FMT>(planes_of<FMT>(prm.P, sh.owners[ip.u].slot, 2), ip.row0, ip.nrows, F, dst, &sh.full[s]);
+                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)Geo<FMT>::row_bytes(F) * rd);
+                    issue_rows<FMT>(planes_of<FMT>(prm.P, sh.owners[ip.u].slot, 2), ip.row0, rd, F, dst, &sh.full[s]);
                 }
             }
         }
@@ -899,7 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         // consumer teams: team tm takes items j = tm, tm + 2, ... of the ring
         const int team = warp / kTeamWarps, wt = warp % kTeamWarps;
         const int tl = (int)threadIdx.x - team * kTeamWarps * 32;
-        float* hst = hs + (size_t)team * hs_floats;
+        uint8_t* hst = hs + (size_t)team * hs_bytes;
+        float* redt = red + (size_t)team * red_team;
         bool ok = true;
         int cur = -1;
         uint32_t gu_done = 0;
@@ -912,30 +746,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
             const int s = j % NS;
             const uint8_t* st = stages + (size_t)s * stage_bytes;
             if (j < ng) {
-                bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
+                // partial sums of successive items alternate between two buffers:
+                // warp 0 reduces item n while the other warps start item n + 1
+                float* redb = redt + ((j / kTeams) & 1) * (kTeamWarps * red_floats<NSLOT>());
+                const bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
                 const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
-                const int u = ip.u, f0 = ip.row0;
-                const Owner& o = sh.owners[u];
                 if (got) {
-                    if constexpr (NTMAX == 1) {
-                        gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs, wt);
-                    } else {
-                        switch (o.ntok) {
-                            case 1: gateup_item<FMT, 1>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
-                            case 2: gateup_item<FMT, 2>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
-                            case 3: gateup_item<FMT, 3>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
-                            default: gateup_item<FMT, 4>(prm, o, u, f0, ip.nrows, st, xs, wt); break;
-                        }
-                    }
+                    if (rf == 16) gateup_partial<FMT, 2, NSLOT>(prm, rf, st, xs, wt, redb + wt * red_floats<NSLOT>());
+                    else gateup_partial<FMT, 1, NSLOT>(prm, rf, st, xs, wt, redb + wt * red_floats<NSLOT>());
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);
-                // the team's h stores of this item are done (and the verdict is
-                // the team's, so every thread leaves the loop together): publish
+                // every warp's partials are in redb (and the verdict is the team's,
+                // so every thread leaves the loop together)
                 ok = team_all(team, got);
                 if (!ok) break;
-                ++gu_done;
-                if (tl == 0) st_release_cta(&sh.team_items[team], gu_done);
+                if (wt == 0) {
+                    gateup_reduce<NSLOT>(prm, ip.u, ip.row0, rf, redb);
+                    __syncwarp();
+                    ++gu_done;
+                    if (lane == 0) st_release_cta(&sh.team_items[team], gu_done);
+                }
             } else {
                 const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
                 const int u = ip.u, r0 = ip.row0;
@@ -944,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                     team_sync(team);                    // the team is done reading hst
                     bool waited = true;
                     if (tl == 0) {
-                        const uint32_t target = (uint32_t)(u == 0 ? 2 * nfb : nfb);   // items of owner u
+                        const uint32_t target = (uint32_t)nfb;   // gate|up items of owner u
                         const uint64_t t0 = globaltimer_ns();
                         while (ld_acquire(done + u) < target) {
                             if (timed_out(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
@@ -957,24 +788,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                     }
                     ok = team_all(team, waited);
                     if (!ok) break;
-                    stage_activations<FMT>(prm.hbuf + (size_t)u * kDecodeMaxT * F, F, o.ntok, F, hst,
-                                           team * kTeamWarps * 32, kTeamWarps * 32, true);
+                    // the owner's h (fragment order, written by other CTAs of this
+                    // launch): L2-coherent 16-byte copies
+                    const uint4* src = reinterpret_cast<const uint4*>(prm.hfrag + (size_t)u * F * NSLOT);
+                    for (int q = tl; q < (int)(hs_bytes / 16); q += kTeamWarps * 32)
+                        reinterpret_cast<uint4*>(hst)[q] = __ldcg(src + q);
                     team_sync(team);
                     cur = u;
                 }
                 const bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
-                if (got) {
-                    if constexpr (NTMAX == 1) {
-                        down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hst, wt);
-                    } else {
-                        switch (o.ntok) {
-                            case 1: down_item<FMT, 1>(prm, o, r0, ip.nrows, st, hst, wt); break;
-                            case 2: down_item<FMT, 2>(prm, o, r0, ip.nrows, st, hst, wt); break;
-                            case 3: down_item<FMT, 3>(prm, o, r0, ip.nrows, st, hst, wt); break;
-                            default: down_item<FMT, 4>(prm, o, r0, ip.nrows, st, hst, wt); break;
-                        }
-                    }
-                }
+                if (got) down_item<FMT, NSLOT>(prm, o, r0, rd, st, hst, wt);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);
                 ok = team_all(team, got);
@@ -998,41 +821,69 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     }
 }
 
-template <int FMT, int NTMAX>
+template <int FMT, int NSLOT>
+size_t smem_for(int D, int F, int rf, int rd, int ns) {
+    const size_t fixed = (size_t)D * NSLOT * 2 + kTeams * (size_t)F * NSLOT * 2 +
+                         kTeams * (size_t)2 * kTeamWarps * red_floats<NSLOT>() * 4;
+    const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf, b = (size_t)Geo<FMT>::row_bytes(F) * rd;
+    return fixed + (size_t)ns * (a > b ? a : b);
+}
+
+// Dynamic shared memory available to decode_ffn_kernel<FMT, NSLOT> on the
+// current device: the opt-in per-block limit less the kernel's static shared
+// memory, capped at kSmemBudget (looked up once per device; 0 if the query fails).
+template <int FMT, int NSLOT>
+int smem_budget() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev >= 0 && dev < 64) {
+        const int v = cache[dev].load(std::memory_order_relaxed);
+        if (v) return v;
+    }
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa, decode_ffn_kernel<FMT, NSLOT>) != cudaSuccess)
+        return 0;
+    int b = optin - (int)fa.sharedSizeBytes;
+    if (b > kSmemBudget) b = kSmemBudget;
+    if (dev >= 0 && dev < 64) cache[dev].store(b, std::memory_order_relaxed);
+    return b;
+}
+
+template <int FMT, int NSLOT>
 moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
-    const int T = prm.T, D = prm.P.D, F = prm.P.F;
-    const size_t xs_bytes = ((size_t)T * (D / 32) * kXStride * 4 + 127) / 128 * 128;
-    const size_t hs_bytes = kTeams * (((size_t)kDecodeMaxT * (F / 32) * kXStride + 31) / 32 * 32) * 4;
-    // gate|up items of rf features, down items of rd rows, one ring of up to 4
-    // stages (~3-4 items in flight per SM cover the copy latency)
+    const int D = prm.P.D, F = prm.P.F;
+    const int budget = smem_budget<FMT, NSLOT>();
+    if (budget <= 0) return MOE_ERR_CUDA;
+    // gate|up items of rf features (two 16-row tiles), down items of rd rows
+    // (eight 16-row tiles, one per warp of a team), up to 4 stages (3-4 items in
+    // flight per SM cover the copy latency)
     int rf = 16, rd = 128;
-    const size_t budget = 216 * 1024;
-    auto stage_of = [&](int rf_, int rd_) {
-        const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf_, b = (size_t)Geo<FMT>::row_bytes(F) * rd_;
-        return a > b ? a : b;
-    };
-    while (rf > 2 && xs_bytes + hs_bytes + 2 * stage_of(rf, rd) > budget) rf /= 2;
+    while (rf > 8 && smem_for<FMT, NSLOT>(D, F, rf, rd, 2) > (size_t)budget) rf /= 2;
     while (rd > 16 && (size_t)Geo<FMT>::row_bytes(F) * rd > 2 * (size_t)Geo<FMT>::row_bytes(D) * rf) rd /= 2;
+    while (rd > 16 && smem_for<FMT, NSLOT>(D, F, rf, rd, 2) > (size_t)budget) rd /= 2;
     int ns = 4;
-    while (ns > 2 && xs_bytes + hs_bytes + ns * stage_of(rf, rd) > budget) --ns;
+    while (ns > 2 && smem_for<FMT, NSLOT>(D, F, rf, rd, ns) > (size_t)budget) --ns;
     prm.rf = rf;
     prm.rd = rd;
-    prm.ns_gu = prm.ns_dn = ns;
-    const size_t smem = xs_bytes + hs_bytes + ns * stage_of(rf, rd);
-    if (smem > kSmemBudget || F % rf || D % rd || rf < 2 || rd < 2) return MOE_ERR_UNSUPPORTED;
-    // every bulk copy (full and half items) must be a multiple of 16 bytes
+    prm.ns = ns;
+    const size_t smem = smem_for<FMT, NSLOT>(D, F, rf, rd, ns);
+    if (smem > (size_t)budget || F % rf || D % rd) return MOE_ERR_UNSUPPORTED;
+    // every bulk copy must be a multiple of 16 bytes
     auto ok16 = [](int K, int n) {
         return ((size_t)Geo<FMT>::code_row(K) * n) % 16 == 0 && ((size_t)Geo<FMT>::meta_row(K) * n) % 16 == 0 &&
                ((size_t)Geo<FMT>::d_row(K) * n) % 16 == 0;
     };
-    if (!ok16(D, rf) || !ok16(D, rf / 2) || !ok16(F, rd) || !ok16(F, rd / 2)) return MOE_ERR_UNSUPPORTED;
+    if (!ok16(D, rf) || !ok16(F, rd)) return MOE_ERR_UNSUPPORTED;
     static std::atomic<uint64_t> attr_done{0};
     if (!once_per_device(attr_done, [] {
-            return cudaFuncSetAttribute(decode_ffn_kernel<FMT, NTMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemBudget) == cudaSuccess;
+            return cudaFuncSetAttribute(decode_ffn_kernel<FMT, NSLOT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        smem_budget<FMT, NSLOT>()) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
-    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NTMAX>, dim3(device_sm_count()), dim3(kThreads), smem, s, prm);
+    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NSLOT>, dim3(device_sm_count()), dim3(kThreads), smem, s, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -1040,15 +891,17 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
 
 // ws layout: [0,4) reserved, [4,8) device error word, [64, 64 + 4*(kMaxPairs+1))
 // completion counters (zero before the first call; every completed call leaves
-// them zero), [1024, ...) h buffer.
+// them zero), [1024, ...) h of every owner (fp16, fragment order, 4 token
+// columns for T <= 4, else 8).
 size_t decode_workspace_bytes(int T, int D, int F, int k) {
-    (void)D; (void)T; (void)k;
-    return 1024 + (size_t)kMaxPairs * kDecodeMaxT * F * sizeof(uint16_t);
+    (void)D; (void)k;
+    return 1024 + (size_t)kMaxPairs * (T <= 4 ? 4 : 8) * F * sizeof(uint16_t);
 }
 
 moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
                                  const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
                                  int32_t* miss_count, void* ws, cudaStream_t s) {
+    if (P.D % kUnitK || P.F % kUnitK) return MOE_ERR_UNSUPPORTED;
     DecodeParams prm;
     prm.P = P;
     prm.slot_table = slot_table;
@@ -1063,12 +916,18 @@ moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, i
     prm.miss_count = miss_count;
     prm.err = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
     prm.done = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 64);
-    prm.hbuf = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 1024);
-    const bool one = (T == 1);
+    prm.hfrag = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 1024);
+    if (T <= 4) {
+        switch (P.fmt) {
+            case MOE_Q2_32: return launch_fmt<MOE_Q2_32, 4>(prm, s);
+            case MOE_Q3_32: return launch_fmt<MOE_Q3_32, 4>(prm, s);
+            default: return launch_fmt<MOE_Q3_S256, 4>(prm, s);
+        }
+    }
     switch (P.fmt) {
-        case MOE_Q2_32: return one ? launch_fmt<MOE_Q2_32, 1>(prm, s) : launch_fmt<MOE_Q2_32, 4>(prm, s);
-        case MOE_Q3_32: return one ? launch_fmt<MOE_Q3_32, 1>(prm, s) : launch_fmt<MOE_Q3_32, 4>(prm, s);
-        default: return one ? launch_fmt<MOE_Q3_S256, 1>(prm, s) : launch_fmt<MOE_Q3_S256, 4>(prm, s);
+        case MOE_Q2_32: return launch_fmt<MOE_Q2_32, 8>(prm, s);
+        case MOE_Q3_32: return launch_fmt<MOE_Q3_32, 8>(prm, s);
+        default: return launch_fmt<MOE_Q3_S256, 8>(prm, s);
     }
 }
 

@@ -12,11 +12,11 @@ namespace moe {
 // Layout of the opaque expert_out buffer:
 //   int32 rowmap[T][k+1]  row index of the output row of (token, rank), -1 = miss;
 //                         rank k is the shared expert
-//   (256-byte aligned) rows: decode path fp32 [T*(k+1)][D], indexed t*(k+1)+r;
+//   (256-byte aligned) rows: decode path (T <= 8) fp32 [T*(k+1)][D], indexed t*(k+1)+r;
 //                         prefill path bf16 [T*(k+1)][D], expert-ordered
 inline size_t rowmap_bytes(int T, int k) { return ((size_t)T * (k + 1) * 4 + 255) / 256 * 256; }
 inline size_t expert_out_bytes(int T, int D, int k) {
-    const size_t row = (T <= 4) ? 4 : 2;
+    const size_t row = (T <= 8) ? 4 : 2;
     return rowmap_bytes(T, k) + (size_t)T * (k + 1) * D * row;
 }
 
@@ -43,6 +43,9 @@ moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, 
                                   int T, const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
                                   int32_t* miss_count, void* ws, cudaStream_t s);
 size_t prefill_workspace_bytes(int T, int D, int F, int E, int k);
+size_t prefill_operand_dump_ws_bytes(int D, int F);
+moe_status launch_prefill_operand_dump(const PoolView& P, int gemm, int slot, int m0, uint32_t* dump, void* ws,
+                                       cudaStream_t s);
 
 moe_status launch_combine(const void* expert_out, const float* gates, int T, int D, int k,
                           const float* miss_partial, const uint16_t* residual, uint16_t* out, cudaStream_t s);

@@ -19,12 +19,10 @@
 // Both are "swap-AB": the weights are the M = 128 operand (A, in tensor
 // memory), the rows are N (B, in shared memory).
 //
-// Operand type.  The MMAs run kind::f16 with fp16 A and B.  Weights are
-// dequantised with packed fp16 arithmetic, which rounds once (Q2_32 / Q3_32:
-// fma(s, q, m); Q3_S256: fp16(d (sc - 32)) (q - 4), two roundings), i.e. to
-// within one fp16 ulp of the exact weight — finer than a bf16 weight.  The bf16
-// activations convert to fp16 exactly inside the fp16 range; an activation
-// of magnitude >= 65520 (x or h) sets kErrRange in the error word.
+// Operand type.  The MMAs run kind::f16 with fp16 A and B.  Every weight is
+// the exact weight rounded once to fp16 (dequant.cuh) — finer than a bf16
+// weight.  The bf16 activations convert to fp16 exactly inside the fp16 range;
+// an activation of magnitude >= 65520 (x or h) sets kErrRange in the error word.
 //
 // K order.  Inside every group of 16 consecutive K indices the operands use
 // the order (0, 8, 1, 9, ..., 7, 15): one 32-bit word of A then holds the
@@ -37,6 +35,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "dequant.cuh"
 #include "kernels.cuh"
 #include "once.cuh"
 #include "sync.cuh"
@@ -286,11 +285,6 @@ __global__ void __launch_bounds__(kChunk) plan_scatter_kernel(PlanArgs a) {
 }
 
 // ---------------------------------------------------------------- x rows -> fp16, group order, K-permuted
-MOE_DEVINL uint32_t pack_f16x2(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
 MOE_DEVINL uint32_t bf16_half(uint32_t w, int hi) { return hi ? (w & 0xffff0000u) : (w << 16); }
 
 // xg[row] = x[perm[row]] in fp16 and K order: one thread per 16-element group,
@@ -408,95 +402,6 @@ MOE_DEVINL bool epilogue_all(bool v, int nthreads_const_128) {
 // Byte offset of the 16-byte chunk c of row r in a K-major 128B-swizzled tile.
 MOE_DEVINL uint32_t sw128(int r, int c) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)); }
 
-// ---------------------------------------------------------------- dequantisation to fp16 pairs
-// fp16 "magic" numbers 2^(10-b): OR-ing a code field that sits at bit b of a
-// half into one gives 2^(10-b) + code exactly; subtracting it back gives the
-// code (exact small integers).
-struct Magic {
-    uint32_t m1024, m256, m128, m64, m16, m8, m4;      // f16x2, both halves
-    uint32_t s1028, s132, s20, s12;                     // magic + 4 (the Q3_S256 code centre)
-};
-MOE_DEVINL uint32_t opaque_u32(uint32_t v) {
-    uint32_t r;
-    asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v));
-    return r;
-}
-MOE_DEVINL Magic make_magic() {
-    Magic m;
-    m.m1024 = opaque_u32(0x64006400u);
-    m.m256 = opaque_u32(0x5C005C00u);
-    m.m128 = opaque_u32(0x58005800u);
-    m.m64 = opaque_u32(0x54005400u);
-    m.m16 = opaque_u32(0x4C004C00u);
-    m.m8 = opaque_u32(0x48004800u);
-    m.m4 = opaque_u32(0x44004400u);
-    m.s1028 = opaque_u32(0x64046404u);
-    m.s132 = opaque_u32(0x58205820u);
-    m.s20 = opaque_u32(0x4D004D00u);
-    m.s12 = opaque_u32(0x4A004A00u);
-    return m;
-}
-template <uint32_t MASK>
-MOE_DEVINL uint32_t field_or(uint32_t w, uint32_t magic) {
-    uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "n"(MASK), "r"(magic));   // (w & MASK) | magic
-    return r;
-}
-MOE_DEVINL uint32_t hsub2u(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-MOE_DEVINL uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t r;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-    return r;
-}
-MOE_DEVINL uint32_t hmul2u(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
-// Q2_32, one 16-weight group: word w holds code i at bits [2i, 2i+2).
-// out[i] = (w_i, w_{i+8}) = fma(s, q, m) in fp16.
-MOE_DEVINL void dq_q2_group(uint32_t w, uint32_t s2, uint32_t m2, const Magic& M, uint32_t* out) {
-    const uint32_t w10 = w >> 10;
-    out[0] = hfma2u(s2, hsub2u(field_or<0x00030003u>(w, M.m1024), M.m1024), m2);
-    out[1] = hfma2u(s2, hsub2u(field_or<0x000C000Cu>(w, M.m256), M.m256), m2);
-    out[2] = hfma2u(s2, hsub2u(field_or<0x00300030u>(w, M.m64), M.m64), m2);
-    out[3] = hfma2u(s2, hsub2u(field_or<0x00C000C0u>(w, M.m16), M.m16), m2);
-    out[4] = hfma2u(s2, hsub2u(field_or<0x03000300u>(w, M.m4), M.m4), m2);
-    out[5] = hfma2u(s2, hsub2u(field_or<0x00030003u>(w10, M.m1024), M.m1024), m2);
-    out[6] = hfma2u(s2, hsub2u(field_or<0x000C000Cu>(w10, M.m256), M.m256), m2);
-    out[7] = hfma2u(s2, hsub2u(field_or<0x00300030u>(w10, M.m64), M.m64), m2);
-}
-
-// 3-bit codes of one 16-weight group, given P = (stream bits [0,16) | [24,40))
-// and P2 = (bits [8,24) | [32,48)) of the group's 48-bit stream: code i of the
-// low half (code i + 8 of the high half) sits at bit 3i of P for i <= 4 and at
-// bit 3i - 8 of P2 for i >= 5.  q[i] = the code pair, minus 4 when CENTRED.
-template <bool CENTRED>
-MOE_DEVINL void q3_codes(uint32_t P, uint32_t P2, const Magic& M, uint32_t* q) {
-    const uint32_t P9 = P >> 9, P10 = P2 >> 10;
-    q[0] = hsub2u(field_or<0x00070007u>(P, M.m1024), CENTRED ? M.s1028 : M.m1024);
-    q[1] = hsub2u(field_or<0x00380038u>(P, M.m128), CENTRED ? M.s132 : M.m128);
-    q[2] = hsub2u(field_or<0x01C001C0u>(P, M.m16), CENTRED ? M.s20 : M.m16);
-    q[3] = hsub2u(field_or<0x00070007u>(P9, M.m1024), CENTRED ? M.s1028 : M.m1024);
-    q[4] = hsub2u(field_or<0x00380038u>(P9, M.m128), CENTRED ? M.s132 : M.m128);
-    q[5] = hsub2u(field_or<0x03800380u>(P2, M.m8), CENTRED ? M.s12 : M.m8);
-    q[6] = hsub2u(field_or<0x00070007u>(P10, M.m1024), CENTRED ? M.s1028 : M.m1024);
-    q[7] = hsub2u(field_or<0x00380038u>(P10, M.m128), CENTRED ? M.s132 : M.m128);
-}
-
-// One 32-weight block (12 code bytes = words c0, c1, c2) of a 3-bit format:
-// group 0 = stream bytes 0..5, group 1 = bytes 6..11.
-template <bool CENTRED>
-MOE_DEVINL void q3_block_codes(uint32_t c0, uint32_t c1, uint32_t c2, const Magic& M, uint32_t* q) {
-    q3_codes<CENTRED>(__byte_perm(c0, c1, 0x4310), __byte_perm(c0, c1, 0x5421), M, q);
-    q3_codes<CENTRED>(__byte_perm(c1, c2, 0x6532), __byte_perm(c1, c2, 0x7643), M, q + 8);
-}
-
 // ---------------------------------------------------------------- grouped GEMM
 struct GemmParams {
     const int4* tiles;
@@ -507,6 +412,8 @@ struct GemmParams {
     int D, F;
     int rps;                     // dequant rounds per code stage (4, 2 or 1: K / 128 is a multiple)
     uint32_t* err;
+    uint32_t* dump;              // test hook, normally null: the A operand of tile dump_tile as read
+    int dump_tile;               // back from TMEM, [K / 128 rounds][128 rows][64 f16x2 words]
 };
 
 template <int FMT>
@@ -533,7 +440,11 @@ constexpr uint32_t kBStepBytes = (uint32_t)kNmax * kKStep * 2;     // one k-step
 constexpr uint32_t kBStageBytes = 2 * kBStepBytes;                  // a round: two k-steps
 constexpr int kCodeSlots = 2;             // code stages of up to 4 rounds (K = 512)
 constexpr uint32_t kCodeSlotBytes = 32768;
-constexpr uint32_t kGemmSmem = kCodeSlots * kCodeSlotBytes + kABufs * kBStageBytes;
+// The row operand lives in a byte ring: each round takes npad * 256 bytes (two
+// k-steps of npad rows x 128 bytes), so small tiles prefetch many rounds ahead.
+constexpr uint32_t kBRingBytes = kABufs * kBStageBytes;
+constexpr int kBSlots = 32;               // rounds of the row operand in flight, at most
+constexpr uint32_t kGemmSmem = kCodeSlots * kCodeSlotBytes + kBRingBytes;
 static_assert(kACol0 + kABufs * kABufCols == 512, "TMEM columns");
 
 // Warp roles: 0..15 dequantise (warp w owns TMEM lanes 32 (w % 4) ..; the four
@@ -552,10 +463,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     using Fm = GemmFmt<FMT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_c[kCodeSlots], empty_c[kCodeSlots];
-    // round slot i (= round % 4): its TMEM A buffer and its row-operand stage are
-    // filled under round_full[i] (the 4 dequant warps of the round arrive, the
-    // row-operand TMA arrives with its byte count) and released by round_empty[i]
+    // round slot i (= round % 4): its TMEM A buffer is filled under round_full[i]
+    // (the 4 dequant warps of the round arrive) and released by round_empty[i];
+    // the round's row operand (ring slot round % kBSlots, at byte b_off of the
+    // ring) lands under b_full and is released by b_free
     __shared__ uint64_t round_full[kABufs], round_empty[kABufs];
+    __shared__ uint64_t b_full[kBSlots], b_free[kBSlots];
+    __shared__ uint32_t b_off[kBSlots], b_use[kBSlots];
     __shared__ uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain_bar;
     __shared__ uint32_t tmem_base;
     __shared__ float gate_x[kGateRows][17];        // epilogue: gate values handed to the up lanes
@@ -576,8 +490,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&empty_c[s], 4 * rps);    // the 4 quadrant warps of each of its rounds
         }
         for (int s = 0; s < kABufs; ++s) {
-            mbar_init(&round_full[s], 5);
+            mbar_init(&round_full[s], 4);
             mbar_init(&round_empty[s], 1);
+        }
+        for (int s = 0; s < kBSlots; ++s) {
+            mbar_init(&b_full[s], 1);
+            mbar_init(&b_free[s], 1);
         }
         for (int s = 0; s < kAccBufs; ++s) {
             mbar_init(&acc_full[s], 1);
@@ -637,7 +555,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty_c[cslot]);
                 // Q3_S256: the super-block's sub-scales and d, straight from global memory
-                float sd = 0.f;
+                uint32_t d2 = 0;
                 uint32_t sub0 = 0, sub1 = 0, sub2 = 0;
                 if constexpr (FMT == MOE_Q3_S256) {
                     const int pm = MODE == 1 ? (r >> 6) : 2;                   // plane: gate, up, down
@@ -649,7 +567,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     sub0 = __ldg(reinterpret_cast<const uint32_t*>(sp));
                     sub1 = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
                     sub2 = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
-                    sd = f16_bits_to_f32(__ldg(reinterpret_cast<const uint16_t*>(base + 3 * blocks * 12) + pm * blocks + sb));
+                    const uint32_t db = __ldg(reinterpret_cast<const uint16_t*>(base + 3 * blocks * 12) + pm * blocks + sb);
+                    d2 = db | (db << 16);
                 }
                 const int buf = par, use = gr >> 2;
                 const uint32_t col0 = (uint32_t)(kACol0 + buf * kABufCols);
@@ -657,25 +576,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int b = 0; b < 4; ++b) {
                     uint32_t o[16];
                     if constexpr (FMT == MOE_Q2_32) {
-                        const uint32_t s2 = __byte_perm(sw[b], 0, 0x1010), m2 = __byte_perm(sw[b], 0, 0x3232);
-                        dq_q2_group(cw[2 * b], s2, m2, Mg, o);
-                        dq_q2_group(cw[2 * b + 1], s2, m2, Mg, o + 8);
-                    } else if constexpr (FMT == MOE_Q3_32) {
-                        const uint32_t s2 = __byte_perm(sw[b], 0, 0x1010), m2 = __byte_perm(sw[b], 0, 0x3232);
-                        q3_block_codes<false>(cw[3 * b], cw[3 * b + 1], cw[3 * b + 2], Mg, o);
+                        const uint32_t s2 = bcast_lo(sw[b]), m2 = bcast_hi(sw[b]);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) o[i] = hfma2u(s2, o[i], m2);
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t w = cw[2 * b + h], w10 = w >> 10;
+                            o[8 * h + 0] = w_sm(q2_codes<0>(w, w10, Mg), s2, m2);
+                            o[8 * h + 1] = w_sm(q2_codes<1>(w, w10, Mg), s2, m2);
+                            o[8 * h + 2] = w_sm(q2_codes<2>(w, w10, Mg), s2, m2);
+                            o[8 * h + 3] = w_sm(q2_codes<3>(w, w10, Mg), s2, m2);
+                            o[8 * h + 4] = w_sm(q2_codes<4>(w, w10, Mg), s2, m2);
+                            o[8 * h + 5] = w_sm(q2_codes<5>(w, w10, Mg), s2, m2);
+                            o[8 * h + 6] = w_sm(q2_codes<6>(w, w10, Mg), s2, m2);
+                            o[8 * h + 7] = w_sm(q2_codes<7>(w, w10, Mg), s2, m2);
+                        }
                     } else {
-                        // sub-blocks 2c and 2c + 1 of the super-block, c = 32-weight chunk (0..7)
-                        const int c = 4 * (rr & 1) + b;
-                        const uint64_t lo = ((uint64_t)sub1 << 32) | sub0, hi = ((uint64_t)sub2 << 32) | sub1;
-                        const uint32_t bits = c < 4 ? (uint32_t)(lo >> (12 * c)) : (uint32_t)(hi >> (12 * c - 32));
-                        const float S0 = sd * (float)((int)(bits & 63u) - 32);
-                        const float S1 = sd * (float)((int)((bits >> 6) & 63u) - 32);
-                        const uint32_t S0h = pack_f16x2(S0, S0), S1h = pack_f16x2(S1, S1);
-                        q3_block_codes<true>(cw[3 * b], cw[3 * b + 1], cw[3 * b + 2], Mg, o);
+                        uint32_t s2 = 0, m2 = 0, sc2[2] = {0, 0};
+                        if constexpr (FMT == MOE_Q3_32) {
+                            s2 = bcast_lo(sw[b]);
+                            m2 = bcast_hi(sw[b]);
+                        } else {
+                            // sub-blocks 2c and 2c + 1 of the super-block, c = 32-weight chunk (0..7)
+                            const int c = 4 * (rr & 1) + b;
+                            const uint64_t lo = ((uint64_t)sub1 << 32) | sub0, hi = ((uint64_t)sub2 << 32) | sub1;
+                            const uint32_t bits = c < 4 ? (uint32_t)(lo >> (12 * c)) : (uint32_t)(hi >> (12 * c - 32));
+                            sc2[0] = s256_sub(bits & 63u);
+                            sc2[1] = s256_sub((bits >> 6) & 63u);
+                        }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) o[i] = hmul2u(i < 8 ? S0h : S1h, o[i]);
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t P, P2;
+                            q3_group_words(cw[3 * b], cw[3 * b + 1], cw[3 * b + 2], h, P, P2);
+                            const uint32_t P9 = P >> 9, P10 = P2 >> 10;
+                            if constexpr (FMT == MOE_Q3_32) {
+                                o[8 * h + 0] = w_sm(q3_codes<0, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 1] = w_sm(q3_codes<1, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 2] = w_sm(q3_codes<2, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 3] = w_sm(q3_codes<3, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 4] = w_sm(q3_codes<4, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 5] = w_sm(q3_codes<5, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 6] = w_sm(q3_codes<6, false>(P, P9, P2, P10, Mg), s2, m2);
+                                o[8 * h + 7] = w_sm(q3_codes<7, false>(P, P9, P2, P10, Mg), s2, m2);
+                            } else {
+                                o[8 * h + 0] = w_s256(q3_codes<0, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 1] = w_s256(q3_codes<1, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 2] = w_s256(q3_codes<2, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 3] = w_s256(q3_codes<3, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 4] = w_s256(q3_codes<4, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 5] = w_s256(q3_codes<5, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 6] = w_s256(q3_codes<6, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                                o[8 * h + 7] = w_s256(q3_codes<7, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                            }
+                        }
                     }
                     if (b == 0 && use > 0) {
                         if (!mbar_wait(&round_empty[buf], (use - 1) & 1, g.err)) { ok = false; break; }
@@ -686,6 +637,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 if (!ok) break;
                 tmem_st_wait();
+                if (g.dump != nullptr && tile == g.dump_tile) {
+                    // test hook: read the round's A operand back from TMEM as the MMAs see it
+                    uint32_t* drow = g.dump + ((size_t)rr * kTileM + r) * 64;
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t v[16];
+                        tmem_ld16(lane_addr + col0 + (uint32_t)(16 * b), v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) drow[16 * b + i] = v[i];
+                    }
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&round_full[buf]);
@@ -791,37 +754,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
     } else if (!dead && warp == kGatherWarp) {
         // ---------------- row operand (K-major, 128B swizzle) by TMA: the tile's rows are
-        // contiguous (group order), read as boxes of 128 / 64 / 32 / 16 rows
+        // contiguous (group order), read as boxes of 128 / 64 / 32 / 16 rows into the
+        // byte ring; a round that does not fit before the ring's end starts at 0
         if (lane == 0) {
             const uint64_t pol = l2_evict_last();
             bool ok = true;
-            int issued = 0;
+            int issued = 0, tail = 0;
+            uint32_t head = 0, used = 0;
             for (int tile = first, h = 0; tile < n_tiles && ok; tile += step) {
                 const int4 td = __ldg(g.tiles + tile);
                 const int row0 = td.x, npad = (td.y + 15) & ~15;
+                const uint32_t nb = (uint32_t)npad * 256u;          // two k-steps of npad rows
                 for (int rr = 0; rr < R; ++rr, ++h) {
-                    const int st = h & 3;
-                    if (h >= kABufs && !mbar_wait(&round_empty[st], ((h >> 2) - 1) & 1, g.err)) { ok = false; break; }
-                    const uint32_t b_base = smem_u32(b_ring + st * kBStageBytes);
-                    mbar_arrive_expect_tx(&round_full[st], 2u * (uint32_t)npad * kKStep * 2);
+                    const uint32_t pad = head + nb > kBRingBytes ? kBRingBytes - head : 0u;
+                    // free the oldest rounds until the bytes and a slot are available
+                    while (kBRingBytes - used < pad + nb || h - tail >= kBSlots) {
+                        if (!mbar_wait(&b_free[tail % kBSlots], (tail / kBSlots) & 1, g.err)) { ok = false; break; }
+                        used -= b_use[tail % kBSlots];
+                        ++tail;
+                    }
+                    if (!ok) break;
+                    const uint32_t off = pad ? 0u : head;
+                    head = off + nb;
+                    used += pad + nb;
+                    const int bs = h % kBSlots;
+                    b_use[bs] = pad + nb;
+                    b_off[bs] = off;
+                    mbar_arrive_expect_tx(&b_full[bs], nb);
+                    const uint32_t b_base = smem_u32(b_ring + off);
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const int x = (2 * rr + j) * kKStep;
-                        const uint32_t dst = b_base + j * kBStepBytes;
+                        const uint32_t dst = b_base + (uint32_t)j * (uint32_t)npad * 128u;
                         for (int n = 0; n < npad;) {
                             const int left = npad - n;
                             const CUtensorMap* m = left >= 128 ? &rows128 : left >= 64 ? &rows64 : left >= 32 ? &rows32 : &rows16;
-                            const int nb = left >= 128 ? 128 : left >= 64 ? 64 : left >= 32 ? 32 : 16;
-                            tma_load_2d(dst + n * 128, m, x, row0 + n, &round_full[st], pol);
-                            n += nb;
+                            const int nbx = left >= 128 ? 128 : left >= 64 ? 64 : left >= 32 ? 32 : 16;
+                            tma_load_2d(dst + n * 128, m, x, row0 + n, &b_full[bs], pol);
+                            n += nbx;
                         }
                     }
                     issued = h + 1;
                 }
             }
-            // every issued stage completes before the CTA exits
-            for (int j = issued - kABufs; j < issued; ++j)
-                if (j >= 0) mbar_drain(&round_full[j & 3], (j >> 2) & 1);
+            // every issued copy lands before the CTA exits
+            for (int j = issued - kBSlots; j < issued; ++j)
+                if (j >= 0) mbar_drain(&b_full[j % kBSlots], (j / kBSlots) & 1);
         }
         __syncwarp();
     } else if (!dead && warp == kMmaWarp) {
@@ -843,19 +821,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int rr = 0; rr < R; ++rr) {
                     const int gr = li * R + rr;
                     const int buf = gr & 3;
-                    if (!mbar_wait(&round_full[buf], (gr >> 2) & 1, g.err)) { ok = false; break; }
+                    const int bs = gr % kBSlots;
+                    if (!mbar_wait(&round_full[buf], (gr >> 2) & 1, g.err) ||
+                        !mbar_wait(&b_full[bs], (gr / kBSlots) & 1, g.err)) { ok = false; break; }
                     tc_fence_after();
                     // descriptor start addresses advance in 16-byte units
-                    const uint64_t bd = bdesc0 + (uint64_t)((buf * kBStageBytes) >> 4);
+                    const uint64_t bd = bdesc0 + (uint64_t)(b_off[bs] >> 4);
+                    const uint32_t kstep = (uint32_t)npad * 128u;
                     const uint32_t at = tmem + (uint32_t)(kACol0 + buf * kABufCols);
 #pragma unroll
                     for (int j = 0; j < 2; ++j)
 #pragma unroll
                         for (int kk = 0; kk < kKStep / 16; ++kk)
-                            mma_ts(d_tmem, at + (uint32_t)(j * 32 + kk * 8), bd + (uint64_t)((j * kBStepBytes + kk * 32) >> 4),
+                            mma_ts(d_tmem, at + (uint32_t)(j * 32 + kk * 8), bd + (uint64_t)((j * kstep + kk * 32) >> 4),
                                    idesc, (rr > 0 || j > 0 || kk > 0) ? 1u : 0u);
                     issued = true;
-                    mma_commit(&round_empty[buf]);     // frees the round's A buffer and row stage
+                    mma_commit(&round_empty[buf]);     // frees the round's A buffer
+                    mma_commit(&b_free[bs]);           // and its row operand
                 }
                 if (ok) mma_commit(&acc_full[ab]);
             }
@@ -971,6 +953,7 @@ moe_status launch_gemms(const PoolView& P, const PrefillWs& w, uint16_t* yrows, 
     GemmParams a1;
     a1.tiles = w.tiles1; a1.n_tiles = w.meta + 1; a1.dst = w.h;
     a1.scales = P.scales; a1.stride_s = P.stride_s; a1.D = P.D; a1.F = P.F; a1.err = w.err;
+    a1.dump = nullptr; a1.dump_tile = -1;
     const uint64_t rows = (uint64_t)T * (k + 1);
     moe_status st = launch_gemm<FMT, 1>(P, a1, w.xg, rows, (int)sz.max_t1, s);
     if (st != MOE_OK) return st;
@@ -979,7 +962,45 @@ moe_status launch_gemms(const PoolView& P, const PrefillWs& w, uint16_t* yrows, 
     return launch_gemm<FMT, 2>(P, a2, w.h, rows, (int)sz.max_t2, s);
 }
 
+template <int FMT>
+moe_status launch_operand_dump(const PoolView& P, int gemm, int slot, int m0, uint32_t* dump, void* ws, cudaStream_t s) {
+    // ws: [0, 1024) error word + tile list + count, then a zero row operand of
+    // 128 rows x max(D, F) fp16 (every row box of the tensor maps fits), then 16
+    // rows of output
+    char* p = reinterpret_cast<char*>(ws);
+    const int Kmax = P.D > P.F ? P.D : P.F;
+    uint16_t* src = reinterpret_cast<uint16_t*>(p + 1024);
+    uint16_t* dst = reinterpret_cast<uint16_t*>(p + 1024 + (size_t)128 * Kmax * 2);
+    int4* tiles = reinterpret_cast<int4*>(p + 256);
+    int32_t* count = reinterpret_cast<int32_t*>(p + 512);
+    const int4 td = make_int4(0, 16, m0, slot);
+    const int32_t one = 1;
+    if (cudaMemsetAsync(p, 0, 1024 + (size_t)128 * Kmax * 2, s) != cudaSuccess ||
+        cudaMemcpyAsync(tiles, &td, sizeof(td), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(count, &one, sizeof(one), cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    GemmParams a;
+    a.tiles = tiles; a.n_tiles = count; a.dst = dst;
+    a.scales = P.scales; a.stride_s = P.stride_s; a.D = P.D; a.F = P.F;
+    a.err = reinterpret_cast<uint32_t*>(p + 4);
+    a.dump = dump; a.dump_tile = 0;
+    return gemm == 1 ? launch_gemm<FMT, 1>(P, a, src, 128, 1, s) : launch_gemm<FMT, 2>(P, a, src, 128, 1, s);
+}
+
 }  // namespace
+
+size_t prefill_operand_dump_ws_bytes(int D, int F) { return 1024 + (size_t)144 * (D > F ? D : F) * 2; }
+
+moe_status launch_prefill_operand_dump(const PoolView& P, int gemm, int slot, int m0, uint32_t* dump, void* ws,
+                                       cudaStream_t s) {
+    if (P.F % kRoundK || P.D % kRoundK) return MOE_ERR_UNSUPPORTED;
+    if (!encode_tiled()) return MOE_ERR_CUDA;
+    switch (P.fmt) {
+        case MOE_Q2_32: return launch_operand_dump<MOE_Q2_32>(P, gemm, slot, m0, dump, ws, s);
+        case MOE_Q3_32: return launch_operand_dump<MOE_Q3_32>(P, gemm, slot, m0, dump, ws, s);
+        default: return launch_operand_dump<MOE_Q3_S256>(P, gemm, slot, m0, dump, ws, s);
+    }
+}
 
 size_t prefill_workspace_bytes(int T, int D, int F, int E, int k) { return ws_sizes(T, D, F, E, k).total; }
 

@@ -13,7 +13,8 @@
 
 namespace moe {
 
-// Decode route (T <= 4): one warp per expert computes its logits for all T
+// Decode route (T <= 8, x staged in shared memory): one warp per expert
+// computes its logits for all T
 // tokens, then the last block to finish selects every token's top-k.  The
 // block counter lives in ws and wraps back to zero on every completed launch.
 // Wr is not produced by the preceding kernel: one bulk copy brings the block's
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
         for (int i = threadIdx.x; i < T * k; i += blockDim.x) { ids[i] = -1; gates[i] = 0.f; }
         return;
     }
-    if (warp < T) topk_warp(logits + (size_t)warp * E, E, k, ids + (size_t)warp * k, gates + (size_t)warp * k);
+    for (int t = warp; t < T; t += 4) topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, gates + (size_t)t * k);
 }
 
 moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, const float* bias, int E,
@@ -93,23 +94,31 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
     uint32_t* rerr = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
     float* lg = logits ? logits : reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256);
     cudaError_t e;
-    if (T <= kDecodeMaxT) {
+    if (T <= kRouteDecodeMaxT && (size_t)(4 * T + 8) * D <= kRouteDecodeSmem) {
         const dim3 grid((E + 3) / 4), block(128);
         const size_t smem = (size_t)T * D * sizeof(float) + (size_t)4 * D * sizeof(uint16_t);
         static std::atomic<uint64_t> attr{0};
         if (!once_per_device(attr, [] {
-                const int b = 192 * 1024;
+                const int b = (int)kRouteDecodeSmem;
                 return cudaFuncSetAttribute(route_decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
                        cudaFuncSetAttribute(route_decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
                        cudaFuncSetAttribute(route_decode_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
-                       cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess;
+                       cudaFuncSetAttribute(route_decode_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<5>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<7>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess &&
+                       cudaFuncSetAttribute(route_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess;
             }))
             return MOE_ERR_CUDA;
         switch (T) {
             case 1: e = launch_pdl(route_decode_kernel<1>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
             case 2: e = launch_pdl(route_decode_kernel<2>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
             case 3: e = launch_pdl(route_decode_kernel<3>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            default: e = launch_pdl(route_decode_kernel<4>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            case 4: e = launch_pdl(route_decode_kernel<4>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            case 5: e = launch_pdl(route_decode_kernel<5>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            case 6: e = launch_pdl(route_decode_kernel<6>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            case 7: e = launch_pdl(route_decode_kernel<7>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+            default: e = launch_pdl(route_decode_kernel<8>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
         }
         return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }

@@ -26,7 +26,8 @@ MOE_Q2_32, MOE_Q3_32, MOE_Q3_S256 = 0, 1, 2
 EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_size", "moe_workspace_size",
            "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
            "moe_status_string", "moe_route_topk_static", "moe_expert_hist", "moe_cache_plan", "moe_slot_fill",
-           "moe_workspace_status", "moe_debug_wait_flag"]
+           "moe_workspace_status", "moe_debug_wait_flag", "moe_debug_operand_workspace_size",
+           "moe_debug_prefill_operand"]
 
 
 class MoeError(RuntimeError):
@@ -82,6 +83,10 @@ def lib():
         L.moe_workspace_status.argtypes = [P, P]
         L.moe_debug_wait_flag.restype = i
         L.moe_debug_wait_flag.argtypes = [P, ctypes.c_uint32, ctypes.c_uint32, P, P]
+        L.moe_debug_operand_workspace_size.restype = sz
+        L.moe_debug_operand_workspace_size.argtypes = [i, i]
+        L.moe_debug_prefill_operand.restype = i
+        L.moe_debug_prefill_operand.argtypes = [ctypes.POINTER(moe_pool), i, i, i, P, P, sz, P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [i]
         _lib = L
@@ -173,6 +178,17 @@ def moe_debug_wait_flag(flag, expect, limit_us, ws, stream=None):
     """Test hook: a bounded device wait for flag[0] == expect (flag: int32/uint32 device tensor)."""
     _check("moe_debug_wait_flag", lib().moe_debug_wait_flag(_p(flag), int(expect), int(limit_us), _p(ws),
                                                             _stream(stream)))
+
+
+def moe_debug_prefill_operand(pool: moe_pool, gemm, slot, m0, dump, stream=None):
+    """Test hook: the dequantised A operand of one prefill GEMM tile as read back
+    from tensor memory.  dump: uint32 device tensor of K/128 * 128 * 64 words."""
+    nb = int(lib().moe_debug_operand_workspace_size(pool.d_model, pool.d_ff))
+    ws = alloc_ws(nb, dump.device)
+    _check("moe_debug_prefill_operand", lib().moe_debug_prefill_operand(ctypes.byref(pool), int(gemm), int(slot),
+                                                                        int(m0), _p(dump), _p(ws), nb,
+                                                                        _stream(stream)))
+    return ws
 
 
 def moe_dequantize(pool: moe_pool, slot, matrix, out, stream=None):

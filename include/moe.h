@@ -34,8 +34,12 @@
  *  - Results are deterministic: no floating-point atomics, fixed summation
  *    orders; two identical calls give identical bits.
  *  - T == 0 is valid and launches nothing (miss_count is still zeroed).
- *  - Path: T <= 4 is the decode path (1 token + up to 3 draft tokens);
- *    T > 4 is the prefill path.  Both compute the same function.
+ *  - Paths: the expert pass (moe_expert_forward) runs its decode path for
+ *    T <= 8 (one token + up to 7 MTP draft tokens) and its prefill path for
+ *    T > 8; the router (moe_route_topk) runs its decode path (CUDA cores)
+ *    for T <= 8 when (4 T + 8) D <= 196608 (every T <= 4; T = 8 up to
+ *    D = 4864) and its prefill path (tensor cores) otherwise.  All paths
+ *    compute the same function.
  *  - Kernels are launched with programmatic dependent launch: each may start
  *    while the previous kernel on the stream is finishing, and waits for it
  *    before reading the activations, ids, gates or expert_out it may have
@@ -114,6 +118,11 @@ typedef struct moe_pool {
  * Shape limits (MOE_ERR_UNSUPPORTED otherwise):
  *   D % 256 == 0, 256 <= D <= 8192;  F % 128 == 0, 128 <= F <= 4096 (Q3_S256:
  *   F % 256 == 0);  1 <= k <= 16;  k <= E <= 1024;  0 <= T <= 65536.
+ *   The expert pass's decode path (T <= 8) also keeps x (8 D bytes; 16 D for
+ *   T > 4), two copies of h (16 F bytes; 32 F for T > 4) and at least two
+ *   pipeline stages of 16 weight rows in 220 KB of shared memory per SM; the
+ *   largest shapes do not fit and return MOE_ERR_UNSUPPORTED from
+ *   moe_expert_forward (every shape with D + F <= 4096 fits).
  */
 
 /* Bytes of one slot's codes / scale data (unpadded). */
@@ -136,8 +145,9 @@ size_t moe_expert_out_size(int T, int D, int k);
  *          equal logits: lower id first)
  *   gates  fp32 [T][k] out: exp(l_r - l_0) / sum_{r'<k} exp(l_r' - l_0)
  *          (reading: softmax restricted to the selected experts; sums to 1)
- *   logits fp32 [T][E] out, or NULL.  Decode path: the canonical-order
- *          values below.  Prefill path: tensor-core values within the bound
+ *   logits fp32 [T][E] out, or NULL.  Decode path of the router: the
+ *          canonical-order values below.  Prefill path: tensor-core values
+ *          within the bound
  *          |l - canonical| <= 2^-12 * |x_t|_2 * |Wr_e|_2 (D <= 8192); the ids
  *          and gates always come from the canonical values.
  *   ws     device scratch of moe_route_workspace_size bytes, 256-byte
@@ -203,22 +213,21 @@ moe_status moe_route_topk_static(const uint16_t* x, int T, int D, const uint16_t
  *            bit 0 (MOE_ERR_TIMEOUT): a bounded device wait gave up; the
  *              call's outputs are not valid, and every later call on this ws
  *              does no work until the caller zeroes its first 1024 bytes;
- *            bit 1 (MOE_ERR_RANGE, prefill path only): some x or h value has
- *              magnitude >= 65520, which the fp16 tensor-core operands cannot
- *              hold; the output rows of those tokens are not valid, the other
- *              rows are, and later calls are not affected (the bit stays set
- *              until the caller clears it).
+ *            bit 1 (MOE_ERR_RANGE): some x or h value has magnitude >= 65520,
+ *              which the fp16 tensor-core operands cannot hold; the output
+ *              rows of those tokens are not valid, the other rows are, and
+ *              later calls are not affected (the bit stays set until the
+ *              caller clears it).
  * Per expert (reading; the pages do not give the FFN form):
  *   h = bf16( silu(Wg x) * (Wu x) ),  y = Wd h,  fp32 accumulation.
  * Missed experts are not computed.
- * Operand precision.  Decode path (T <= 4): the inner products consume the
- * codes directly, s * sum(q x) + m * sum(x) in fp32, without forming weights.
- * Prefill path (T > 4): the tensor cores take fp16 operands.  Each weight is
- * formed in fp16 arithmetic: Q2_32/Q3_32 fp16(s*q + m) (one rounding);
- * Q3_S256 fp16( fp16(d*(sc-32)) * (q-4) ) (two roundings); x and h (bf16
- * values) convert to fp16 exactly when their magnitude is below 65520.
- * Outputs of both paths are within the relative L2 bound of 1e-2 per token of
- * the exact-weight result.
+ * Operand precision (both paths): the tensor cores take fp16 operands with
+ * fp32 accumulation.  Each weight is the exact weight of its block format
+ * rounded once to fp16 (round to nearest even; see moe_debug_prefill_operand);
+ * x and h (bf16 values) convert to fp16 exactly when their magnitude is below
+ * 65520 (bit 1 of the error word otherwise).  Q3_S256 pools also need
+ * |d*(sc-32)| < 65504.  Outputs are within the relative L2 bound of 1e-2 per
+ * token of the exact-weight result.
  */
 moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, int E,
                               const uint16_t* x, int T, const int32_t* ids, int k,
@@ -266,6 +275,26 @@ moe_status moe_workspace_status(const void* ws, moe_stream_t stream);
  */
 moe_status moe_debug_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t limit_us, void* ws,
                                moe_stream_t stream);
+
+/*
+ * Test hook: the weight operand of one tile of the prefill path's tensor-core
+ * GEMM, exactly as the MMAs read it.  Runs the prefill GEMM kernel on a single
+ * tile of `slot` (against zero rows) and copies its dequantised A operand back
+ * out of tensor memory after each K = 128 round.
+ *   gemm 1 (gate|up): A rows 0..63 are gate features m0..m0+63 and rows
+ *          64..127 the up features m0..m0+63 (m0 % 64 == 0, m0 < d_ff), K = d_model;
+ *   gemm 2 (down): A rows are output features m0..m0+127 (m0 % 128 == 0,
+ *          m0 < d_model), K = d_ff.
+ *   dump   uint32 [K / 128][128][64] (device): word 16b + i of row r in round
+ *          rr holds the fp16 pair (lo, hi) of weights K0 + (i & 7) and
+ *          K0 + (i & 7) + 8, with K0 = 128 rr + 32 b + 16 (i >> 3).
+ *   ws     device scratch of moe_debug_operand_workspace_size bytes, 256-byte
+ *          aligned (overwritten).
+ * Each fp16 weight is the exact weight (moe_dequantize) rounded once to fp16.
+ */
+size_t moe_debug_operand_workspace_size(int d_model, int d_ff);
+moe_status moe_debug_prefill_operand(const moe_pool* pool, int gemm, int slot, int m0, uint32_t* dump, void* ws,
+                                     size_t ws_bytes, moe_stream_t stream);
 
 /* Static text for a status code. */
 const char* moe_status_string(moe_status s);

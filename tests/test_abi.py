@@ -142,3 +142,17 @@ def test_status_query_and_wait_hook_argument_errors(L):
     assert L.moe_debug_wait_flag(f, 1, 1000, None, None) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_debug_wait_flag(f, 1, 0, f, None) == moe.MOE_ERR_INVALID_ARG             # no limit
     assert L.moe_debug_wait_flag(f, 1, 2000000, f, None) == moe.MOE_ERR_INVALID_ARG       # above 1 s
+
+
+def test_operand_hook_argument_errors(L):
+    f = _fake()
+    assert L.moe_debug_operand_workspace_size(3072, 512) > 128 * 3072 * 2
+    op = lambda pool=_pool(), gemm=1, slot=0, m0=0, dump=f, ws=f, nb=1 << 30: L.moe_debug_prefill_operand(
+        ctypes.byref(pool), gemm, slot, m0, dump, ws, nb, None)
+    assert op(gemm=3) == moe.MOE_ERR_INVALID_ARG
+    assert op(slot=4) == moe.MOE_ERR_INVALID_ARG
+    assert op(m0=32) == moe.MOE_ERR_INVALID_ARG            # gate|up tiles start at multiples of 64
+    assert op(gemm=2, m0=64) == moe.MOE_ERR_INVALID_ARG    # down tiles start at multiples of 128
+    assert op(m0=512) == moe.MOE_ERR_INVALID_ARG           # beyond d_ff
+    assert op(dump=None) == moe.MOE_ERR_INVALID_ARG
+    assert op(nb=64) == moe.MOE_ERR_WORKSPACE

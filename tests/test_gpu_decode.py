@@ -1,4 +1,4 @@
-"""GPU parity of the decode path (T <= 4) against the CPU oracle, called through
+"""GPU parity of the decode path (T <= 8) against the CPU oracle, called through
 the C ABI.  Bars: routing ids, miss lists and dequantised weights bit-exact;
 decode-path logits bit-exact (same canonical order); gates within 1e-6
 relative (the GPU forms them in double and rounds once to fp32, the oracle
@@ -37,7 +37,9 @@ def _check_layer(wl, x, layer_idx=0, miss_partial=None, residual=None, k=None):
     ref = oracle_layer(wl.pool, L, k, u16(x),
                        miss_partial=None if miss_partial is None else miss_partial.cpu().numpy(),
                        residual_bits=None if residual is None else u16(residual))
-    assert np.array_equal(layer.logits.cpu().numpy().view(np.uint32), ref.logits.view(np.uint32))
+    T, D = x.shape
+    if T <= 8 and (4 * T + 8) * D <= 196608:   # the CUDA-core router returns the canonical logits themselves
+        assert np.array_equal(layer.logits.cpu().numpy().view(np.uint32), ref.logits.view(np.uint32))
     assert np.array_equal(layer.ids.cpu().numpy(), ref.ids)
     g = layer.gates.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(g - ref.gates) <= TOL_GATE * np.abs(ref.gates))
@@ -54,7 +56,7 @@ def test_tiny_parity():
     _check_layer(wl, wl.x)
 
 
-@pytest.mark.parametrize("T", [1, 2, 3, 4])
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 6, 8])
 def test_decode_parity(T):
     wl = _workload("decode", T=T)
     layer, ref, err = _check_layer(wl, wl.x)
@@ -170,10 +172,12 @@ def test_decode48_chain_per_layer():
     assert 0.85 < hit_rate <= 1.0
 
 
-def test_decode_65_owners():
-    """T = 4, k = 16, every selected expert distinct and resident: the shared
-    expert plus 64 routed owners, the most the decode path serves."""
-    cfg = configs.Config("edge65", 1, 256, 128, 128, 16, 4, synth.Q2_32, None, None, None, seed=3)
+@pytest.mark.parametrize("T", [4, 8])
+def test_decode_all_distinct_owners(T):
+    """k = 16, every selected expert distinct and resident: the shared expert
+    plus 64 (T = 4) or 128 (T = 8, the most the decode path serves) routed
+    owners."""
+    cfg = configs.Config("edge_owners", 1, 256, 128, 128, 16, T, synth.Q2_32, None, None, None, seed=3)
     wl = configs.build(cfg, device="cuda")
     L = wl.layers[0]
     # token t prefers experts 16t .. 16t+15 (strictly decreasing logits, no ties)
@@ -188,4 +192,4 @@ def test_decode_65_owners():
     x[:, cfg.T:] = 0.01 * torch.randn(cfg.T, cfg.D - cfg.T, generator=torch.Generator().manual_seed(5))
     x = x.to(torch.bfloat16).cuda()
     layer, ref, err = _check_layer(wl, x, k=16)
-    assert len(np.unique(ref.ids)) == 64 and int(layer.miss_count.item()) == 0
+    assert len(np.unique(ref.ids)) == 16 * T and int(layer.miss_count.item()) == 0

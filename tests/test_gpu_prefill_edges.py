@@ -1,8 +1,10 @@
 """GPU parity of the edges between and inside the two paths, against the CPU
 oracle through the C ABI:
 
-* the decode/prefill crossover: T = 5 is the smallest prefill batch; its
-  first four rows also match the decode path on the same tokens;
+* the path crossovers: T = 5 is the smallest batch of the tensor-core router
+  (the expert pass still takes its decode path), T = 9 the smallest batch of
+  the prefill expert pass; their first rows match the decode path on the same
+  tokens;
 * one expert set takes every token (router weights zero, a strictly
   decreasing bias): expert groups of 300 rows span several 128-row tiles and
   two 256-token plan chunks, on both paths;
@@ -54,14 +56,15 @@ def _check_full(wl, L, x, k, residual=None):
     return layer, out, ref
 
 
-def test_crossover_T5_prefill_path_and_decode_rows():
-    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=5, layers=1)
+@pytest.mark.parametrize("T", [5, 8, 9])
+def test_crossover_batches_and_decode_rows(T):
+    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=T, layers=1)
     L = wl.layers[0]
-    _, out5, _ = _check_full(wl, L, wl.x, wl.cfg.k)
+    _, outT, _ = _check_full(wl, L, wl.x, wl.cfg.k)
     layer4 = _layer(wl, L, wl.cfg.k, 4)
     out4 = layer4(wl.x[:4].contiguous())
     torch.cuda.synchronize()
-    assert rel_l2_per_token(u16(out5)[:4], u16(out4)).max() <= TOL_OUT
+    assert rel_l2_per_token(u16(outT)[:4], u16(out4)).max() <= TOL_OUT
 
 
 @pytest.mark.parametrize("T", [4, 300])
