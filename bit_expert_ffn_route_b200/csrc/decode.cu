@@ -121,23 +121,29 @@ struct DecodeParams {
     int32_t* miss_count;
     uint16_t* hfrag;       // [kMaxPairs][F * NSLOT] fp16, fragment order
     uint32_t* err;
-    uint32_t* done;        // [kMaxPairs + 1]: per-owner gate|up completion counters + CTA ticket
+    uint32_t* done;        // [kMaxPairs + 2]: per-owner gate|up completion counters, CTA ticket, work queue
     int rf;                // gate|up: features per item (8 or 16)
     int rd;                // down: rows per item (multiple of 16)
     int ns;                // pipeline stages
 };
 
+constexpr int kRedBufs = 3;                        // partial-sum buffers per team (items in flight)
+constexpr int kPubRing = 64;                       // finished gate|up items awaiting release
+
 struct Shared {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
+    int stage_item[kMaxStages];    // the work item in each stage (-1: no more work)
     Owner owners[kMaxPairs];
     int slot_of[kMaxPairs];
-    int table[kMaxE];          // the slot table, staged before the dependency wait
+    int table[kMaxE];              // the slot table, staged before the dependency wait
     int n_owners;
-    int abort[kTeams];         // set by a consumer team that stopped on an error
-    int d_range[2];            // this CTA's down items [d_range[0], d_range[1])
-    uint64_t range_bar;        // completes once d_range is written
-    uint32_t team_items[kTeams];   // gate|up items finished by each team (release.cta by its reducer)
+    int abort;                     // set by any warp that stopped on an error
+    uint32_t red_cnt[kTeams][kRedBufs];   // warps that wrote their partials into a buffer
+    uint32_t red_gen[kTeams][kRedBufs];   // reductions completed on a buffer
+    uint32_t pub_head;             // finished gate|up items queued for the publisher
+    int pubq[kPubRing];            // their owners + 1 (0: free; -1: no more items)
+    uint32_t finished;             // warps (consumers, producer) that are done
 };
 
 // The slot table is an input of the layer, not produced by the router: stage it
@@ -543,15 +549,6 @@ __device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int r
     }
 }
 
-MOE_DEVINL void team_sync(int team) { asm volatile("bar.sync %0, %1;" ::"r"(2 + team), "n"(kTeamWarps * 32) : "memory"); }
-// A team barrier that also returns whether v held on every thread of the team.
-MOE_DEVINL bool team_all(int team, bool v) {
-    uint32_t r;
-    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                 : "=r"(r) : "r"((uint32_t)v), "r"(2 + team), "n"(kTeamWarps * 32) : "memory");
-    return r != 0;
-}
-
 MOE_DEVINL void st_release_cta(uint32_t* p, uint32_t v) {
     asm volatile("st.release.cta.shared.u32 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(p)), "r"(v) : "memory");
 }
@@ -570,41 +567,20 @@ MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
     return v;
 }
 
-// Work is balanced by weight count: gate|up item i (n_owners * nfb of them, gw
-// weights each) runs on CTA i mod G; down items cost dw weights each, and CTA b
-// takes a contiguous range of them.  The down work before CTA b is its share
-// of all work less the gate|up work of CTAs 0 .. b-1, clamped to [0, all down
-// work]; any such sequence from 0 to the total covers every item (a decrease
-// only makes two neighbouring ranges overlap, and an overlapped item is
-// computed twice with identical results).
-MOE_DEVINL void down_range(int n, int b, int G, int nfb, long long gw, int nrb, long long dw, int& d0, int& d1) {
-    const long long ng = (long long)n * nfb, nd = (long long)n * nrb;
-    auto below = [&](long long m, int cb) {    // #{i < m : i mod G < cb}
-        const long long q = m / G, r = m % G;
-        return q * cb + (r < cb ? r : (long long)cb);
-    };
-    const long long all = ng * gw + nd * dw;
-    auto start = [&](int cb) -> long long {   // first down item of CTA cb
-        if (cb <= 0) return 0;
-        if (cb >= G) return nd;
-        long long work = (all * cb + G - 1) / G - below(ng, cb) * gw;
-        if (work < 0) work = 0;
-        const long long it = (work + dw - 1) / dw;
-        return it > nd ? nd : it;
-    };
-    d0 = (int)start(b);
-    d1 = (int)start(b + 1);
-}
-
 // ---------------------------------------------------------------- the fused kernel
-// One persistent CTA per SM.  Each CTA takes its gate|up items (round-robin),
-// then a contiguous range of down items (balancing the weights of both),
-// through one ring of stages.  A down item of owner u waits until every
-// gate|up item of u has published its h: a per-owner item counter in ws,
-// advanced by a publisher warp that releases each finished item at gpu scope,
-// off the computing warps' path.  The down weights stream in meanwhile.  The
-// last CTA to finish resets the counters, so every completed call leaves them
-// zero.
+// One persistent CTA per SM.  Work items come from one queue shared by all
+// CTAs (an atomic counter): first the gate|up items of every owner (owner by
+// owner), then the down items (owner by owner).  A CTA's producer warp takes
+// the next item whenever a stage is free, so the CTAs finish within about one
+// item of each other, and by the time a down item of owner u is taken, the
+// gate|up items of u were taken long before.  A down item needs the owner's h:
+// the producer waits for the owner's gate|up count (a per-owner counter in ws,
+// advanced at gpu scope by the publisher warp of whichever CTA finished the
+// item) and copies h into the stage after the weights.  Consumer warps never
+// wait on each other: each warp of a gate|up item adds its partial sums to the
+// team's buffer, and the last one to do so reduces them and queues the item for
+// the publisher.  The last CTA to finish resets the counters, so every
+// completed call leaves them zero.
 template <int FMT, int NSLOT>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams prm) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -612,23 +588,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = prm.P.D, F = prm.P.F, rf = prm.rf, rd = prm.rd, NS = prm.ns;
     const size_t xs_bytes = (size_t)D * NSLOT * 2;
-    const size_t hs_bytes = (size_t)F * NSLOT * 2;                               // one per team
-    const size_t red_team = (size_t)2 * kTeamWarps * red_floats<NSLOT>();        // per team, double-buffered
+    const uint32_t hbytes = (uint32_t)F * NSLOT * 2;                           // one owner's h
+    const size_t red_team = (size_t)kRedBufs * kTeamWarps * red_floats<NSLOT>();
     uint8_t* xs = smem;
-    uint8_t* hs = smem + xs_bytes;
-    float* red = reinterpret_cast<float*>(smem + xs_bytes + kTeams * hs_bytes);
-    uint8_t* stages = smem + xs_bytes + kTeams * hs_bytes + kTeams * red_team * 4;
+    float* red = reinterpret_cast<float*>(smem + xs_bytes);
+    uint8_t* stages = smem + xs_bytes + kTeams * red_team * 4;
     const uint32_t gu_bytes = 2u * Geo<FMT>::row_bytes(D) * rf;
     const uint32_t dn_bytes = (uint32_t)Geo<FMT>::row_bytes(F) * rd;
-    const uint32_t stage_bytes = gu_bytes > dn_bytes ? gu_bytes : dn_bytes;
+    const uint32_t stage_bytes = gu_bytes > dn_bytes + hbytes ? gu_bytes : dn_bytes + hbytes;
     const int nfb = F / rf, nrb = D / rd;
     uint32_t* done = prm.done;
+    uint32_t* queue = done + kMaxPairs + 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], kTeamWarps); }
-        mbar_init(&sh.range_bar, 1);
         fence_mbar_init();
-        for (int tm = 0; tm < kTeams; ++tm) { sh.abort[tm] = 0; sh.team_items[tm] = 0; }
+        sh.abort = 0;
+        sh.pub_head = 0;
+        sh.finished = 0;
+        for (int tm = 0; tm < kTeams; ++tm)
+            for (int b = 0; b < kRedBufs; ++b) { sh.red_cnt[tm][b] = 0; sh.red_gen[tm][b] = 0; }
     }
+    for (int i = threadIdx.x; i < kPubRing; i += blockDim.x) sh.pubq[i] = 0;
     // a call on a workspace whose timeout bit is set does no work (every CTA
     // still takes its ticket below, so the counters are left zero); one read,
     // shared by the whole CTA, so that every warp takes the same branch.  The
@@ -655,159 +635,185 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         asm volatile("bar.sync 1, 96;" ::: "memory");
     }
     pdl_launch_dependents();
-    // gate|up items round-robin over the CTAs; down items in contiguous ranges
-    const int n_g = sh.n_owners * nfb;
-    const int ng = n_g > (int)blockIdx.x ? (n_g - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-    // the down range is computed by the publisher warp, off the producer's path;
-    // the others wait for it only when they reach their first down item
-    int d0r = 0, d1r = 0;
-    bool have_range = false;
-    auto get_range = [&]() -> bool {
-        if (!have_range) {
-            if (!mbar_wait(&sh.range_bar, 0, prm.err)) return false;
-            d0r = sh.d_range[0];
-            d1r = sh.d_range[1];
-            have_range = true;
-        }
-        return true;
-    };
-    if (warp == kPublisherWarp) {    // publisher: the down range, then release finished gate|up items
+    const int n_g = sh.n_owners * nfb, n_all = n_g + sh.n_owners * nrb;
+    auto stopped = [&]() { return timed_out(prm.err) || *reinterpret_cast<volatile int*>(&sh.abort) != 0; };
+    if (warp == kPublisherWarp) {
+        // publisher: release each finished gate|up item to the other CTAs (one
+        // gpu-scope fence per batch, then relaxed adds to the owners' counters)
         if (lane == 0) {
-            int r0, r1;
-            down_range(sh.n_owners, (int)blockIdx.x, (int)gridDim.x, nfb, 2ll * rf * D, nrb, (long long)rd * F, r0, r1);
-            sh.d_range[0] = r0;
-            sh.d_range[1] = r1;
-            mbar_arrive(&sh.range_bar);
-            uint32_t pub[kTeams] = {0u, 0u};
-            const uint32_t want[kTeams] = {(uint32_t)((ng + 1) / 2), (uint32_t)(ng / 2)};
-            const uint64_t t0 = globaltimer_ns();
-            while (pub[0] < want[0] || pub[1] < want[1]) {
-                const uint32_t c0 = ld_acquire_cta(&sh.team_items[0]), c1 = ld_acquire_cta(&sh.team_items[1]);
-                if (c0 > pub[0] || c1 > pub[1]) {
-                    fence_acq_rel_gpu();             // with the relaxed adds below: one release per batch
-                    const uint32_t cn[kTeams] = {c0, c1};
-                    for (int tm = 0; tm < kTeams; ++tm)
-                        for (uint32_t n = pub[tm]; n < cn[tm]; ++n) {
-                            const int j = tm + kTeams * (int)n;
-                            red_relaxed_add(done + item_pos(blockIdx.x + j * gridDim.x, nfb, rf).u, 1u);
-                        }
-                    pub[0] = c0;
-                    pub[1] = c1;
-                } else {
-                    if (timed_out(prm.err) ||
-                        *reinterpret_cast<volatile int*>(&sh.abort[0]) || *reinterpret_cast<volatile int*>(&sh.abort[1]))
-                        break;
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                        atomicOr(prm.err, kErrTimeout);
-                        break;
+            uint32_t tail = 0;
+            uint64_t t0 = globaltimer_ns();
+            for (bool more = true; more;) {
+                // every item queued so far (up to 8), then one fence for the batch
+                int v[8];
+                int nb = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    v[q] = 0;
+                    if (nb == q) {
+                        v[q] = (int)ld_acquire_cta(reinterpret_cast<uint32_t*>(&sh.pubq[(tail + q) % kPubRing]));
+                        if (v[q] != 0) ++nb;
                     }
+                }
+                if (nb) {
+                    fence_acq_rel_gpu();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (q < nb) {
+                            if (v[q] > 0) red_relaxed_add(done + (v[q] - 1), 1u);
+                            else more = false;                  // the end marker
+                            st_release_cta(reinterpret_cast<uint32_t*>(&sh.pubq[(tail + q) % kPubRing]), 0u);
+                        }
+                    }
+                    tail += nb;
+                    t0 = globaltimer_ns();
+                } else {
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicOr(prm.err, kErrTimeout); break; }
                     __nanosleep(32);
                 }
             }
         }
-    } else if (warp == kProducerWarp) {    // producer: gate|up items, then down items
+    } else if (warp == kProducerWarp) {    // producer: take items from the queue, stage them
         if (lane == 0) {
-            for (int j = 0;; ++j) {
-                if (j >= ng && !get_range()) break;
-                if (j >= ng + (d1r - d0r)) break;
+            int j = 0, issued = 0;
+            bool ok = true;
+            for (;; ++j) {
                 const int s = j % NS;
-                if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) break;
-                if (*reinterpret_cast<volatile int*>(&sh.abort[0]) | *reinterpret_cast<volatile int*>(&sh.abort[1])) break;
+                if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) { ok = false; break; }
+                if (stopped()) { ok = false; break; }
+                const int idx = (int)atomicAdd(queue, 1u);
                 uint8_t* dst = stages + (size_t)s * stage_bytes;
-                if (j < ng) {
-                    const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
+                if (idx >= n_all) {                       // no more work: tell this stage's team
+                    sh.stage_item[s] = -1;
+                    mbar_arrive(&sh.full[s]);
+                    ++j;
+                    break;
+                }
+                sh.stage_item[s] = idx;
+                if (idx < n_g) {
+                    const ItemPos ip = item_pos(idx, nfb, rf);
                     const int slot = sh.owners[ip.u].slot;
                     const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * rf;
                     mbar_arrive_expect_tx(&sh.full[s], 2 * half);
                     issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 0), ip.row0, rf, D, dst, &sh.full[s]);
                     issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 1), ip.row0, rf, D, dst + half, &sh.full[s]);
                 } else {
-                    const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
-                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)Geo<FMT>::row_bytes(F) * rd);
+                    const ItemPos ip = item_pos(idx - n_g, nrb, rd);
+                    mbar_arrive_expect_tx(&sh.full[s], dn_bytes + hbytes);
                     issue_rows<FMT>(planes_of<FMT>(prm.P, sh.owners[ip.u].slot, 2), ip.row0, rd, F, dst, &sh.full[s]);
+                    // the owner's h, once every gate|up item of the owner is published
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire(done + ip.u) < (uint32_t)nfb) {
+                        if (timed_out(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
+                            atomicOr(prm.err, kErrTimeout);
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    // (after a give-up the copy still completes the stage's byte count)
+                    asm volatile("fence.proxy.async.global;" ::: "memory");   // h was written through the generic proxy
+                    bulk_g2s(dst + dn_bytes, prm.hfrag + (size_t)ip.u * F * NSLOT, hbytes, &sh.full[s]);
                 }
-            }
-        }
-    } else {
-        // consumer teams: team tm takes items j = tm, tm + 2, ... of the ring
-        const int team = warp / kTeamWarps, wt = warp % kTeamWarps;
-        const int tl = (int)threadIdx.x - team * kTeamWarps * 32;
-        uint8_t* hst = hs + (size_t)team * hs_bytes;
-        float* redt = red + (size_t)team * red_team;
-        bool ok = true;
-        int cur = -1;
-        uint32_t gu_done = 0;
-        for (int j = team;; j += kTeams) {
-            if (j >= ng) {
-                ok = team_all(team, get_range());     // the same verdict on every thread of the team
+                issued = j + 1;
                 if (!ok) break;
-                if (j >= ng + (d1r - d0r)) break;
             }
-            const int s = j % NS;
-            const uint8_t* st = stages + (size_t)s * stage_bytes;
-            if (j < ng) {
-                // partial sums of successive items alternate between two buffers:
-                // warp 0 reduces item n while the other warps start item n + 1
-                float* redb = redt + ((j / kTeams) & 1) * (kTeamWarps * red_floats<NSLOT>());
-                const bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
-                const ItemPos ip = item_pos(blockIdx.x + j * gridDim.x, nfb, rf);
-                if (got) {
-                    if (rf == 16) gateup_partial<FMT, 2, NSLOT>(prm, rf, st, xs, wt, redb + wt * red_floats<NSLOT>());
-                    else gateup_partial<FMT, 1, NSLOT>(prm, rf, st, xs, wt, redb + wt * red_floats<NSLOT>());
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.empty[s]);
-                // every warp's partials are in redb (and the verdict is the team's,
-                // so every thread leaves the loop together)
-                ok = team_all(team, got);
-                if (!ok) break;
-                if (wt == 0) {
-                    gateup_reduce<NSLOT>(prm, ip.u, ip.row0, rf, redb);
-                    __syncwarp();
-                    ++gu_done;
-                    if (lane == 0) st_release_cta(&sh.team_items[team], gu_done);
+            // the other team's next stage also learns that the work is over
+            if (ok) {
+                const int s = j % NS;
+                if (j < NS || mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) {
+                    sh.stage_item[s] = -1;
+                    mbar_arrive(&sh.full[s]);
                 }
             } else {
-                const ItemPos ip = item_pos(d0r + (j - ng), nrb, rd);
-                const int u = ip.u, r0 = ip.row0;
-                const Owner& o = sh.owners[u];
-                if (u != cur) {
-                    team_sync(team);                    // the team is done reading hst
-                    bool waited = true;
-                    if (tl == 0) {
-                        const uint32_t target = (uint32_t)nfb;   // gate|up items of owner u
-                        const uint64_t t0 = globaltimer_ns();
-                        while (ld_acquire(done + u) < target) {
-                            if (timed_out(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
-                                atomicOr(prm.err, kErrTimeout);
-                                waited = false;
-                                break;
-                            }
-                            __nanosleep(64);
+                sh.abort = 1;
+            }
+            // after a give-up, every issued copy lands before the CTA exits (on the
+            // normal path the consumers wait for each staged item themselves)
+            if (!ok)
+                for (int q = issued - NS; q < issued; ++q)
+                    if (q >= 0) mbar_drain(&sh.full[q % NS], (q / NS) & 1);
+        }
+        __syncwarp();
+        if (lane == 0 && atomicAdd(&sh.finished, 1u) == kConsumerWarps) {   // the last worker warp
+            const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
+            st_release_cta(reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]), 0xffffffffu);
+        }
+    } else {
+        // consumer teams: team tm takes stages j = tm, tm + 2, ... of the ring;
+        // the warps of a team work through the same items without waiting on
+        // each other (the last one to finish a gate|up item reduces it)
+        const int team = warp / kTeamWarps, wt = warp % kTeamWarps;
+        float* redt = red + (size_t)team * red_team;
+        uint32_t n_gu = 0;                       // gate|up items this team has seen (same order in every warp)
+        for (int j = team;; j += kTeams) {
+            const int s = j % NS;
+            if (!mbar_wait(&sh.full[s], (j / NS) & 1, prm.err)) { if (lane == 0) sh.abort = 1; break; }
+            const int idx = sh.stage_item[s];
+            if (idx < 0) break;
+            const uint8_t* st = stages + (size_t)s * stage_bytes;
+            if (idx < n_g) {
+                const ItemPos ip = item_pos(idx, nfb, rf);
+                const int b = (int)(n_gu % kRedBufs);
+                const uint32_t use = n_gu / kRedBufs;     // earlier reductions of buffer b
+                ++n_gu;
+                float* redb = redt + (size_t)b * (kTeamWarps * red_floats<NSLOT>());
+                // buffer b is free once its previous reduction is done (rarely waits)
+                bool ok = true;
+                if (lane == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_cta(&sh.red_gen[team][b]) < use) {
+                        if (stopped() || globaltimer_ns() - t0 > kWaitLimitNs) {
+                            atomicOr(prm.err, kErrTimeout);
+                            ok = false;
+                            break;
                         }
                     }
-                    ok = team_all(team, waited);
-                    if (!ok) break;
-                    // the owner's h (fragment order, written by other CTAs of this
-                    // launch): L2-coherent 16-byte copies
-                    const uint4* src = reinterpret_cast<const uint4*>(prm.hfrag + (size_t)u * F * NSLOT);
-                    for (int q = tl; q < (int)(hs_bytes / 16); q += kTeamWarps * 32)
-                        reinterpret_cast<uint4*>(hst)[q] = __ldcg(src + q);
-                    team_sync(team);
-                    cur = u;
                 }
-                const bool got = mbar_wait(&sh.full[s], (j / NS) & 1, prm.err);
-                if (got) down_item<FMT, NSLOT>(prm, o, r0, rd, st, hst, wt);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (rf == 16) gateup_partial<FMT, 2, NSLOT>(prm, rf, st, xs, wt, redb + wt * red_floats<NSLOT>());
+                else gateup_partial<FMT, 1, NSLOT>(prm, rf, st, xs, wt, redb + wt * red_floats<NSLOT>());
+                __syncwarp();
+                uint32_t prev = 0;
+                if (lane == 0) {
+                    mbar_arrive(&sh.empty[s]);
+                    asm volatile("atom.acq_rel.cta.shared.add.u32 %0, [%1], 1;"
+                                 : "=r"(prev)
+                                 : "r"((uint32_t)__cvta_generic_to_shared(&sh.red_cnt[team][b]))
+                                 : "memory");
+                }
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == kTeamWarps - 1) {            // the last warp of the item reduces it
+                    __syncwarp();                        // (orders the other warps' partials, seen by lane 0)
+                    gateup_reduce<NSLOT>(prm, ip.u, ip.row0, rf, redb);
+                    __syncwarp();
+                    if (lane == 0) {
+                        sh.red_cnt[team][b] = 0;
+                        st_release_cta(&sh.red_gen[team][b], use + 1);
+                        const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
+                        uint32_t* slot = reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]);
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_cta(slot) != 0u && globaltimer_ns() - t0 < kWaitLimitNs) {}   // ring slot free
+                        st_release_cta(slot, (uint32_t)(ip.u + 1));
+                    }
+                }
+            } else {
+                const ItemPos ip = item_pos(idx - n_g, nrb, rd);
+                down_item<FMT, NSLOT>(prm, sh.owners[ip.u], ip.row0, rd, st, st + dn_bytes, wt);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.empty[s]);
-                ok = team_all(team, got);
-                if (!ok) break;
             }
         }
-        if (!ok && tl == 0) sh.abort[team] = 1;
+        // the last worker warp to finish tells the publisher that no more items come
+        __syncwarp();
+        if (lane == 0 && atomicAdd(&sh.finished, 1u) == kConsumerWarps) {
+            const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
+            st_release_cta(reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]), 0xffffffffu);
+        }
     }
     }   // !dead
-    // last CTA out resets the per-owner counters for the next call
+    // last CTA out resets the per-owner counters and the queue for the next call
     // (acq_rel ticket: this CTA's counter updates, ordered before it by the
     // barrier, precede the reset; the last CTA sees every other CTA's)
     __syncthreads();
@@ -817,15 +823,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
         if (ticket == gridDim.x - 1) {
             for (int u = 0; u < kMaxPairs; ++u) done[u] = 0u;
             done[kMaxPairs] = 0u;
+            done[kMaxPairs + 1] = 0u;
         }
     }
 }
 
 template <int FMT, int NSLOT>
 size_t smem_for(int D, int F, int rf, int rd, int ns) {
-    const size_t fixed = (size_t)D * NSLOT * 2 + kTeams * (size_t)F * NSLOT * 2 +
-                         kTeams * (size_t)2 * kTeamWarps * red_floats<NSLOT>() * 4;
-    const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf, b = (size_t)Geo<FMT>::row_bytes(F) * rd;
+    const size_t fixed = (size_t)D * NSLOT * 2 + kTeams * (size_t)kRedBufs * kTeamWarps * red_floats<NSLOT>() * 4;
+    const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf, b = (size_t)Geo<FMT>::row_bytes(F) * rd + (size_t)F * NSLOT * 2;
     return fixed + (size_t)ns * (a > b ? a : b);
 }
 

@@ -766,7 +766,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int row0 = td.x, npad = (td.y + 15) & ~15;
                 const uint32_t nb = (uint32_t)npad * 256u;          // two k-steps of npad rows
                 for (int rr = 0; rr < R; ++rr, ++h) {
-                    const uint32_t pad = head + nb > kBRingBytes ? kBRingBytes - head : 0u;
+                    const bool wrap = head + nb > kBRingBytes;       // (head may equal kBRingBytes)
+                    const uint32_t pad = wrap ? kBRingBytes - head : 0u;
                     // free the oldest rounds until the bytes and a slot are available
                     while (kBRingBytes - used < pad + nb || h - tail >= kBSlots) {
                         if (!mbar_wait(&b_free[tail % kBSlots], (tail / kBSlots) & 1, g.err)) { ok = false; break; }
@@ -774,7 +775,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ++tail;
                     }
                     if (!ok) break;
-                    const uint32_t off = pad ? 0u : head;
+                    const uint32_t off = wrap ? 0u : head;
                     head = off + nb;
                     used += pad + nb;
                     const int bs = h % kBSlots;
