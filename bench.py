@@ -47,7 +47,7 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 EXTRA = ["prefill", "decode48", "prefill48"]
-# kernels per layer and step: decode (T <= 4) route 1, expert pass 1, combine 1;
+# kernels per layer and step: decode (T <= 8) route 1, expert pass 1, combine 1;
 # prefill route 3 (norms, tensor-core logits, selection), expert pass 6 (3
 # plan, gather, 2 GEMMs), combine 1
 LAUNCHES = {"decode": 3, "prefill": 10}
@@ -226,7 +226,7 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     pool_bytes = wl.pool.n_slots * slot_bytes
     # decode touches ~(U+1) experts + Wr (~65 MB) per step: 8 replicas put ~450 MB
     # of other traffic between two uses of one replica (L2 is 126 MB)
-    R = args.replicas or (8 if T <= 4 else 2)
+    R = args.replicas or (8 if T <= 8 else 2)
     pools, Wrs, xs = [], [], []
     for r in range(R):
         if r == 0:
@@ -258,29 +258,38 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     # every token's shared-expert row costs gate + up + down = 3 * 2 * D * F
     fwd_flops = [(h * T * k + T) * 6.0 * D * F for h in hits]
 
-    G = _divisor_at_most(K, 512 if T <= 4 else 64)
+    G = _divisor_at_most(K, 512 if T <= 8 else 64)
     ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
           for _ in range(G)]
 
-    def step(i):
+    def step(i, events=False):
         lay = layers[i % R]
         moe.moe_route_topk(xs[i % R], lay.Wr, lay.bias, k, lay.ids, lay.gates, lay.route_ws, stream=stream)
-        ev[i][0].record(stream)
+        if events:
+            ev[i][0].record(stream)
         moe.moe_expert_forward(lay.pool, lay.slot_table, xs[i % R], lay.ids, k, lay.expert_out, lay.miss_list,
                                lay.miss_count, lay.ws, stream=stream)
-        ev[i][1].record(stream)
+        if events:
+            ev[i][1].record(stream)
         moe.moe_combine(lay.expert_out, lay.gates, T, D, k, lay.out, stream=stream)
 
+    # the throughput graph has no event nodes: an event recorded between two
+    # kernels ends the programmatic-launch overlap of the second with the first
     graph = _graph_of(step, G, stream)
+    graph_ev = _graph_of(lambda i: step(i, True), G, stream)
     with torch.cuda.stream(stream):
         for _ in range(max(1, -(-W // G))):
             graph.replay()
+            graph_ev.replay()
     ms, clocks = _timed_replays(graph, K // G, stream, ws_, dev, local)
+    # the expert pass's own duration: the same steps with an event pair around
+    # each moe_expert_forward launch (so launched without the overlap)
+    _timed_replays(graph_ev, K // G, stream, ws_, dev, local, clocks=False)
     fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(G)]
     value = ws_ * T * K / (ms / 1e3)
     fwd_avg_ms = float(np.mean(fwd_ms))
     peaks = _peaks()
-    if T <= 4:
+    if T <= 8:
         roof = _roofline("hbm", float(np.mean([fwd_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks, "decode")
         roof["kernel"] = "moe_expert_forward (decode_ffn_kernel: gate|up + down dequant-GEMV)"
     else:
@@ -301,7 +310,7 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
         layers[r](xd[r], stream=stream)
         oh[r].copy_(layers[r].out, non_blocking=True)
 
-    Ge = _divisor_at_most(K, 256 if T <= 4 else 32)
+    Ge = _divisor_at_most(K, 256 if T <= 8 else 32)
     g2 = _graph_of(e2e_step, Ge, stream)
     with torch.cuda.stream(stream):
         g2.replay()
@@ -313,7 +322,7 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
         "l2": f"rotating {R} replicas of pool+Wr+x ({R * pool_bytes / 1e9:.2f} GB)",
         "e2e": {"value": round(ws_ * T * K / (ems / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": T * D * 2,
                 "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": LAUNCHES["decode" if T <= 4 else "prefill"] * K,
+        "gpu_launches": LAUNCHES["decode" if T <= 8 else "prefill"] * K,
         "roofline": roof,
         "hit_rate": round(float(np.mean(hits)), 4), "u_hit_mean": round(float(np.mean(u_hit)), 2),
         "step_alg_bytes": round(float(np.mean(step_bytes))),
@@ -325,7 +334,7 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
                                "below_16": int((loads < 16).sum())}
     if with_cpu:
         res["cpu_baseline"] = cpu_baseline(cfg, wl, seconds=args.cpu_seconds)
-    del layers, pools, Wrs, xs, graph, g2, wl
+    del layers, pools, Wrs, xs, graph, graph_ev, g2, wl
     return res
 
 
@@ -358,7 +367,7 @@ def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 16, 64), K=64)
         ms, _ = _timed_replays(graph, K // G, stream, ws_, dev, local, clocks=False)
         out[str(T)] = {"ms_per_step": round(ms / K, 5), "tokens_per_s": round(ws_ * T * K / (ms / 1e3), 1),
                        "expert_pass": "decode" if T <= 8 else "prefill",
-                       "router": "canonical CUDA-core" if T <= 4 else "tensor-core + canonical recheck"}
+                       "router": "canonical CUDA-core" if T <= 8 else "tensor-core + canonical recheck"}
         del layers, xs, graph
     del pools, wl
     return {"workload": "decode layer shapes (D=3072, F=512, E=512, top-10+1, Q2_32, 320/512 resident), "
@@ -425,18 +434,23 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
     ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
           for _ in range(NL)]
 
-    def step(i):
+    def step(i, events=False):
         for l in range(NL):
-            buf.layer(wl, l, stream, ev=ev[l] if i == 0 else None)
+            buf.layer(wl, l, stream, ev=ev[l] if events else None)
 
+    # no event nodes in the throughput graph (they end the programmatic-launch
+    # overlap between kernels); a second graph times each expert pass
     graph = _graph_of(step, 1, stream)
+    graph_ev = _graph_of(lambda i: step(i, True), 1, stream)
     with torch.cuda.stream(stream):
         for _ in range(W):
             graph.replay()
+        graph_ev.replay()
     ms, clocks = _timed_replays(graph, K, stream, ws_, dev, local)
+    _timed_replays(graph_ev, 1, stream, ws_, dev, local, clocks=False)
     fwd_ms = [ev[l][0].elapsed_time(ev[l][1]) for l in range(NL)]
     peaks = _peaks()
-    if T <= 4:
+    if T <= 8:
         roof = _roofline("hbm", float(np.sum(fwd_bytes)) / NL, float(np.sum(fwd_ms)) / NL, peaks, "decode48")
         roof["kernel"] = "moe_expert_forward (decode_ffn_kernel), averaged over the 48 layers"
     else:
@@ -467,14 +481,14 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
         "e2e": {"value": round(ws_ * T * NL * K / (ems / 1e3), 1), "unit": "tokens/s (per layer)",
                 "chain_tokens_per_s": round(ws_ * T * K / (ems / 1e3), 2), "h2d_bytes_per_step": T * D * 2,
                 "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": LAUNCHES["decode" if T <= 4 else "prefill"] * NL * K,
+        "gpu_launches": LAUNCHES["decode" if T <= 8 else "prefill"] * NL * K,
         "roofline": roof,
         "hit_rate": round(hits / n_sel, 4),
         "clocks": clocks,
     }
     if with_cpu:
         res["cpu_baseline"] = cpu_baseline_chain(cfg, wl)
-    del buf, graph, g2, wl
+    del buf, graph, graph_ev, g2, wl
     return res
 
 
@@ -511,7 +525,7 @@ def cpu_baseline_chain(cfg, wl):
     prefill48 — a 64-token sample through one layer (per-layer rate)."""
     from tests.harness import oracle_layer, u16
     ncores = os.cpu_count() or 1
-    if cfg.T <= 4:
+    if cfg.T <= 8:
         x = u16(wl.x)
         t0 = time.time()
         for L in wl.layers:

@@ -45,6 +45,7 @@
 #include "kernels.cuh"
 #include "once.cuh"
 #include "sync.cuh"
+#include "tmap.cuh"
 
 namespace moe {
 namespace {
@@ -79,6 +80,39 @@ struct Geo {
     static constexpr int row_bytes(int K) { return code_row(K) + meta_row(K) + d_row(K); }
 };
 
+// Smallest y >= x with y % m == r.
+constexpr uint32_t pad_to(uint32_t x, uint32_t m, uint32_t r) { return x + ((r + m - x % m) % m); }
+
+// A staged region of n matrix rows of K weights: the n code rows, then the n
+// meta rows, then (Q3_S256) the n d rows, each plane at its own smem row
+// stride.  Code and Q2/Q3_32 scale rows are copied one row at a time into
+// padded rows, so that the eight rows read by one load instruction (lanes g =
+// 0..7, four lanes a row) fall on distinct banks:
+//   Q2 codes      8-byte loads, 32 bytes a row:  stride = 32 (mod 64)
+//   Q3 codes      three 4-byte loads, 12 bytes a lane: stride = 16 (mod 32)
+//   (s, m) words  4-byte loads, 16 bytes a row:  stride = 16 (mod 32)
+// (rows r * stride then start at distinct 32-byte (resp. 16-byte) slots of the
+// 128-byte bank window, since stride / 16 is odd).  The Q3_S256 sub-scale and
+// d rows are read with broadcasts (one super-block a row) and copied unpadded
+// in one piece.
+template <int FMT>
+struct Rows {
+    uint32_t c, m, d;     // smem row strides of the planes
+    uint32_t cr, mr, dr;  // bytes of one row in the pool (padding: zeros past cr, mr)
+    static constexpr Rows of(int K) {
+        Rows R{};
+        R.cr = Geo<FMT>::code_row(K);
+        R.mr = Geo<FMT>::meta_row(K);
+        R.dr = Geo<FMT>::d_row(K);
+        R.c = FMT == MOE_Q2_32 ? pad_to(R.cr, 64, 32) : pad_to(R.cr, 32, 16);
+        R.m = FMT == MOE_Q3_S256 ? R.mr : pad_to(R.mr, 32, 16);
+        R.d = R.dr;
+        return R;
+    }
+    constexpr uint32_t bytes(int n) const { return (uint32_t)n * (c + m + d); }      // staged (and copied)
+    constexpr uint32_t region(int n) const { return (bytes(n) + 127u) & ~127u; }     // 128-byte aligned slot
+};
+
 struct Planes {
     const uint8_t* c;   // code plane
     const uint8_t* m;   // (s,m) plane or sub-scale plane
@@ -99,6 +133,16 @@ MOE_DEVINL Planes planes_of(const PoolView& P, int slot, int mat) {
         pl.d = nullptr;
     }
     return pl;
+}
+
+// One stage of the ring: a gate|up item (gate rows, then up rows, each in a
+// 128-byte aligned region) or a down item (rows, then the owner's h), 128-byte
+// aligned (tensor copies land on 128-byte boundaries).
+template <int FMT, int NSLOT>
+constexpr uint32_t stage_size(int D, int F, int rf, int rd) {
+    const uint32_t a = 2u * Rows<FMT>::of(D).region(rf);
+    const uint32_t b = Rows<FMT>::of(F).bytes(rd) + (uint32_t)F * NSLOT * 2;
+    return ((a > b ? a : b) + 127u) & ~127u;
 }
 
 // ---------------------------------------------------------------- work resolution
@@ -125,6 +169,10 @@ struct DecodeParams {
     int rf;                // gate|up: features per item (8 or 16)
     int rd;                // down: rows per item (multiple of 16)
     int ns;                // pipeline stages
+    // padded-row boxes (Rows<FMT>): gate|up matrices as one tensor of 2F rows
+    // of D weights, down as D rows of F weights; codes and (s, m) planes
+    // (Q3_S256: the code maps only)
+    CUtensorMap tm_gu_c, tm_gu_m, tm_dn_c, tm_dn_m;
 };
 
 constexpr int kRedBufs = 3;                        // partial-sum buffers per team (items in flight)
@@ -135,8 +183,8 @@ struct Shared {
     uint64_t empty[kMaxStages];
     int stage_item[kMaxStages];    // the work item in each stage (-1: no more work)
     Owner owners[kMaxPairs];
-    int slot_of[kMaxPairs];
     int table[kMaxE];              // the slot table, staged before the dependency wait
+    int oidx[kMaxPairs];           // per owning pair: its owner index
     int n_owners;
     int abort;                     // set by any warp that stopped on an error
     uint32_t red_cnt[kTeams][kRedBufs];   // warps that wrote their partials into a buffer
@@ -148,10 +196,12 @@ struct Shared {
 
 // The slot table is an input of the layer, not produced by the router: stage it
 // while the router may still run.
-__device__ void stage_table(const DecodeParams& prm, Shared& sh) {
+// `first` (E ints, scratch for resolve_owners) starts at kMaxPairs.
+__device__ void stage_table(const DecodeParams& prm, Shared& sh, int* first) {
     for (int e = threadIdx.x; e < prm.E; e += blockDim.x) {
         const int s = __ldg(prm.slot_table + e);
         sh.table[e] = (s < 0 || s >= prm.P.n_slots) ? -1 : s;
+        first[e] = kMaxPairs;
     }
 }
 
@@ -171,10 +221,14 @@ MOE_DEVINL int lookup_slot(const DecodeParams& prm, const Shared& sh, int e) {
 }
 
 // One warp: resolve every pair's slot and the owners — owner 0 is the shared
-// expert, then the first pair of each distinct resident slot in pair order —
+// expert, then the first pair of each distinct resident expert in pair order —
 // and, with `book`, the row map, miss list and miss count.  Lane L handles
-// pairs L + 32h (h = 0..3; T * k <= 128).
-__device__ void resolve_owners(const DecodeParams& prm, Shared& sh, bool book) {
+// pairs L + 32h (h = 0..3; T * k <= 128).  Pairs of one expert find their
+// owner through a shared-memory minimum per expert id (`first`: E ints, all
+// kMaxPairs on entry); each pair then sets its rank bit in its owner's token
+// mask.  (Two expert ids on one slot would get
+// two owners over the same weights: the same outputs, computed twice.)
+__device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, bool book) {
     constexpr int H = (kMaxPairs - 1 + 31) / 32;
     const int lane = threadIdx.x & 31;
     const int T = prm.T, k = prm.k, n = T * k;   // n <= 128
@@ -185,8 +239,12 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, bool book) {
     for (int h = 0; h < H; ++h) {
         const int p = lane + 32 * h;
         e[h] = p < n ? __ldg(prm.ids + p) : -1;
+    }
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        const int p = lane + 32 * h;
         s[h] = p < n ? lookup_slot(prm, sh, e[h]) : -1;
-        if (p < n) sh.slot_of[p] = s[h];
+        if (s[h] >= 0) atomicMin(first + e[h], p);
         missb[h] = __ballot_sync(0xffffffffu, p < n && s[h] < 0);
     }
     if (book) {
@@ -208,62 +266,31 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, bool book) {
         if (lane == 0) prm.miss_count[0] = base;
     }
     __syncwarp();
-    // eq[h]: the pairs q with the same slot as pair lane + 32h (bits of 2 words)
-    uint64_t eq[H][2];
-    bool own[H];
-#pragma unroll
-    for (int h = 0; h < H; ++h) { eq[h][0] = eq[h][1] = 0; }
-    for (int q = 0; q < n && q < 64; ++q) {
-        const int sq = sh.slot_of[q];
-#pragma unroll
-        for (int h = 0; h < H; ++h)
-            if (sq == s[h]) eq[h][0] |= 1ull << q;
-    }
-    for (int q = 64; q < n; ++q) {
-        const int sq = sh.slot_of[q];
-#pragma unroll
-        for (int h = 0; h < H; ++h)
-            if (sq == s[h]) eq[h][1] |= 1ull << (q - 64);
-    }
-    uint32_t ownb[H];
-#pragma unroll
-    for (int h = 0; h < H; ++h) {
-        const int p = lane + 32 * h;
-        bool o = p < n && s[h] >= 0;
-        if (o) {   // an earlier pair with the same slot owns it
-            const uint64_t lo = p >= 64 ? eq[h][0] : (eq[h][0] & ((1ull << p) - 1ull));
-            const uint64_t hi = p >= 64 ? (eq[h][1] & ((1ull << (p - 64)) - 1ull)) : 0ull;
-            if (lo | hi) o = false;
-        }
-        own[h] = o;
-        ownb[h] = __ballot_sync(0xffffffffu, o);
-    }
     int base = 1;
 #pragma unroll
     for (int h = 0; h < H; ++h) {
-        if (own[h]) {
-            Owner& o = sh.owners[base + __popc(ownb[h] & below)];
+        const int p = lane + 32 * h;
+        const bool own = s[h] >= 0 && first[e[h]] == p;
+        const uint32_t ownb = __ballot_sync(0xffffffffu, own);
+        if (own) {
+            const int o = base + __popc(ownb & below);
+            sh.oidx[p] = o;
+            sh.owners[o].slot = s[h];
 #pragma unroll
-            for (int t = 0; t < kDecodeMaxT; ++t) {
-                uint32_t m = 0;
-                if (t < T) {
-                    const int b0 = t * k;                       // bits [b0, b0 + k) of the 128-bit eq
-                    uint64_t w;
-                    if (b0 >= 64) w = eq[h][1] >> (b0 - 64);
-                    else if (b0 == 0) w = eq[h][0];
-                    else w = (eq[h][0] >> b0) | (eq[h][1] << (64 - b0));
-                    m = (uint32_t)w & ((1u << k) - 1u);
-                }
-                o.rmask[t] = m;
-            }
-            o.slot = s[h];
+            for (int t = 0; t < kDecodeMaxT; ++t) sh.owners[o].rmask[t] = 0u;
         }
-        base += __popc(ownb[h]);
+        base += __popc(ownb);
     }
     if (lane < kDecodeMaxT) sh.owners[0].rmask[lane] = lane < T ? 1u << k : 0u;
     if (lane == 0) {
         sh.owners[0].slot = prm.P.shared_slot;
         sh.n_owners = base;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        const int p = lane + 32 * h;
+        if (s[h] >= 0) atomicOr(&sh.owners[sh.oidx[first[e[h]]]].rmask[p / k], 1u << (p % k));
     }
     __syncwarp();
 }
@@ -339,33 +366,32 @@ struct RowBlock {
     uint32_t d2;             // Q3_S256: d broadcast to f16x2
 };
 
-// Load block (4U + c) of local row r of a staged region (codes | meta | d,
-// rows of K weights).
+// Load block (4U + c) of local row r of a staged region (planes at cbase,
+// mbase, dbase; row strides R).
 template <int FMT>
-MOE_DEVINL void load_row_block(const uint8_t* cbase, const uint8_t* mbase, const uint8_t* dbase, int r, int K, int U,
-                               int c, RowBlock<FMT>& rb) {
+MOE_DEVINL void load_row_block(const uint8_t* cbase, const uint8_t* mbase, const uint8_t* dbase, int r,
+                               const Rows<FMT>& R, int U, int c, RowBlock<FMT>& rb) {
     const int blk = 4 * U + c;
     if constexpr (FMT == MOE_Q2_32) {
-        const uint2 v = *reinterpret_cast<const uint2*>(cbase + (size_t)r * Geo<FMT>::code_row(K) + blk * 8);
+        const uint2 v = *reinterpret_cast<const uint2*>(cbase + (size_t)r * R.c + blk * 8);
         rb.w[0] = v.x; rb.w[1] = v.y; rb.w[2] = 0;
     } else {
-        const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)r * Geo<FMT>::code_row(K) + blk * 12);
+        const uint32_t* p = reinterpret_cast<const uint32_t*>(cbase + (size_t)r * R.c + blk * 12);
         rb.w[0] = p[0]; rb.w[1] = p[1]; rb.w[2] = p[2];
     }
     if constexpr (FMT != MOE_Q3_S256) {
-        const uint32_t sm = *reinterpret_cast<const uint32_t*>(mbase + (size_t)r * Geo<FMT>::meta_row(K) + blk * 4);
+        const uint32_t sm = *reinterpret_cast<const uint32_t*>(mbase + (size_t)r * R.m + blk * 4);
         rb.sa = bcast_lo(sm);
         rb.sb = bcast_hi(sm);
         rb.d2 = 0;
     } else {
         // super-block U / 2; the block's two sub-blocks: 12 bits at bit 12 * (4 (U & 1) + c)
-        const uint32_t* scp =
-            reinterpret_cast<const uint32_t*>(mbase + (size_t)r * Geo<FMT>::meta_row(K) + (U >> 1) * 12);
+        const uint32_t* scp = reinterpret_cast<const uint32_t*>(mbase + (size_t)r * R.m + (U >> 1) * 12);
         const int cc = 4 * (U & 1) + c, bit = 12 * cc, wi = bit >> 5, sh = bit & 31;
         const uint32_t lo = scp[wi];
         const uint32_t hi = wi < 2 ? scp[wi + 1] : 0u;
         const uint32_t bits = __funnelshift_r(lo, hi, sh);
-        const uint32_t db = *reinterpret_cast<const uint16_t*>(dbase + (size_t)r * Geo<FMT>::d_row(K) + (U >> 1) * 2);
+        const uint32_t db = *reinterpret_cast<const uint16_t*>(dbase + (size_t)r * R.d + (U >> 1) * 2);
         rb.d2 = db | (db << 16);
         rb.sa = s256_sub(bits & 63u);
         rb.sb = s256_sub((bits >> 6) & 63u);
@@ -409,14 +435,14 @@ MOE_DEVINL void static_for(Fn&& fn) {
 // fragment-order buffer bs.  Accumulates into acc[t].
 template <int FMT, int NT, int NSLOT>
 MOE_DEVINL void unit_mma(const uint8_t* ca, const uint8_t* ma, const uint8_t* da, const uint8_t* cb,
-                         const uint8_t* mb, const uint8_t* db, const int (&rt)[NT], const int (&rbm)[NT], int K, int U,
-                         const uint8_t* bs, const Magic& M, float (&acc)[NT][4]) {
+                         const uint8_t* mb, const uint8_t* db, const int (&rt)[NT], const int (&rbm)[NT],
+                         const Rows<FMT>& R, int U, const uint8_t* bs, const Magic& M, float (&acc)[NT][4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     RowBlock<FMT> top[NT], bot[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-        load_row_block<FMT>(ca, ma, da, rt[t], K, U, c, top[t]);
-        load_row_block<FMT>(cb, mb, db, rbm[t], K, U, c, bot[t]);
+        load_row_block<FMT>(ca, ma, da, rt[t], R, U, c, top[t]);
+        load_row_block<FMT>(cb, mb, db, rbm[t], R, U, c, bot[t]);
     }
     static_for<0, 8>([&](auto S) {
         constexpr int s = decltype(S)::value, I = s >> 2, J = s & 3;
@@ -438,14 +464,25 @@ MOE_DEVINL void unit_mma(const uint8_t* ca, const uint8_t* ma, const uint8_t* da
 
 MOE_DEVINL float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-// Issue the bulk copies of `nrows` rows starting at `row0` of matrix planes pl
-// (rows of K weights) into dst (codes | meta | d), completing on bar.
+// The copies of `nrows` rows starting at row y of a matrix set (tensor maps
+// mc, mm over the slot's rows; pl: the slot's planes of the matrix, rows from
+// row0) into the region at dst (layout Rows<FMT>), completing on bar: one
+// padded-row box per code and (s, m) plane; the Q3_S256 sub-scale and d planes
+// in one bulk copy each.  Every copied byte, padding included, counts toward
+// the barrier's transaction bytes: Rows<FMT>::bytes(nrows).
 template <int FMT>
-MOE_DEVINL void issue_rows(const Planes& pl, int row0, int nrows, int K, uint8_t* dst, uint64_t* bar) {
-    const uint32_t cr = Geo<FMT>::code_row(K), mr = Geo<FMT>::meta_row(K), dr = Geo<FMT>::d_row(K);
-    bulk_g2s(dst, pl.c + (size_t)row0 * cr, cr * nrows, bar);
-    bulk_g2s(dst + cr * nrows, pl.m + (size_t)row0 * mr, mr * nrows, bar);
-    if constexpr (FMT == MOE_Q3_S256) bulk_g2s(dst + (cr + mr) * nrows, pl.d + (size_t)row0 * dr, dr * nrows, bar);
+MOE_DEVINL void issue_rows(const CUtensorMap* mc, const CUtensorMap* mm, const Planes& pl, int y, int row0,
+                           int slot, int nrows, const Rows<FMT>& R, uint8_t* dst, uint64_t* bar) {
+    tma_box_3d(dst, mc, 0, y, slot, bar);
+    uint8_t* dm = dst + (size_t)nrows * R.c;
+    if constexpr (FMT != MOE_Q3_S256) {
+        (void)pl; (void)row0;
+        tma_box_3d(dm, mm, 0, y, slot, bar);
+    } else {
+        (void)mm;
+        bulk_g2s(dm, pl.m + (size_t)row0 * R.mr, R.mr * nrows, bar);
+        bulk_g2s(dm + (size_t)nrows * R.m, pl.d + (size_t)row0 * R.dr, R.dr * nrows, bar);
+    }
 }
 
 // ---------------------------------------------------------------- gate | up
@@ -459,14 +496,13 @@ __device__ void gateup_partial(const DecodeParams& prm, int rf, const uint8_t* s
                                float* red_w) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     const int D = prm.P.D;
-    const uint32_t cr = Geo<FMT>::code_row(D), mr = Geo<FMT>::meta_row(D);
-    const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * rf;   // gate rows then up rows
-    const uint8_t* gc = stage;
-    const uint8_t* gm = stage + cr * rf;
-    const uint8_t* gd = stage + (cr + mr) * rf;
-    const uint8_t* uc = stage + half;
-    const uint8_t* um = uc + cr * rf;
-    const uint8_t* ud = uc + (cr + mr) * rf;
+    const Rows<FMT> R = Rows<FMT>::of(D);
+    const uint8_t* gc = stage;                     // gate rows, then up rows
+    const uint8_t* gm = gc + R.c * rf;
+    const uint8_t* gd = gm + R.m * rf;
+    const uint8_t* uc = stage + R.region(rf);
+    const uint8_t* um = uc + R.c * rf;
+    const uint8_t* ud = um + R.m * rf;
     const Magic M = make_magic();
     float acc[NT][4];
     int rt[NT];
@@ -476,7 +512,7 @@ __device__ void gateup_partial(const DecodeParams& prm, int rf, const uint8_t* s
         acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
     }
     for (int U = wt; U < D / kUnitK; U += kTeamWarps)
-        unit_mma<FMT, NT, NSLOT>(gc, gm, gd, uc, um, ud, rt, rt, D, U, xs, M, acc);
+        unit_mma<FMT, NT, NSLOT>(gc, gm, gd, uc, um, ud, rt, rt, R, U, xs, M, acc);
     // lanes with c < NSLOT / 2 hold token columns 2c, 2c + 1 (the columns in use)
     if (c < NSLOT / 2) {
 #pragma unroll
@@ -525,14 +561,14 @@ __device__ void down_item(const DecodeParams& prm, const Owner& o, int d0, int r
     if (16 * wt >= rd) return;
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     const int D = prm.P.D, F = prm.P.F, k = prm.k;
-    const uint32_t cr = Geo<FMT>::code_row(F), mr = Geo<FMT>::meta_row(F);
+    const Rows<FMT> R = Rows<FMT>::of(F);
     const uint8_t* dc = stage;
-    const uint8_t* dm = stage + cr * rd;
-    const uint8_t* dd = stage + (cr + mr) * rd;
+    const uint8_t* dm = dc + R.c * rd;
+    const uint8_t* dd = dm + R.m * rd;
     const Magic M = make_magic();
     float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
     const int rt[1] = {16 * wt + g}, rbm[1] = {16 * wt + g + 8};
-    for (int U = 0; U < F / kUnitK; ++U) unit_mma<FMT, 1, NSLOT>(dc, dm, dd, dc, dm, dd, rt, rbm, F, U, hs, M, acc);
+    for (int U = 0; U < F / kUnitK; ++U) unit_mma<FMT, 1, NSLOT>(dc, dm, dd, dc, dm, dd, rt, rbm, R, U, hs, M, acc);
     if (c < NSLOT / 2) {
         const int row = d0 + 16 * wt + g;
 #pragma unroll
@@ -582,9 +618,11 @@ MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
 // the publisher.  The last CTA to finish resets the counters, so every
 // completed call leaves them zero.
 template <int FMT, int NSLOT>
-__global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams prm) {
-    extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_constant__ DecodeParams prm) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ Shared sh;
+    // tensor copies land on 128-byte boundaries (the launch adds 128 bytes)
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = prm.P.D, F = prm.P.F, rf = prm.rf, rd = prm.rd, NS = prm.ns;
     const size_t xs_bytes = (size_t)D * NSLOT * 2;
@@ -593,9 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     uint8_t* xs = smem;
     float* red = reinterpret_cast<float*>(smem + xs_bytes);
     uint8_t* stages = smem + xs_bytes + kTeams * red_team * 4;
-    const uint32_t gu_bytes = 2u * Geo<FMT>::row_bytes(D) * rf;
-    const uint32_t dn_bytes = (uint32_t)Geo<FMT>::row_bytes(F) * rd;
-    const uint32_t stage_bytes = gu_bytes > dn_bytes + hbytes ? gu_bytes : dn_bytes + hbytes;
+    const Rows<FMT> RD = Rows<FMT>::of(D), RF = Rows<FMT>::of(F);
+    const uint32_t dn_bytes = RF.bytes(rd);                                    // down rows, then h
+    const uint32_t stage_bytes = stage_size<FMT, NSLOT>(D, F, rf, rd);         // gate rows | up rows
     const int nfb = F / rf, nrb = D / rd;
     uint32_t* done = prm.done;
     uint32_t* queue = done + kMaxPairs + 1;
@@ -617,7 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     // precedes this launch passed its own wait.
     __shared__ int dead;
     if (threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
-    stage_table(prm, sh);
+    // the partial-sum buffers are free until the first item: owner resolution
+    // keeps its per-expert scratch there
+    int* first = reinterpret_cast<int*>(red);
+    stage_table(prm, sh, first);
     __syncthreads();
     pdl_wait();                      // ids come from the router
     if (!dead) {
@@ -625,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
     // (barrier 1) while the other consumers stage x; the consumers meet at
     // barrier 4 before computing
     if (warp == 0) {
-        resolve_owners(prm, sh, blockIdx.x == 0);
+        resolve_owners(prm, sh, first, blockIdx.x == 0);
         asm volatile("bar.arrive 1, 96;" ::: "memory");
         asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
     } else if (warp < kConsumerWarps) {
@@ -673,40 +714,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                 }
             }
         }
-    } else if (warp == kProducerWarp) {    // producer: take items from the queue, stage them
-        if (lane == 0) {
-            int j = 0, issued = 0;
-            bool ok = true;
-            for (;; ++j) {
-                const int s = j % NS;
-                if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) { ok = false; break; }
-                if (stopped()) { ok = false; break; }
-                const int idx = (int)atomicAdd(queue, 1u);
-                uint8_t* dst = stages + (size_t)s * stage_bytes;
-                if (idx >= n_all) {                       // no more work: tell this stage's team
+    } else if (warp == kProducerWarp) {
+        // producer (lane 0): take items from the queue, wait for free stages,
+        // issue the copies
+        int j = 0, issued = 0;
+        bool ok = true;
+        // the next item is taken from the queue one step ahead, so the
+        // atomic's round trip overlaps the wait for a free stage
+        int next = 0;
+        if (lane == 0) next = (int)atomicAdd(queue, 1u);
+        for (;; ++j) {
+            const int s = j % NS;
+            int idx = next, go = 1;
+            if (lane == 0) {
+                if (idx < n_all) next = (int)atomicAdd(queue, 1u);
+                if (j >= NS && !mbar_wait(&sh.empty[s], ((j / NS) - 1) & 1, prm.err)) go = 0;
+                else if (stopped()) go = 0;
+            }
+            go = __shfl_sync(0xffffffffu, go, 0);
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            if (!go) { ok = false; break; }
+            uint8_t* dst = stages + (size_t)s * stage_bytes;
+            if (idx >= n_all) {                       // no more work: tell this stage's team
+                if (lane == 0) {
                     sh.stage_item[s] = -1;
                     mbar_arrive(&sh.full[s]);
-                    ++j;
-                    break;
                 }
-                sh.stage_item[s] = idx;
-                if (idx < n_g) {
-                    const ItemPos ip = item_pos(idx, nfb, rf);
+                ++j;
+                break;
+            }
+            if (idx < n_g) {
+                const ItemPos ip = item_pos(idx, nfb, rf);
+                const int slot = sh.owners[ip.u].slot;
+                if (lane == 0) {
+                    sh.stage_item[s] = idx;
+                    mbar_arrive_expect_tx(&sh.full[s], 2 * RD.bytes(rf));
+                    issue_rows<FMT>(&prm.tm_gu_c, &prm.tm_gu_m, planes_of<FMT>(prm.P, slot, 0), ip.row0, ip.row0, slot,
+                                    rf, RD, dst, &sh.full[s]);
+                    issue_rows<FMT>(&prm.tm_gu_c, &prm.tm_gu_m, planes_of<FMT>(prm.P, slot, 1), F + ip.row0, ip.row0,
+                                    slot, rf, RD, dst + RD.region(rf), &sh.full[s]);
+                }
+            } else {
+                const ItemPos ip = item_pos(idx - n_g, nrb, rd);
+                int fine = 1;
+                if (lane == 0) {
                     const int slot = sh.owners[ip.u].slot;
-                    const uint32_t half = (uint32_t)Geo<FMT>::row_bytes(D) * rf;
-                    mbar_arrive_expect_tx(&sh.full[s], 2 * half);
-                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 0), ip.row0, rf, D, dst, &sh.full[s]);
-                    issue_rows<FMT>(planes_of<FMT>(prm.P, slot, 1), ip.row0, rf, D, dst + half, &sh.full[s]);
-                } else {
-                    const ItemPos ip = item_pos(idx - n_g, nrb, rd);
+                    sh.stage_item[s] = idx;
                     mbar_arrive_expect_tx(&sh.full[s], dn_bytes + hbytes);
-                    issue_rows<FMT>(planes_of<FMT>(prm.P, sh.owners[ip.u].slot, 2), ip.row0, rd, F, dst, &sh.full[s]);
+                    issue_rows<FMT>(&prm.tm_dn_c, &prm.tm_dn_m, planes_of<FMT>(prm.P, slot, 2), ip.row0, ip.row0, slot,
+                                    rd, RF, dst, &sh.full[s]);
                     // the owner's h, once every gate|up item of the owner is published
                     const uint64_t t0 = globaltimer_ns();
                     while (ld_acquire(done + ip.u) < (uint32_t)nfb) {
                         if (timed_out(prm.err) || globaltimer_ns() - t0 > kWaitLimitNs) {
                             atomicOr(prm.err, kErrTimeout);
-                            ok = false;
+                            fine = 0;
                             break;
                         }
                         __nanosleep(64);
@@ -715,9 +777,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
                     asm volatile("fence.proxy.async.global;" ::: "memory");   // h was written through the generic proxy
                     bulk_g2s(dst + dn_bytes, prm.hfrag + (size_t)ip.u * F * NSLOT, hbytes, &sh.full[s]);
                 }
-                issued = j + 1;
-                if (!ok) break;
+                ok = __shfl_sync(0xffffffffu, fine, 0) != 0;
             }
+            issued = j + 1;
+            if (!ok) break;
+        }
+        if (lane == 0) {
             // the other team's next stage also learns that the work is over
             if (ok) {
                 const int s = j % NS;
@@ -831,8 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(DecodeParams pr
 template <int FMT, int NSLOT>
 size_t smem_for(int D, int F, int rf, int rd, int ns) {
     const size_t fixed = (size_t)D * NSLOT * 2 + kTeams * (size_t)kRedBufs * kTeamWarps * red_floats<NSLOT>() * 4;
-    const size_t a = 2 * (size_t)Geo<FMT>::row_bytes(D) * rf, b = (size_t)Geo<FMT>::row_bytes(F) * rd + (size_t)F * NSLOT * 2;
-    return fixed + (size_t)ns * (a > b ? a : b);
+    return 128 + fixed + (size_t)ns * stage_size<FMT, NSLOT>(D, F, rf, rd);
 }
 
 // Dynamic shared memory available to decode_ffn_kernel<FMT, NSLOT> on the
@@ -860,7 +924,8 @@ int smem_budget() {
 
 template <int FMT, int NSLOT>
 moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
-    const int D = prm.P.D, F = prm.P.F;
+    const PoolView& P = prm.P;
+    const int D = P.D, F = P.F;
     const int budget = smem_budget<FMT, NSLOT>();
     if (budget <= 0) return MOE_ERR_CUDA;
     // gate|up items of rf features (two 16-row tiles), down items of rd rows
@@ -868,7 +933,7 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
     // flight per SM cover the copy latency)
     int rf = 16, rd = 128;
     while (rf > 8 && smem_for<FMT, NSLOT>(D, F, rf, rd, 2) > (size_t)budget) rf /= 2;
-    while (rd > 16 && (size_t)Geo<FMT>::row_bytes(F) * rd > 2 * (size_t)Geo<FMT>::row_bytes(D) * rf) rd /= 2;
+    while (rd > 16 && (size_t)Rows<FMT>::of(F).bytes(rd) > 2 * (size_t)Rows<FMT>::of(D).region(rf)) rd /= 2;
     while (rd > 16 && smem_for<FMT, NSLOT>(D, F, rf, rd, 2) > (size_t)budget) rd /= 2;
     int ns = 4;
     while (ns > 2 && smem_for<FMT, NSLOT>(D, F, rf, rd, ns) > (size_t)budget) --ns;
@@ -883,6 +948,23 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
                ((size_t)Geo<FMT>::d_row(K) * n) % 16 == 0;
     };
     if (!ok16(D, rf) || !ok16(F, rd)) return MOE_ERR_UNSUPPORTED;
+    // tensor maps over every slot: gate|up as 2F rows of D weights, down as D
+    // rows of F weights (after the gate and up matrices of the slot)
+    const Rows<FMT> RD = Rows<FMT>::of(D), RF = Rows<FMT>::of(F);
+    const uint8_t* dn_codes = P.codes + 2 * (size_t)F * RD.cr;
+    const uint64_t slots = (uint64_t)P.n_slots;
+    if (!padded_rows_map(&prm.tm_gu_c, P.codes, RD.cr, 2 * (uint64_t)F, slots, P.stride_c, RD.c, (uint32_t)rf) ||
+        !padded_rows_map(&prm.tm_dn_c, dn_codes, RF.cr, (uint64_t)D, slots, P.stride_c, RF.c, (uint32_t)rd))
+        return MOE_ERR_UNSUPPORTED;
+    if constexpr (FMT != MOE_Q3_S256) {
+        const uint8_t* dn_scales = P.scales + 2 * (size_t)F * RD.mr;
+        if (!padded_rows_map(&prm.tm_gu_m, P.scales, RD.mr, 2 * (uint64_t)F, slots, P.stride_s, RD.m, (uint32_t)rf) ||
+            !padded_rows_map(&prm.tm_dn_m, dn_scales, RF.mr, (uint64_t)D, slots, P.stride_s, RF.m, (uint32_t)rd))
+            return MOE_ERR_UNSUPPORTED;
+    } else {
+        prm.tm_gu_m = prm.tm_gu_c;
+        prm.tm_dn_m = prm.tm_dn_c;
+    }
     static std::atomic<uint64_t> attr_done{0};
     if (!once_per_device(attr_done, [] {
             return cudaFuncSetAttribute(decode_ffn_kernel<FMT, NSLOT>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tmap.cuh"
 #include "once.cuh"
 #include "route_warp.cuh"
 #include "sync.cuh"
@@ -269,25 +270,9 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
     topk_row_warp(row, E, k, ids + (size_t)t * k, gates + (size_t)t * k);
 }
 
-typedef CUresult (*EncodeTiledFnR)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFnR encode_tiled_r() {
-    static EncodeTiledFnR fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFnR>(p);
-    }
-    return fn;
-}
-
 // bf16 [rows][D], boxes of 64 x 128 rows, 128B swizzle
 bool bf16_rows_map(CUtensorMap* m, const void* base, int D, int rows) {
-    EncodeTiledFnR fn = encode_tiled_r();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
