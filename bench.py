@@ -47,10 +47,10 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 EXTRA = ["prefill", "decode48", "prefill48"]
-# kernels per layer and step: decode (T <= 8) route 1, expert pass 1, combine 1;
-# prefill route 3 (norms, tensor-core logits, selection), expert pass 6 (3
+# kernels per layer and step: the one-call decode layer (T <= 8) 1; decode as
+# three calls: route 1, expert pass 1, combine 1; prefill route 3 (norms, tensor-core logits, selection), expert pass 6 (3
 # plan, gather, 2 GEMMs), combine 1
-LAUNCHES = {"decode": 3, "prefill": 10}
+LAUNCHES = {"layer": 1, "decode": 3, "prefill": 10}
 
 
 def _peaks():
@@ -254,6 +254,9 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     wr_bytes = E * D * 2
     fwd_bytes = [(u + 1) * slot_bytes + x_bytes for u in u_hit]         # expert weights read + x
     step_bytes = [fb + wr_bytes + x_bytes for fb in fwd_bytes]           # + router weights + out
+    # the decode step is the one-call layer (routing, expert pass and combine
+    # in one kernel): its algorithmic bytes are the whole step's
+    fused = T <= 8 and layers[0].layer_ws is not None
     # algorithmic FLOPs of the expert FFNs: every resident (token, rank) row and
     # every token's shared-expert row costs gate + up + down = 3 * 2 * D * F
     fwd_flops = [(h * T * k + T) * 6.0 * D * F for h in hits]
@@ -263,6 +266,17 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
           for _ in range(G)]
 
     def step(i, events=False):
+        lay = layers[i % R]
+        if fused:
+            if events:
+                ev[i][0].record(stream)
+            lay.fused(xs[i % R], stream=stream)
+            if events:
+                ev[i][1].record(stream)
+            return
+        three_calls(i, events)
+
+    def three_calls(i, events=False):
         lay = layers[i % R]
         moe.moe_route_topk(xs[i % R], lay.Wr, lay.bias, k, lay.ids, lay.gates, lay.route_ws, stream=stream)
         if events:
@@ -282,14 +296,28 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
             graph.replay()
             graph_ev.replay()
     ms, clocks = _timed_replays(graph, K // G, stream, ws_, dev, local)
-    # the expert pass's own duration: the same steps with an event pair around
-    # each moe_expert_forward launch (so launched without the overlap)
+    # the dominant kernel's own duration: the same steps with an event pair
+    # around each moe_layer_forward (decode) or moe_expert_forward (prefill)
+    # launch, so launched without the overlap
     _timed_replays(graph_ev, K // G, stream, ws_, dev, local, clocks=False)
     fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(G)]
     value = ws_ * T * K / (ms / 1e3)
     fwd_avg_ms = float(np.mean(fwd_ms))
     peaks = _peaks()
-    if T <= 8:
+    three = None
+    if fused:
+        # the same layer as three calls (router, expert pass, combine), for comparison
+        g3 = _graph_of(three_calls, G, stream)
+        with torch.cuda.stream(stream):
+            g3.replay()
+        ms3, _ = _timed_replays(g3, K // G, stream, ws_, dev, local, clocks=False)
+        three = {"ms_per_step": round(ms3 / K, 6), "value": round(ws_ * T * K / (ms3 / 1e3), 1),
+                 "calls": "moe_route_topk + moe_expert_forward + moe_combine"}
+        del g3
+        roof = _roofline("hbm", float(np.mean([step_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks, "decode")
+        roof["kernel"] = ("moe_layer_forward (decode_ffn_kernel, one-call layer: logits + top-k, gate|up and down "
+                          "dequant-GEMV, combine); bytes = Wr + resident experts read + x + out")
+    elif T <= 8:
         roof = _roofline("hbm", float(np.mean([fwd_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks, "decode")
         roof["kernel"] = "moe_expert_forward (decode_ffn_kernel: gate|up + down dequant-GEMV)"
     else:
@@ -307,7 +335,10 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     def e2e_step(i):
         r = i % R
         xd[r].copy_(xh[r], non_blocking=True)
-        layers[r](xd[r], stream=stream)
+        if fused:
+            layers[r].fused(xd[r], stream=stream)
+        else:
+            layers[r](xd[r], stream=stream)
         oh[r].copy_(layers[r].out, non_blocking=True)
 
     Ge = _divisor_at_most(K, 256 if T <= 8 else 32)
@@ -322,13 +353,15 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
         "l2": f"rotating {R} replicas of pool+Wr+x ({R * pool_bytes / 1e9:.2f} GB)",
         "e2e": {"value": round(ws_ * T * K / (ems / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": T * D * 2,
                 "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": LAUNCHES["decode" if T <= 8 else "prefill"] * K,
+        "gpu_launches": LAUNCHES["layer" if fused else ("decode" if T <= 8 else "prefill")] * K,
         "roofline": roof,
         "hit_rate": round(float(np.mean(hits)), 4), "u_hit_mean": round(float(np.mean(u_hit)), 2),
         "step_alg_bytes": round(float(np.mean(step_bytes))),
         "clocks": clocks,
     }
-    if T > 4:
+    if three is not None:
+        res["three_calls"] = three
+    if T > 8:
         loads = np.bincount(layers[0].ids.cpu().numpy().ravel(), minlength=E)
         res["expert_loads"] = {"max": int(loads.max()), "zero": int((loads == 0).sum()),
                                "below_16": int((loads < 16).sum())}
@@ -368,6 +401,14 @@ def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 16, 64), K=64)
         out[str(T)] = {"ms_per_step": round(ms / K, 5), "tokens_per_s": round(ws_ * T * K / (ms / 1e3), 1),
                        "expert_pass": "decode" if T <= 8 else "prefill",
                        "router": "canonical CUDA-core" if T <= 8 else "tensor-core + canonical recheck"}
+        if layers[0].layer_ws is not None:
+            g1 = _graph_of(lambda i: layers[i % R].fused(xs[i % R], stream=stream), G, stream)
+            with torch.cuda.stream(stream):
+                g1.replay()
+            ms1, _ = _timed_replays(g1, K // G, stream, ws_, dev, local, clocks=False)
+            out[str(T)]["one_call"] = {"ms_per_step": round(ms1 / K, 5),
+                                       "tokens_per_s": round(ws_ * T * K / (ms1 / 1e3), 1)}
+            del g1
         del layers, xs, graph
     del pools, wl
     return {"workload": "decode layer shapes (D=3072, F=512, E=512, top-10+1, Q2_32, 320/512 resident), "
@@ -392,10 +433,23 @@ class ChainBuffers:
         self.miss_count = torch.zeros(1, dtype=torch.int32, device=dev)
         self.x = [torch.empty(T, D, dtype=torch.bfloat16, device=dev) for _ in range(len(wl.layers) + 1)]
         self.x[0].copy_(wl.x)
+        n = moe.layer_workspace_size(T, D, cfg.F, E, k, cfg.fmt)     # the one-call layer (T <= 8)
+        self.layer_ws = moe.alloc_ws(n, dev) if n else None
 
     def layer(self, wl, l, stream, ev=None, ids_out=None):
         cfg, L = wl.cfg, wl.layers[l]
         T, D, k = cfg.T, cfg.D, cfg.k
+        if self.layer_ws is not None:
+            if ev is not None:
+                ev[0].record(stream)
+            moe.moe_layer_forward(self.pools[l], L.slot_table, self.x[l], L.Wr, L.bias, k, self.ids, self.gates,
+                                  self.expert_out, self.miss_list, self.miss_count, self.x[l + 1], self.layer_ws,
+                                  residual=self.x[l], stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            if ids_out is not None:
+                ids_out[l].copy_(self.ids)
+            return
         moe.moe_route_topk(self.x[l], L.Wr, L.bias, k, self.ids, self.gates, self.route_ws, stream=stream)
         if ids_out is not None:
             ids_out[l].copy_(self.ids)
@@ -426,7 +480,7 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
     for l in range(NL):
         sl = wl.layers[l].slot_table.cpu().numpy()[ids_all[l].cpu().numpy()]
         u = len(np.unique(sl[sl >= 0]))
-        fwd_bytes.append((u + 1) * slot_bytes + T * D * 2)
+        fwd_bytes.append((u + 1) * slot_bytes + T * D * 2 + (E * D * 2 + T * D * 2 if buf.layer_ws is not None else 0))
         h = int((sl >= 0).sum())
         fwd_flops.append((h + T) * 6.0 * D * F)
         hits += h
@@ -452,7 +506,8 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
     peaks = _peaks()
     if T <= 8:
         roof = _roofline("hbm", float(np.sum(fwd_bytes)) / NL, float(np.sum(fwd_ms)) / NL, peaks, "decode48")
-        roof["kernel"] = "moe_expert_forward (decode_ffn_kernel), averaged over the 48 layers"
+        roof["kernel"] = ("moe_layer_forward (decode_ffn_kernel, one-call layer), averaged over the 48 layers; "
+                          "bytes = Wr + resident experts read + x + out")
     else:
         roof = _roofline("tensor", float(np.sum(fwd_flops)) / NL, float(np.sum(fwd_ms)) / NL, peaks, "prefill48")
         roof["kernel"] = "moe_expert_forward (plan + gather + tcgen05 GEMMs), averaged over the 48 layers"
@@ -481,7 +536,7 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
         "e2e": {"value": round(ws_ * T * NL * K / (ems / 1e3), 1), "unit": "tokens/s (per layer)",
                 "chain_tokens_per_s": round(ws_ * T * K / (ems / 1e3), 2), "h2d_bytes_per_step": T * D * 2,
                 "d2h_bytes_per_step": T * D * 2},
-        "gpu_launches": LAUNCHES["decode" if T <= 8 else "prefill"] * NL * K,
+        "gpu_launches": LAUNCHES["layer" if buf.layer_ws is not None else "prefill"] * NL * K,
         "roofline": roof,
         "hit_rate": round(hits / n_sel, 4),
         "clocks": clocks,
@@ -595,7 +650,7 @@ def run_ours(args, ws_, rank, local):
         "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "roofline": head["roofline"],
         "clocks": head["clocks"],
     }
-    for key in ("hit_rate", "u_hit_mean", "step_alg_bytes", "chain_tokens_per_s", "expert_loads"):
+    for key in ("hit_rate", "u_hit_mean", "step_alg_bytes", "chain_tokens_per_s", "expert_loads", "three_calls"):
         if key in head:
             line[key] = head[key]
     if "cpu_baseline" in head:

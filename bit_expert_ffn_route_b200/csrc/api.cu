@@ -137,6 +137,36 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
                                            (cudaStream_t)stream));
 }
 
+size_t moe_layer_workspace_size(int T, int D, int F, int E, int k, int fmt) {
+    if (check_shapes(T, D, E, k) != MOE_OK || F <= 0 || !fmt_ok(fmt) || T > kDecodeMaxT) return 0;
+    return layer_workspace_bytes(T, D, F, E, k);
+}
+
+moe_status moe_layer_forward(const moe_pool* pool, const int32_t* slot_table, int E, const uint16_t* x, int T,
+                             const uint16_t* Wr, const float* bias, int k, int32_t* ids, float* gates,
+                             void* expert_out, size_t expert_out_bytes_, int32_t* miss_list, int32_t* miss_count,
+                             const uint16_t* residual, uint16_t* out, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
+    PoolView v;
+    moe_status st = check_pool(pool, v);
+    if (st != MOE_OK) return st;
+    st = check_shapes(T, v.D, E, k);
+    if (st != MOE_OK) return st;
+    if (T > kDecodeMaxT) return MOE_ERR_UNSUPPORTED;
+    if (!miss_count) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return cuda_status(cudaMemsetAsync(miss_count, 0, sizeof(int32_t), (cudaStream_t)stream));
+    if (!slot_table || !x || !Wr || !ids || !gates || !expert_out || !miss_list || !out || !ws)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(Wr, 16) || !aligned(expert_out, 256) || !aligned(ws, 256) ||
+        !aligned(out, 16) || (residual && !aligned(residual, 16)))
+        return MOE_ERR_INVALID_ARG;
+    if (out == x) return MOE_ERR_INVALID_ARG;
+    if (expert_out_bytes_ < expert_out_bytes(T, v.D, k)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < layer_workspace_bytes(T, v.D, v.F, E, k)) return MOE_ERR_WORKSPACE;
+    return reported(launch_layer_forward(v, slot_table, E, x, T, Wr, bias, k, ids, gates, expert_out, miss_list,
+                                         miss_count, residual, out, ws, (cudaStream_t)stream));
+}
+
 moe_status moe_combine(const void* expert_out, const float* gates, int T, int D, int k, const float* miss_partial,
                        const uint16_t* residual, uint16_t* out, moe_stream_t stream) {
     if (T < 0 || D <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;

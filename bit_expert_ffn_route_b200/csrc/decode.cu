@@ -44,6 +44,7 @@
 #include "dequant.cuh"
 #include "kernels.cuh"
 #include "once.cuh"
+#include "route_warp.cuh"
 #include "sync.cuh"
 #include "tmap.cuh"
 
@@ -173,10 +174,22 @@ struct DecodeParams {
     // of D weights, down as D rows of F weights; codes and (s, m) planes
     // (Q3_S256: the code maps only)
     CUtensorMap tm_gu_c, tm_gu_m, tm_dn_c, tm_dn_m;
+    // the one-call layer (moe_layer_forward): routing in the kernel, combine
+    // at the end (unused otherwise)
+    const uint16_t* Wr;    // [E][D] bf16
+    const float* bias;     // [E] or null
+    int route_j;           // experts whose logits each CTA computes (CTA b: route_j * b + j)
+    int route_wr_smem;     // 1: those Wr rows are copied into the stage ring (after x), else read from L2
+    float* logits;         // [T][E] fp32 scratch
+    int32_t* ids_out;      // [T][k]
+    float* gates_out;      // [T][k]
+    const uint16_t* residual;   // [T][D] bf16 or null
+    uint16_t* out;         // [T][D] bf16
 };
 
 constexpr int kRedBufs = 3;                        // partial-sum buffers per team (items in flight)
 constexpr int kPubRing = 64;                       // finished gate|up items awaiting release
+constexpr uint32_t kPubEnd = 0xffffffffu;          // ring entry: no more items (others: owner + 1)
 
 struct Shared {
     uint64_t full[kMaxStages];
@@ -190,8 +203,11 @@ struct Shared {
     uint32_t red_cnt[kTeams][kRedBufs];   // warps that wrote their partials into a buffer
     uint32_t red_gen[kTeams][kRedBufs];   // reductions completed on a buffer
     uint32_t pub_head;             // finished gate|up items queued for the publisher
-    int pubq[kPubRing];            // their owners + 1 (0: free; -1: no more items)
+    int pubq[kPubRing];            // their owners + 1 (0: free; kPubEnd: no more items)
     uint32_t finished;             // warps (consumers, producer) that are done
+    int32_t sids[kDecodeMaxT * kMaxTopK];   // one-call layer: the selected ids and gates
+    float sgates[kDecodeMaxT * kMaxTopK];
+    float sbias[kConsumerWarps];    // the router bias of this CTA's logit experts
 };
 
 // The slot table is an input of the layer, not produced by the router: stage it
@@ -222,26 +238,33 @@ MOE_DEVINL int lookup_slot(const DecodeParams& prm, const Shared& sh, int e) {
 
 // One warp: resolve every pair's slot and the owners — owner 0 is the shared
 // expert, then the first pair of each distinct resident expert in pair order —
-// and, with `book`, the row map, miss list and miss count.  Lane L handles
+// and, with `book`, the row map, miss list and miss count.  The ids come
+// from global memory (prm.ids) or, in the one-call layer, from shared memory
+// (ids_smem).  Lane L handles
 // pairs L + 32h (h = 0..3; T * k <= 128).  Pairs of one expert find their
 // owner through a shared-memory minimum per expert id (`first`: E ints, all
 // kMaxPairs on entry); each pair then sets its rank bit in its owner's token
 // mask.  (Two expert ids on one slot would get
 // two owners over the same weights: the same outputs, computed twice.)
-__device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, bool book) {
+__device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, bool book,
+                               const int32_t* ids_smem) {
     constexpr int H = (kMaxPairs - 1 + 31) / 32;
     const int lane = threadIdx.x & 31;
     const int T = prm.T, k = prm.k, n = T * k;   // n <= 128
+    const int hn = (n + 31) >> 5;                // pair groups in use (warp-uniform)
     const uint32_t below = (1u << lane) - 1u;
-    int e[H], s[H];
+    int e[H], s[H], tt[H], rr[H];
     uint32_t missb[H];
 #pragma unroll
     for (int h = 0; h < H; ++h) {
         const int p = lane + 32 * h;
-        e[h] = p < n ? __ldg(prm.ids + p) : -1;
+        e[h] = h < hn && p < n ? (ids_smem ? ids_smem[p] : __ldg(prm.ids + p)) : -1;
+        tt[h] = p / k;
+        rr[h] = p - tt[h] * k;
     }
 #pragma unroll
     for (int h = 0; h < H; ++h) {
+        if (h >= hn) break;
         const int p = lane + 32 * h;
         s[h] = p < n ? lookup_slot(prm, sh, e[h]) : -1;
         if (s[h] >= 0) atomicMin(first + e[h], p);
@@ -251,9 +274,10 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, 
         int base = 0;
 #pragma unroll
         for (int h = 0; h < H; ++h) {
+            if (h >= hn) break;
             const int p = lane + 32 * h;
             if (p < n) {
-                const int t = p / k, r = p % k;
+                const int t = tt[h], r = rr[h];
                 prm.rowmap[t * (k + 1) + r] = s[h] >= 0 ? t * (k + 1) + r : -1;
                 if (s[h] < 0) {
                     const int pos = base + __popc(missb[h] & below);
@@ -269,6 +293,7 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, 
     int base = 1;
 #pragma unroll
     for (int h = 0; h < H; ++h) {
+        if (h >= hn) break;
         const int p = lane + 32 * h;
         const bool own = s[h] >= 0 && first[e[h]] == p;
         const uint32_t ownb = __ballot_sync(0xffffffffu, own);
@@ -289,8 +314,8 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, 
     __syncwarp();
 #pragma unroll
     for (int h = 0; h < H; ++h) {
-        const int p = lane + 32 * h;
-        if (s[h] >= 0) atomicOr(&sh.owners[sh.oidx[first[e[h]]]].rmask[p / k], 1u << (p % k));
+        if (h >= hn) break;
+        if (s[h] >= 0) atomicOr(&sh.owners[sh.oidx[first[e[h]]]].rmask[tt[h]], 1u << rr[h]);
     }
     __syncwarp();
 }
@@ -322,7 +347,7 @@ MOE_DEVINL bool half_block_frag(const uint4 a, const uint4 b, uint2 (&out)[4]) {
 // columns >= T zero).  Run by `nthreads` threads starting at thread `first`.
 template <int NSLOT>
 __device__ void stage_x_frag(const uint16_t* __restrict__ x, int T, int K, uint8_t* xs, uint32_t* err, int first,
-                             int nthreads) {
+                             int nthreads, uint16_t* xcopy = nullptr) {
     const int nhb = K / 16;
     bool ok = true;
     for (int idx = (int)threadIdx.x - first; idx < NSLOT * nhb; idx += nthreads) {
@@ -330,7 +355,13 @@ __device__ void stage_x_frag(const uint16_t* __restrict__ x, int T, int K, uint8
         uint2 o[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
         if (n < T) {
             const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)n * K + 16 * hb);
-            ok &= half_block_frag(__ldg(p), __ldg(p + 1), o);
+            const uint4 a = __ldg(p), b = __ldg(p + 1);
+            ok &= half_block_frag(a, b, o);
+            if (xcopy) {                 // and the rows as they are (bf16 [T][K])
+                uint4* c = reinterpret_cast<uint4*>(xcopy + (size_t)n * K + 16 * hb);
+                c[0] = a;
+                c[1] = b;
+            }
         }
         // hb = U * 8 + c * 2 + i
         const int U = hb >> 3, c = (hb >> 1) & 3, i = hb & 1;
@@ -617,7 +648,139 @@ MOE_DEVINL uint32_t ld_acquire(const uint32_t* p) {
 // team's buffer, and the last one to do so reduces them and queues the item for
 // the publisher.  The last CTA to finish resets the counters, so every
 // completed call leaves them zero.
-template <int FMT, int NSLOT>
+// ---------------------------------------------------------------- one-call layer
+// The 512 consumer threads meet at named barrier 5.
+MOE_DEVINL void consumers_sync() { asm volatile("bar.sync 5, %0;" ::"n"(kConsumers) : "memory"); }
+
+// Queue one entry for the publisher warp (one lane): waits (bounded) for the
+// ring slot to be free, then releases the entry (with the caller's prior
+// writes, ordered before it by the caller's __syncwarp).
+MOE_DEVINL void pub_push(Shared& sh, uint32_t v) {
+    const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]);
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_cta(slot) != 0u && globaltimer_ns() - t0 < kWaitLimitNs) {}
+    st_release_cta(slot, v);
+}
+
+// Byte offset of the routing Wr rows in the stage ring (after x, bf16 [T][D]).
+__host__ __device__ constexpr size_t wr_ring_offset(int T, int D) { return ((size_t)T * D * 2 + 127) & ~(size_t)127; }
+
+// Grid-wide barrier over one counter (thread 0 of each CTA; every CTA of the
+// grid is resident: one CTA per SM).  False, with the timeout bit set, if the
+// other CTAs did not all arrive within the wait limit.
+MOE_DEVINL bool grid_arrive_wait(uint32_t* count, uint32_t* err) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire(count) < gridDim.x) {
+        if (timed_out(err) || globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Routing inside the expert-pass kernel, by the consumer warps of every CTA:
+// x staged in fp16 fragment order for the expert pass and, as it is (bf16), in
+// the stage ring for the logits; the logits of this CTA's experts route_j * b + j (warp j, the
+// router's canonical order and bias; their Wr rows copied into the ring after
+// x before the dependency wait, completing on wbar, or read from L2 when they
+// do not fit); a grid-wide barrier; then every CTA selects every token's top-k
+// itself (the router's selection) into shared memory, and CTA 0 writes the
+// ids and gates.  Returns false (on every consumer thread) when a wait gave
+// up: the CTA then does no expert work, and CTA 0 writes ids -1 and gates 0.
+template <int NSLOT>
+__device__ bool route_phase(const DecodeParams& prm, Shared& sh, uint8_t* xs, uint8_t* ring, uint64_t* wbar,
+                            bool rows_issued, uint32_t* grid_count) {
+    const int warp = threadIdx.x >> 5;
+    const int T = prm.T, D = prm.P.D, E = prm.E, k = prm.k, J = prm.route_j;
+    uint16_t* xb = reinterpret_cast<uint16_t*>(ring);
+    const uint16_t* wsm = reinterpret_cast<const uint16_t*>(ring + wr_ring_offset(T, D));
+    stage_x_frag<NSLOT>(prm.x, T, D, xs, prm.err, 0, kConsumers, xb);
+    __shared__ int x_ok;
+    if (threadIdx.x == 0) {
+        bool ok = true;
+        if (rows_issued) {
+            ok = mbar_wait(wbar, 0, prm.err);
+            if (!ok) mbar_drain(wbar, 0);        // the copy lands before the ring is reused
+        }
+        x_ok = ok;
+    }
+    consumers_sync();
+    // one (expert, token) logit per warp at a time: the per-token sums are
+    // independent, so spreading them over the warps keeps the canonical order
+    for (int q = warp; x_ok && q < J * T; q += kConsumerWarps) {
+        const int j = q % J, t = q / J, e = J * (int)blockIdx.x + j;
+        if (e >= E) continue;
+        if (prm.route_wr_smem)
+            canon_logits_warp_xbf16<1, true>(xb + (size_t)t * D, 1, D, wsm + (size_t)j * D, prm.bias != nullptr,
+                                             sh.sbias[j], E, e, prm.logits + (size_t)t * E);
+        else
+            canon_logits_warp_xbf16<1, false>(xb + (size_t)t * D, 1, D, prm.Wr + (size_t)e * D, prm.bias != nullptr,
+                                              sh.sbias[j], E, e, prm.logits + (size_t)t * E);
+    }
+    // generic reads of the ring precede the bulk copies that land there later
+    fence_proxy_async();
+    consumers_sync();
+    __shared__ int routed;           // one decision for the whole CTA
+    if (threadIdx.x == 0) routed = grid_arrive_wait(grid_count, prm.err) && !timed_out(prm.err) ? 1 : 0;
+    consumers_sync();
+    if (!routed) {
+        if (blockIdx.x == 0)
+            for (int i = threadIdx.x; i < T * k; i += kConsumers) { prm.ids_out[i] = -1; prm.gates_out[i] = 0.f; }
+        return false;
+    }
+    if (warp < T) topk_warp(prm.logits + (size_t)warp * E, E, k, sh.sids + warp * k, sh.sgates + warp * k);
+    consumers_sync();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < T * k; i += kConsumers) { prm.ids_out[i] = sh.sids[i]; prm.gates_out[i] = sh.sgates[i]; }
+    return true;
+}
+
+// The gate-weighted combine of this CTA's slice of the outputs, after every
+// expert row is written: task i = (t, feature pair 2q) of the T * D / 2 tasks,
+// CTA b taking a contiguous range; each sums its two features in
+// moe_combine's order (hit ranks ascending with fmaf, then the shared expert,
+// then the residual), rounds to bf16 and writes out.  Every row of a task is
+// loaded before the sums (one round trip); rows written by other CTAs are read
+// from L2.
+__device__ void combine_slice(const DecodeParams& prm, const Shared& sh) {
+    const int T = prm.T, D = prm.P.D, k = prm.k, half = D / 2;
+    const int total = T * half, per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int end = min(total, ((int)blockIdx.x + 1) * per);
+    const float* rows = prm.yrows;
+    for (int task = (int)blockIdx.x * per + (int)threadIdx.x; task < end; task += (int)blockDim.x) {
+        const int t = task / half, d = 2 * (task - t * half);
+        float2 y[kMaxTopK];
+        bool hit[kMaxTopK];
+#pragma unroll
+        for (int r = 0; r < kMaxTopK; ++r) {
+            hit[r] = r < k && lookup_slot(prm, sh, sh.sids[t * k + r]) >= 0;
+            y[r] = hit[r] ? __ldcg(reinterpret_cast<const float2*>(rows + (size_t)(t * (k + 1) + r) * D + d))
+                          : make_float2(0.f, 0.f);
+        }
+        const float2 ys = __ldcg(reinterpret_cast<const float2*>(rows + (size_t)(t * (k + 1) + k) * D + d));
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxTopK; ++r) {
+            if (hit[r]) {
+                const float g = sh.sgates[t * k + r];
+                a0 = __fmaf_rn(g, y[r].x, a0);
+                a1 = __fmaf_rn(g, y[r].y, a1);
+            }
+        }
+        a0 += ys.x; a1 += ys.y;
+        if (prm.residual) {
+            const uint32_t rv = *reinterpret_cast<const uint32_t*>(prm.residual + (size_t)t * D + d);
+            a0 += bf16lo(rv); a1 += bf16hi(rv);
+        }
+        *reinterpret_cast<uint32_t*>(prm.out + (size_t)t * D + d) =
+            (uint32_t)f32_to_bf16_rne(a0) | ((uint32_t)f32_to_bf16_rne(a1) << 16);
+    }
+}
+
+template <int FMT, int NSLOT, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_constant__ DecodeParams prm) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ Shared sh;
@@ -653,24 +816,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
     // word is read before the dependency wait: only this kernel writes it, and
     // its previous launch on the stream completed before the router that
     // precedes this launch passed its own wait.
+    // (one-call layer: the word is read after the dependency wait, since the
+    // previous launch on the workspace may still run until then)
     __shared__ int dead;
-    if (threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
+    if (!FUSED && threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
     // the partial-sum buffers are free until the first item: owner resolution
     // keeps its per-expert scratch there
     int* first = reinterpret_cast<int*>(red);
     stage_table(prm, sh, first);
+    // one-call layer: this CTA's Wr rows (weights, not produced by the
+    // preceding kernel) are prefetched into L2 before the wait, and the bias of
+    // each logit warp's expert is loaded
+    __shared__ uint64_t wbar;
+    const int e0 = prm.route_j * (int)blockIdx.x;
+    const bool rows_issued = FUSED && prm.route_wr_smem && min(prm.route_j, prm.E - e0) > 0;
+    if constexpr (FUSED) {
+        const int nrows = min(prm.route_j, prm.E - e0);
+        if (threadIdx.x == 0) {
+            mbar_init(&wbar, 1);
+            fence_mbar_init();
+            if (rows_issued) {
+                mbar_arrive_expect_tx(&wbar, (uint32_t)nrows * D * 2u);
+                bulk_g2s(stages + wr_ring_offset(prm.T, D), prm.Wr + (size_t)e0 * D, (uint32_t)nrows * D * 2u, &wbar);
+            } else if (nrows > 0) {
+                prefetch_l2(prm.Wr + (size_t)e0 * D, (uint32_t)nrows * D * 2u);
+            }
+        }
+        if (threadIdx.x < prm.route_j)
+            sh.sbias[threadIdx.x] = e0 + (int)threadIdx.x < prm.E && prm.bias ? __ldg(prm.bias + e0 + threadIdx.x) : 0.f;
+    }
     __syncthreads();
-    pdl_wait();                      // ids come from the router
+    pdl_wait();                      // ids come from the router (x: from the previous layer)
+    if constexpr (FUSED) {
+        if (threadIdx.x == 0) dead = timed_out(prm.err) ? 1 : 0;
+        __syncthreads();
+    }
     if (!dead) {
     // warp 0 resolves the owners and releases the producer and publisher
     // (barrier 1) while the other consumers stage x; the consumers meet at
-    // barrier 4 before computing
+    // barrier 4 before computing.  One-call layer: all consumers first route
+    // (and stage x), and a CTA whose routing gave up has no owners.
+    bool routed = true;
+    if constexpr (FUSED)
+        if (warp < kConsumerWarps)
+            routed = route_phase<NSLOT>(prm, sh, xs, stages, &wbar, rows_issued, queue + 1);
     if (warp == 0) {
-        resolve_owners(prm, sh, first, blockIdx.x == 0);
+        if (routed) {
+            resolve_owners(prm, sh, first, blockIdx.x == 0, FUSED ? sh.sids : nullptr);
+        } else if (lane == 0) {
+            sh.n_owners = 0;
+        }
+        __syncwarp();
         asm volatile("bar.arrive 1, 96;" ::: "memory");
         asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
     } else if (warp < kConsumerWarps) {
-        stage_x_frag<NSLOT>(prm.x, prm.T, D, xs, prm.err, 32, kConsumers - 32);
+        if constexpr (!FUSED) stage_x_frag<NSLOT>(prm.x, prm.T, D, xs, prm.err, 32, kConsumers - 32);
         asm volatile("bar.sync 4, %0;" ::"n"(kConsumers) : "memory");
     } else {
         asm volatile("bar.sync 1, 96;" ::: "memory");
@@ -719,6 +919,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         // issue the copies
         int j = 0, issued = 0;
         bool ok = true;
+        // the next item is taken from the queue one step ahead, so the
+        // atomic's round trip overlaps the wait for a free stage
         // the next item is taken from the queue one step ahead, so the
         // atomic's round trip overlaps the wait for a free stage
         int next = 0;
@@ -800,10 +1002,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     if (q >= 0) mbar_drain(&sh.full[q % NS], (q / NS) & 1);
         }
         __syncwarp();
-        if (lane == 0 && atomicAdd(&sh.finished, 1u) == kConsumerWarps) {   // the last worker warp
-            const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
-            st_release_cta(reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]), 0xffffffffu);
-        }
+        if (lane == 0 && atomicAdd(&sh.finished, 1u) == kConsumerWarps) pub_push(sh, kPubEnd);   // the last worker warp
     } else {
         // consumer teams: team tm takes stages j = tm, tm + 2, ... of the ring;
         // the warps of a team work through the same items without waiting on
@@ -856,11 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
                     if (lane == 0) {
                         sh.red_cnt[team][b] = 0;
                         st_release_cta(&sh.red_gen[team][b], use + 1);
-                        const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
-                        uint32_t* slot = reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]);
-                        const uint64_t t0 = globaltimer_ns();
-                        while (ld_acquire_cta(slot) != 0u && globaltimer_ns() - t0 < kWaitLimitNs) {}   // ring slot free
-                        st_release_cta(slot, (uint32_t)(ip.u + 1));
+                        pub_push(sh, (uint32_t)(ip.u + 1));
                     }
                 }
             } else {
@@ -872,12 +1067,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
         }
         // the last worker warp to finish tells the publisher that no more items come
         __syncwarp();
-        if (lane == 0 && atomicAdd(&sh.finished, 1u) == kConsumerWarps) {
-            const uint32_t pos = atomicAdd(&sh.pub_head, 1u);
-            st_release_cta(reinterpret_cast<uint32_t*>(&sh.pubq[pos % kPubRing]), 0xffffffffu);
-        }
+        if (lane == 0 && atomicAdd(&sh.finished, 1u) == kConsumerWarps) pub_push(sh, kPubEnd);
     }
     }   // !dead
+    if constexpr (FUSED) {
+        if (dead && rows_issued && threadIdx.x == 0) mbar_drain(&wbar, 0);   // the Wr copy lands before exit
+        // one-call layer: once every CTA's expert rows are written (a grid-wide
+        // barrier: release, this CTA's rows; acquire, every other CTA's), each
+        // CTA combines its slice of the outputs
+        __syncthreads();
+        __shared__ int comb_ok;
+        if (threadIdx.x == 0) {
+            const bool arrived = grid_arrive_wait(queue + 2, prm.err);
+            comb_ok = arrived && !dead && sh.n_owners > 0 && !timed_out(prm.err);
+        }
+        __syncthreads();
+        if (comb_ok) combine_slice(prm, sh);
+    }
     // last CTA out resets the per-owner counters and the queue for the next call
     // (acq_rel ticket: this CTA's counter updates, ordered before it by the
     // barrier, precede the reset; the last CTA sees every other CTA's)
@@ -889,6 +1095,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_ffn_kernel(const __grid_co
             for (int u = 0; u < kMaxPairs; ++u) done[u] = 0u;
             done[kMaxPairs] = 0u;
             done[kMaxPairs + 1] = 0u;
+            if constexpr (FUSED) {
+                done[kMaxPairs + 2] = 0u;                       // the routing barrier
+                done[kMaxPairs + 3] = 0u;                       // the combine barrier
+            }
         }
     }
 }
@@ -902,7 +1112,7 @@ size_t smem_for(int D, int F, int rf, int rd, int ns) {
 // Dynamic shared memory available to decode_ffn_kernel<FMT, NSLOT> on the
 // current device: the opt-in per-block limit less the kernel's static shared
 // memory, capped at kSmemBudget (looked up once per device; 0 if the query fails).
-template <int FMT, int NSLOT>
+template <int FMT, int NSLOT, bool FUSED>
 int smem_budget() {
     static std::atomic<int> cache[64];
     int dev = 0;
@@ -914,7 +1124,7 @@ int smem_budget() {
     int optin = 0;
     cudaFuncAttributes fa;
     if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-        cudaFuncGetAttributes(&fa, decode_ffn_kernel<FMT, NSLOT>) != cudaSuccess)
+        cudaFuncGetAttributes(&fa, decode_ffn_kernel<FMT, NSLOT, FUSED>) != cudaSuccess)
         return 0;
     int b = optin - (int)fa.sharedSizeBytes;
     if (b > kSmemBudget) b = kSmemBudget;
@@ -922,11 +1132,11 @@ int smem_budget() {
     return b;
 }
 
-template <int FMT, int NSLOT>
+template <int FMT, int NSLOT, bool FUSED>
 moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
     const PoolView& P = prm.P;
     const int D = P.D, F = P.F;
-    const int budget = smem_budget<FMT, NSLOT>();
+    const int budget = smem_budget<FMT, NSLOT, FUSED>();
     if (budget <= 0) return MOE_ERR_CUDA;
     // gate|up items of rf features (two 16-row tiles), down items of rd rows
     // (eight 16-row tiles, one per warp of a team), up to 4 stages (3-4 items in
@@ -967,11 +1177,18 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
     }
     static std::atomic<uint64_t> attr_done{0};
     if (!once_per_device(attr_done, [] {
-            return cudaFuncSetAttribute(decode_ffn_kernel<FMT, NSLOT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        smem_budget<FMT, NSLOT>()) == cudaSuccess;
+            return cudaFuncSetAttribute(decode_ffn_kernel<FMT, NSLOT, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        smem_budget<FMT, NSLOT, FUSED>()) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
-    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NSLOT>, dim3(device_sm_count()), dim3(kThreads), smem, s, prm);
+    if constexpr (FUSED) {
+        // routing in the kernel: x (bf16) fits in the stage ring, one logit warp per expert
+        prm.route_j = (prm.E + device_sm_count() - 1) / device_sm_count();
+        const size_t ring = (size_t)ns * stage_size<FMT, NSLOT>(D, F, rf, rd);
+        if ((size_t)prm.T * D * 2 > ring || prm.route_j > kConsumerWarps) return MOE_ERR_UNSUPPORTED;
+        prm.route_wr_smem = wr_ring_offset(prm.T, D) + (size_t)prm.route_j * D * 2 <= ring ? 1 : 0;
+    }
+    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NSLOT, FUSED>, dim3(device_sm_count()), dim3(kThreads), smem, s, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -986,11 +1203,10 @@ size_t decode_workspace_bytes(int T, int D, int F, int k) {
     return 1024 + (size_t)kMaxPairs * (T <= 4 ? 4 : 8) * F * sizeof(uint16_t);
 }
 
-moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
-                                 const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
-                                 int32_t* miss_count, void* ws, cudaStream_t s) {
-    if (P.D % kUnitK || P.F % kUnitK) return MOE_ERR_UNSUPPORTED;
-    DecodeParams prm;
+namespace {
+DecodeParams expert_params(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
+                           const int32_t* ids, int k, void* expert_out, int32_t* miss_list, int32_t* miss_count) {
+    DecodeParams prm{};
     prm.P = P;
     prm.slot_table = slot_table;
     prm.E = E;
@@ -1002,21 +1218,65 @@ moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, i
     prm.yrows = reinterpret_cast<float*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T, k));
     prm.miss_list = miss_list;
     prm.miss_count = miss_count;
+    return prm;
+}
+
+template <bool FUSED>
+moe_status launch_any(DecodeParams prm, cudaStream_t s) {
+    if (prm.T <= 4) {
+        switch (prm.P.fmt) {
+            case MOE_Q2_32: return launch_fmt<MOE_Q2_32, 4, FUSED>(prm, s);
+            case MOE_Q3_32: return launch_fmt<MOE_Q3_32, 4, FUSED>(prm, s);
+            default: return launch_fmt<MOE_Q3_S256, 4, FUSED>(prm, s);
+        }
+    }
+    switch (prm.P.fmt) {
+        case MOE_Q2_32: return launch_fmt<MOE_Q2_32, 8, FUSED>(prm, s);
+        case MOE_Q3_32: return launch_fmt<MOE_Q3_32, 8, FUSED>(prm, s);
+        default: return launch_fmt<MOE_Q3_S256, 8, FUSED>(prm, s);
+    }
+}
+
+// one-call layer ws: [4,8) error word, [64, ...) counters (as the expert
+// pass's, plus the routing and combine barriers), [1024, 33792) logits [T][E]
+// fp32, then h.
+constexpr size_t kLayerLogits = 1024, kLayerH = 1024 + (size_t)kDecodeMaxT * 1024 * 4;
+}  // namespace
+
+moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
+                                 const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
+                                 int32_t* miss_count, void* ws, cudaStream_t s) {
+    if (P.D % kUnitK || P.F % kUnitK) return MOE_ERR_UNSUPPORTED;
+    DecodeParams prm = expert_params(P, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count);
     prm.err = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
     prm.done = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 64);
     prm.hfrag = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 1024);
-    if (T <= 4) {
-        switch (P.fmt) {
-            case MOE_Q2_32: return launch_fmt<MOE_Q2_32, 4>(prm, s);
-            case MOE_Q3_32: return launch_fmt<MOE_Q3_32, 4>(prm, s);
-            default: return launch_fmt<MOE_Q3_S256, 4>(prm, s);
-        }
-    }
-    switch (P.fmt) {
-        case MOE_Q2_32: return launch_fmt<MOE_Q2_32, 8>(prm, s);
-        case MOE_Q3_32: return launch_fmt<MOE_Q3_32, 8>(prm, s);
-        default: return launch_fmt<MOE_Q3_S256, 8>(prm, s);
-    }
+    return launch_any<false>(prm, s);
+}
+
+size_t layer_workspace_bytes(int T, int D, int F, int E, int k) {
+    (void)D; (void)E; (void)k;
+    return kLayerH + (size_t)kMaxPairs * (T <= 4 ? 4 : 8) * F * sizeof(uint16_t);
+}
+
+moe_status launch_layer_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
+                                const uint16_t* Wr, const float* bias, int k, int32_t* ids, float* gates,
+                                void* expert_out, int32_t* miss_list, int32_t* miss_count, const uint16_t* residual,
+                                uint16_t* out, void* ws, cudaStream_t s) {
+    if (P.D % kUnitK || P.F % kUnitK || T > kDecodeMaxT || E > 1024) return MOE_ERR_UNSUPPORTED;
+    char* w = reinterpret_cast<char*>(ws);
+    DecodeParams prm = expert_params(P, slot_table, E, x, T, nullptr, k, expert_out, miss_list, miss_count);
+    prm.err = reinterpret_cast<uint32_t*>(w + 4);
+    prm.done = reinterpret_cast<uint32_t*>(w + 64);
+    prm.logits = reinterpret_cast<float*>(w + kLayerLogits);
+    prm.hfrag = reinterpret_cast<uint16_t*>(w + kLayerH);
+    prm.Wr = Wr;
+    prm.bias = bias;
+    prm.ids_out = ids;
+    prm.gates_out = gates;
+    prm.residual = residual;
+    prm.out = out;
+    return launch_any<true>(prm, s);
 }
 
 }  // namespace moe

@@ -38,6 +38,11 @@ moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, i
                                  int T, const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
                                  int32_t* miss_count, void* ws, cudaStream_t s);
 size_t decode_workspace_bytes(int T, int D, int F, int k);
+moe_status launch_layer_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
+                                const uint16_t* Wr, const float* bias, int k, int32_t* ids, float* gates,
+                                void* expert_out, int32_t* miss_list, int32_t* miss_count, const uint16_t* residual,
+                                uint16_t* out, void* ws, cudaStream_t s);
+size_t layer_workspace_bytes(int T, int D, int F, int E, int k);
 
 moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x,
                                   int T, const int32_t* ids, int k, void* expert_out, int32_t* miss_list,

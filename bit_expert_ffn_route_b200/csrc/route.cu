@@ -43,27 +43,7 @@ __global__ void __launch_bounds__(128) route_decode_kernel(const uint16_t* __res
     }
     const float bias_e = (bias && e < E) ? __ldg(bias + e) : 0.0f;   // a weight too: load it now
     pdl_wait();
-    // stage x: every load of a batch is in flight before the first store
-    constexpr int kBatch = 16;
-    const int n16 = T * D / 8;
-    for (int i0 = 0; i0 < n16; i0 += kBatch * 128) {
-        uint4 v[kBatch];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int i = i0 + q * 128 + (int)threadIdx.x;
-            v[q] = i < n16 ? __ldg(reinterpret_cast<const uint4*>(x) + i) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int i = i0 + q * 128 + (int)threadIdx.x;
-            if (i < n16) {
-                const int t = (8 * i) / D, d = 8 * i - t * D;
-                float* dst = xsf + (size_t)t * D + canon_stage_pos(d);
-                *reinterpret_cast<float4*>(dst) = make_float4(bf16lo(v[q].x), bf16hi(v[q].x), bf16lo(v[q].y), bf16hi(v[q].y));
-                *reinterpret_cast<float4*>(dst + 128) = make_float4(bf16lo(v[q].z), bf16hi(v[q].z), bf16lo(v[q].w), bf16hi(v[q].w));
-            }
-        }
-    }
+    stage_x_canon(x, T, D, xsf, (int)threadIdx.x, 128);
     __syncthreads();
     pdl_launch_dependents();
     const bool have_w = mbar_wait(&wbar, 0, err);

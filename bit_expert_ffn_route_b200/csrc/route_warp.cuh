@@ -15,6 +15,33 @@ __device__ __forceinline__ int canon_stage_pos(int d) {
     return (c << 8) + ((j >> 2) << 7) + (L << 2) + (j & 3);
 }
 
+// Stage T bf16 token rows [T][D] into xsf as fp32 in the canon_stage_pos
+// layout, threads tid = 0..nthreads-1 of the caller; every load of a batch is
+// in flight before the first store.
+__device__ __forceinline__ void stage_x_canon(const uint16_t* __restrict__ x, int T, int D, float* xsf, int tid,
+                                              int nthreads) {
+    constexpr int kBatch = 16;
+    const int n16 = T * D / 8;
+    for (int i0 = 0; i0 < n16; i0 += kBatch * nthreads) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int i = i0 + q * nthreads + tid;
+            v[q] = i < n16 ? __ldg(reinterpret_cast<const uint4*>(x) + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int i = i0 + q * nthreads + tid;
+            if (i < n16) {
+                const int t = (8 * i) / D, d = 8 * i - t * D;
+                float* dst = xsf + (size_t)t * D + canon_stage_pos(d);
+                *reinterpret_cast<float4*>(dst) = make_float4(bf16lo(v[q].x), bf16hi(v[q].x), bf16lo(v[q].y), bf16hi(v[q].y));
+                *reinterpret_cast<float4*>(dst + 128) = make_float4(bf16lo(v[q].z), bf16hi(v[q].z), bf16lo(v[q].w), bf16hi(v[q].w));
+            }
+        }
+    }
+}
+
 // Canonical logits of expert e for NT tokens: lane L accumulates elements
 // 256c + 8L + j (c ascending), then the xor butterfly, then + bias.  The token
 // rows are staged in shared memory as fp32 (exact copies of the bf16 values)
@@ -67,6 +94,63 @@ __device__ __forceinline__ void canon_logits_warp_staged(const float* __restrict
     }
 }
 
+// The same logits (same order, same arithmetic) with the token rows staged as
+// bf16 [nt][D] in natural order in shared memory and the expert's Wr row read
+// from shared memory (W_SHARED) or global memory (eight 16-byte loads of a
+// lane in flight at a time).
+template <int NT, bool W_SHARED>
+__device__ __forceinline__ void canon_logits_warp_xbf16(const uint16_t* __restrict__ xs /* [NT][D] */, int nt, int D,
+                                                        const uint16_t* __restrict__ wrow, bool has_bias,
+                                                        float bias_e, int E, int e,
+                                                        float* __restrict__ lout /* + t*E */) {
+    const int lane = threadIdx.x & 31;
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
+    const int nc = D >> 8;
+    for (int c0 = 0; c0 < nc; c0 += 8) {
+        uint4 wl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            wl[i] = c0 + i >= nc ? make_uint4(0, 0, 0, 0)
+                    : W_SHARED ? *reinterpret_cast<const uint4*>(wrow + 256 * (c0 + i) + 8 * lane)
+                               : ld_nc_u128(wrow + 256 * (c0 + i) + 8 * lane);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (c0 + i < nc) {
+                const int c = c0 + i;
+                const uint32_t wv[4] = {wl[i].x, wl[i].y, wl[i].z, wl[i].w};
+                float wf[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) { wf[2 * q] = bf16lo(wv[q]); wf[2 * q + 1] = bf16hi(wv[q]); }
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (t < nt) {
+                        const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)t * D + 256 * c + 8 * lane);
+                        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            acc[t] = __fmaf_rn(bf16lo(xw[q]), wf[2 * q], acc[t]);
+                            acc[t] = __fmaf_rn(bf16hi(xw[q]), wf[2 * q + 1], acc[t]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+            acc[t] = __fadd_rn(acc[t], __shfl_xor_sync(0xffffffffu, acc[t], off));
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            if (t < nt) lout[(size_t)t * E + e] = has_bias ? __fadd_rn(acc[t], bias_e) : acc[t];
+    }
+}
+
 // Order-preserving map of a float to an unsigned key (larger float, larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -97,6 +181,7 @@ __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_
                             float* __restrict__ gates) {
     __shared__ uint64_t s_keys[8][32];   // per warp: lane maxima, then the candidates
     __shared__ uint64_t s_sel[8][32];    // per warp: the selected keys by rank
+    __shared__ int s_n[8];               // per warp: candidates placed so far
     const int lane = threadIdx.x & 31, w = (threadIdx.x >> 5) & 7;
     uint64_t key[NV];
 #pragma unroll
@@ -118,9 +203,10 @@ __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_
     };
     uint64_t best = lane_best();
     s_keys[w][lane] = best;
+    if (lane == 0) s_n[w] = 0;
     __syncwarp();
     int above = 0;                           // lane maxima larger than this lane's
-#pragma unroll 8
+#pragma unroll
     for (int i = 0; i < 32; ++i) above += s_keys[w][i] > best;
     const uint32_t at_k = __ballot_sync(0xffffffffu, above == k - 1);   // keys are distinct: one lane
     const uint64_t tau = __shfl_sync(0xffffffffu, best, __ffs(at_k) - 1);
@@ -130,14 +216,9 @@ __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_
     const int total = (int)__reduce_add_sync(0xffffffffu, (uint32_t)cnt);
     uint64_t my = 0;
     if (total <= 32) {
-        int pos = cnt;                       // inclusive scan of the counts
-#pragma unroll
-        for (int off = 1; off < 32; off *= 2) {
-            const int o = __shfl_up_sync(0xffffffffu, pos, off);
-            if (lane >= off) pos += o;
-        }
-        pos -= cnt;
+        // the candidates in any order (each one's rank among them is counted)
         __syncwarp();
+        int pos = cnt ? atomicAdd(&s_n[w], cnt) : 0;
 #pragma unroll
         for (int i = 0; i < NV; ++i)
             if (key[i] >= tau) s_keys[w][pos++] = key[i];
@@ -145,7 +226,8 @@ __device__ void topk_warp_n(const float* __restrict__ lrow, int E, int k, int32_
         if (lane < total) {
             const uint64_t c = s_keys[w][lane];
             int rank = 0;
-            for (int i = 0; i < total; ++i) rank += s_keys[w][i] > c;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rank += (i < total && s_keys[w][i] > c);
             if (rank < k) s_sel[w][rank] = c;
         }
         __syncwarp();

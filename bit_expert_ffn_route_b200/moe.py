@@ -27,7 +27,7 @@ EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_s
            "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
            "moe_status_string", "moe_route_topk_static", "moe_expert_hist", "moe_cache_plan", "moe_slot_fill",
            "moe_workspace_status", "moe_debug_wait_flag", "moe_debug_operand_workspace_size",
-           "moe_debug_prefill_operand"]
+           "moe_debug_prefill_operand", "moe_layer_workspace_size", "moe_layer_forward"]
 
 
 class MoeError(RuntimeError):
@@ -87,6 +87,11 @@ def lib():
         L.moe_debug_operand_workspace_size.argtypes = [i, i]
         L.moe_debug_prefill_operand.restype = i
         L.moe_debug_prefill_operand.argtypes = [ctypes.POINTER(moe_pool), i, i, i, P, P, sz, P]
+        L.moe_layer_workspace_size.restype = sz
+        L.moe_layer_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.moe_layer_forward.restype = i
+        L.moe_layer_forward.argtypes = [ctypes.POINTER(moe_pool), P, i, P, i, P, P, i, P, P, P, sz, P, P, P, P, P, sz,
+                                        P]
         L.moe_status_string.restype = ctypes.c_char_p
         L.moe_status_string.argtypes = [i]
         _lib = L
@@ -128,6 +133,10 @@ def workspace_size(T, D, F, E, k, fmt) -> int:
     return int(lib().moe_workspace_size(T, D, F, E, k, fmt))
 
 
+def layer_workspace_size(T, D, F, E, k, fmt) -> int:
+    return int(lib().moe_layer_workspace_size(T, D, F, E, k, fmt))
+
+
 def expert_out_size(T, D, k) -> int:
     return int(lib().moe_expert_out_size(T, D, k))
 
@@ -161,6 +170,17 @@ def moe_expert_forward(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_l
                                   _p(expert_out), expert_out.numel(), _p(miss_list), _p(miss_count),
                                   _p(ws), ws.numel(), _stream(stream))
     _check("moe_expert_forward", st)
+
+
+def moe_layer_forward(pool: moe_pool, slot_table, x, Wr, bias, k, ids, gates, expert_out, miss_list, miss_count,
+                      out, ws, residual=None, stream=None):
+    """The one-call layer (T <= 8): routing, expert pass and combine in one launch."""
+    T = x.shape[0]
+    E = slot_table.shape[0]
+    st = lib().moe_layer_forward(ctypes.byref(pool), _p(slot_table), E, _p(x), T, _p(Wr), _p(bias), k, _p(ids),
+                                 _p(gates), _p(expert_out), expert_out.numel(), _p(miss_list), _p(miss_count),
+                                 _p(residual), _p(out), _p(ws), ws.numel(), _stream(stream))
+    _check("moe_layer_forward", st)
 
 
 def moe_combine(expert_out, gates, T, D, k, out, miss_partial=None, residual=None, stream=None):
@@ -250,6 +270,18 @@ class Layer:
         self.miss_list = torch.empty(max(T * k, 1), 3, dtype=torch.int32, device=device)
         self.miss_count = torch.zeros(1, dtype=torch.int32, device=device)
         self.out = torch.empty(T, D, dtype=torch.bfloat16, device=device)
+        n = layer_workspace_size(T, D, pool.d_ff, E, k, pool.fmt)
+        self.layer_ws = alloc_ws(n, device) if n else None
+
+    def fused(self, x, residual=None, out=None, stream=None):
+        """The same layer through moe_layer_forward (T <= 8; no miss_partial)."""
+        out = self.out if out is None else out
+        if self.layer_ws is None:
+            raise MoeError("moe_layer_forward", MOE_ERR_UNSUPPORTED)
+        moe_layer_forward(self.pool, self.slot_table, x, self.Wr, self.bias, self.k, self.ids, self.gates,
+                          self.expert_out, self.miss_list, self.miss_count, out, self.layer_ws, residual=residual,
+                          stream=stream)
+        return out
 
     def __call__(self, x, miss_partial=None, residual=None, out=None, stream=None, with_logits=False):
         out = self.out if out is None else out

@@ -251,6 +251,40 @@ moe_status moe_combine(const void* expert_out, const float* gates, int T, int D,
                        uint16_t* out, moe_stream_t stream);
 
 /*
+ * One MoE layer for a small batch (T <= 8) in one launch: the results of
+ *   moe_route_topk(x, ...) ; moe_expert_forward(...) ;
+ *   moe_combine(expert_out, gates, T, D, k, NULL, residual, out)
+ * bit for bit (ids, gates, expert_out rows of every hit and of the shared
+ * expert, the row map, miss_list, miss_count and out).  The pages do not split
+ * a decode layer into launches; this call is an addition of this library that
+ * keeps the routing, the expert pass and the combine in one persistent kernel:
+ * every CTA computes the logits of ceil(E / #SMs) experts, all CTAs meet at a
+ * grid-wide barrier (one CTA per SM, all resident), every CTA then selects
+ * every token's top-k itself; after the expert pass a second grid-wide
+ * barrier, then each CTA combines a slice of the outputs.
+ *   Arguments as in the three calls; residual bf16 [T][D] or NULL; out bf16
+ *   [T][D] (may alias residual, not x).  Missed experts contribute nothing to
+ *   out (to add them, call moe_combine again with miss_partial).
+ *   ws     device scratch of moe_layer_workspace_size bytes, 256-byte aligned,
+ *          zero before the first call (every completed call leaves its counters
+ *          zero); word 1 is the device error word (moe_workspace_status).
+ *          A call on a ws whose timeout bit is set does no work.  A bounded
+ *          wait that gives up sets the timeout bit and the call writes ids -1
+ *          and gates 0 (out is then not written).
+ *   T > 8, or shapes whose routing does not fit the kernel's shared memory
+ *   (the CTA's Wr rows and x as fp32 beside the expert pipeline; every shape
+ *   with D + F <= 4096 and E <= 1024 fits): MOE_ERR_UNSUPPORTED, nothing
+ *   launched (use the three calls).
+ */
+size_t moe_layer_workspace_size(int T, int D, int F, int E, int k, int fmt);
+moe_status moe_layer_forward(const moe_pool* pool, const int32_t* slot_table, int E,
+                             const uint16_t* x, int T, const uint16_t* Wr, const float* bias, int k,
+                             int32_t* ids, float* gates, void* expert_out, size_t expert_out_bytes,
+                             int32_t* miss_list, int32_t* miss_count,
+                             const uint16_t* residual, uint16_t* out,
+                             void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Test hook: dequantise one matrix of one slot to fp32, row-major
  * (matrix 0 = gate [F][D], 1 = up [F][D], 2 = down [D][F]).  Exact:
  * Q2_32/Q3_32 w = fmaf(s, q, m); Q3_S256 w = d*(sc-32)*(q-4).

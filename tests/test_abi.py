@@ -156,3 +156,21 @@ def test_operand_hook_argument_errors(L):
     assert op(m0=512) == moe.MOE_ERR_INVALID_ARG           # beyond d_ff
     assert op(dump=None) == moe.MOE_ERR_INVALID_ARG
     assert op(nb=64) == moe.MOE_ERR_WORKSPACE
+
+
+def test_layer_size_and_argument_errors(L):
+    assert L.moe_layer_workspace_size(4, 3072, 512, 512, 10, 0) >= 1024 + 32768
+    assert L.moe_layer_workspace_size(8, 3072, 512, 512, 10, 2) > L.moe_layer_workspace_size(4, 3072, 512, 512, 10, 2)
+    assert L.moe_layer_workspace_size(9, 3072, 512, 512, 10, 0) == 0      # one call covers T <= 8
+    assert L.moe_layer_workspace_size(4, 3000, 512, 512, 10, 0) == 0
+    f, g = _fake(), _fake(1 << 21)
+    lf = lambda pool, T=4, E=512, k=10, eo=1 << 30, ws=1 << 30, x=f, out=g: L.moe_layer_forward(
+        ctypes.byref(pool), f, E, x, T, f, None, k, f, f, f, eo, f, f, None, out, f, ws, None)
+    assert lf(_pool(fmt=5)) == moe.MOE_ERR_INVALID_ARG
+    assert lf(_pool(D=3000)) == moe.MOE_ERR_UNSUPPORTED
+    assert lf(_pool(), T=9) == moe.MOE_ERR_UNSUPPORTED
+    assert lf(_pool(), k=17) == moe.MOE_ERR_UNSUPPORTED
+    assert lf(_pool(), eo=16) == moe.MOE_ERR_WORKSPACE
+    assert lf(_pool(), ws=16) == moe.MOE_ERR_WORKSPACE
+    assert lf(_pool(), out=None) == moe.MOE_ERR_INVALID_ARG
+    assert lf(_pool(), x=f, out=f) == moe.MOE_ERR_INVALID_ARG        # out may not alias x
