@@ -12,6 +12,9 @@
  *   moe_combine         gate-weighted sum of the expert outputs + shared
  *                       expert (+ caller's partial for the misses) (+ residual)
  *
+ * and, for decode batches (T <= 8), moe_layer_forward: the three in one launch
+ * (without the misses' partial), with the same results.
+ *
  * Sources: 512 routed experts per layer, 10 routed + 1 shared per token
  * (wiselychen RTX 5090 report, "30 秒定位"; greenbean-ai "Strata 如何讓 12GB
  * 顯卡跑 Qwen3.8-Flash-Next", §一).  The GPU runs the routing and the shared
