@@ -324,25 +324,51 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
         roof = _roofline("tensor", float(np.mean([fwd_flops[i % R] for i in range(G)])), fwd_avg_ms, peaks, "prefill")
         roof["kernel"] = "moe_expert_forward (plan + gather + tcgen05 gate|up and down grouped GEMMs)"
 
-    # end to end through the public API: pinned host input -> device, the three
-    # calls, device -> pinned host output, every step
+    # end to end through the public API: pinned host input -> device, the layer
+    # call(s), device -> pinned host output, every step.  The copies run on a
+    # copy stream, pipelined with the neighbouring steps' compute: step i's
+    # input is copied in during step i - 1 and its output copied out during
+    # step i + 1 (buffers rotate over R replicas; step i's layer waits for the
+    # copy-out of step i - R, the last reader of its output buffer)
     xh = [torch.empty(T, D, dtype=torch.bfloat16).pin_memory() for _ in range(R)]
     oh = [torch.empty(T, D, dtype=torch.bfloat16).pin_memory() for _ in range(R)]
     for r in range(R):
         xh[r].copy_(xs[r].cpu())
     xd = [torch.empty(T, D, dtype=torch.bfloat16, device=dev) for _ in range(R)]
-
-    def e2e_step(i):
-        r = i % R
-        xd[r].copy_(xh[r], non_blocking=True)
-        if fused:
-            layers[r].fused(xd[r], stream=stream)
-        else:
-            layers[r](xd[r], stream=stream)
-        oh[r].copy_(layers[r].out, non_blocking=True)
-
+    copy_stream = torch.cuda.Stream(device=dev)
     Ge = _divisor_at_most(K, 256 if T <= 8 else 32)
-    g2 = _graph_of(e2e_step, Ge, stream)
+    ev_in = [torch.cuda.Event() for _ in range(Ge)]
+    ev_done = [torch.cuda.Event() for _ in range(Ge)]
+    ev_out = [torch.cuda.Event() for _ in range(Ge)]
+
+    def e2e_steps():
+        copy_stream.wait_stream(stream)
+        with torch.cuda.stream(copy_stream):
+            xd[0].copy_(xh[0], non_blocking=True)
+            ev_in[0].record(copy_stream)
+        for i in range(Ge):
+            r = i % R
+            if i + 1 < Ge:
+                with torch.cuda.stream(copy_stream):
+                    xd[(i + 1) % R].copy_(xh[(i + 1) % R], non_blocking=True)
+                    ev_in[i + 1].record(copy_stream)
+            stream.wait_event(ev_in[i])
+            if i >= R:
+                stream.wait_event(ev_out[i - R])
+            if fused:
+                layers[r].fused(xd[r], stream=stream)
+            else:
+                layers[r](xd[r], stream=stream)
+            ev_done[i].record(stream)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(ev_done[i])
+                oh[r].copy_(layers[r].out, non_blocking=True)
+                ev_out[i].record(copy_stream)
+        stream.wait_stream(copy_stream)
+
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=stream):
+        e2e_steps()
     with torch.cuda.stream(stream):
         g2.replay()
     ems, _ = _timed_replays(g2, K // Ge, stream, ws_, dev, local, clocks=False)
@@ -352,7 +378,8 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
                     f"{synth.FMT_NAMES[cfg.fmt]}, {int((table >= 0).sum())}/{E} resident",
         "l2": f"rotating {R} replicas of pool+Wr+x ({R * pool_bytes / 1e9:.2f} GB)",
         "e2e": {"value": round(ws_ * T * K / (ems / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": T * D * 2,
-                "d2h_bytes_per_step": T * D * 2},
+                "d2h_bytes_per_step": T * D * 2, "copies": "pinned host buffers, on a copy stream overlapping the "
+                                                           "neighbouring steps' compute"},
         "gpu_launches": LAUNCHES["layer" if fused else ("decode" if T <= 8 else "prefill")] * K,
         "roofline": roof,
         "hit_rate": round(float(np.mean(hits)), 4), "u_hit_mean": round(float(np.mean(u_hit)), 2),
