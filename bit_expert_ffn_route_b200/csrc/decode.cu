@@ -348,26 +348,40 @@ MOE_DEVINL bool half_block_frag(const uint4 a, const uint4 b, uint2 (&out)[4]) {
 template <int NSLOT>
 __device__ void stage_x_frag(const uint16_t* __restrict__ x, int T, int K, uint8_t* xs, uint32_t* err, int first,
                              int nthreads, uint16_t* xcopy = nullptr) {
-    const int nhb = K / 16;
+    const int nhb = K / 16, total = NSLOT * nhb;
     bool ok = true;
-    for (int idx = (int)threadIdx.x - first; idx < NSLOT * nhb; idx += nthreads) {
-        const int n = idx / nhb, hb = idx - n * nhb;
-        uint2 o[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
-        if (n < T) {
-            const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)n * K + 16 * hb);
-            const uint4 a = __ldg(p), b = __ldg(p + 1);
-            ok &= half_block_frag(a, b, o);
-            if (xcopy) {                 // and the rows as they are (bf16 [T][K])
-                uint4* c = reinterpret_cast<uint4*>(xcopy + (size_t)n * K + 16 * hb);
-                c[0] = a;
-                c[1] = b;
+    // two half blocks per thread and round, both loads in flight before the stores
+    for (int idx0 = (int)threadIdx.x - first; idx0 < total; idx0 += 2 * nthreads) {
+        uint4 a[2], b[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int idx = idx0 + q * nthreads, n = idx / nhb, hb = idx - n * nhb;
+            a[q] = b[q] = make_uint4(0, 0, 0, 0);
+            if (idx < total && n < T) {
+                const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)n * K + 16 * hb);
+                a[q] = __ldg(p);
+                b[q] = __ldg(p + 1);
             }
         }
-        // hb = U * 8 + c * 2 + i
-        const int U = hb >> 3, c = (hb >> 1) & 3, i = hb & 1;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint2*>(xs + frag_off<NSLOT>((U * 2 + i) * 4 + j, n, c)) = o[j];
+        for (int q = 0; q < 2; ++q) {
+            const int idx = idx0 + q * nthreads, n = idx / nhb, hb = idx - n * nhb;
+            if (idx >= total) continue;
+            uint2 o[4] = {make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0), make_uint2(0, 0)};
+            if (n < T) {
+                ok &= half_block_frag(a[q], b[q], o);
+                if (xcopy) {             // and the rows as they are (bf16 [T][K])
+                    uint4* c = reinterpret_cast<uint4*>(xcopy + (size_t)n * K + 16 * hb);
+                    c[0] = a[q];
+                    c[1] = b[q];
+                }
+            }
+            // hb = U * 8 + c * 2 + i
+            const int U = hb >> 3, c = (hb >> 1) & 3, i = hb & 1;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint2*>(xs + frag_off<NSLOT>((U * 2 + i) * 4 + j, n, c)) = o[j];
+        }
     }
     if (!ok) atomicOr(err, kErrRange);
 }
