@@ -1202,7 +1202,9 @@ moe_status launch_fmt(DecodeParams prm, cudaStream_t s) {
         if ((size_t)prm.T * D * 2 > ring || prm.route_j > kConsumerWarps) return MOE_ERR_UNSUPPORTED;
         prm.route_wr_smem = wr_ring_offset(prm.T, D) + (size_t)prm.route_j * D * 2 <= ring ? 1 : 0;
     }
-    cudaError_t e = launch_pdl(decode_ffn_kernel<FMT, NSLOT, FUSED>, dim3(device_sm_count()), dim3(kThreads), smem, s, prm);
+    // the one-call layer's CTAs meet at grid-wide barriers: a cooperative launch
+    cudaError_t e = launch_pdl_ex(FUSED, decode_ffn_kernel<FMT, NSLOT, FUSED>, dim3(device_sm_count()), dim3(kThreads),
+                                  smem, s, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -99,21 +99,30 @@ MOE_DEVINL void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_de
 
 }  // namespace moe
 
-// Host: launch with the programmatic-stream-serialization attribute.
+// Host: launch with the programmatic-stream-serialization attribute; with
+// `cooperative`, also as a cooperative launch (every CTA resident at once, or
+// the launch fails), for kernels whose CTAs wait on one another.
 namespace moe {
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                              Args&&... args) {
+inline cudaError_t launch_pdl_ex(bool cooperative, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, Args&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = cooperative ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+    return launch_pdl_ex(false, kernel, grid, block, smem, s, std::forward<Args>(args)...);
 }
 }  // namespace moe

@@ -262,7 +262,8 @@ moe_status moe_combine(const void* expert_out, const float* gates, int T, int D,
  * a decode layer into launches; this call is an addition of this library that
  * keeps the routing, the expert pass and the combine in one persistent kernel:
  * every CTA computes the logits of ceil(E / #SMs) experts, all CTAs meet at a
- * grid-wide barrier (one CTA per SM, all resident), every CTA then selects
+ * grid-wide barrier (a cooperative launch: one CTA per SM, all resident, so the
+ * call waits for the whole GPU to be free of other work), every CTA then selects
  * every token's top-k itself; after the expert pass a second grid-wide
  * barrier, then each CTA combines a slice of the outputs.
  *   Arguments as in the three calls; residual bf16 [T][D] or NULL; out bf16
