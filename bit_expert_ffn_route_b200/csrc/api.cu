@@ -219,7 +219,7 @@ moe_status moe_debug_prefill_operand(const moe_pool* pool, int gemm, int slot, i
     if (st != MOE_OK) return st;
     if (gemm != 1 && gemm != 2) return MOE_ERR_INVALID_ARG;
     if (slot < 0 || slot >= v.n_slots || !dump || !ws || !aligned(ws, 256) || !aligned(dump, 4)) return MOE_ERR_INVALID_ARG;
-    if (m0 < 0 || (gemm == 1 ? (m0 % 64 || m0 >= v.F) : (m0 % 128 || m0 >= v.D))) return MOE_ERR_INVALID_ARG;
+    if (m0 < 0 || (gemm == 1 ? (m0 % 128 || m0 >= v.F) : (m0 % 256 || m0 >= v.D))) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < prefill_operand_dump_ws_bytes(v.D, v.F)) return MOE_ERR_WORKSPACE;
     return reported(launch_prefill_operand_dump(v, gemm, slot, m0, dump, ws, (cudaStream_t)stream));
 }

@@ -46,13 +46,12 @@ namespace {
 
 constexpr int kChunk = 256;            // tokens per plan chunk
 constexpr int kMaxE = 1024;
-constexpr int kTileM = 128;            // weight rows per tile (MMA M)
 constexpr int kN1 = 128;               // max rows per gate|up tile
 constexpr int kN2 = 128;               // max rows per down tile
-constexpr int kGateRows = 64;          // gate|up tile: 64 gate + the same 64 up features
-constexpr int kKStep = 64;             // K per row-operand stage: one 128-byte swizzle atom of fp16
-constexpr int kRoundK = 128;           // K per dequant round (two k-steps)
-constexpr int kDqWarps = 16;           // 4 per TMEM lane quadrant
+constexpr int kGateFeat = 128;         // gate|up tile: 128 gate + the same 128 up features
+constexpr int kDownRows = 256;         // down tile: 256 outputs
+constexpr int kKAlign = 128;           // D and F are multiples of this
+constexpr int kDqWarps = 16;           // dequantisation warps: two halves of 256 threads (one per weight row)
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = kDqWarps + kEpiWarps;
 constexpr int kGatherWarp = kTmaWarp + 1;
@@ -84,8 +83,8 @@ inline WsSizes ws_sizes(int T, int D, int F, int E, int k) {
     const size_t rows = (size_t)T * (k + 1);
     WsSizes s;
     // bound on sum over groups of ceil(n / N): rows / N + (number of groups)
-    s.max_t1 = (rows / kN1 + (size_t)E + 2) * (F / kGateRows);
-    s.max_t2 = (rows / kN2 + (size_t)E + 2) * (D / kTileM);
+    s.max_t1 = (rows / kN1 + (size_t)E + 2) * (F / kGateFeat);
+    s.max_t2 = (rows / kN2 + (size_t)E + 2) * (D / kDownRows);
     s.hist = align256((size_t)nchunk * E * 4);
     s.miss = align256((size_t)nchunk * 4);
     s.meta = 256;
@@ -206,8 +205,8 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
         }
         t1off[a.E + 1] = n1;
         t2off[a.E + 1] = n2;
-        a.w.meta[1] = n1 * (a.F / kGateRows);
-        a.w.meta[2] = n2 * (a.D / kTileM);
+        a.w.meta[1] = n1 * (a.F / kGateFeat);
+        a.w.meta[2] = n2 * (a.D / kDownRows);
     }
     __syncthreads();
     // per-chunk base rows of every expert
@@ -220,7 +219,7 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
         }
     }
     // tile lists: group, row tile, then weight-row tile (the fastest index)
-    const int mt1 = a.F / kGateRows, mt2 = a.D / kTileM;
+    const int mt1 = a.F / kGateFeat, mt2 = a.D / kDownRows;
     for (int g = threadIdx.x; g <= a.E; g += blockDim.x) {
         const int n = g < a.E ? tot[g] : a.T;
         const int row0 = g < a.E ? off[g] : off[a.E];
@@ -228,12 +227,12 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
         for (int j = 0; j < t1off[g + 1] - t1off[g]; ++j) {
             const int r0 = row0 + j * kN1, rows = min(kN1, n - j * kN1);
             for (int m = 0; m < mt1; ++m)
-                a.w.tiles1[(size_t)(t1off[g] + j) * mt1 + m] = make_int4(r0, rows, m * kGateRows, slot);
+                a.w.tiles1[(size_t)(t1off[g] + j) * mt1 + m] = make_int4(r0, rows, m * kGateFeat, slot);
         }
         for (int j = 0; j < t2off[g + 1] - t2off[g]; ++j) {
             const int r0 = row0 + j * kN2, rows = min(kN2, n - j * kN2);
             for (int m = 0; m < mt2; ++m)
-                a.w.tiles2[(size_t)(t2off[g] + j) * mt2 + m] = make_int4(r0, rows, m * kTileM, slot);
+                a.w.tiles2[(size_t)(t2off[g] + j) * mt2 + m] = make_int4(r0, rows, m * kDownRows, slot);
         }
     }
 }
@@ -327,16 +326,51 @@ MOE_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
     d |= (uint64_t)2 << 61;                           // 128-byte swizzle
     return d;
 }
-// kind::f16, A = B = fp16, D = f32, A and B K-major, M = 128.
-MOE_DEVINL uint32_t instr_desc_f16(int n) {
-    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+// Tile: 128 rows (tokens) x 256 weight rows.  MODE 1 (gate|up): weight rows
+// 0..127 are the gate features f0..f0+127 and rows 128..255 the same up
+// features, so one accumulator holds both halves of the SwiGLU; MODE 2 (down):
+// weight rows are the outputs d0..d0+255.  The MMA is M = 128 (the rows, A,
+// from shared memory by TMA) x N = 256 (the weights, B, dequantised into
+// shared memory) x K = 16: at small row counts an instruction costs about the
+// same for any N, so the weights take the wide side.
+constexpr int kTileRows = 128;             // rows (tokens) per tile: MMA M
+constexpr int kTileW = 256;                // weight rows per tile: MMA N
+constexpr int kRound = 64;                 // K per round: one 128-byte swizzle atom of fp16
+constexpr uint32_t kWRoundBytes = (uint32_t)kTileW * 128;     // a round of the weight operand
+constexpr uint32_t kRRoundBytes = (uint32_t)kTileRows * 128;  // a round of the row operand
+constexpr int kWBufs = 4;                  // weight rounds in flight: two per dequant half
+#ifndef MOE_GEMM_RBUFS
+#define MOE_GEMM_RBUFS 3
+#endif
+#ifndef MOE_GEMM_CSLOTS
+#define MOE_GEMM_CSLOTS 3
+#endif
+constexpr int kRBufs = MOE_GEMM_RBUFS;     // row rounds in flight (they hide the row loads' latency)
+// Code stages (2 rounds each: K = 128) in flight.  The weight stream is read
+// from HBM by these loads alone, so their depth sets its bandwidth: bytes in
+// flight per SM / load latency.
+constexpr int kCodeSlots = MOE_GEMM_CSLOTS;
+#ifndef MOE_GEMM_CSLOT_BYTES
+#define MOE_GEMM_CSLOT_BYTES 16384
+#endif
+constexpr int kSpr = 2;                    // rounds per code stage: one for each dequant half
+constexpr uint32_t kCodeSlotBytes = MOE_GEMM_CSLOT_BYTES;
+constexpr int kAccCols = kTileW;           // one accumulator: 128 lanes x 256 fp32 columns
+constexpr int kAccBufs = 2;
+constexpr uint32_t kGemmSmem = kCodeSlots * kCodeSlotBytes + kWBufs * kWRoundBytes + kRBufs * kRRoundBytes;
+static_assert(kAccBufs * kAccCols == 512, "TMEM columns");
+static_assert(kGemmSmem + 1024 + 512 <= 232448, "shared memory per block");
+
+// kind::f16, A = B = fp16, D = f32, both K-major, M = 128, N = 256.
+MOE_DEVINL uint32_t instr_desc_tile() {
+    return (1u << 4) | ((uint32_t)(kTileW >> 3) << 17) | ((uint32_t)(kTileRows >> 4) << 24);
 }
-// D[tmem] (+)= A[tmem] * B[smem]^T
-MOE_DEVINL void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+// D[tmem] (+)= A[smem] * B[smem]^T
+MOE_DEVINL void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 MOE_DEVINL void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -352,15 +386,6 @@ MOE_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 MOE_DEVINL void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-MOE_DEVINL void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-MOE_DEVINL void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // L2 policies: the weight stream is read once (evict first); the activation
 // rows are re-read by every weight tile of their group (evict last).
@@ -388,39 +413,26 @@ MOE_DEVINL void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, 
         "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
 }
-// AND of `v` over the epilogue warps (named barrier 1): they leave their loop
-// together, so none is left waiting at a named barrier.
-MOE_DEVINL bool epilogue_all(bool v, int nthreads_const_128) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(nthreads_const_128)
-        : "memory");
-    return r != 0;
-}
 
 // Byte offset of the 16-byte chunk c of row r in a K-major 128B-swizzled tile.
 MOE_DEVINL uint32_t sw128(int r, int c) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)); }
 
 // ---------------------------------------------------------------- grouped GEMM
 struct GemmParams {
-    const int4* tiles;
+    const int4* tiles;           // (row0, rows, w0, slot): w0 = first gate feature (MODE 1) / output (MODE 2)
     const int32_t* n_tiles;      // device count
     uint16_t* dst;               // MODE 1: h [rows][F] fp16; MODE 2: y rows [rows][D] bf16
     const uint8_t* scales;       // Q3_S256: the pool's scale base (sub-scales, d)
     size_t stride_s;
     int D, F;
-    int rps;                     // dequant rounds per code stage (4, 2 or 1: K / 128 is a multiple)
     uint32_t* err;
-    uint32_t* dump;              // test hook, normally null: the A operand of tile dump_tile as read
-    int dump_tile;               // back from TMEM, [K / 128 rounds][128 rows][64 f16x2 words]
+    uint32_t* dump;              // test hook, normally null: the weight operand of tile dump_tile as the
+    int dump_tile;               // MMAs read it, [K / 64 rounds][256 rows][32 f16x2 words]
 };
 
 template <int FMT>
 struct GemmFmt {
     static constexpr int kCb = FMT == MOE_Q2_32 ? 8 : 12;                  // code bytes per 32 weights
-    static constexpr int kRb = 4 * kCb;                                    // code bytes per row per round
     static constexpr bool kTmaScales = FMT != MOE_Q3_S256;
 };
 
@@ -431,30 +443,61 @@ MOE_DEVINL uint32_t swz_chunk(int r, int c, int pitch) {
     return (uint32_t)(r * pitch + ((c ^ sw) << 4));
 }
 
-constexpr int kNmax = 128;                 // rows per tile (MMA N <= 128)
-constexpr int kAccCols = 128;              // one accumulator: 128 lanes x N fp32 columns
-constexpr int kAccBufs = 2;                // double-buffered accumulators
-constexpr int kABufs = 4;                  // dequantised A round buffers, one per warp group
-constexpr int kABufCols = 2 * 32;          // a round: 2 k-steps x 32 columns (64 fp16 per lane)
-constexpr int kACol0 = kAccBufs * kAccCols;
-constexpr uint32_t kBStepBytes = (uint32_t)kNmax * kKStep * 2;     // one k-step of the row operand
-constexpr uint32_t kBStageBytes = 2 * kBStepBytes;                  // a round: two k-steps
-constexpr int kCodeSlots = 2;             // code stages of up to 4 rounds (K = 512)
-constexpr uint32_t kCodeSlotBytes = 32768;
-// The row operand lives in a byte ring: each round takes npad * 256 bytes (two
-// k-steps of npad rows x 128 bytes), so small tiles prefetch many rounds ahead.
-constexpr uint32_t kBRingBytes = kABufs * kBStageBytes;
-constexpr int kBSlots = 32;               // rounds of the row operand in flight, at most
-constexpr uint32_t kGemmSmem = kCodeSlots * kCodeSlotBytes + kBRingBytes;
-static_assert(kACol0 + kABufs * kABufCols == 512, "TMEM columns");
+// One 32-weight block of one weight row -> 16 fp16 pair words: word 8h + i =
+// weights (16h + i, 16h + i + 8), each the exact weight rounded once to fp16.
+// cw: the block's code words; sm: its (s, m) word (Q2/Q3_32); sc2: sub-scales
+// of its two 16-weight halves and d2 (Q3_S256).
+template <int FMT>
+MOE_DEVINL void dequant_block(const uint32_t (&cw)[3], uint32_t sm, const uint32_t (&sc2)[2], uint32_t d2,
+                              const Magic& Mg, uint32_t (&o)[16]) {
+    if constexpr (FMT == MOE_Q2_32) {
+        const uint32_t s2 = bcast_lo(sm), m2 = bcast_hi(sm);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t w = cw[h], w10 = w >> 10;
+            o[8 * h + 0] = w_sm(q2_codes<0>(w, w10, Mg), s2, m2);
+            o[8 * h + 1] = w_sm(q2_codes<1>(w, w10, Mg), s2, m2);
+            o[8 * h + 2] = w_sm(q2_codes<2>(w, w10, Mg), s2, m2);
+            o[8 * h + 3] = w_sm(q2_codes<3>(w, w10, Mg), s2, m2);
+            o[8 * h + 4] = w_sm(q2_codes<4>(w, w10, Mg), s2, m2);
+            o[8 * h + 5] = w_sm(q2_codes<5>(w, w10, Mg), s2, m2);
+            o[8 * h + 6] = w_sm(q2_codes<6>(w, w10, Mg), s2, m2);
+            o[8 * h + 7] = w_sm(q2_codes<7>(w, w10, Mg), s2, m2);
+        }
+    } else {
+        const uint32_t s2 = FMT == MOE_Q3_32 ? bcast_lo(sm) : 0u, m2 = FMT == MOE_Q3_32 ? bcast_hi(sm) : 0u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t P, P2;
+            q3_group_words(cw[0], cw[1], cw[2], h, P, P2);
+            const uint32_t P9 = P >> 9, P10 = P2 >> 10;
+            if constexpr (FMT == MOE_Q3_32) {
+                o[8 * h + 0] = w_sm(q3_codes<0, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 1] = w_sm(q3_codes<1, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 2] = w_sm(q3_codes<2, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 3] = w_sm(q3_codes<3, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 4] = w_sm(q3_codes<4, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 5] = w_sm(q3_codes<5, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 6] = w_sm(q3_codes<6, false>(P, P9, P2, P10, Mg), s2, m2);
+                o[8 * h + 7] = w_sm(q3_codes<7, false>(P, P9, P2, P10, Mg), s2, m2);
+            } else {
+                o[8 * h + 0] = w_s256(q3_codes<0, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 1] = w_s256(q3_codes<1, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 2] = w_s256(q3_codes<2, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 3] = w_s256(q3_codes<3, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 4] = w_s256(q3_codes<4, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 5] = w_s256(q3_codes<5, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 6] = w_s256(q3_codes<6, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+                o[8 * h + 7] = w_s256(q3_codes<7, true>(P, P9, P2, P10, Mg), sc2[h], d2);
+            }
+        }
+    }
+}
 
-// Warp roles: 0..15 dequantise (warp w owns TMEM lanes 32 (w % 4) ..; the four
-// warps of a lane quadrant take rounds in turn), 16..19 epilogue, 20 TMA for
-// the code tiles (one stage per rps rounds), 21 TMA for the row operand, 22 MMA issue.
-// The A operand of a tile has 128 rows: MODE 1 rows 0..63 are the gate
-// features m0..m0+63 and rows 64..127 the same up features, so one M = 128
-// accumulator holds both halves of the SwiGLU; MODE 2 rows are 128 outputs.
-// TMEM columns: two accumulators [0, 256), then four A round buffers.
+// Warp roles: 0..15 dequantise (thread i: weight row i % 256, 32-weight block
+// i / 256 of each K = 64 round), 16..19 epilogue (TMEM lane quadrant w % 4 =
+// rows 32q..), 20 TMA of the code stages (two rounds each), 21 TMA of the row
+// operand, 22 MMA issue.  TMEM: two 128 x 256 fp32 accumulators.
 template <int FMT, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_scales,
@@ -464,44 +507,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     using Fm = GemmFmt<FMT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_c[kCodeSlots], empty_c[kCodeSlots];
-    // round slot i (= round % 4): its TMEM A buffer is filled under round_full[i]
-    // (the 4 dequant warps of the round arrive) and released by round_empty[i];
-    // the round's row operand (ring slot round % kBSlots, at byte b_off of the
-    // ring) lands under b_full and is released by b_free
-    __shared__ uint64_t round_full[kABufs], round_empty[kABufs];
-    __shared__ uint64_t b_full[kBSlots], b_free[kBSlots];
-    __shared__ uint32_t b_off[kBSlots], b_use[kBSlots];
+    // round b (mod kWBufs): ready = its weights dequantised (one arrive per warp of the
+    // half) and its rows landed (the row producer's arrive + bytes); done = its MMAs
+    // completed, which frees both its weight buffer and its row buffer
+    __shared__ uint64_t ready[kWBufs], done[kWBufs];
     __shared__ uint64_t acc_full[kAccBufs], acc_empty[kAccBufs], drain_bar;
     __shared__ uint32_t tmem_base;
-    __shared__ float gate_x[kGateRows][17];        // epilogue: gate values handed to the up lanes
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* code_ring = smem;
-    uint8_t* b_ring = smem + kCodeSlots * kCodeSlotBytes;
+    uint8_t* w_ring = smem + kCodeSlots * kCodeSlotBytes;
+    uint8_t* r_ring = w_ring + kWBufs * kWRoundBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = g.D, F = g.F;
     const int K = MODE == 1 ? D : F;
-    const int R = K / kRoundK;                  // dequant rounds per tile
-    const int rps = g.rps;                      // rounds per code stage
-    const int CP = rps * Fm::kRb, SP = rps * 16;  // code / scale bytes per row of a code stage
+    const int R = K / kRound;                   // rounds per tile
+    constexpr int CP = kSpr * 2 * Fm::kCb, SP = kSpr * 8;   // code / scale bytes per weight row of a stage
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCodeSlots; ++s) {
             mbar_init(&full_c[s], 1);
-            mbar_init(&empty_c[s], 4 * rps);    // the 4 quadrant warps of each of its rounds
+            mbar_init(&empty_c[s], kDqWarps);       // every dequant warp, once it has read the stage
         }
-        for (int s = 0; s < kABufs; ++s) {
-            mbar_init(&round_full[s], 4);
-            mbar_init(&round_empty[s], 1);
-        }
-        for (int s = 0; s < kBSlots; ++s) {
-            mbar_init(&b_full[s], 1);
-            mbar_init(&b_free[s], 1);
-        }
-        for (int s = 0; s < kAccBufs; ++s) {
-            mbar_init(&acc_full[s], 1);
-            mbar_init(&acc_empty[s], kEpiWarps);
-        }
+        for (int s = 0; s < kWBufs; ++s) { mbar_init(&ready[s], kDqWarps / 2 + 1); mbar_init(&done[s], 1); }
+        for (int s = 0; s < kAccBufs; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
         mbar_init(&drain_bar, 1);
         fence_mbar_init();
     }
@@ -524,186 +553,175 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int first = blockIdx.x, step = gridDim.x;
 
     if (!dead && warp < kDqWarps) {
-        // ---------------- dequantisation into TMEM
-        const int q = warp & 3, par = warp >> 2;
-        const int r = 32 * q + lane;
+        // ---------------- dequantisation into the weight operand (shared memory).  Half h
+        // (warps 8h..8h+7) takes the rounds of parity h: round 2c + h of a tile is sub-round
+        // h of code stage c, and its weights go to buffer h or h + 2 in turn.  Thread:
+        // weight row r, both 32-weight blocks of the round (16 contiguous code bytes).
+        const int r = (int)threadIdx.x & (kTileW - 1), half = (int)threadIdx.x >> 8;
         const Magic Mg = make_magic();
-        const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
-        int li = 0;
+        int li = 0, j = 0;                         // j: rounds of this half so far
+        int cslot = 0;
+        uint32_t cph = 0;
         bool ok = true;
         for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
             const int4 td = __ldg(g.tiles + tile);
-            const int m0 = td.z, slot = td.w;
-            for (int rr = 0; rr < R; ++rr) {
-                const int gr = li * R + rr;
-                if ((gr & 3) != par) continue;
-                const int cst = gr / rps, sub = gr % rps, cslot = cst & 1;
-                if (!mbar_wait(&full_c[cslot], (cst >> 1) & 1, g.err)) { ok = false; break; }
+            const int w0 = td.z, slot = td.w;
+            // Q3_S256: the row's super-block words (sub-scales, d), one super-block (two
+            // rounds of this half) ahead of their use so that the loads' latency hides
+            uint32_t sbw[4] = {0, 0, 0, 0}, nxt[4] = {0, 0, 0, 0};
+            const uint8_t* sbase = nullptr;
+            size_t sb_row = 0, d_row = 0;
+            if constexpr (FMT == MOE_Q3_S256) {
+                const int pm = MODE == 1 ? (r >> 7) : 2;                   // plane: gate, up, down
+                const int wrow = w0 + (MODE == 1 ? (r & 127) : r);
+                const size_t blocks = (size_t)D * F / 256;                 // super-blocks per plane
+                sbase = g.scales + (size_t)slot * g.stride_s;
+                sb_row = (size_t)pm * blocks * 12 + (size_t)wrow * (K / 256) * 12;
+                d_row = 3 * blocks * 12 + ((size_t)pm * blocks + (size_t)wrow * (K / 256)) * 2;
+                const uint8_t* sp = sbase + sb_row;
+                nxt[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
+                nxt[1] = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
+                nxt[2] = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
+                nxt[3] = __ldg(reinterpret_cast<const uint16_t*>(sbase + d_row));
+            }
+            for (int rr = half; rr < R; rr += 2, ++j) {
+                if (!mbar_wait_sleep(&full_c[cslot], cph, g.err)) { ok = false; break; }
                 const uint8_t* cs = code_ring + cslot * kCodeSlotBytes;
-                // codes of this row for the round's 4 blocks (bytes sub * kRb .. of the
-                // stage row), and the (s, m) words
-                uint32_t cw[3 * 4];
-                uint32_t sw[4] = {0, 0, 0, 0};
-#pragma unroll
-                for (int i = 0; i < Fm::kRb / 16; ++i) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(cs + swz_chunk(r, sub * (Fm::kRb / 16) + i, CP));
-                    cw[4 * i] = a.x; cw[4 * i + 1] = a.y; cw[4 * i + 2] = a.z; cw[4 * i + 3] = a.w;
+                // both blocks' code bytes [half * 2 kCb, +2 kCb) and (s, m) words of the row
+                uint32_t cw[2][3], sm[2] = {0, 0};
+                if constexpr (Fm::kCb == 8) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(cs + swz_chunk(r, half, CP));
+                    cw[0][0] = v.x; cw[0][1] = v.y; cw[0][2] = 0;
+                    cw[1][0] = v.z; cw[1][1] = v.w; cw[1][2] = 0;
+                } else {
+                    const uint8_t* rowp = cs + r * CP + half * 24;            // CP = 48: not swizzled
+                    const uint2 a = *reinterpret_cast<const uint2*>(rowp);
+                    const uint2 b = *reinterpret_cast<const uint2*>(rowp + 8);
+                    const uint2 c = *reinterpret_cast<const uint2*>(rowp + 16);
+                    cw[0][0] = a.x; cw[0][1] = a.y; cw[0][2] = b.x;
+                    cw[1][0] = b.y; cw[1][1] = c.x; cw[1][2] = c.y;
                 }
                 if constexpr (Fm::kTmaScales) {
-                    const uint4 a = *reinterpret_cast<const uint4*>(cs + 128 * CP + swz_chunk(r, sub, SP));
-                    sw[0] = a.x; sw[1] = a.y; sw[2] = a.z; sw[3] = a.w;
+                    const uint2 v = *reinterpret_cast<const uint2*>(cs + kTileW * CP + r * SP + half * 8);
+                    sm[0] = v.x; sm[1] = v.y;
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty_c[cslot]);
-                // Q3_S256: the super-block's sub-scales and d, straight from global memory
-                uint32_t d2 = 0;
-                uint32_t sub0 = 0, sub1 = 0, sub2 = 0;
+                uint32_t sc2[2][2] = {{0, 0}, {0, 0}}, d2 = 0;
                 if constexpr (FMT == MOE_Q3_S256) {
-                    const int pm = MODE == 1 ? (r >> 6) : 2;                   // plane: gate, up, down
-                    const int wrow = m0 + (MODE == 1 ? (r & 63) : r);
-                    const size_t blocks = (size_t)D * F / 256;                 // super-blocks per plane
-                    const size_t sb = (size_t)wrow * (K / 256) + (size_t)(rr >> 1);
-                    const uint8_t* base = g.scales + (size_t)slot * g.stride_s;
-                    const uint8_t* sp = base + (size_t)pm * blocks * 12 + sb * 12;
-                    sub0 = __ldg(reinterpret_cast<const uint32_t*>(sp));
-                    sub1 = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
-                    sub2 = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
-                    const uint32_t db = __ldg(reinterpret_cast<const uint16_t*>(base + 3 * blocks * 12) + pm * blocks + sb);
-                    d2 = db | (db << 16);
-                }
-                const int buf = par, use = gr >> 2;
-                const uint32_t col0 = (uint32_t)(kACol0 + buf * kABufCols);
+                    if ((rr >> 1) % 2 == 0) {              // rounds 4m + half: a new super-block
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    uint32_t o[16];
-                    if constexpr (FMT == MOE_Q2_32) {
-                        const uint32_t s2 = bcast_lo(sw[b]), m2 = bcast_hi(sw[b]);
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t w = cw[2 * b + h], w10 = w >> 10;
-                            o[8 * h + 0] = w_sm(q2_codes<0>(w, w10, Mg), s2, m2);
-                            o[8 * h + 1] = w_sm(q2_codes<1>(w, w10, Mg), s2, m2);
-                            o[8 * h + 2] = w_sm(q2_codes<2>(w, w10, Mg), s2, m2);
-                            o[8 * h + 3] = w_sm(q2_codes<3>(w, w10, Mg), s2, m2);
-                            o[8 * h + 4] = w_sm(q2_codes<4>(w, w10, Mg), s2, m2);
-                            o[8 * h + 5] = w_sm(q2_codes<5>(w, w10, Mg), s2, m2);
-                            o[8 * h + 6] = w_sm(q2_codes<6>(w, w10, Mg), s2, m2);
-                            o[8 * h + 7] = w_sm(q2_codes<7>(w, w10, Mg), s2, m2);
-                        }
-                    } else {
-                        uint32_t s2 = 0, m2 = 0, sc2[2] = {0, 0};
-                        if constexpr (FMT == MOE_Q3_32) {
-                            s2 = bcast_lo(sw[b]);
-                            m2 = bcast_hi(sw[b]);
-                        } else {
-                            // sub-blocks 2c and 2c + 1 of the super-block, c = 32-weight chunk (0..7)
-                            const int c = 4 * (rr & 1) + b;
-                            const uint64_t lo = ((uint64_t)sub1 << 32) | sub0, hi = ((uint64_t)sub2 << 32) | sub1;
-                            const uint32_t bits = c < 4 ? (uint32_t)(lo >> (12 * c)) : (uint32_t)(hi >> (12 * c - 32));
-                            sc2[0] = s256_sub(bits & 63u);
-                            sc2[1] = s256_sub((bits >> 6) & 63u);
-                        }
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t P, P2;
-                            q3_group_words(cw[3 * b], cw[3 * b + 1], cw[3 * b + 2], h, P, P2);
-                            const uint32_t P9 = P >> 9, P10 = P2 >> 10;
-                            if constexpr (FMT == MOE_Q3_32) {
-                                o[8 * h + 0] = w_sm(q3_codes<0, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 1] = w_sm(q3_codes<1, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 2] = w_sm(q3_codes<2, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 3] = w_sm(q3_codes<3, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 4] = w_sm(q3_codes<4, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 5] = w_sm(q3_codes<5, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 6] = w_sm(q3_codes<6, false>(P, P9, P2, P10, Mg), s2, m2);
-                                o[8 * h + 7] = w_sm(q3_codes<7, false>(P, P9, P2, P10, Mg), s2, m2);
-                            } else {
-                                o[8 * h + 0] = w_s256(q3_codes<0, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 1] = w_s256(q3_codes<1, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 2] = w_s256(q3_codes<2, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 3] = w_s256(q3_codes<3, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 4] = w_s256(q3_codes<4, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 5] = w_s256(q3_codes<5, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 6] = w_s256(q3_codes<6, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                                o[8 * h + 7] = w_s256(q3_codes<7, true>(P, P9, P2, P10, Mg), sc2[h], d2);
-                            }
+                        for (int i = 0; i < 4; ++i) sbw[i] = nxt[i];
+                        const int jn = (rr >> 2) + 1;
+                        if (jn < K / 256) {
+                            const uint8_t* sp = sbase + sb_row + (size_t)jn * 12;
+                            nxt[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
+                            nxt[1] = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
+                            nxt[2] = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
+                            nxt[3] = __ldg(reinterpret_cast<const uint16_t*>(sbase + d_row) + jn);
                         }
                     }
-                    if (b == 0 && use > 0) {
-                        if (!mbar_wait(&round_empty[buf], (use - 1) & 1, g.err)) { ok = false; break; }
-                        tc_fence_after();
-                    }
-                    // block b -> k-step b / 2, columns (b % 2) * 16 of the step's 32
-                    tmem_st16(lane_addr + col0 + (uint32_t)((b >> 1) * 32 + (b & 1) * 16), o);
-                }
-                if (!ok) break;
-                tmem_st_wait();
-                if (g.dump != nullptr && tile == g.dump_tile) {
-                    // test hook: read the round's A operand back from TMEM as the MMAs see it
-                    uint32_t* drow = g.dump + ((size_t)rr * kTileM + r) * 64;
+                    d2 = sbw[3] | (sbw[3] << 16);
+                    const uint64_t lo = ((uint64_t)sbw[1] << 32) | sbw[0], hi = ((uint64_t)sbw[2] << 32) | sbw[1];
 #pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        uint32_t v[16];
-                        tmem_ld16(lane_addr + col0 + (uint32_t)(16 * b), v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) drow[16 * b + i] = v[i];
+                    for (int b = 0; b < 2; ++b) {
+                        const int c = (2 * rr + b) & 7;                        // sub-blocks 2c, 2c + 1
+                        const uint32_t bits = c < 4 ? (uint32_t)(lo >> (12 * c)) : (uint32_t)(hi >> (12 * c - 32));
+                        sc2[b][0] = s256_sub(bits & 63u);
+                        sc2[b][1] = s256_sub((bits >> 6) & 63u);
                     }
                 }
-                tc_fence_before();
+                uint32_t o[2][16];
+                dequant_block<FMT>(cw[0], sm[0], sc2[0], d2, Mg, o[0]);
+                dequant_block<FMT>(cw[1], sm[1], sc2[1], d2, Mg, o[1]);
+                // the stage is released once every value read from it has been used
+                const uint32_t dep = o[0][0] ^ o[0][15] ^ o[1][0] ^ o[1][15];
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&round_full[buf]);
+                if (lane == 0) mbar_arrive_dep(&empty_c[cslot], dep);
+                if (++cslot == kCodeSlots) { cslot = 0; cph ^= 1u; }
+                // the buffer is free once the MMAs of its previous use completed
+                const int wb = half + 2 * (j & 1);
+                if (j >= 2) {
+                    if (!mbar_wait_sleep(&done[wb], ((j >> 1) - 1) & 1, g.err)) { ok = false; break; }
+                    tc_fence_after();
+                }
+                uint8_t* wbuf = w_ring + wb * kWRoundBytes;
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4*>(wbuf + sw128(r, 4 * b + q)) =
+                            make_uint4(o[b][4 * q], o[b][4 * q + 1], o[b][4 * q + 2], o[b][4 * q + 3]);
+                if (g.dump != nullptr && tile == g.dump_tile) {
+                    // test hook: the round's weight operand as the MMAs will read it
+                    uint32_t* drow = g.dump + ((size_t)rr * kTileW + r) * 32;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(wbuf + sw128(r, q));
+                        drow[4 * q] = v.x; drow[4 * q + 1] = v.y; drow[4 * q + 2] = v.z; drow[4 * q + 3] = v.w;
+                    }
+                }
+                fence_proxy_async();                 // generic stores -> the tensor core's reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ready[wb]);
             }
         }
     } else if (!dead && warp < kTmaWarp) {
-        // ---------------- epilogue: TMEM -> registers -> global
+        // ---------------- epilogue: TMEM -> registers -> global; lane = row of the tile
         const int q = warp & 3;
-        const int r = 32 * q + lane;
+        const int t = 32 * q + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
         int li = 0;
-        bool range_bad = false, ok = true;
-        for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
+        bool range_bad = false;
+        for (int tile = first; tile < n_tiles; tile += step, ++li) {
             const int4 td = __ldg(g.tiles + tile);
-            const int row0 = td.x, nrows = td.y, m0 = td.z;
-            const int npad = (nrows + 15) & ~15;
+            const int row0 = td.x, nrows = td.y, w0 = td.z;
             const int ab = li & 1;
-            bool got = mbar_wait(&acc_full[ab], (li >> 1) & 1, g.err);
-            if constexpr (MODE == 1) got = epilogue_all(got, kEpiWarps * 32);
-            if (!got) { ok = false; break; }
+            if (!mbar_wait_sleep(&acc_full[ab], (li >> 1) & 1, g.err)) break;
             tc_fence_after();
             const uint32_t acc = lane_addr + (uint32_t)(ab * kAccCols);
-            for (int c = 0; c < npad; c += 16) {
-                uint32_t v[16];
-                tmem_ld16(acc + (uint32_t)c, v);
-                tmem_ld_wait();
-                if constexpr (MODE == 1) {
-                    // lanes 0..63 hold gate, 64..127 up of the same features
-                    if (q < 2) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) gate_x[r][i] = __uint_as_float(v[i]);
-                    }
-                    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-                    if (q >= 2) {
-                        const int f = m0 + (r - 64);
-                        const int fpos = (f & ~15) | ((f & 7) << 1) | ((f >> 3) & 1);
+            if constexpr (MODE == 1) {
+                // columns c: gate feature w0 + c, columns 128 + c: the same up feature
+                for (int c = 0; c < kTileW / 2; c += 16) {
+                    uint32_t gv[16], uv[16];
+                    tmem_ld16(acc + (uint32_t)c, gv);
+                    tmem_ld16(acc + (uint32_t)(kTileW / 2 + c), uv);
+                    tmem_ld_wait();
+                    if (t < nrows) {
+                        float hb[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const int n = c + i;
-                            if (n < nrows) {
-                                const float gte = gate_x[r - 64][i], up = __uint_as_float(v[i]);
-                                const float hv = gte / (1.0f + expf(-gte)) * up;
-                                const float hb = bf16_bits_to_f32(f32_to_bf16_rne(hv));   // h is a bf16 value
-                                range_bad |= !(fabsf(hb) < 65520.f);
-                                g.dst[(size_t)(row0 + n) * F + fpos] = __half_as_ushort(__float2half_rn(hb));
-                            }
+                            const float gte = __uint_as_float(gv[i]), up = __uint_as_float(uv[i]);
+                            hb[i] = bf16_bits_to_f32(f32_to_bf16_rne(gte / (1.0f + expf(-gte)) * up));   // h is a bf16 value
+                            range_bad |= !(fabsf(hb[i]) < 65520.f);
                         }
-                    }
-                    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-                } else {
+                        // the 16 features in the K order of the down GEMM's row operand: word i = (i, i + 8)
+                        uint32_t w[8];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int n = c + i;
-                        if (n < nrows) g.dst[(size_t)(row0 + n) * D + m0 + r] = f32_to_bf16_rne(__uint_as_float(v[i]));
+                        for (int i = 0; i < 8; ++i)
+                            w[i] = (uint32_t)__half_as_ushort(__float2half_rn(hb[i])) |
+                                   ((uint32_t)__half_as_ushort(__float2half_rn(hb[i + 8])) << 16);
+                        uint4* dst = reinterpret_cast<uint4*>(g.dst + (size_t)(row0 + t) * F + w0 + c);
+                        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                }
+            } else {
+                for (int c = 0; c < kTileW; c += 32) {   // two loads in flight per wait
+                    uint32_t v[2][16];
+                    tmem_ld16(acc + (uint32_t)c, v[0]);
+                    tmem_ld16(acc + (uint32_t)(c + 16), v[1]);
+                    tmem_ld_wait();
+                    if (t < nrows) {
+                        uint4* dst = reinterpret_cast<uint4*>(g.dst + (size_t)(row0 + t) * D + w0 + c);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                w[i] = (uint32_t)f32_to_bf16_rne(__uint_as_float(v[h][2 * i])) |
+                                       ((uint32_t)f32_to_bf16_rne(__uint_as_float(v[h][2 * i + 1])) << 16);
+                            dst[2 * h] = make_uint4(w[0], w[1], w[2], w[3]);
+                            dst[2 * h + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        }
                     }
                 }
             }
@@ -713,137 +731,110 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (range_bad) atomicOr(g.err, kErrRange);
     } else if (!dead && warp == kTmaWarp) {
-        // ---------------- TMA loads of the code (and scale) tiles, one stage per rps rounds
+        // ---------------- TMA loads of the code (and scale) stages: rows 0..127 and 128..255
         if (lane == 0) {
             const uint64_t pol = l2_evict_first();
-            const uint32_t bytes = 128u * CP + (Fm::kTmaScales ? 128u * SP : 0u);
-            int li = 0, issued = 0;
+            const uint32_t bytes = (uint32_t)kTileW * CP + (Fm::kTmaScales ? (uint32_t)kTileW * SP : 0u);
+            int issued = 0, cst = 0, slot = 0;
+            uint32_t ph = 0;
             bool ok = true;
-            for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
+            for (int tile = first; tile < n_tiles && ok; tile += step) {
                 const int4 td = __ldg(g.tiles + tile);
-                const int m0 = td.z, slot_id = td.w;
-                for (int c = 0; c < R / rps; ++c) {
-                    const int cst = li * (R / rps) + c, slot = cst & 1;
-                    if (cst >= kCodeSlots && !mbar_wait(&empty_c[slot], ((cst >> 1) - 1) & 1, g.err)) {
+                const int w0 = td.z, slot_id = td.w;
+                for (int c = 0; c < R / kSpr; ++c, ++cst) {
+                    if (cst >= kCodeSlots && !mbar_wait_sleep(&empty_c[slot], ph ^ 1u, g.err)) {
                         ok = false;
                         break;
                     }
                     uint8_t* cs = code_ring + slot * kCodeSlotBytes;
                     mbar_arrive_expect_tx(&full_c[slot], bytes);
-                    if constexpr (MODE == 1) {
-                        // gate rows m0.. into rows 0..63, up rows F + m0.. into rows 64..127
 #pragma unroll
-                        for (int m = 0; m < 2; ++m) {
-                            const int y = m * F + m0;
-                            tma_load_3d(smem_u32(cs + m * 64 * CP), &map_codes, c * CP, y, slot_id, &full_c[slot], pol);
-                            if constexpr (Fm::kTmaScales)
-                                tma_load_3d(smem_u32(cs + 128 * CP + m * 64 * SP), &map_scales, c * SP, y, slot_id,
-                                            &full_c[slot], pol);
-                        }
-                    } else {
-                        tma_load_3d(smem_u32(cs), &map_codes, c * CP, m0, slot_id, &full_c[slot], pol);
+                    for (int m = 0; m < 2; ++m) {
+                        // MODE 1: gate rows w0.., then up rows F + w0..; MODE 2: outputs w0.., w0 + 128..
+                        const int y = MODE == 1 ? m * F + w0 : w0 + 128 * m;
+                        tma_load_3d(smem_u32(cs + m * 128 * CP), &map_codes, c * CP, y, slot_id, &full_c[slot], pol);
                         if constexpr (Fm::kTmaScales)
-                            tma_load_3d(smem_u32(cs + 128 * CP), &map_scales, c * SP, m0, slot_id, &full_c[slot], pol);
+                            tma_load_3d(smem_u32(cs + kTileW * CP + m * 128 * SP), &map_scales, c * SP, y, slot_id,
+                                        &full_c[slot], pol);
                     }
                     issued = cst + 1;
+                    if (++slot == kCodeSlots) { slot = 0; ph ^= 1u; }
                 }
             }
             // every issued stage completes before the CTA exits
             for (int j = issued - kCodeSlots; j < issued; ++j)
-                if (j >= 0) mbar_drain(&full_c[j & 1], (j >> 1) & 1);
+                if (j >= 0) mbar_drain(&full_c[j % kCodeSlots], (j / kCodeSlots) & 1);
         }
         __syncwarp();
     } else if (!dead && warp == kGatherWarp) {
-        // ---------------- row operand (K-major, 128B swizzle) by TMA: the tile's rows are
-        // contiguous (group order), read as boxes of 128 / 64 / 32 / 16 rows into the
-        // byte ring; a round that does not fit before the ring's end starts at 0
+        // ---------------- row operand: the tile's rows x 64 K per round (K-major, 128B
+        // swizzle) in one box of 16, 32, 64 or 128 rows; the rest of the round's
+        // 128 MMA rows hold stale values, whose results are not stored
         if (lane == 0) {
             const uint64_t pol = l2_evict_last();
             bool ok = true;
-            int issued = 0, tail = 0;
-            uint32_t head = 0, used = 0;
-            for (int tile = first, h = 0; tile < n_tiles && ok; tile += step) {
+            int issued = 0, gr = 0, rb = 0, b = 0, lb = 0;      // lb: round gr - kRBufs (mod kWBufs)
+            uint32_t ph = 0, lph = 0;
+            for (int tile = first; tile < n_tiles && ok; tile += step) {
                 const int4 td = __ldg(g.tiles + tile);
-                const int row0 = td.x, npad = (td.y + 15) & ~15;
-                const uint32_t nb = (uint32_t)npad * 256u;          // two k-steps of npad rows
-                for (int rr = 0; rr < R; ++rr, ++h) {
-                    const bool wrap = head + nb > kBRingBytes;       // (head may equal kBRingBytes)
-                    const uint32_t pad = wrap ? kBRingBytes - head : 0u;
-                    // free the oldest rounds until the bytes and a slot are available
-                    while (kBRingBytes - used < pad + nb || h - tail >= kBSlots) {
-                        if (!mbar_wait(&b_free[tail % kBSlots], (tail / kBSlots) & 1, g.err)) { ok = false; break; }
-                        used -= b_use[tail % kBSlots];
-                        ++tail;
+                const int row0 = td.x, nrows = td.y;
+                const CUtensorMap* m = nrows > 64 ? &rows128 : nrows > 32 ? &rows64 : nrows > 16 ? &rows32 : &rows16;
+                const uint32_t bytes = (nrows > 64 ? 128u : nrows > 32 ? 64u : nrows > 16 ? 32u : 16u) * 128u;
+                for (int rr = 0; rr < R; ++rr, ++gr) {
+                    if (gr >= kRBufs) {      // row buffer rb is free once round gr - kRBufs is done
+                        if (!mbar_wait_sleep(&done[lb], lph, g.err)) { ok = false; break; }
+                        if (++lb == kWBufs) { lb = 0; lph ^= 1u; }
                     }
-                    if (!ok) break;
-                    const uint32_t off = wrap ? 0u : head;
-                    head = off + nb;
-                    used += pad + nb;
-                    const int bs = h % kBSlots;
-                    b_use[bs] = pad + nb;
-                    b_off[bs] = off;
-                    mbar_arrive_expect_tx(&b_full[bs], nb);
-                    const uint32_t b_base = smem_u32(b_ring + off);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const int x = (2 * rr + j) * kKStep;
-                        const uint32_t dst = b_base + (uint32_t)j * (uint32_t)npad * 128u;
-                        for (int n = 0; n < npad;) {
-                            const int left = npad - n;
-                            const CUtensorMap* m = left >= 128 ? &rows128 : left >= 64 ? &rows64 : left >= 32 ? &rows32 : &rows16;
-                            const int nbx = left >= 128 ? 128 : left >= 64 ? 64 : left >= 32 ? 32 : 16;
-                            tma_load_2d(dst + n * 128, m, x, row0 + n, &b_full[bs], pol);
-                            n += nbx;
-                        }
-                    }
-                    issued = h + 1;
+                    mbar_arrive_expect_tx(&ready[b], bytes);
+                    tma_load_2d(smem_u32(r_ring + rb * kRRoundBytes), m, rr * kRound, row0, &ready[b], pol);
+                    issued = gr + 1;
+                    if (++rb == kRBufs) rb = 0;
+                    if (++b == kWBufs) { b = 0; ph ^= 1u; }
                 }
             }
-            // every issued copy lands before the CTA exits
-            for (int j = issued - kBSlots; j < issued; ++j)
-                if (j >= 0) mbar_drain(&b_full[j % kBSlots], (j / kBSlots) & 1);
+            // every issued row load lands before the CTA exits
+            for (int j = issued - kRBufs; j < issued; ++j)
+                if (j >= 0) mbar_drain(&ready[j % kWBufs], (j / kWBufs) & 1);
         }
         __syncwarp();
     } else if (!dead && warp == kMmaWarp) {
-        // ---------------- single-thread MMA issue: per round, 2 k-steps x 4 MMAs of K = 16
+        // ---------------- single-thread MMA issue: per round, 4 MMAs of K = 16
         if (lane == 0) {
-            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(b_ring));
-            int li = 0;
+            const uint32_t idesc = instr_desc_tile();
+            int li = 0, wb = 0, rb = 0;
+            uint32_t wph = 0;
             bool ok = true, issued = false;
+            bool pre = false;                            // the round's ready phase already seen complete
             for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
-                const int4 td = __ldg(g.tiles + tile);
-                const int npad = (td.y + 15) & ~15;
-                const uint32_t idesc = instr_desc_f16(npad);
                 const int ab = li & 1;
                 if (li >= kAccBufs) {
-                    if (!mbar_wait(&acc_empty[ab], ((li >> 1) - 1) & 1, g.err)) { ok = false; break; }
+                    if (!mbar_wait_sleep(&acc_empty[ab], ((li >> 1) - 1) & 1, g.err)) { ok = false; break; }
                     tc_fence_after();
                 }
                 const uint32_t d_tmem = tmem + (uint32_t)(ab * kAccCols);
                 for (int rr = 0; rr < R; ++rr) {
-                    const int gr = li * R + rr;
-                    const int buf = gr & 3;
-                    const int bs = gr % kBSlots;
-                    if (!mbar_wait(&round_full[buf], (gr >> 2) & 1, g.err) ||
-                        !mbar_wait(&b_full[bs], (gr / kBSlots) & 1, g.err)) { ok = false; break; }
+                    if (!pre && !mbar_wait_sleep(&ready[wb], wph, g.err)) { ok = false; break; }
                     tc_fence_after();
-                    // descriptor start addresses advance in 16-byte units
-                    const uint64_t bd = bdesc0 + (uint64_t)(b_off[bs] >> 4);
-                    const uint32_t kstep = (uint32_t)npad * 128u;
-                    const uint32_t at = tmem + (uint32_t)(kACol0 + buf * kABufCols);
+                    const uint64_t ad = smem_desc_sw128(smem_u32(r_ring + rb * kRRoundBytes));
+                    const uint64_t bd = smem_desc_sw128(smem_u32(w_ring + wb * kWRoundBytes));
+                    // test the next round's barrier now: the test's latency then passes while
+                    // this round's MMAs hold the thread (a phase, once complete, stays so until
+                    // the round's MMAs are done)
+                    const int nb = wb + 1 == kWBufs ? 0 : wb + 1;
+                    const uint32_t nph = wb + 1 == kWBufs ? wph ^ 1u : wph;
+                    pre = mbar_try_wait(&ready[nb], nph);
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int kk = 0; kk < kKStep / 16; ++kk)
-                            mma_ts(d_tmem, at + (uint32_t)(j * 32 + kk * 8), bd + (uint64_t)((j * kstep + kk * 32) >> 4),
-                                   idesc, (rr > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kRound / 16; ++kk)     // descriptor start addresses in 16-byte units
+                        mma_ss(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (rr > 0 || kk > 0) ? 1u : 0u);
                     issued = true;
-                    mma_commit(&round_empty[buf]);     // frees the round's A buffer
-                    mma_commit(&b_free[bs]);           // and its row operand
+                    mma_commit(&done[wb]);               // frees the round's weight and row buffers
+                    wb = nb;
+                    wph = nph;
+                    if (++rb == kRBufs) rb = 0;
                 }
                 if (ok) mma_commit(&acc_full[ab]);
             }
-            if (issued) {                              // every MMA completes before TMEM is released
+            if (issued) {                                // every MMA completes before TMEM is released
                 mma_commit(&drain_bar);
                 mbar_drain(&drain_bar, 0);
             }
@@ -880,7 +871,7 @@ bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32
     if (!fn) return false;
     const cuuint64_t dims[2] = {K, rows};
     const cuuint64_t strides[1] = {K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kKStep, box_rows};
+    const cuuint32_t box[2] = {(cuuint32_t)kRound, box_rows};
     const cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -901,23 +892,23 @@ moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, u
     const uint64_t rows = MODE == 1 ? 2 * (uint64_t)F : (uint64_t)D;
     const uint64_t code_row = (uint64_t)Kg / 32 * Fm::kCb;
     const uint8_t* codes = P.codes + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * Fm::kCb));
-    CUtensorMap mc, ms;
-    const int R = Kg / kRoundK;
-    prm.rps = R % 4 == 0 ? 4 : (R % 2 == 0 ? 2 : 1);
-    const uint32_t cp = (uint32_t)(prm.rps * Fm::kRb), sp = (uint32_t)(prm.rps * 16);
-    const uint32_t box_y = MODE == 1 ? kGateRows : kTileM;   // gate|up: two 64-row boxes per stage
-    if (!byte_map(&mc, codes, code_row, rows, (uint64_t)P.n_slots, P.stride_c, cp, box_y, swizzle_for(cp)))
+    CUtensorMap mc, ms, mr;
+    const int R = Kg / kRound;
+    const uint32_t cp = (uint32_t)(kSpr * 2 * Fm::kCb), sp = (uint32_t)(kSpr * 8);
+    if ((uint64_t)kTileW * (cp + (Fm::kTmaScales ? sp : 0u)) > kCodeSlotBytes || R % kSpr) return MOE_ERR_UNSUPPORTED;
+    // code (and scale) stages: two boxes of 128 weight rows
+    if (!byte_map(&mc, codes, code_row, rows, (uint64_t)P.n_slots, P.stride_c, cp, 128, swizzle_for(cp)))
         return MOE_ERR_CUDA;
     if constexpr (Fm::kTmaScales) {
         const uint64_t scale_row = (uint64_t)Kg / 32 * 4;
         const uint8_t* scales = P.scales + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * 4));
-        if (!byte_map(&ms, scales, scale_row, rows, (uint64_t)P.n_slots, P.stride_s, sp, box_y, swizzle_for(sp)))
+        if (!byte_map(&ms, scales, scale_row, rows, (uint64_t)P.n_slots, P.stride_s, sp, 128, swizzle_for(sp)))
             return MOE_ERR_CUDA;
     } else {
         ms = mc;
     }
-    CUtensorMap r128, r64, r32, r16;
-    if (!row_map(&r128, src, (uint64_t)Kg, src_rows, 128) || !row_map(&r64, src, (uint64_t)Kg, src_rows, 64) ||
+    CUtensorMap r64, r32, r16;
+    if (!row_map(&mr, src, (uint64_t)Kg, src_rows, 128) || !row_map(&r64, src, (uint64_t)Kg, src_rows, 64) ||
         !row_map(&r32, src, (uint64_t)Kg, src_rows, 32) || !row_map(&r16, src, (uint64_t)Kg, src_rows, 16))
         return MOE_ERR_CUDA;
     const size_t smem = kGemmSmem + 1024;
@@ -929,7 +920,7 @@ moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, u
         return MOE_ERR_CUDA;
     const int grid = max_tiles < device_sm_count() ? (max_tiles > 0 ? max_tiles : 1) : device_sm_count();
     const cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms,
-                                     r128, r64, r32, r16, prm);
+                                     mr, r64, r32, r16, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -979,7 +970,7 @@ size_t prefill_operand_dump_ws_bytes(int D, int F) { return 1024 + (size_t)144 *
 
 moe_status launch_prefill_operand_dump(const PoolView& P, int gemm, int slot, int m0, uint32_t* dump, void* ws,
                                        cudaStream_t s) {
-    if (P.F % kRoundK || P.D % kRoundK) return MOE_ERR_UNSUPPORTED;
+    if (P.F % kKAlign || P.D % kKAlign || P.D % kDownRows) return MOE_ERR_UNSUPPORTED;
     if (!encode_tiled()) return MOE_ERR_CUDA;
     switch (P.fmt) {
         case MOE_Q2_32: return launch_operand_dump<MOE_Q2_32>(P, gemm, slot, m0, dump, ws, s);
@@ -993,7 +984,7 @@ size_t prefill_workspace_bytes(int T, int D, int F, int E, int k) { return ws_si
 moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
                                   const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
                                   int32_t* miss_count, void* ws, cudaStream_t s) {
-    if (P.F % kRoundK || P.D % kRoundK || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+    if (P.F % kKAlign || P.D % kDownRows || E > kMaxE) return MOE_ERR_UNSUPPORTED;
     if (!encode_tiled()) return MOE_ERR_CUDA;
     const PrefillWs w = carve(ws, T, P.D, P.F, E, k);
     PlanArgs a;

@@ -38,6 +38,13 @@ MOE_DEVINL void fence_proxy_async() { asm volatile("fence.proxy.async.shared::ct
 MOE_DEVINL void mbar_arrive(uint64_t* bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar)) : "memory");
 }
+// Arrive once `dep` is known: a value computed from everything this warp read
+// out of the buffer the arrive releases, so that no read of it is still in
+// flight when its producer may overwrite it.
+MOE_DEVINL void mbar_arrive_dep(uint64_t* bar, uint32_t dep) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar)), "r"(dep)
+                 : "memory");
+}
 MOE_DEVINL void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
                  "r"(bytes)
@@ -68,6 +75,38 @@ MOE_DEVINL bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             if (err) atomicOr(err, kErrTimeout);
             return false;
+        }
+    }
+}
+
+// Bounded wait as mbar_wait, but each poll suspends the thread in hardware
+// (up to 20 us) until the phase completes: a waiting warp takes no issue
+// slots from the warps that do the work.
+MOE_DEVINL bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+// The error word is a global load: it is read every 20 us of waiting, not at
+// every poll, so that its latency does not delay the wake-up.
+MOE_DEVINL bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t check = t0 + 20000;
+    for (;;) {
+        if (mbar_try_wait_suspend(bar, parity)) return true;
+        const uint64_t t = globaltimer_ns();
+        if (t >= check) {
+            if (timed_out(err)) return false;
+            if (t - t0 > kWaitLimitNs) {
+                if (err) atomicOr(err, kErrTimeout);
+                return false;
+            }
+            check = t + 20000;
         }
     }
 }

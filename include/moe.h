@@ -317,15 +317,15 @@ moe_status moe_debug_wait_flag(const uint32_t* flag, uint32_t expect, uint32_t l
 /*
  * Test hook: the weight operand of one tile of the prefill path's tensor-core
  * GEMM, exactly as the MMAs read it.  Runs the prefill GEMM kernel on a single
- * tile of `slot` (against zero rows) and copies its dequantised A operand back
- * out of tensor memory after each K = 128 round.
- *   gemm 1 (gate|up): A rows 0..63 are gate features m0..m0+63 and rows
- *          64..127 the up features m0..m0+63 (m0 % 64 == 0, m0 < d_ff), K = d_model;
- *   gemm 2 (down): A rows are output features m0..m0+127 (m0 % 128 == 0,
+ * tile of `slot` (against zero rows) and copies its dequantised weight operand
+ * back out of shared memory after each K = 64 round.
+ *   gemm 1 (gate|up): weight rows 0..127 are gate features m0..m0+127 and rows
+ *          128..255 the same up features (m0 % 128 == 0, m0 < d_ff), K = d_model;
+ *   gemm 2 (down): weight rows are output features m0..m0+255 (m0 % 256 == 0,
  *          m0 < d_model), K = d_ff.
- *   dump   uint32 [K / 128][128][64] (device): word 16b + i of row r in round
- *          rr holds the fp16 pair (lo, hi) of weights K0 + (i & 7) and
- *          K0 + (i & 7) + 8, with K0 = 128 rr + 32 b + 16 (i >> 3).
+ *   dump   uint32 [K / 64][256][32] (device): word j of row r in round rr holds
+ *          the fp16 pair (lo, hi) of weights K0 and K0 + 8, with c = j / 4,
+ *          K0 = 64 rr + 16 (c / 2) + 4 (c % 2) + j % 4.
  *   ws     device scratch of moe_debug_operand_workspace_size bytes, 256-byte
  *          aligned (overwritten).
  * Each fp16 weight is the exact weight (moe_dequantize) rounded once to fp16.

@@ -1,12 +1,12 @@
 """The weight operand the prefill tensor cores consume, bit for bit.
 
 moe_debug_prefill_operand runs the prefill GEMM kernel on one tile and reads
-its dequantised A operand back out of tensor memory.  Every fp16 weight must
+its dequantised weight operand back out of shared memory.  Every fp16 weight must
 be the exact weight of the block format rounded once to fp16 (round to nearest
 even): the oracle's fp32 dequantisation (exact for these pools: s*q + m and
 d*(sc-32)*(q-4) need at most 17 significant bits) converted by numpy's
 float32 -> float16 cast.  Covers the three formats, both GEMMs (gate|up rows
-0..63 gate and 64..127 up; down rows = outputs) and first / last tiles."""
+0..127 gate and 128..255 up; down rows = outputs) and first / last tiles."""
 import numpy as np
 import pytest
 import torch
@@ -20,18 +20,18 @@ D, F = 3072, 512
 
 
 def decode_dump(dump, K):
-    """uint32 [K/128][128][64] -> fp16 bit patterns [128][K] (the documented word order)."""
-    R = K // 128
-    d = dump.reshape(R, 128, 64)
+    """uint32 [K/64][256][32] -> fp16 bit patterns [256][K] (the documented word order)."""
+    R = K // 64
+    d = dump.reshape(R, 256, 32)
     lo = (d & 0xFFFF).astype(np.uint16)
     hi = (d >> 16).astype(np.uint16)
-    W = np.zeros((128, K), np.uint16)
+    W = np.zeros((256, K), np.uint16)
     for rr in range(R):
-        for col in range(64):
-            b, i = col // 16, col % 16
-            k0 = 128 * rr + 32 * b + 16 * (i >> 3) + (i & 7)
-            W[:, k0] = lo[rr, :, col]
-            W[:, k0 + 8] = hi[rr, :, col]
+        for j in range(32):
+            c = j // 4
+            k0 = 64 * rr + 16 * (c // 2) + 4 * (c % 2) + j % 4
+            W[:, k0] = lo[rr, :, j]
+            W[:, k0 + 8] = hi[rr, :, j]
     return W
 
 
@@ -43,16 +43,16 @@ def test_prefill_operand_is_rne_fp16_of_exact_weight(fmt):
                            pool.stride_codes, pool.stride_scales)
     for slot in (1, 2):
         gate, up, down = (oracle.dequant(host, slot, m) for m in range(3))
-        for gemm, m0 in ((1, 0), (1, F - 64), (2, 0), (2, D - 128)):
+        for gemm, m0 in ((1, 0), (1, F - 128), (2, 0), (2, D - 256)):
             K = D if gemm == 1 else F
-            dump = torch.zeros(K // 128 * 128 * 64, dtype=torch.int32, device="cuda")
+            dump = torch.zeros(K // 64 * 256 * 32, dtype=torch.int32, device="cuda")
             moe.moe_debug_prefill_operand(p, gemm, slot, m0, dump)
             torch.cuda.synchronize()
             got = decode_dump(dump.cpu().numpy().view(np.uint32), K)
             if gemm == 1:
-                want32 = np.concatenate([gate[m0:m0 + 64], up[m0:m0 + 64]])
+                want32 = np.concatenate([gate[m0:m0 + 128], up[m0:m0 + 128]])
             else:
-                want32 = down[m0:m0 + 128]
+                want32 = down[m0:m0 + 256]
             want = want32.astype(np.float16).view(np.uint16)
             bad = np.argwhere(got != want)[:6]
             detail = [(int(r), int(c), float(got[r, c:c + 1].view(np.float16)[0]),
