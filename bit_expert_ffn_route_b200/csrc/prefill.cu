@@ -387,6 +387,13 @@ MOE_DEVINL void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 MOE_DEVINL void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Two fp32 values rounded to bf16 (nearest even) and packed: lo in bits 0..15.
+MOE_DEVINL uint32_t pack_bf16x2_rn(float lo, float hi) {
+    uint32_t d;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
 // L2 policies: the weight stream is read once (evict first); the activation
 // rows are re-read by every weight tile of their group (evict last).
 MOE_DEVINL uint64_t l2_evict_first() {
@@ -563,8 +570,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int cslot = 0;
         uint32_t cph = 0;
         bool ok = true;
+        int4 nxt = first < n_tiles ? __ldg(g.tiles + first) : make_int4(0, 0, 0, 0);   // one tile ahead
         for (int tile = first; tile < n_tiles && ok; tile += step, ++li) {
-            const int4 td = __ldg(g.tiles + tile);
+            const int4 td = nxt;
+            if (tile + step < n_tiles) nxt = __ldg(g.tiles + tile + step);
             const int w0 = td.z, slot = td.w;
             // Q3_S256: the row's super-block words (sub-scales, d), one super-block (two
             // rounds of this half) ahead of their use so that the loads' latency hides
@@ -671,8 +680,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
         int li = 0;
         bool range_bad = false;
+        int4 nxt = first < n_tiles ? __ldg(g.tiles + first) : make_int4(0, 0, 0, 0);   // one tile ahead
         for (int tile = first; tile < n_tiles; tile += step, ++li) {
-            const int4 td = __ldg(g.tiles + tile);
+            const int4 td = nxt;
+            if (tile + step < n_tiles) nxt = __ldg(g.tiles + tile + step);
             const int row0 = td.x, nrows = td.y, w0 = td.z;
             const int ab = li & 1;
             if (!mbar_wait_sleep(&acc_full[ab], (li >> 1) & 1, g.err)) break;
@@ -686,41 +697,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld16(acc + (uint32_t)(kTileW / 2 + c), uv);
                     tmem_ld_wait();
                     if (t < nrows) {
-                        float hb[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float gte = __uint_as_float(gv[i]), up = __uint_as_float(uv[i]);
-                            hb[i] = bf16_bits_to_f32(f32_to_bf16_rne(gte / (1.0f + expf(-gte)) * up));   // h is a bf16 value
-                            range_bad |= !(fabsf(hb[i]) < 65520.f);
-                        }
-                        // the 16 features in the K order of the down GEMM's row operand: word i = (i, i + 8)
+                        // the 16 features in the K order of the down GEMM's row operand: word i = (i, i + 8);
+                        // h is a bf16 value, carried exactly in fp16 when in range
                         uint32_t w[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            w[i] = (uint32_t)__half_as_ushort(__float2half_rn(hb[i])) |
-                                   ((uint32_t)__half_as_ushort(__float2half_rn(hb[i + 8])) << 16);
+                        for (int i = 0; i < 8; ++i) {
+                            const float g0 = __uint_as_float(gv[i]), u0 = __uint_as_float(uv[i]);
+                            const float g1 = __uint_as_float(gv[i + 8]), u1 = __uint_as_float(uv[i + 8]);
+                            const uint32_t hp = pack_bf16x2_rn(g0 / (1.0f + expf(-g0)) * u0, g1 / (1.0f + expf(-g1)) * u1);
+                            const float h0 = __uint_as_float(hp << 16), h1 = __uint_as_float(hp & 0xffff0000u);
+                            range_bad |= !(fabsf(h0) < 65520.f) || !(fabsf(h1) < 65520.f);
+                            const __half2 hh = __floats2half2_rn(h0, h1);
+                            w[i] = *reinterpret_cast<const uint32_t*>(&hh);
+                        }
                         uint4* dst = reinterpret_cast<uint4*>(g.dst + (size_t)(row0 + t) * F + w0 + c);
                         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
                         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     }
                 }
             } else {
-                for (int c = 0; c < kTileW; c += 32) {   // two loads in flight per wait
-                    uint32_t v[2][16];
-                    tmem_ld16(acc + (uint32_t)c, v[0]);
-                    tmem_ld16(acc + (uint32_t)(c + 16), v[1]);
-                    tmem_ld_wait();
-                    if (t < nrows) {
-                        uint4* dst = reinterpret_cast<uint4*>(g.dst + (size_t)(row0 + t) * D + w0 + c);
+                if (32 * q < nrows) {                    // a quadrant with no rows of the tile skips its loads
+                    for (int c = 0; c < kTileW; c += 32) {   // two loads in flight per wait
+                        uint32_t v[2][16];
+                        tmem_ld16(acc + (uint32_t)c, v[0]);
+                        tmem_ld16(acc + (uint32_t)(c + 16), v[1]);
+                        tmem_ld_wait();
+                        if (t < nrows) {
+                            uint4* dst = reinterpret_cast<uint4*>(g.dst + (size_t)(row0 + t) * D + w0 + c);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t w[8];
+                            for (int h = 0; h < 2; ++h) {
+                                uint32_t w[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                w[i] = (uint32_t)f32_to_bf16_rne(__uint_as_float(v[h][2 * i])) |
-                                       ((uint32_t)f32_to_bf16_rne(__uint_as_float(v[h][2 * i + 1])) << 16);
-                            dst[2 * h] = make_uint4(w[0], w[1], w[2], w[3]);
-                            dst[2 * h + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+                                for (int i = 0; i < 8; ++i)
+                                    w[i] = pack_bf16x2_rn(__uint_as_float(v[h][2 * i]), __uint_as_float(v[h][2 * i + 1]));
+                                dst[2 * h] = make_uint4(w[0], w[1], w[2], w[3]);
+                                dst[2 * h + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+                            }
                         }
                     }
                 }
@@ -738,8 +750,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int issued = 0, cst = 0, slot = 0;
             uint32_t ph = 0;
             bool ok = true;
+            int4 nxt = first < n_tiles ? __ldg(g.tiles + first) : make_int4(0, 0, 0, 0);   // one tile ahead
             for (int tile = first; tile < n_tiles && ok; tile += step) {
-                const int4 td = __ldg(g.tiles + tile);
+                const int4 td = nxt;
+                if (tile + step < n_tiles) nxt = __ldg(g.tiles + tile + step);
                 const int w0 = td.z, slot_id = td.w;
                 for (int c = 0; c < R / kSpr; ++c, ++cst) {
                     if (cst >= kCodeSlots && !mbar_wait_sleep(&empty_c[slot], ph ^ 1u, g.err)) {
@@ -775,8 +789,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             int issued = 0, gr = 0, rb = 0, b = 0, lb = 0;      // lb: round gr - kRBufs (mod kWBufs)
             uint32_t ph = 0, lph = 0;
+            int4 nxt = first < n_tiles ? __ldg(g.tiles + first) : make_int4(0, 0, 0, 0);   // one tile ahead
             for (int tile = first; tile < n_tiles && ok; tile += step) {
-                const int4 td = __ldg(g.tiles + tile);
+                const int4 td = nxt;
+                if (tile + step < n_tiles) nxt = __ldg(g.tiles + tile + step);
                 const int row0 = td.x, nrows = td.y;
                 const CUtensorMap* m = nrows > 64 ? &rows128 : nrows > 32 ? &rows64 : nrows > 16 ? &rows32 : &rows16;
                 const uint32_t bytes = (nrows > 64 ? 128u : nrows > 32 ? 64u : nrows > 16 ? 32u : 16u) * 128u;
