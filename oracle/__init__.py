@@ -64,6 +64,14 @@ def lib():
         L.orc_expert.argtypes = [ctypes.POINTER(_Pool), i, P, P, P]
         L.orc_moe_layer.argtypes = [ctypes.POINTER(_Pool), P, i, i, P, i, P, P, P, P,
                                     P, P, P, P, P, P, i]
+        L.orc_moe_layer_fp8.argtypes = L.orc_moe_layer.argtypes
+        L.orc_expert_fp8.argtypes = [ctypes.POINTER(_Pool), i, P, P]
+        L.orc_e4m3_rne.restype = ctypes.c_uint8
+        L.orc_e4m3_rne.argtypes = [ctypes.c_double]
+        L.orc_e4m3_to_f64.restype = ctypes.c_double
+        L.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.orc_f16_round.restype = ctypes.c_double
+        L.orc_f16_round.argtypes = [ctypes.c_double]
         L.orc_bf16_rne.restype = ctypes.c_uint16
         L.orc_bf16_rne.argtypes = [ctypes.c_double]
         L.orc_f16_to_f32.restype = ctypes.c_float
@@ -173,8 +181,9 @@ class LayerResult:
 
 
 def moe_layer(pool: HostPool, slot_table, k, x, Wr, bias=None, miss_partial=None,
-              residual=None, n_threads: int = 1) -> LayerResult:
-    """The whole expert pass for T tokens (see moe_oracle.h)."""
+              residual=None, n_threads: int = 1, fp8: bool = False) -> LayerResult:
+    """The whole expert pass for T tokens (see moe_oracle.h); fp8=True is the
+    e4m3-operand variant (orc_moe_layer_fp8)."""
     x = _c(x, np.uint16); Wr = _c(Wr, np.uint16); bias = _c(bias, np.float32)
     st = _c(slot_table, np.int32)
     mp = _c(miss_partial, np.float32); res = _c(residual, np.uint16)
@@ -187,7 +196,8 @@ def moe_layer(pool: HostPool, slot_table, k, x, Wr, bias=None, miss_partial=None
     slots = np.empty((T, k), np.int32)
     miss = np.empty((max(T * k, 1), 3), np.int32)
     p = pool._c()
-    n = lib().orc_moe_layer(ctypes.byref(p), _ptr(st), E, k, _ptr(x), T, _ptr(Wr), _ptr(bias),
+    fn = lib().orc_moe_layer_fp8 if fp8 else lib().orc_moe_layer
+    n = fn(ctypes.byref(p), _ptr(st), E, k, _ptr(x), T, _ptr(Wr), _ptr(bias),
                             _ptr(mp), _ptr(res), _ptr(out), _ptr(logits), _ptr(ids), _ptr(gates),
                             _ptr(slots), _ptr(miss), int(n_threads))
     if n < 0:
@@ -201,3 +211,26 @@ def bf16_rne(v: float) -> int:
 
 def f16_to_f32(h: int) -> float:
     return float(lib().orc_f16_to_f32(int(h)))
+
+
+def e4m3_rne(v: float) -> int:
+    """The e4m3 byte nearest to v (ties to even, saturating at +-448)."""
+    return int(lib().orc_e4m3_rne(float(v)))
+
+
+def e4m3_to_f64(b: int) -> float:
+    return float(lib().orc_e4m3_to_f64(int(b)))
+
+
+def f16_round(v: float) -> float:
+    return float(lib().orc_f16_round(float(v)))
+
+
+def expert_fp8(pool: HostPool, slot: int, x):
+    """The e4m3-operand variant of one expert on one token: y float64 [D]."""
+    x = _c(x, np.uint16)
+    y = np.empty(pool.d_model, np.float64)
+    p = pool._c()
+    if lib().orc_expert_fp8(ctypes.byref(p), slot, _ptr(x), _ptr(y)) != 0:
+        raise ValueError("orc_expert_fp8: bad arguments")
+    return y

@@ -66,6 +66,60 @@ uint16_t orc_bf16_rne(double v)
     return (uint16_t)(bits | (v < 0 ? 0x8000 : 0));
 }
 
+/* Round a double to the nearest IEEE binary16 value (ties to even) and return
+ * that value.  11 significant bits; smallest normal 2^-14, subnormal spacing
+ * 2^-24; magnitudes that round above 65504 become infinite. */
+static double f16_round(double v)
+{
+    if (isnan(v) || v == 0.0) return v;
+    double a = fabs(v);
+    int e;
+    frexp(a, &e);
+    int E = e - 1;
+    double quantum = (E < -14) ? ldexp(1.0, -24) : ldexp(1.0, E - 10);
+    double r = rint(a / quantum) * quantum;
+    if (r > 65504.0) r = INFINITY;
+    return v < 0 ? -r : r;
+}
+
+/* E4M3 (8-bit float: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities, S.1111.111 is NaN, largest finite 448 = 1.75 * 2^8, subnormals
+ * m * 2^-9).  Round to nearest, ties to even, saturating at +-448; NaN -> 0x7f. */
+uint8_t orc_e4m3_rne(double v)
+{
+    if (isnan(v)) return 0x7f;
+    const uint8_t sign = (v < 0 || (v == 0.0 && signbit(v))) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7e);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);
+    int E = e - 1;                                   /* a = 1.xxx * 2^E */
+    double quantum = (E < -6) ? ldexp(1.0, -9) : ldexp(1.0, E - 3);
+    double r = rint(a / quantum) * quantum;          /* nearest, ties to even */
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return sign;
+    frexp(r, &e);
+    E = e - 1;
+    if (E < -6)                                      /* subnormal: m * 2^-9 */
+        return (uint8_t)(sign | (int)(r / ldexp(1.0, -9)));
+    int m = (int)(r / ldexp(1.0, E - 3)) - 8;        /* 1.mmm */
+    return (uint8_t)(sign | ((E + 7) << 3) | m);
+}
+
+double orc_e4m3_to_f64(uint8_t b)
+{
+    const int e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return (b & 0x80) ? -v : v;
+}
+
+static double e4m3_value(double v) { return orc_e4m3_to_f64(orc_e4m3_rne(v)); }
+
+/* the fp16 value nearest to v (ties to even), exposed for the oracle's pins */
+double orc_f16_round(double v) { return f16_round(v); }
+
 /* ------------------------------------------------------------------ */
 /* block formats                                                        */
 /*                                                                     */
@@ -321,6 +375,45 @@ int orc_expert(const orc_pool* P, int slot, const uint16_t* x, uint16_t* h_out, 
     return 0;
 }
 
+/* The e4m3-operand variant of the expert (the library's lossy option; the
+ * pages fix no such variant, its definition is this library's):
+ *   weight operand  W8 = e4m3( fp16( 64 w ) )  (w the exact block weight)
+ *   x operand       x8 = e4m3( x )
+ *   gate_pre = sum W8g x8 / 64,  up_pre = sum W8u x8 / 64   (double)
+ *   h8 = e4m3( silu(gate_pre) * up_pre )
+ *   y[d] = sum_f W8d[d][f] h8[f] / 64                       (double)  */
+int orc_expert_fp8(const orc_pool* P, int slot, const uint16_t* x, double* y)
+{
+    if (!pool_ok(P) || slot < 0 || slot >= P->n_slots || !x || !y) return -1;
+    const int D = P->d_model, F = P->d_ff;
+    float* rowg = (float*)malloc(sizeof(float) * (size_t)(D > F ? D : F));
+    float* rowu = (float*)malloc(sizeof(float) * (size_t)(D > F ? D : F));
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* x8 = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!rowg || !rowu || !h || !x8) { free(rowg); free(rowu); free(h); free(x8); return -1; }
+    for (int i = 0; i < D; ++i) x8[i] = e4m3_value(bf16_to_f32(x[i]));
+    for (int f = 0; f < F; ++f) {
+        dequant_row(P, slot, 0, f, rowg);
+        dequant_row(P, slot, 1, f, rowu);
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < D; ++i) {
+            g += e4m3_value(f16_round(64.0 * rowg[i])) * x8[i];
+            u += e4m3_value(f16_round(64.0 * rowu[i])) * x8[i];
+        }
+        g /= 64.0;
+        u /= 64.0;
+        h[f] = e4m3_value(g / (1.0 + exp(-g)) * u);
+    }
+    for (int d = 0; d < D; ++d) {
+        dequant_row(P, slot, 2, d, rowg);
+        double acc = 0.0;
+        for (int f = 0; f < F; ++f) acc += e4m3_value(f16_round(64.0 * rowg[f])) * h[f];
+        y[d] = acc / 64.0;
+    }
+    free(rowg); free(rowu); free(h); free(x8);
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* 1-6: one layer                                                       */
 /*   out[t] = bf16( sum_{r<k, hit} g[t,r] y[t,r] + y_shared[t]          */
@@ -330,11 +423,11 @@ int orc_expert(const orc_pool* P, int slot, const uint16_t* x, uint16_t* h_out, 
 /* path leaves misses to the caller, who may pass their partial sum).    */
 /* The shared expert has weight 1 and always sits in pool->shared_slot.  */
 /* ------------------------------------------------------------------ */
-int orc_moe_layer(const orc_pool* P, const int32_t* slot_table, int E, int k,
-                  const uint16_t* x, int T, const uint16_t* Wr, const float* bias,
-                  const float* miss_partial, const uint16_t* residual,
-                  uint16_t* out, float* logits_out, int32_t* ids_out, double* gates_out,
-                  int32_t* slots_out, int32_t* miss_list, int n_threads)
+static int moe_layer_impl(const orc_pool* P, const int32_t* slot_table, int E, int k,
+                          const uint16_t* x, int T, const uint16_t* Wr, const float* bias,
+                          const float* miss_partial, const uint16_t* residual,
+                          uint16_t* out, float* logits_out, int32_t* ids_out, double* gates_out,
+                          int32_t* slots_out, int32_t* miss_list, int n_threads, int fp8)
 {
     if (!pool_ok(P) || !slot_table || !x || !Wr || !out || T < 0 || k <= 0 || k > E) return -1;
     if (P->shared_slot < 0 || P->shared_slot >= P->n_slots) return -1;
@@ -365,7 +458,9 @@ int orc_moe_layer(const orc_pool* P, const int32_t* slot_table, int E, int k,
         int t = pr / per_tok, r = pr % per_tok;
         int s = (r < k) ? slots[(size_t)t * k + r] : P->shared_slot;
         if (s < 0) continue;
-        if (orc_expert(P, s, x + (size_t)t * D, NULL, ys + (size_t)pr * D) != 0) failed += 1;
+        const int rc_e = fp8 ? orc_expert_fp8(P, s, x + (size_t)t * D, ys + (size_t)pr * D)
+                             : orc_expert(P, s, x + (size_t)t * D, NULL, ys + (size_t)pr * D);
+        if (rc_e != 0) failed += 1;
     }
     for (int t = 0; t < T && !failed; ++t) {
         for (int d = 0; d < D; ++d) {
@@ -387,4 +482,24 @@ int orc_moe_layer(const orc_pool* P, const int32_t* slot_table, int E, int k,
     if (slots_out) memcpy(slots_out, slots, sizeof(int32_t) * (size_t)T * k);
     free(logits); free(ids); free(gates); free(slots);
     return failed ? -1 : n_miss;
+}
+
+int orc_moe_layer(const orc_pool* P, const int32_t* slot_table, int E, int k,
+                  const uint16_t* x, int T, const uint16_t* Wr, const float* bias,
+                  const float* miss_partial, const uint16_t* residual,
+                  uint16_t* out, float* logits_out, int32_t* ids_out, double* gates_out,
+                  int32_t* slots_out, int32_t* miss_list, int n_threads)
+{
+    return moe_layer_impl(P, slot_table, E, k, x, T, Wr, bias, miss_partial, residual, out, logits_out, ids_out,
+                          gates_out, slots_out, miss_list, n_threads, 0);
+}
+
+int orc_moe_layer_fp8(const orc_pool* P, const int32_t* slot_table, int E, int k,
+                      const uint16_t* x, int T, const uint16_t* Wr, const float* bias,
+                      const float* miss_partial, const uint16_t* residual,
+                      uint16_t* out, float* logits_out, int32_t* ids_out, double* gates_out,
+                      int32_t* slots_out, int32_t* miss_list, int n_threads)
+{
+    return moe_layer_impl(P, slot_table, E, k, x, T, Wr, bias, miss_partial, residual, out, logits_out, ids_out,
+                          gates_out, slots_out, miss_list, n_threads, 1);
 }

@@ -72,9 +72,22 @@ int orc_moe_layer(const orc_pool* pool, const int32_t* slot_table, int E, int k,
                   uint16_t* out, float* logits, int32_t* ids, double* gates,
                   int32_t* slots, int32_t* miss_list, int n_threads);
 
+/* The e4m3-operand variant (weights e4m3(fp16(64 w)), x and h e4m3, products
+ * in double scaled by 1/64): one expert, and 1-6 for T tokens with the same
+ * arguments and results as orc_moe_layer. */
+int orc_expert_fp8(const orc_pool* pool, int slot, const uint16_t* x, double* y);
+int orc_moe_layer_fp8(const orc_pool* pool, const int32_t* slot_table, int E, int k,
+                      const uint16_t* x, int T, const uint16_t* Wr, const float* bias,
+                      const float* miss_partial, const uint16_t* residual,
+                      uint16_t* out, float* logits, int32_t* ids, double* gates,
+                      int32_t* slots, int32_t* miss_list, int n_threads);
+
 /* helpers exposed for the oracle's own pins */
 uint16_t orc_bf16_rne(double v);
 float    orc_f16_to_f32(uint16_t h);
+uint8_t  orc_e4m3_rne(double v);         /* nearest even, saturating at +-448 */
+double   orc_e4m3_to_f64(uint8_t b);
+double   orc_f16_round(double v);         /* nearest fp16 value, ties to even */
 
 #ifdef __cplusplus
 }
