@@ -216,6 +216,45 @@ def _roofline(kind, per_launch, avg_ms, peaks, traffic_kind):
             "algorithmic_flops_per_launch": round(per_launch), "avg_launch_us": round(avg_ms * 1e3, 3)}
 
 
+def _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_flops, peaks):
+    """The same prefill steps with the e4m3-operand expert pass
+    (moe_expert_forward_fp8): step time and the expert pass against the e4m3
+    tensor peak (the measured bf16 peak x 2, the nominal dense ratio)."""
+    with torch.cuda.stream(stream):
+        for r in range(R):
+            layers[r](xs[r], stream=stream, fp8=True)          # allocates each layer's e4m3 workspace
+    torch.cuda.synchronize()
+
+    def fp8_step(i, events=False):
+        lay = layers[i % R]
+        moe.moe_route_topk(xs[i % R], lay.Wr, lay.bias, k, lay.ids, lay.gates, lay.route_ws, stream=stream)
+        if events:
+            ev[i][0].record(stream)
+        moe.moe_expert_forward_fp8(lay.pool, lay.slot_table, xs[i % R], lay.ids, k, lay.expert_out, lay.miss_list,
+                                   lay.miss_count, lay.ws_fp8, stream=stream)
+        if events:
+            ev[i][1].record(stream)
+        moe.moe_combine(lay.expert_out, lay.gates, T, D, k, lay.out, stream=stream)
+
+    g8 = _graph_of(fp8_step, G, stream)
+    g8e = _graph_of(lambda i: fp8_step(i, True), G, stream)
+    with torch.cuda.stream(stream):
+        g8.replay()
+        g8e.replay()
+    ms8, _ = _timed_replays(g8, K // G, stream, ws_, dev, local, clocks=False)
+    _timed_replays(g8e, K // G, stream, ws_, dev, local, clocks=False)
+    fwd8 = float(np.mean([ev[i][0].elapsed_time(ev[i][1]) for i in range(G)]))
+    hbm, tf, tf_sus, kind = peaks
+    roof8 = _roofline("tensor", float(np.mean([fwd_flops[i % R] for i in range(G)])), fwd8,
+                      (hbm, round(2 * tf, 1), round(2 * tf_sus, 1), kind), "prefill_fp8")
+    roof8["peak_kind"] = f"measured bf16 burst x 2 (e4m3 nominal dense ratio); sustained {round(2 * tf_sus, 1)}"
+    roof8["kernel"] = "moe_expert_forward_fp8 (plan + e4m3 gather + tcgen05 kind::f8f6f4 grouped GEMMs)"
+    del g8, g8e
+    return {"value": round(ws_ * T * K / (ms8 / 1e3), 1), "unit": "tokens/s", "ms_per_step": round(ms8 / K, 6),
+            "dtype": "e4m3 operands (weights x64, x, h), fp32 accumulate; lossy, see tests/test_gpu_fp8.py",
+            "roofline": roof8}
+
+
 # ---------------------------------------------------------------- one-layer workloads
 def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     cfg = configs.CONFIGS[name]
@@ -388,6 +427,8 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     }
     if three is not None:
         res["three_calls"] = three
+    if T > 8:
+        res["fp8_variant"] = _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_flops, peaks)
     if T > 8:
         loads = np.bincount(layers[0].ids.cpu().numpy().ravel(), minlength=E)
         res["expert_loads"] = {"max": int(loads.max()), "zero": int((loads == 0).sum()),
@@ -677,7 +718,8 @@ def run_ours(args, ws_, rank, local):
         "e2e": head["e2e"], "gpu_launches": head["gpu_launches"], "roofline": head["roofline"],
         "clocks": head["clocks"],
     }
-    for key in ("hit_rate", "u_hit_mean", "step_alg_bytes", "chain_tokens_per_s", "expert_loads", "three_calls"):
+    for key in ("hit_rate", "u_hit_mean", "step_alg_bytes", "chain_tokens_per_s", "expert_loads", "three_calls",
+                "fp8_variant"):
         if key in head:
             line[key] = head[key]
     if "cpu_baseline" in head:

@@ -134,7 +134,32 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
         return reported(launch_decode_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
                                               (cudaStream_t)stream));
     return reported(launch_prefill_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
-                                           (cudaStream_t)stream));
+                                           (cudaStream_t)stream, false));
+}
+
+size_t moe_workspace_size_fp8(int T, int D, int F, int E, int k, int fmt) {
+    if (check_shapes(T, D, E, k) != MOE_OK || F <= 0 || !fmt_ok(fmt) || T <= kDecodeMaxT) return 0;
+    return prefill_workspace_bytes(T, D, F, E, k);
+}
+
+moe_status moe_expert_forward_fp8(const moe_pool* pool, const int32_t* slot_table, int E, const uint16_t* x, int T,
+                                  const int32_t* ids, int k, void* expert_out, size_t expert_out_bytes_,
+                                  int32_t* miss_list, int32_t* miss_count, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream) {
+    PoolView v;
+    moe_status st = check_pool(pool, v);
+    if (st != MOE_OK) return st;
+    st = check_shapes(T, v.D, E, k);
+    if (st != MOE_OK) return st;
+    if (!miss_count) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return cuda_status(cudaMemsetAsync(miss_count, 0, sizeof(int32_t), (cudaStream_t)stream));
+    if (T <= kDecodeMaxT) return MOE_ERR_UNSUPPORTED;    // moe_combine reads the small-batch layout there
+    if (!slot_table || !x || !ids || !expert_out || !miss_list || !ws) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(expert_out, 256) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    if (expert_out_bytes_ < expert_out_bytes(T, v.D, k)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < moe_workspace_size_fp8(T, v.D, v.F, E, k, v.fmt)) return MOE_ERR_WORKSPACE;
+    return reported(launch_prefill_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
+                                           (cudaStream_t)stream, true));
 }
 
 size_t moe_layer_workspace_size(int T, int D, int F, int E, int k, int fmt) {

@@ -46,7 +46,7 @@ size_t layer_workspace_bytes(int T, int D, int F, int E, int k);
 
 moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x,
                                   int T, const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
-                                  int32_t* miss_count, void* ws, cudaStream_t s);
+                                  int32_t* miss_count, void* ws, cudaStream_t s, bool fp8);
 size_t prefill_workspace_bytes(int T, int D, int F, int E, int k);
 size_t prefill_operand_dump_ws_bytes(int D, int F);
 moe_status launch_prefill_operand_dump(const PoolView& P, int gemm, int slot, int m0, uint32_t* dump, void* ws,

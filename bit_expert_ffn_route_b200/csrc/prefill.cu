@@ -316,6 +316,48 @@ __global__ void __launch_bounds__(256) gather_f16p_kernel(const uint16_t* __rest
     if (bad) atomicOr(err, kErrRange);
 }
 
+// Two fp16 values (a pair word) to two e4m3 bytes, rounded to nearest even and
+// saturated to the finite range: the low half to bits 0..7.
+MOE_DEVINL uint32_t e4m3x2_of_f16x2(uint32_t h2) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(d) : "r"(h2));
+    return d;
+}
+// Two fp32 values to two e4m3 bytes (nearest even, saturated): lo in bits 0..7.
+MOE_DEVINL uint32_t e4m3x2_of_f32(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+// The e4m3 variant: x rows in group order as e4m3 bytes, K-permuted the same way
+// (bytes 2i, 2i + 1 of a 16-group = elements i, i + 8), rounded to nearest even
+// and saturated; |x| >= 448 sets the range bit.
+__global__ void __launch_bounds__(256) gather_f8p_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+                                                         const int32_t* __restrict__ meta, int T, int D,
+                                                         uint8_t* __restrict__ xg, uint32_t* err) {
+    pdl_wait();
+    const int row_groups = D / 16;
+    const size_t ngroups = (size_t)(__ldg(meta) + T) * row_groups;
+    bool bad = false;
+    for (size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x; gi < ngroups; gi += (size_t)gridDim.x * blockDim.x) {
+        const size_t row = gi / row_groups, gc = gi % row_groups;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)__ldg(perm + row) * D + gc * 16);
+        const uint4 a = __ldg(src), b = __ldg(src + 1);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+        uint32_t o[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float lo = __uint_as_float(bf16_half(aw[i >> 1], i & 1));
+            const float hi = __uint_as_float(bf16_half(bw[i >> 1], i & 1));
+            bad |= !(fabsf(lo) < 448.f) || !(fabsf(hi) < 448.f);
+            o[i >> 1] |= e4m3x2_of_f32(lo, hi) << (16 * (i & 1));
+        }
+        *reinterpret_cast<uint4*>(xg + row * D + gc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (bad) atomicOr(err, kErrRange);
+}
+
 // ---------------------------------------------------------------- tcgen05 / TMA helpers
 MOE_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
     uint64_t d = 0;
@@ -365,12 +407,20 @@ static_assert(kGemmSmem + 1024 + 512 <= 232448, "shared memory per block");
 MOE_DEVINL uint32_t instr_desc_tile() {
     return (1u << 4) | ((uint32_t)(kTileW >> 3) << 17) | ((uint32_t)(kTileRows >> 4) << 24);
 }
-// D[tmem] (+)= A[smem] * B[smem]^T
+// D[tmem] (+)= A[smem] * B[smem]^T; kind::f16 (K = 16) or, with F8, kind::f8f6f4
+// (K = 32, both operands e4m3: the format fields of the descriptor are 0 as for fp16)
+template <bool F8>
 MOE_DEVINL void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+    if constexpr (F8)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 MOE_DEVINL void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -505,7 +555,7 @@ MOE_DEVINL void dequant_block(const uint32_t (&cw)[3], uint32_t sm, const uint32
 // i / 256 of each K = 64 round), 16..19 epilogue (TMEM lane quadrant w % 4 =
 // rows 32q..), 20 TMA of the code stages (two rounds each), 21 TMA of the row
 // operand, 22 MMA issue.  TMEM: two 128 x 256 fp32 accumulators.
-template <int FMT, int MODE>
+template <int FMT, int MODE, bool F8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_scales,
                        const __grid_constant__ CUtensorMap rows128, const __grid_constant__ CUtensorMap rows64,
@@ -528,15 +578,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = g.D, F = g.F;
     const int K = MODE == 1 ? D : F;
-    const int R = K / kRound;                   // rounds per tile
-    constexpr int CP = kSpr * 2 * Fm::kCb, SP = kSpr * 8;   // code / scale bytes per weight row of a stage
+    // a round is one 128-byte swizzle row of each operand: K = 64 fp16 or K = 128 e4m3
+    constexpr int kKR = F8 ? 128 : kRound;
+    const int R = K / kKR;                      // rounds per tile
+    constexpr int CP = kSpr * 2 * Fm::kCb, SP = kSpr * 8;   // code / scale bytes per weight row of a stage (K = 128)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCodeSlots; ++s) {
             mbar_init(&full_c[s], 1);
             mbar_init(&empty_c[s], kDqWarps);       // every dequant warp, once it has read the stage
         }
-        for (int s = 0; s < kWBufs; ++s) { mbar_init(&ready[s], kDqWarps / 2 + 1); mbar_init(&done[s], 1); }
+        for (int s = 0; s < kWBufs; ++s) {
+            mbar_init(&ready[s], (F8 ? kDqWarps : kDqWarps / 2) + 1);
+            mbar_init(&done[s], 1);
+        }
         for (int s = 0; s < kAccBufs; ++s) { mbar_init(&acc_full[s], 1); mbar_init(&acc_empty[s], kEpiWarps); }
         mbar_init(&drain_bar, 1);
         fence_mbar_init();
@@ -560,13 +615,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int first = blockIdx.x, step = gridDim.x;
 
     if (!dead && warp < kDqWarps) {
-        // ---------------- dequantisation into the weight operand (shared memory).  Half h
-        // (warps 8h..8h+7) takes the rounds of parity h: round 2c + h of a tile is sub-round
-        // h of code stage c, and its weights go to buffer h or h + 2 in turn.  Thread:
-        // weight row r, both 32-weight blocks of the round (16 contiguous code bytes).
-        const int r = (int)threadIdx.x & (kTileW - 1), half = (int)threadIdx.x >> 8;
+        // ---------------- dequantisation into the weight operand (shared memory).  Thread:
+        // weight row r and part hp of each code stage (the 16 contiguous code bytes of two
+        // 32-weight blocks).  fp16: a round is half a stage; half hp (warps 8hp..8hp+7)
+        // takes the rounds of parity hp, i.e. part hp of every stage, and writes the whole
+        // 128-byte row of its round into buffer hp or hp + 2 in turn.  e4m3: a round is a
+        // stage; all 16 warps take every round, part hp fills bytes [64 hp, 64 hp + 64) of
+        // the row, buffers in turn.
+        const int r = (int)threadIdx.x & (kTileW - 1), hp = (int)threadIdx.x >> 8;
+        constexpr int kStep = F8 ? 1 : 2;          // rounds between two of this thread's rounds
+        constexpr int kSeq = F8 ? kWBufs : 2;      // buffers in this thread's sequence
         const Magic Mg = make_magic();
-        int li = 0, j = 0;                         // j: rounds of this half so far
+        int li = 0, j = 0;                         // j: this thread's rounds so far
         int cslot = 0;
         uint32_t cph = 0;
         bool ok = true;
@@ -575,9 +635,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int4 td = nxt;
             if (tile + step < n_tiles) nxt = __ldg(g.tiles + tile + step);
             const int w0 = td.z, slot = td.w;
-            // Q3_S256: the row's super-block words (sub-scales, d), one super-block (two
-            // rounds of this half) ahead of their use so that the loads' latency hides
-            uint32_t sbw[4] = {0, 0, 0, 0}, nxt[4] = {0, 0, 0, 0};
+            // Q3_S256: the row's super-block words (sub-scales, d), one super-block ahead of
+            // their use so that the loads' latency hides behind the rounds before
+            uint32_t sbw[4] = {0, 0, 0, 0}, sbn[4] = {0, 0, 0, 0};
+            int sb_cur = -1;
             const uint8_t* sbase = nullptr;
             size_t sb_row = 0, d_row = 0;
             if constexpr (FMT == MOE_Q3_S256) {
@@ -588,22 +649,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 sb_row = (size_t)pm * blocks * 12 + (size_t)wrow * (K / 256) * 12;
                 d_row = 3 * blocks * 12 + ((size_t)pm * blocks + (size_t)wrow * (K / 256)) * 2;
                 const uint8_t* sp = sbase + sb_row;
-                nxt[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
-                nxt[1] = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
-                nxt[2] = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
-                nxt[3] = __ldg(reinterpret_cast<const uint16_t*>(sbase + d_row));
+                sbn[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
+                sbn[1] = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
+                sbn[2] = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
+                sbn[3] = __ldg(reinterpret_cast<const uint16_t*>(sbase + d_row));
             }
-            for (int rr = half; rr < R; rr += 2, ++j) {
+            for (int rr = F8 ? 0 : hp; rr < R; rr += kStep, ++j) {
                 if (!mbar_wait_sleep(&full_c[cslot], cph, g.err)) { ok = false; break; }
                 const uint8_t* cs = code_ring + cslot * kCodeSlotBytes;
-                // both blocks' code bytes [half * 2 kCb, +2 kCb) and (s, m) words of the row
+                // both blocks' code bytes [hp * 2 kCb, +2 kCb) and (s, m) words of the row
                 uint32_t cw[2][3], sm[2] = {0, 0};
                 if constexpr (Fm::kCb == 8) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(cs + swz_chunk(r, half, CP));
+                    const uint4 v = *reinterpret_cast<const uint4*>(cs + swz_chunk(r, hp, CP));
                     cw[0][0] = v.x; cw[0][1] = v.y; cw[0][2] = 0;
                     cw[1][0] = v.z; cw[1][1] = v.w; cw[1][2] = 0;
                 } else {
-                    const uint8_t* rowp = cs + r * CP + half * 24;            // CP = 48: not swizzled
+                    const uint8_t* rowp = cs + r * CP + hp * 24;              // CP = 48: not swizzled
                     const uint2 a = *reinterpret_cast<const uint2*>(rowp);
                     const uint2 b = *reinterpret_cast<const uint2*>(rowp + 8);
                     const uint2 c = *reinterpret_cast<const uint2*>(rowp + 16);
@@ -611,28 +672,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     cw[1][0] = b.y; cw[1][1] = c.x; cw[1][2] = c.y;
                 }
                 if constexpr (Fm::kTmaScales) {
-                    const uint2 v = *reinterpret_cast<const uint2*>(cs + kTileW * CP + r * SP + half * 8);
+                    const uint2 v = *reinterpret_cast<const uint2*>(cs + kTileW * CP + r * SP + hp * 8);
                     sm[0] = v.x; sm[1] = v.y;
+                    if constexpr (F8) {                    // e4m3 operand: weights x 64 (exact in fp16)
+                        sm[0] = hmul2u(sm[0], 0x54005400u);
+                        sm[1] = hmul2u(sm[1], 0x54005400u);
+                    }
                 }
                 uint32_t sc2[2][2] = {{0, 0}, {0, 0}}, d2 = 0;
                 if constexpr (FMT == MOE_Q3_S256) {
-                    if ((rr >> 1) % 2 == 0) {              // rounds 4m + half: a new super-block
+                    const int kb0 = F8 ? 4 * rr + 2 * hp : 2 * rr;             // the thread's first block in the row
+                    const int sbi = kb0 >> 3;
+                    if (sbi != sb_cur) {                   // a new super-block: take the prefetched words
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) sbw[i] = nxt[i];
-                        const int jn = (rr >> 2) + 1;
-                        if (jn < K / 256) {
-                            const uint8_t* sp = sbase + sb_row + (size_t)jn * 12;
-                            nxt[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
-                            nxt[1] = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
-                            nxt[2] = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
-                            nxt[3] = __ldg(reinterpret_cast<const uint16_t*>(sbase + d_row) + jn);
+                        for (int i = 0; i < 4; ++i) sbw[i] = sbn[i];
+                        sb_cur = sbi;
+                        if (sbi + 1 < K / 256) {
+                            const uint8_t* sp = sbase + sb_row + (size_t)(sbi + 1) * 12;
+                            sbn[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
+                            sbn[1] = __ldg(reinterpret_cast<const uint32_t*>(sp + 4));
+                            sbn[2] = __ldg(reinterpret_cast<const uint32_t*>(sp + 8));
+                            sbn[3] = __ldg(reinterpret_cast<const uint16_t*>(sbase + d_row) + sbi + 1);
                         }
                     }
                     d2 = sbw[3] | (sbw[3] << 16);
+                    if constexpr (F8) d2 = hmul2u(d2, 0x54005400u);
                     const uint64_t lo = ((uint64_t)sbw[1] << 32) | sbw[0], hi = ((uint64_t)sbw[2] << 32) | sbw[1];
 #pragma unroll
                     for (int b = 0; b < 2; ++b) {
-                        const int c = (2 * rr + b) & 7;                        // sub-blocks 2c, 2c + 1
+                        const int c = (kb0 + b) & 7;                           // sub-blocks 2c, 2c + 1
                         const uint32_t bits = c < 4 ? (uint32_t)(lo >> (12 * c)) : (uint32_t)(hi >> (12 * c - 32));
                         sc2[b][0] = s256_sub(bits & 63u);
                         sc2[b][1] = s256_sub((bits >> 6) & 63u);
@@ -647,25 +715,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (lane == 0) mbar_arrive_dep(&empty_c[cslot], dep);
                 if (++cslot == kCodeSlots) { cslot = 0; cph ^= 1u; }
                 // the buffer is free once the MMAs of its previous use completed
-                const int wb = half + 2 * (j & 1);
-                if (j >= 2) {
-                    if (!mbar_wait_sleep(&done[wb], ((j >> 1) - 1) & 1, g.err)) { ok = false; break; }
+                const int wb = F8 ? (j & (kWBufs - 1)) : hp + 2 * (j & 1);
+                const int use = j / kSeq;
+                if (use >= 1) {
+                    if (!mbar_wait_sleep(&done[wb], (use - 1) & 1, g.err)) { ok = false; break; }
                     tc_fence_after();
                 }
                 uint8_t* wbuf = w_ring + wb * kWRoundBytes;
+                if constexpr (F8) {
+                    // e4m3 pairs: word i of a block's fp16 pairs (16h + i, 16h + i + 8) -> bytes 2i, 2i + 1
 #pragma unroll
-                for (int b = 0; b < 2; ++b)
+                    for (int b = 0; b < 2; ++b)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        *reinterpret_cast<uint4*>(wbuf + sw128(r, 4 * b + q)) =
-                            make_uint4(o[b][4 * q], o[b][4 * q + 1], o[b][4 * q + 2], o[b][4 * q + 3]);
-                if (g.dump != nullptr && tile == g.dump_tile) {
-                    // test hook: the round's weight operand as the MMAs will read it
-                    uint32_t* drow = g.dump + ((size_t)rr * kTileW + r) * 32;
+                        for (int q = 0; q < 2; ++q) {
+                            uint32_t e[4];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(wbuf + sw128(r, q));
-                        drow[4 * q] = v.x; drow[4 * q + 1] = v.y; drow[4 * q + 2] = v.z; drow[4 * q + 3] = v.w;
+                            for (int i = 0; i < 4; ++i)
+                                e[i] = e4m3x2_of_f16x2(o[b][8 * q + 2 * i]) | (e4m3x2_of_f16x2(o[b][8 * q + 2 * i + 1]) << 16);
+                            *reinterpret_cast<uint4*>(wbuf + sw128(r, 4 * hp + 2 * b + q)) = make_uint4(e[0], e[1], e[2], e[3]);
+                        }
+                } else {
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            *reinterpret_cast<uint4*>(wbuf + sw128(r, 4 * b + q)) =
+                                make_uint4(o[b][4 * q], o[b][4 * q + 1], o[b][4 * q + 2], o[b][4 * q + 3]);
+                    if (g.dump != nullptr && tile == g.dump_tile) {
+                        // test hook: the round's weight operand as the MMAs will read it
+                        uint32_t* drow = g.dump + ((size_t)rr * kTileW + r) * 32;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const uint4 v = *reinterpret_cast<const uint4*>(wbuf + sw128(r, q));
+                            drow[4 * q] = v.x; drow[4 * q + 1] = v.y; drow[4 * q + 2] = v.z; drow[4 * q + 3] = v.w;
+                        }
                     }
                 }
                 fence_proxy_async();                 // generic stores -> the tensor core's reads
@@ -675,6 +758,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else if (!dead && warp < kTmaWarp) {
         // ---------------- epilogue: TMEM -> registers -> global; lane = row of the tile
+        constexpr float kDescale = F8 ? 0.015625f : 1.0f;    // e4m3 weights carry a factor 64
         const int q = warp & 3;
         const int t = 32 * q + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(32 * q) << 16);
@@ -696,7 +780,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tmem_ld16(acc + (uint32_t)c, gv);
                     tmem_ld16(acc + (uint32_t)(kTileW / 2 + c), uv);
                     tmem_ld_wait();
-                    if (t < nrows) {
+                    if (F8 && t < nrows) {
+                        // acc = 64 x the products (the e4m3 weights carry a factor 64); h in e4m3, the 16
+                        // features in the K order of the down GEMM's row operand: bytes 2i, 2i + 1 = (i, i + 8)
+                        uint32_t e[4] = {0, 0, 0, 0};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float g0 = __uint_as_float(gv[i]) * kDescale, u0 = __uint_as_float(uv[i]) * kDescale;
+                            const float g1 = __uint_as_float(gv[i + 8]) * kDescale, u1 = __uint_as_float(uv[i + 8]) * kDescale;
+                            const float h0 = g0 / (1.0f + expf(-g0)) * u0, h1 = g1 / (1.0f + expf(-g1)) * u1;
+                            range_bad |= !(fabsf(h0) < 448.f) || !(fabsf(h1) < 448.f);
+                            e[i >> 1] |= e4m3x2_of_f32(h0, h1) << (16 * (i & 1));
+                        }
+                        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(g.dst) + (size_t)(row0 + t) * F + w0 + c) =
+                            make_uint4(e[0], e[1], e[2], e[3]);
+                    } else if (t < nrows) {
                         // the 16 features in the K order of the down GEMM's row operand: word i = (i, i + 8);
                         // h is a bf16 value, carried exactly in fp16 when in range
                         uint32_t w[8];
@@ -729,7 +827,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 uint32_t w[8];
 #pragma unroll
                                 for (int i = 0; i < 8; ++i)
-                                    w[i] = pack_bf16x2_rn(__uint_as_float(v[h][2 * i]), __uint_as_float(v[h][2 * i + 1]));
+                                    w[i] = pack_bf16x2_rn(__uint_as_float(v[h][2 * i]) * kDescale,
+                                                          __uint_as_float(v[h][2 * i + 1]) * kDescale);
                                 dst[2 * h] = make_uint4(w[0], w[1], w[2], w[3]);
                                 dst[2 * h + 1] = make_uint4(w[4], w[5], w[6], w[7]);
                             }
@@ -755,7 +854,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int4 td = nxt;
                 if (tile + step < n_tiles) nxt = __ldg(g.tiles + tile + step);
                 const int w0 = td.z, slot_id = td.w;
-                for (int c = 0; c < R / kSpr; ++c, ++cst) {
+                for (int c = 0; c < K / 128; ++c, ++cst) {
                     if (cst >= kCodeSlots && !mbar_wait_sleep(&empty_c[slot], ph ^ 1u, g.err)) {
                         ok = false;
                         break;
@@ -802,7 +901,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         if (++lb == kWBufs) { lb = 0; lph ^= 1u; }
                     }
                     mbar_arrive_expect_tx(&ready[b], bytes);
-                    tma_load_2d(smem_u32(r_ring + rb * kRRoundBytes), m, rr * kRound, row0, &ready[b], pol);
+                    tma_load_2d(smem_u32(r_ring + rb * kRRoundBytes), m, rr * kKR, row0, &ready[b], pol);
                     issued = gr + 1;
                     if (++rb == kRBufs) rb = 0;
                     if (++b == kWBufs) { b = 0; ph ^= 1u; }
@@ -840,8 +939,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint32_t nph = wb + 1 == kWBufs ? wph ^ 1u : wph;
                     pre = mbar_try_wait(&ready[nb], nph);
 #pragma unroll
-                    for (int kk = 0; kk < kRound / 16; ++kk)     // descriptor start addresses in 16-byte units
-                        mma_ss(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (rr > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk)     // 32 bytes of K per MMA: descriptor start in 16-byte units
+                        mma_ss<F8>(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (rr > 0 || kk > 0) ? 1u : 0u);
                     issued = true;
                     mma_commit(&done[wb]);               // frees the round's weight and row buffers
                     wb = nb;
@@ -881,15 +980,17 @@ bool byte_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t row
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The row operand: fp16 [rows][K] with boxes of 64 x box_rows, 128B swizzle.
-bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+// The row operand: fp16 [rows][K] with boxes of 64 x box_rows, or e4m3 bytes
+// [rows][K] with boxes of 128 x box_rows (F8); 128B swizzle.
+bool row_map(CUtensorMap* m, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows, bool f8) {
     EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[2] = {K, rows};
-    const cuuint64_t strides[1] = {K * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)kRound, box_rows};
+    const cuuint64_t strides[1] = {K * (f8 ? 1 : 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)(f8 ? 128 : kRound), box_rows};
     const cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+    return fn(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims,
+              strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -899,8 +1000,8 @@ CUtensorMapSwizzle swizzle_for(uint32_t pitch) {
                         : pitch == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : pitch == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
 }
 
-template <int FMT, int MODE>
-moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, uint64_t src_rows, int max_tiles,
+template <int FMT, int MODE, bool F8>
+moe_status launch_gemm(const PoolView& P, GemmParams prm, const void* src, uint64_t src_rows, int max_tiles,
                        cudaStream_t s) {
     using Fm = GemmFmt<FMT>;
     const int D = P.D, F = P.F;
@@ -909,9 +1010,8 @@ moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, u
     const uint64_t code_row = (uint64_t)Kg / 32 * Fm::kCb;
     const uint8_t* codes = P.codes + (MODE == 1 ? 0 : 2 * (uint64_t)F * ((uint64_t)D / 32 * Fm::kCb));
     CUtensorMap mc, ms, mr;
-    const int R = Kg / kRound;
     const uint32_t cp = (uint32_t)(kSpr * 2 * Fm::kCb), sp = (uint32_t)(kSpr * 8);
-    if ((uint64_t)kTileW * (cp + (Fm::kTmaScales ? sp : 0u)) > kCodeSlotBytes || R % kSpr) return MOE_ERR_UNSUPPORTED;
+    if ((uint64_t)kTileW * (cp + (Fm::kTmaScales ? sp : 0u)) > kCodeSlotBytes || Kg % 128) return MOE_ERR_UNSUPPORTED;
     // code (and scale) stages: two boxes of 128 weight rows
     if (!byte_map(&mc, codes, code_row, rows, (uint64_t)P.n_slots, P.stride_c, cp, 128, swizzle_for(cp)))
         return MOE_ERR_CUDA;
@@ -924,23 +1024,23 @@ moe_status launch_gemm(const PoolView& P, GemmParams prm, const uint16_t* src, u
         ms = mc;
     }
     CUtensorMap r64, r32, r16;
-    if (!row_map(&mr, src, (uint64_t)Kg, src_rows, 128) || !row_map(&r64, src, (uint64_t)Kg, src_rows, 64) ||
-        !row_map(&r32, src, (uint64_t)Kg, src_rows, 32) || !row_map(&r16, src, (uint64_t)Kg, src_rows, 16))
+    if (!row_map(&mr, src, (uint64_t)Kg, src_rows, 128, F8) || !row_map(&r64, src, (uint64_t)Kg, src_rows, 64, F8) ||
+        !row_map(&r32, src, (uint64_t)Kg, src_rows, 32, F8) || !row_map(&r16, src, (uint64_t)Kg, src_rows, 16, F8))
         return MOE_ERR_CUDA;
     const size_t smem = kGemmSmem + 1024;
     static std::atomic<uint64_t> attr{0};
     if (!once_per_device(attr, [&] {
-            return cudaFuncSetAttribute(expert_gemm_kernel<FMT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            return cudaFuncSetAttribute(expert_gemm_kernel<FMT, MODE, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)smem) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
     const int grid = max_tiles < device_sm_count() ? (max_tiles > 0 ? max_tiles : 1) : device_sm_count();
-    const cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, MODE>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms,
+    const cudaError_t e = launch_pdl(expert_gemm_kernel<FMT, MODE, F8>, dim3(grid), dim3(kGemmThreads), smem, s, mc, ms,
                                      mr, r64, r32, r16, prm);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int FMT>
+template <int FMT, bool F8>
 moe_status launch_gemms(const PoolView& P, const PrefillWs& w, uint16_t* yrows, const WsSizes& sz, int T, int k,
                         cudaStream_t s) {
     GemmParams a1;
@@ -948,11 +1048,11 @@ moe_status launch_gemms(const PoolView& P, const PrefillWs& w, uint16_t* yrows, 
     a1.scales = P.scales; a1.stride_s = P.stride_s; a1.D = P.D; a1.F = P.F; a1.err = w.err;
     a1.dump = nullptr; a1.dump_tile = -1;
     const uint64_t rows = (uint64_t)T * (k + 1);
-    moe_status st = launch_gemm<FMT, 1>(P, a1, w.xg, rows, (int)sz.max_t1, s);
+    moe_status st = launch_gemm<FMT, 1, F8>(P, a1, w.xg, rows, (int)sz.max_t1, s);
     if (st != MOE_OK) return st;
     GemmParams a2 = a1;
     a2.tiles = w.tiles2; a2.n_tiles = w.meta + 2; a2.dst = yrows;
-    return launch_gemm<FMT, 2>(P, a2, w.h, rows, (int)sz.max_t2, s);
+    return launch_gemm<FMT, 2, F8>(P, a2, w.h, rows, (int)sz.max_t2, s);
 }
 
 template <int FMT>
@@ -977,7 +1077,7 @@ moe_status launch_operand_dump(const PoolView& P, int gemm, int slot, int m0, ui
     a.scales = P.scales; a.stride_s = P.stride_s; a.D = P.D; a.F = P.F;
     a.err = reinterpret_cast<uint32_t*>(p + 4);
     a.dump = dump; a.dump_tile = 0;
-    return gemm == 1 ? launch_gemm<FMT, 1>(P, a, src, 128, 1, s) : launch_gemm<FMT, 2>(P, a, src, 128, 1, s);
+    return gemm == 1 ? launch_gemm<FMT, 1, false>(P, a, src, 128, 1, s) : launch_gemm<FMT, 2, false>(P, a, src, 128, 1, s);
 }
 
 }  // namespace
@@ -999,7 +1099,7 @@ size_t prefill_workspace_bytes(int T, int D, int F, int E, int k) { return ws_si
 
 moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
                                   const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
-                                  int32_t* miss_count, void* ws, cudaStream_t s) {
+                                  int32_t* miss_count, void* ws, cudaStream_t s, bool fp8) {
     if (P.F % kKAlign || P.D % kDownRows || E > kMaxE) return MOE_ERR_UNSUPPORTED;
     if (!encode_tiled()) return MOE_ERR_CUDA;
     const PrefillWs w = carve(ws, T, P.D, P.F, E, k);
@@ -1017,15 +1117,24 @@ moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, 
     e = launch_pdl(plan_scatter_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const size_t gblocks = ((size_t)T * (k + 1) * (P.D / 16) + 255) / 256;
-    e = launch_pdl(gather_f16p_kernel, dim3((unsigned)(gblocks < 2368 ? gblocks : 2368)), dim3(256), 0, s, x, w.perm,
-                   w.meta, T, P.D, w.xg, w.err);
+    const dim3 ggrid((unsigned)(gblocks < 2368 ? gblocks : 2368));
+    e = fp8 ? launch_pdl(gather_f8p_kernel, ggrid, dim3(256), 0, s, x, w.perm, w.meta, T, P.D,
+                         reinterpret_cast<uint8_t*>(w.xg), w.err)
+            : launch_pdl(gather_f16p_kernel, ggrid, dim3(256), 0, s, x, w.perm, w.meta, T, P.D, w.xg, w.err);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const WsSizes sz = ws_sizes(T, P.D, P.F, E, k);
     uint16_t* yrows = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T, k));
+    if (fp8) {
+        switch (P.fmt) {
+            case MOE_Q2_32: return launch_gemms<MOE_Q2_32, true>(P, w, yrows, sz, T, k, s);
+            case MOE_Q3_32: return launch_gemms<MOE_Q3_32, true>(P, w, yrows, sz, T, k, s);
+            default: return launch_gemms<MOE_Q3_S256, true>(P, w, yrows, sz, T, k, s);
+        }
+    }
     switch (P.fmt) {
-        case MOE_Q2_32: return launch_gemms<MOE_Q2_32>(P, w, yrows, sz, T, k, s);
-        case MOE_Q3_32: return launch_gemms<MOE_Q3_32>(P, w, yrows, sz, T, k, s);
-        default: return launch_gemms<MOE_Q3_S256>(P, w, yrows, sz, T, k, s);
+        case MOE_Q2_32: return launch_gemms<MOE_Q2_32, false>(P, w, yrows, sz, T, k, s);
+        case MOE_Q3_32: return launch_gemms<MOE_Q3_32, false>(P, w, yrows, sz, T, k, s);
+        default: return launch_gemms<MOE_Q3_S256, false>(P, w, yrows, sz, T, k, s);
     }
 }
 

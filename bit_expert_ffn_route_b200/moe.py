@@ -27,7 +27,8 @@ EXPORTS = ["moe_slot_code_bytes", "moe_slot_scale_bytes", "moe_route_workspace_s
            "moe_expert_out_size", "moe_route_topk", "moe_expert_forward", "moe_combine", "moe_dequantize",
            "moe_status_string", "moe_route_topk_static", "moe_expert_hist", "moe_cache_plan", "moe_slot_fill",
            "moe_workspace_status", "moe_debug_wait_flag", "moe_debug_operand_workspace_size",
-           "moe_debug_prefill_operand", "moe_layer_workspace_size", "moe_layer_forward"]
+           "moe_debug_prefill_operand", "moe_layer_workspace_size", "moe_layer_forward",
+           "moe_workspace_size_fp8", "moe_expert_forward_fp8"]
 
 
 class MoeError(RuntimeError):
@@ -67,6 +68,10 @@ def lib():
         L.moe_route_topk.argtypes = [P, i, i, P, P, i, i, P, P, P, P, sz, P]
         L.moe_expert_forward.restype = i
         L.moe_expert_forward.argtypes = [ctypes.POINTER(moe_pool), P, i, P, i, P, i, P, sz, P, P, P, sz, P]
+        L.moe_expert_forward_fp8.restype = i
+        L.moe_expert_forward_fp8.argtypes = [ctypes.POINTER(moe_pool), P, i, P, i, P, i, P, sz, P, P, P, sz, P]
+        L.moe_workspace_size_fp8.restype = sz
+        L.moe_workspace_size_fp8.argtypes = [i, i, i, i, i, i]
         L.moe_combine.restype = i
         L.moe_combine.argtypes = [P, P, i, i, i, P, P, P, P]
         L.moe_dequantize.restype = i
@@ -172,6 +177,21 @@ def moe_expert_forward(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_l
     _check("moe_expert_forward", st)
 
 
+def moe_expert_forward_fp8(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_list, miss_count, ws,
+                           stream=None):
+    """The expert pass with e4m3 tensor-core operands (lossy; any T)."""
+    T = x.shape[0]
+    E = slot_table.shape[0]
+    st = lib().moe_expert_forward_fp8(ctypes.byref(pool), _p(slot_table), E, _p(x), T, _p(ids), k,
+                                      _p(expert_out), expert_out.numel(), _p(miss_list), _p(miss_count),
+                                      _p(ws), ws.numel(), _stream(stream))
+    _check("moe_expert_forward_fp8", st)
+
+
+def workspace_size_fp8(T, D, F, E, k, fmt):
+    return lib().moe_workspace_size_fp8(T, D, F, E, k, fmt)
+
+
 def moe_layer_forward(pool: moe_pool, slot_table, x, Wr, bias, k, ids, gates, expert_out, miss_list, miss_count,
                       out, ws, residual=None, stream=None):
     """The one-call layer (T <= 8): routing, expert pass and combine in one launch."""
@@ -272,6 +292,7 @@ class Layer:
         self.out = torch.empty(T, D, dtype=torch.bfloat16, device=device)
         n = layer_workspace_size(T, D, pool.d_ff, E, k, pool.fmt)
         self.layer_ws = alloc_ws(n, device) if n else None
+        self.ws_fp8 = None
 
     def fused(self, x, residual=None, out=None, stream=None):
         """The same layer through moe_layer_forward (T <= 8; no miss_partial)."""
@@ -283,12 +304,20 @@ class Layer:
                           stream=stream)
         return out
 
-    def __call__(self, x, miss_partial=None, residual=None, out=None, stream=None, with_logits=False):
+    def __call__(self, x, miss_partial=None, residual=None, out=None, stream=None, with_logits=False, fp8=False):
+        """The three calls; fp8=True takes moe_expert_forward_fp8 for the expert pass."""
         out = self.out if out is None else out
         moe_route_topk(x, self.Wr, self.bias, self.k, self.ids, self.gates, self.route_ws,
                        logits=self.logits if with_logits else None, stream=stream)
-        moe_expert_forward(self.pool, self.slot_table, x, self.ids, self.k, self.expert_out, self.miss_list,
-                           self.miss_count, self.ws, stream=stream)
+        if fp8:
+            if self.ws_fp8 is None:
+                self.ws_fp8 = alloc_ws(workspace_size_fp8(self.T, self.D, self.pool_data.d_ff, self.E, self.k,
+                                                          self.pool_data.fmt), x.device)
+            moe_expert_forward_fp8(self.pool, self.slot_table, x, self.ids, self.k, self.expert_out, self.miss_list,
+                                   self.miss_count, self.ws_fp8, stream=stream)
+        else:
+            moe_expert_forward(self.pool, self.slot_table, x, self.ids, self.k, self.expert_out, self.miss_list,
+                               self.miss_count, self.ws, stream=stream)
         moe_combine(self.expert_out, self.gates, x.shape[0], self.D, self.k, out, miss_partial=miss_partial,
                     residual=residual, stream=stream)
         return out

@@ -239,6 +239,29 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * The expert pass with e4m3 tensor-core operands (a lossy variant of
+ * moe_expert_forward's tensor-core path, T > 8; T <= 8 returns
+ * MOE_ERR_UNSUPPORTED and moe_workspace_size_fp8 returns 0 there, T = 0 only
+ * clears miss_count).  Same arguments, results and error word; ws of
+ * moe_workspace_size_fp8 bytes.
+ * Operands: each weight is the exact weight of its block format times 64,
+ * rounded once to fp16 and then to e4m3 (nearest even, saturating); x and h
+ * are rounded to e4m3 (nearest even, saturating; magnitude >= 448 sets bit 1
+ * of the error word); the products accumulate in fp32 and are scaled back by
+ * 1/64.  The e4m3 roundings bound the accuracy, not the 1e-2 of
+ * moe_expert_forward: on the 2,048-token synthetic workload the per-token
+ * relative L2 error to the exact-weight result measured median 6.6e-2, max
+ * 8.2e-2 (within 3e-3 of this variant's own definition).  Status as
+ * moe_expert_forward.
+ */
+size_t moe_workspace_size_fp8(int T, int D, int F, int E, int k, int fmt);
+moe_status moe_expert_forward_fp8(const moe_pool* pool, const int32_t* slot_table, int E,
+                                  const uint16_t* x, int T, const int32_t* ids, int k,
+                                  void* expert_out, size_t expert_out_bytes,
+                                  int32_t* miss_list, int32_t* miss_count,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * Gate-weighted combine:
  *   out[t] = bf16( sum_{r<k, hit} gates[t][r] * y[t][r] + y_shared[t]
  *                  (+ miss_partial[t]) (+ residual[t]) )

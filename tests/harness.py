@@ -44,9 +44,9 @@ def mini_pool(pool, slots, shared_slot):
     return hp, remap
 
 
-def oracle_layer(pool, layer, k, x_bits, miss_partial=None, residual_bits=None, n_threads=8):
+def oracle_layer(pool, layer, k, x_bits, miss_partial=None, residual_bits=None, n_threads=8, fp8=False):
     """The oracle's full expert pass for the tokens x_bits, reading only the
-    slots it needs from the generated pool."""
+    slots it needs from the generated pool (fp8: its e4m3-operand variant)."""
     Wr = u16(layer.Wr)
     bias = None if layer.bias is None else layer.bias.detach().float().cpu().numpy()
     table = layer.slot_table.detach().cpu().numpy().astype(np.int32)
@@ -59,4 +59,4 @@ def oracle_layer(pool, layer, k, x_bits, miss_partial=None, residual_bits=None, 
         if 0 <= s < pool.n_slots:
             mini_table[e] = remap[s]
     return oracle.moe_layer(hp, mini_table, k, x_bits, Wr, bias, miss_partial=miss_partial,
-                            residual=residual_bits, n_threads=n_threads)
+                            residual=residual_bits, n_threads=n_threads, fp8=fp8)
