@@ -172,68 +172,122 @@ __global__ void __launch_bounds__(kChunk) plan_count_kernel(PlanArgs a) {
 }
 
 // One CTA: expert offsets, per-chunk bases, miss bases and the two tile lists.
+// Exclusive prefix sum of v over the 1024 threads of the block; *total gets the
+// block's sum.  Every thread calls it.
+MOE_DEVINL int block_exscan1024(int v, int* total) {
+    __shared__ int wsum[32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int t = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        wsum[lane] = t;
+    }
+    __syncthreads();
+    const int r = (w > 0 ? wsum[w - 1] : 0) + x - v;
+    *total = wsum[31];
+    __syncthreads();                              // wsum is reused by the next call
+    return r;
+}
+
+// Largest g in [0, last] with off[g] <= i (off non-decreasing, off[0] = 0 <= i).
+MOE_DEVINL int group_of(const int* off, int last, int i) {
+    int lo = 0, hi = last;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// One block of 1024 threads: groups' totals, row offsets and tile offsets (block
+// scans over the E routed groups and the shared group E), the misses' chunk
+// offsets, every chunk's base row per expert, and the two tile lists (group, row
+// tile, then weight-row tile, the fastest index), one entry per thread in turn.
 __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
     __shared__ int tot[kMaxE];
     __shared__ int off[kMaxE + 1];
     __shared__ int t1off[kMaxE + 2];
     __shared__ int t2off[kMaxE + 2];
+    __shared__ int gslot[kMaxE + 1];
     pdl_wait();
     const int nchunk = (a.T + kChunk - 1) / kChunk;
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
+        if (e == a.E) { gslot[e] = a.shared_slot; continue; }
         int run = 0;
+#pragma unroll 4
         for (int c = 0; c < nchunk; ++c) run += a.w.hist[(size_t)c * a.E + e];
         tot[e] = run;
+        gslot[e] = plan_slot(a, e);
     }
     __syncthreads();
+    // groups 0..E-1 routed (rows tot[e]), group E the shared expert (T rows)
+    int c_rows = 0, c_t1 = 0, c_t2 = 0;
+    for (int base = 0; base <= a.E; base += 1024) {
+        const int g = base + (int)threadIdx.x;
+        const int n = g < a.E ? tot[g] : (g == a.E ? a.T : 0);
+        int s_rows, s_t1, s_t2;
+        const int x_rows = block_exscan1024(g < a.E ? n : 0, &s_rows);
+        const int x_t1 = block_exscan1024((n + kN1 - 1) / kN1, &s_t1);
+        const int x_t2 = block_exscan1024((n + kN2 - 1) / kN2, &s_t2);
+        if (g <= a.E) {
+            off[g] = c_rows + x_rows;
+            t1off[g] = c_t1 + x_t1;
+            t2off[g] = c_t2 + x_t2;
+        }
+        c_rows += s_rows;
+        c_t1 += s_t1;
+        c_t2 += s_t2;
+    }
     if (threadIdx.x == 0) {
-        int run = 0;
-        for (int e = 0; e < a.E; ++e) { off[e] = run; run += tot[e]; }
-        off[a.E] = run;
+        t1off[a.E + 1] = c_t1;
+        t2off[a.E + 1] = c_t2;
+        a.w.meta[0] = c_rows;
+        a.w.meta[1] = c_t1 * (a.F / kGateFeat);
+        a.w.meta[2] = c_t2 * (a.D / kDownRows);
         // misses: exclusive scan over chunks (token-major order)
         int m = 0;
         for (int c = 0; c < nchunk; ++c) { const int v = a.w.miss_hist[c]; a.w.miss_hist[c] = m; m += v; }
         a.miss_count[0] = m;
-        a.w.meta[0] = run;
-        // row tiles per group (routed groups in id order, then the shared group)
-        int n1 = 0, n2 = 0;
-        for (int e = 0; e <= a.E; ++e) {
-            t1off[e] = n1;
-            t2off[e] = n2;
-            const int n = e < a.E ? tot[e] : a.T;
-            n1 += (n + kN1 - 1) / kN1;
-            n2 += (n + kN2 - 1) / kN2;
-        }
-        t1off[a.E + 1] = n1;
-        t2off[a.E + 1] = n2;
-        a.w.meta[1] = n1 * (a.F / kGateFeat);
-        a.w.meta[2] = n2 * (a.D / kDownRows);
     }
     __syncthreads();
     // per-chunk base rows of every expert
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int run = off[e];
+#pragma unroll 4
         for (int c = 0; c < nchunk; ++c) {
             const int v = a.w.hist[(size_t)c * a.E + e];
             a.w.hist[(size_t)c * a.E + e] = run;
             run += v;
         }
     }
-    // tile lists: group, row tile, then weight-row tile (the fastest index)
+    // tile lists
     const int mt1 = a.F / kGateFeat, mt2 = a.D / kDownRows;
-    for (int g = threadIdx.x; g <= a.E; g += blockDim.x) {
+    const int n1 = c_t1 * mt1, n2 = c_t2 * mt2;
+    for (int i = threadIdx.x; i < n1 + n2; i += blockDim.x) {
+        const bool first_list = i < n1;
+        const int ii = first_list ? i : i - n1;
+        const int mt = first_list ? mt1 : mt2;
+        const int tile = ii / mt, m = ii % mt;
+        const int* toff = first_list ? t1off : t2off;
+        const int g = group_of(toff, a.E, tile);
         const int n = g < a.E ? tot[g] : a.T;
-        const int row0 = g < a.E ? off[g] : off[a.E];
-        const int slot = g < a.E ? (n > 0 ? plan_slot(a, g) : -1) : a.shared_slot;
-        for (int j = 0; j < t1off[g + 1] - t1off[g]; ++j) {
-            const int r0 = row0 + j * kN1, rows = min(kN1, n - j * kN1);
-            for (int m = 0; m < mt1; ++m)
-                a.w.tiles1[(size_t)(t1off[g] + j) * mt1 + m] = make_int4(r0, rows, m * kGateFeat, slot);
-        }
-        for (int j = 0; j < t2off[g + 1] - t2off[g]; ++j) {
-            const int r0 = row0 + j * kN2, rows = min(kN2, n - j * kN2);
-            for (int m = 0; m < mt2; ++m)
-                a.w.tiles2[(size_t)(t2off[g] + j) * mt2 + m] = make_int4(r0, rows, m * kDownRows, slot);
-        }
+        const int j = tile - toff[g];
+        const int nr = first_list ? kN1 : kN2;
+        const int4 td = make_int4(off[g] + j * nr, min(nr, n - j * nr), m * (first_list ? kGateFeat : kDownRows), gslot[g]);
+        if (first_list) a.w.tiles1[ii] = td;
+        else a.w.tiles2[ii] = td;
     }
 }
 
