@@ -4,7 +4,8 @@ all GPU memory through a fixed arena, or code that must not call cudaMalloc
 while a stream is being captured).  It keeps its scratch in a library-owned
 static device array instead of a caller-provided workspace.
 
-The test calls it through the C ABI twice in a row and checks each result
+The tests call it through the C ABI twice in a row (and captured in a CUDA
+graph, replayed) and check each result
 against the workspace-taking moe_route_topk on the same inputs: expert ids and
 logits identical, gates within the 1e-6 relative tolerance the other GPU tests
 use.  It also checks ragged shapes against the CPU oracle directly, and that
@@ -78,3 +79,43 @@ def test_static_router_ragged_shapes_match_oracle(T, E, k):
         assert np.array_equal(ids.cpu().numpy(), want_ids), call
         g = gates.double().cpu().numpy()
         assert np.all(np.abs(g - want_g) <= TOL_GATE * np.abs(want_g)), call
+
+
+def test_static_router_under_graph_capture():
+    """The use its header names: one call before any capture, then calls
+    captured in a CUDA graph (each issues its memset on the stream) and the
+    graph replayed; ids and logits identical to the workspace router."""
+    cfg = configs.CONFIGS["decode"]
+    wl = configs.build(cfg, device="cuda", layers=1)
+    L = wl.layers[0]
+    T, E, D, k = cfg.T, cfg.E, cfg.D, cfg.k
+    xs = [synth.hidden(T, D, seed=cfg.seed, stream=700 + i, device="cuda") for i in range(2)]
+    ids = [torch.empty(T, k, dtype=torch.int32, device="cuda") for _ in range(2)]
+    gates = [torch.empty(T, k, dtype=torch.float32, device="cuda") for _ in range(2)]
+    logits = [torch.empty(T, E, dtype=torch.float32, device="cuda") for _ in range(2)]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        moe.moe_route_topk_static(xs[0], L.Wr, L.bias, k, ids[0], gates[0], stream=stream)   # before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(2):
+            moe.moe_route_topk_static(xs[i], L.Wr, L.bias, k, ids[i], gates[i], logits=logits[i], stream=stream)
+    ws = moe.alloc_ws(moe.route_workspace_size(T, D, E, k))
+    for rep in range(2):
+        for i in range(2):
+            ids[i].fill_(-5)
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        for i in range(2):
+            ids_a = torch.empty(T, k, dtype=torch.int32, device="cuda")
+            gates_a = torch.empty(T, k, dtype=torch.float32, device="cuda")
+            logits_a = torch.empty(T, E, dtype=torch.float32, device="cuda")
+            moe.moe_route_topk(xs[i], L.Wr, L.bias, k, ids_a, gates_a, ws, logits=logits_a)
+            torch.cuda.synchronize()
+            assert torch.equal(ids[i], ids_a), (rep, i)
+            assert torch.equal(logits[i].view(torch.int32), logits_a.view(torch.int32)), (rep, i)
+            ga = gates_a.double().cpu().numpy()
+            assert np.all(np.abs(gates[i].double().cpu().numpy() - ga) <= TOL_GATE * np.abs(ga)), (rep, i)
+    del g
