@@ -440,10 +440,11 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
 
 
 # ---------------------------------------------------------------- small verify batches
-def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 16, 64), K=64):
+def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 12, 16, 24, 25, 32, 64), K=64):
     """The decode layer's shapes at other batch sizes (MTP draft verification):
     per-step time and tokens/s of the three calls, and which expert-pass path
-    ran (decode: T <= 8, tensor-core GEMV; prefill: T > 8, grouped GEMMs)."""
+    ran (decode: T <= 24, tensor-core GEMV in launches of up to 8 tokens;
+    prefill: T > 24, grouped GEMMs)."""
     cfg = configs.CONFIGS["decode"]
     wl = configs.build(cfg, device=dev, T=max(Ts))
     L0 = wl.layers[0]
@@ -467,8 +468,8 @@ def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 16, 64), K=64)
             graph.replay()
         ms, _ = _timed_replays(graph, K // G, stream, ws_, dev, local, clocks=False)
         out[str(T)] = {"ms_per_step": round(ms / K, 5), "tokens_per_s": round(ws_ * T * K / (ms / 1e3), 1),
-                       "expert_pass": "decode" if T <= 8 else "prefill",
-                       "router": "canonical CUDA-core" if T <= 8 else "tensor-core + canonical recheck"}
+                       "expert_pass": (f"decode, {(T + 7) // 8} launches" if T > 8 else "decode") if T <= 24 else "prefill",
+                       "router": "canonical CUDA-core" if T <= 24 else "tensor-core + canonical recheck"}
         if layers[0].layer_ws is not None:
             g1 = _graph_of(lambda i: layers[i % R].fused(xs[i % R], stream=stream), G, stream)
             with torch.cuda.stream(stream):

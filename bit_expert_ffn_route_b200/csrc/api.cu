@@ -80,7 +80,7 @@ size_t moe_route_workspace_size(int T, int D, int E, int k) {
 
 size_t moe_workspace_size(int T, int D, int F, int E, int k, int fmt) {
     if (check_shapes(T, D, E, k) != MOE_OK || F <= 0 || !fmt_ok(fmt)) return 0;
-    if (T <= kDecodeMaxT) return decode_workspace_bytes(T, D, F, k);
+    if (T <= kDecodeLayoutMaxT) return decode_workspace_bytes(T < kDecodeMaxT ? T : kDecodeMaxT, D, F, k);
     return prefill_workspace_bytes(T, D, F, E, k);
 }
 
@@ -130,7 +130,7 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
     if (!aligned(x, 16) || !aligned(expert_out, 256) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
     if (expert_out_bytes_ < expert_out_bytes(T, v.D, k)) return MOE_ERR_WORKSPACE;
     if (ws_bytes < moe_workspace_size(T, v.D, v.F, E, k, v.fmt)) return MOE_ERR_WORKSPACE;
-    if (T <= kDecodeMaxT)
+    if (T <= kDecodeLayoutMaxT)
         return reported(launch_decode_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
                                               (cudaStream_t)stream));
     return reported(launch_prefill_forward(v, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count, ws,
@@ -138,7 +138,7 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
 }
 
 size_t moe_workspace_size_fp8(int T, int D, int F, int E, int k, int fmt) {
-    if (check_shapes(T, D, E, k) != MOE_OK || F <= 0 || !fmt_ok(fmt) || T <= kDecodeMaxT) return 0;
+    if (check_shapes(T, D, E, k) != MOE_OK || F <= 0 || !fmt_ok(fmt) || T <= kDecodeLayoutMaxT) return 0;
     return prefill_workspace_bytes(T, D, F, E, k);
 }
 
@@ -153,7 +153,7 @@ moe_status moe_expert_forward_fp8(const moe_pool* pool, const int32_t* slot_tabl
     if (st != MOE_OK) return st;
     if (!miss_count) return MOE_ERR_INVALID_ARG;
     if (T == 0) return cuda_status(cudaMemsetAsync(miss_count, 0, sizeof(int32_t), (cudaStream_t)stream));
-    if (T <= kDecodeMaxT) return MOE_ERR_UNSUPPORTED;    // moe_combine reads the small-batch layout there
+    if (T <= kDecodeLayoutMaxT) return MOE_ERR_UNSUPPORTED;    // moe_combine reads the small-batch layout there
     if (!slot_table || !x || !ids || !expert_out || !miss_list || !ws) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(expert_out, 256) || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
     if (expert_out_bytes_ < expert_out_bytes(T, v.D, k)) return MOE_ERR_WORKSPACE;

@@ -129,7 +129,7 @@ moe_status launch_combine(const void* expert_out, const float* gates, int T, int
     const int32_t* rowmap = reinterpret_cast<const int32_t*>(expert_out);
     const char* rows = reinterpret_cast<const char*>(expert_out) + rowmap_bytes(T, k);
     cudaError_t e;
-    if (T <= kDecodeMaxT) {
+    if (T <= kDecodeLayoutMaxT) {
         e = launch_pdl(combine_f32_kernel, dim3((D / 4 + 127) / 128, T), dim3(128), 0, s, rowmap,
                        reinterpret_cast<const float*>(rows), gates, T, D, k, miss_partial, residual, out);
     } else {

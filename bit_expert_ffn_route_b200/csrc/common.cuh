@@ -12,7 +12,8 @@
 namespace moe {
 
 constexpr int kMaxTopK = 16;
-constexpr int kDecodeMaxT = 8;        // T <= 8: decode expert pass (tensor-core GEMV over bulk-copied codes)
+constexpr int kDecodeMaxT = 8;        // tokens per launch of the decode expert pass (tensor-core GEMV over bulk-copied codes)
+constexpr int kDecodeLayoutMaxT = 24; // T <= 24: the decode expert pass (launches of up to 8 tokens) and its fp32 row layout
 // The router computes logits on CUDA cores in the canonical order for T <= 8
 // tokens when x (fp32) and four rows of Wr fit in its shared memory
 // ((4 T + 8) D bytes <= kRouteDecodeSmem); otherwise on the tensor cores, with

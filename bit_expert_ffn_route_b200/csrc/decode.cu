@@ -164,6 +164,8 @@ struct DecodeParams {
     float* yrows;          // [T*(k+1)][D]
     int32_t* miss_list;
     int32_t* miss_count;
+    int t0;                // the batch's first token in the caller's batch (rowmap, yrows: already offset)
+    int miss_append;       // 1: misses follow those already counted in miss_count (a batch's second launch)
     uint16_t* hfrag;       // [kMaxPairs][F * NSLOT] fp16, fragment order
     uint32_t* err;
     uint32_t* done;        // [kMaxPairs + 2]: per-owner gate|up completion counters, CTA ticket, work queue
@@ -271,22 +273,26 @@ __device__ void resolve_owners(const DecodeParams& prm, Shared& sh, int* first, 
         missb[h] = __ballot_sync(0xffffffffu, p < n && s[h] < 0);
     }
     if (book) {
-        int base = 0;
+        // row-map values and miss tokens are the caller's batch indices (t0 + t); a
+        // batch's second launch appends its misses after the first launch's
+        const int t0 = prm.t0;
+        int base = prm.miss_append ? *reinterpret_cast<volatile const int32_t*>(prm.miss_count) : 0;
 #pragma unroll
         for (int h = 0; h < H; ++h) {
             if (h >= hn) break;
             const int p = lane + 32 * h;
             if (p < n) {
                 const int t = tt[h], r = rr[h];
-                prm.rowmap[t * (k + 1) + r] = s[h] >= 0 ? t * (k + 1) + r : -1;
+                prm.rowmap[t * (k + 1) + r] = s[h] >= 0 ? (t0 + t) * (k + 1) + r : -1;
                 if (s[h] < 0) {
                     const int pos = base + __popc(missb[h] & below);
-                    prm.miss_list[3 * pos + 0] = t; prm.miss_list[3 * pos + 1] = r; prm.miss_list[3 * pos + 2] = e[h];
+                    prm.miss_list[3 * pos + 0] = t0 + t; prm.miss_list[3 * pos + 1] = r; prm.miss_list[3 * pos + 2] = e[h];
                 }
             }
             base += __popc(missb[h]);
         }
-        if (lane < T) prm.rowmap[lane * (k + 1) + k] = lane * (k + 1) + k;
+        if (lane < T) prm.rowmap[lane * (k + 1) + k] = (t0 + lane) * (k + 1) + k;
+        __syncwarp();                                 // every lane has read the count before lane 0 rewrites it
         if (lane == 0) prm.miss_count[0] = base;
     }
     __syncwarp();
@@ -1220,8 +1226,12 @@ size_t decode_workspace_bytes(int T, int D, int F, int k) {
 }
 
 namespace {
+// tokens [t0, t0 + T) of a batch of T_all tokens whose expert_out layout is
+// rowmap [T_all][k+1], then fp32 rows [T_all * (k+1)][D]
 DecodeParams expert_params(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
-                           const int32_t* ids, int k, void* expert_out, int32_t* miss_list, int32_t* miss_count) {
+                           const int32_t* ids, int k, void* expert_out, int32_t* miss_list, int32_t* miss_count,
+                           int T_all = 0, int t0 = 0) {
+    if (T_all == 0) T_all = T;
     DecodeParams prm{};
     prm.P = P;
     prm.slot_table = slot_table;
@@ -1230,10 +1240,13 @@ DecodeParams expert_params(const PoolView& P, const int32_t* slot_table, int E, 
     prm.T = T;
     prm.ids = ids;
     prm.k = k;
-    prm.rowmap = reinterpret_cast<int32_t*>(expert_out);
-    prm.yrows = reinterpret_cast<float*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T, k));
+    prm.rowmap = reinterpret_cast<int32_t*>(expert_out) + (size_t)t0 * (k + 1);
+    prm.yrows = reinterpret_cast<float*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T_all, k)) +
+                (size_t)t0 * (k + 1) * P.D;
     prm.miss_list = miss_list;
     prm.miss_count = miss_count;
+    prm.t0 = t0;
+    prm.miss_append = t0 > 0 ? 1 : 0;
     return prm;
 }
 
@@ -1262,12 +1275,20 @@ constexpr size_t kLayerLogits = 1024, kLayerH = 1024 + (size_t)kDecodeMaxT * 102
 moe_status launch_decode_forward(const PoolView& P, const int32_t* slot_table, int E, const uint16_t* x, int T,
                                  const int32_t* ids, int k, void* expert_out, int32_t* miss_list,
                                  int32_t* miss_count, void* ws, cudaStream_t s) {
-    if (P.D % kUnitK || P.F % kUnitK) return MOE_ERR_UNSUPPORTED;
-    DecodeParams prm = expert_params(P, slot_table, E, x, T, ids, k, expert_out, miss_list, miss_count);
-    prm.err = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
-    prm.done = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 64);
-    prm.hfrag = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 1024);
-    return launch_any<false>(prm, s);
+    if (P.D % kUnitK || P.F % kUnitK || T > kDecodeLayoutMaxT) return MOE_ERR_UNSUPPORTED;
+    // up to 8 tokens per launch, in token order (each later launch appends its misses
+    // and writes its rows after the earlier ones')
+    for (int t0 = 0; t0 < T; t0 += kDecodeMaxT) {
+        const int n = T - t0 < kDecodeMaxT ? T - t0 : kDecodeMaxT;
+        DecodeParams prm = expert_params(P, slot_table, E, x + (size_t)t0 * P.D, n, ids + (size_t)t0 * k, k,
+                                         expert_out, miss_list, miss_count, T, t0);
+        prm.err = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
+        prm.done = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 64);
+        prm.hfrag = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + 1024);
+        const moe_status st = launch_any<false>(prm, s);
+        if (st != MOE_OK) return st;
+    }
+    return MOE_OK;
 }
 
 size_t layer_workspace_bytes(int T, int D, int F, int E, int k) {

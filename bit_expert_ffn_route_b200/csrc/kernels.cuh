@@ -5,6 +5,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "common.cuh"
 #include "moe.h"
 
 namespace moe {
@@ -16,7 +17,7 @@ namespace moe {
 //                         prefill path bf16 [T*(k+1)][D], expert-ordered
 inline size_t rowmap_bytes(int T, int k) { return ((size_t)T * (k + 1) * 4 + 255) / 256 * 256; }
 inline size_t expert_out_bytes(int T, int D, int k) {
-    const size_t row = (T <= 8) ? 4 : 2;
+    const size_t row = (T <= kDecodeLayoutMaxT) ? 4 : 2;     // fp32 rows (decode path) or bf16 rows (prefill)
     return rowmap_bytes(T, k) + (size_t)T * (k + 1) * D * row;
 }
 

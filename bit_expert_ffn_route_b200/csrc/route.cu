@@ -74,9 +74,12 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
     uint32_t* rerr = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + 4);
     float* lg = logits ? logits : reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256);
     cudaError_t e;
-    if (T <= kRouteDecodeMaxT && (size_t)(4 * T + 8) * D <= kRouteDecodeSmem) {
+    // decode router: up to 8 tokens per launch, as many launches as the decode
+    // expert pass takes (each launch stages its tokens' x as fp32 and four router
+    // rows in shared memory)
+    const int tc = T < kRouteDecodeMaxT ? T : kRouteDecodeMaxT;
+    if (T <= kDecodeLayoutMaxT && (size_t)(4 * tc + 8) * D <= kRouteDecodeSmem) {
         const dim3 grid((E + 3) / 4), block(128);
-        const size_t smem = (size_t)T * D * sizeof(float) + (size_t)4 * D * sizeof(uint16_t);
         static std::atomic<uint64_t> attr{0};
         if (!once_per_device(attr, [] {
                 const int b = (int)kRouteDecodeSmem;
@@ -90,17 +93,26 @@ moe_status launch_route(const uint16_t* x, int T, int D, const uint16_t* Wr, con
                        cudaFuncSetAttribute(route_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, b) == cudaSuccess;
             }))
             return MOE_ERR_CUDA;
-        switch (T) {
-            case 1: e = launch_pdl(route_decode_kernel<1>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            case 2: e = launch_pdl(route_decode_kernel<2>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            case 3: e = launch_pdl(route_decode_kernel<3>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            case 4: e = launch_pdl(route_decode_kernel<4>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            case 5: e = launch_pdl(route_decode_kernel<5>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            case 6: e = launch_pdl(route_decode_kernel<6>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            case 7: e = launch_pdl(route_decode_kernel<7>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
-            default: e = launch_pdl(route_decode_kernel<8>, grid, block, smem, s, x, T, D, Wr, bias, E, k, lg, ids, gates, counter, rerr); break;
+        for (int t0 = 0; t0 < T; t0 += kRouteDecodeMaxT) {
+            const int n = T - t0 < kRouteDecodeMaxT ? T - t0 : kRouteDecodeMaxT;
+            const size_t smem = (size_t)n * D * sizeof(float) + (size_t)4 * D * sizeof(uint16_t);
+            const uint16_t* xc = x + (size_t)t0 * D;
+            float* lc = lg + (size_t)t0 * E;
+            int32_t* ic = ids + (size_t)t0 * k;
+            float* gc = gates + (size_t)t0 * k;
+            switch (n) {
+                case 1: e = launch_pdl(route_decode_kernel<1>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                case 2: e = launch_pdl(route_decode_kernel<2>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                case 3: e = launch_pdl(route_decode_kernel<3>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                case 4: e = launch_pdl(route_decode_kernel<4>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                case 5: e = launch_pdl(route_decode_kernel<5>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                case 6: e = launch_pdl(route_decode_kernel<6>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                case 7: e = launch_pdl(route_decode_kernel<7>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+                default: e = launch_pdl(route_decode_kernel<8>, grid, block, smem, s, xc, n, D, Wr, bias, E, k, lc, ic, gc, counter, rerr); break;
+            }
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
-        return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+        return MOE_OK;
     }
     // prefill: tensor-core logits, then canonical logits of each token's candidates
     float* wnorm = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256 +

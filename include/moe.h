@@ -38,11 +38,12 @@
  *    orders; two identical calls give identical bits.
  *  - T == 0 is valid and launches nothing (miss_count is still zeroed).
  *  - Paths: the expert pass (moe_expert_forward) runs its decode path for
- *    T <= 8 (one token + up to 7 MTP draft tokens) and its prefill path for
- *    T > 8; the router (moe_route_topk) runs its decode path (CUDA cores)
- *    for T <= 8 when (4 T + 8) D <= 196608 (every T <= 4; T = 8 up to
- *    D = 4864) and its prefill path (tensor cores) otherwise.  All paths
- *    compute the same function.
+ *    T <= 24 (one token + MTP draft tokens; up to 8 tokens per launch, in
+ *    token order) and its prefill path for T > 24.  The router
+ *    (moe_route_topk) runs its decode path (CUDA cores) for T <= 24, in
+ *    launches of n = min(T, 8) tokens, when (4 n + 8) D <= 196608 (every
+ *    T <= 4; 8 tokens per launch up to D = 4864), and its prefill path
+ *    (tensor cores) otherwise.  All paths compute the same function.
  *  - Kernels are launched with programmatic dependent launch: each may start
  *    while the previous kernel on the stream is finishing, and waits for it
  *    before reading the activations, ids, gates or expert_out it may have
@@ -121,8 +122,8 @@ typedef struct moe_pool {
  * Shape limits (MOE_ERR_UNSUPPORTED otherwise):
  *   D % 256 == 0, 256 <= D <= 8192;  F % 128 == 0, 128 <= F <= 4096 (Q3_S256:
  *   F % 256 == 0);  1 <= k <= 16;  k <= E <= 1024;  0 <= T <= 65536.
- *   The expert pass's decode path (T <= 8) also keeps x (8 D bytes; 16 D for
- *   T > 4), two copies of h (16 F bytes; 32 F for T > 4) and at least two
+ *   The expert pass's decode path (T <= 24) also keeps x (8 D bytes; 16 D for
+ *   more than 4 tokens in a launch), two copies of h (16 F bytes; 32 F for T > 4) and at least two
  *   pipeline stages of 16 weight rows in 220 KB of shared memory per SM; the
  *   largest shapes do not fit and return MOE_ERR_UNSUPPORTED from
  *   moe_expert_forward (every shape with D + F <= 4096 fits).
@@ -240,7 +241,7 @@ moe_status moe_expert_forward(const moe_pool* pool, const int32_t* slot_table, i
 
 /*
  * The expert pass with e4m3 tensor-core operands (a lossy variant of
- * moe_expert_forward's tensor-core path, T > 8; T <= 8 returns
+ * moe_expert_forward's tensor-core path, T > 24; 1 <= T <= 24 returns
  * MOE_ERR_UNSUPPORTED and moe_workspace_size_fp8 returns 0 there, T = 0 only
  * clears miss_count).  Same arguments, results and error word; ws of
  * moe_workspace_size_fp8 bytes.

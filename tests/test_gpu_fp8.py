@@ -77,17 +77,17 @@ def test_fp8_other_formats(fmt):
 
 
 def test_fp8_small_prefill_with_misses():
-    # decode-layer shapes with 320/512 resident, 12 tokens (the smallest batches the e4m3 entry takes)
-    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=12)
+    # decode-layer shapes with 320/512 resident, 25 tokens (the smallest batches the e4m3 entry takes)
+    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=25)
     layer, _, _, _ = _check(wl, wl.x)
     assert int(layer.miss_count.item()) > 0
 
 
 def test_fp8_rejects_small_batches():
-    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=8, layers=1)
+    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=24, layers=1)
     L = wl.layers[0]
-    assert moe.workspace_size_fp8(8, wl.cfg.D, wl.cfg.F, wl.cfg.E, wl.cfg.k, wl.cfg.fmt) == 0
-    lay = moe.Layer(wl.pool, L.shared_slot, L.slot_table, L.Wr, L.bias, wl.cfg.k, 8)
+    assert moe.workspace_size_fp8(24, wl.cfg.D, wl.cfg.F, wl.cfg.E, wl.cfg.k, wl.cfg.fmt) == 0
+    lay = moe.Layer(wl.pool, L.shared_slot, L.slot_table, L.Wr, L.bias, wl.cfg.k, 24)
     with pytest.raises(moe.MoeError) as e:
         moe.moe_expert_forward_fp8(lay.pool, L.slot_table, wl.x, lay.ids, wl.cfg.k, lay.expert_out, lay.miss_list,
                                    lay.miss_count, moe.alloc_ws(1 << 24))

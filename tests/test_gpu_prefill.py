@@ -1,4 +1,4 @@
-"""GPU parity of the prefill path (T > 8: permute + tcgen05 grouped GEMMs)
+"""GPU parity of the prefill path (T > 24: permute + tcgen05 grouped GEMMs)
 against the CPU oracle, through the C ABI.  Bars as for the decode path:
 routing ids and miss lists bit-exact; outputs within relative L2 1e-2 per token
 (fp16 tensor-core operands and bf16 y rows on this path, fp32 accumulation)."""
@@ -63,10 +63,10 @@ def test_prefill_decode_shapes_with_misses():
 
 
 def test_prefill_matches_decode_path():
-    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=12)
-    _, out12 = _run(wl, wl.x)
+    wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=32)
+    _, out32 = _run(wl, wl.x)
     _, out4 = _run(wl, wl.x[:4].contiguous())
-    err = rel_l2_per_token(u16(out12)[:4], u16(out4))
+    err = rel_l2_per_token(u16(out32)[:4], u16(out4))
     assert err.max() <= TOL_OUT, err
 
 

@@ -56,7 +56,7 @@ def _check_full(wl, L, x, k, residual=None):
     return layer, out, ref
 
 
-@pytest.mark.parametrize("T", [5, 8, 9])
+@pytest.mark.parametrize("T", [5, 8, 9, 24, 25])
 def test_crossover_batches_and_decode_rows(T):
     wl = configs.build(configs.CONFIGS["decode"], device="cuda", T=T, layers=1)
     L = wl.layers[0]

@@ -39,7 +39,7 @@ def _bias(kind, E, rng):
 
 CASES = [(kind, T, E, k)
          for kind in ("hot_lanes", "all_equal", "ties_stride7", "quarter_steps", "random")
-         for T in (4, 8, 64)
+         for T in (4, 8, 12, 64)
          for (E, k) in ((512, 10), (80, 16), (1024, 8))]
 
 
