@@ -45,6 +45,7 @@ namespace moe {
 namespace {
 
 constexpr int kChunk = 256;            // tokens per plan chunk
+constexpr int kGatherThreads = 64;     // threads per row of the x gather (D / 16 groups of 16 elements)
 constexpr int kMaxE = 1024;
 constexpr int kN1 = 128;               // max rows per gate|up tile
 constexpr int kN2 = 128;               // max rows per down tile
@@ -343,16 +344,19 @@ MOE_DEVINL uint32_t bf16_half(uint32_t w, int hi) { return hi ? (w & 0xffff0000u
 
 // xg[row] = x[perm[row]] in fp16 and K order: one thread per 16-element group,
 // out word i = (x[i], x[i + 8]).  Rows: the routed rows, then the T shared rows.
-__global__ void __launch_bounds__(256) gather_f16p_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
-                                                          const int32_t* __restrict__ meta, int T, int D,
-                                                          uint16_t* __restrict__ xg, uint32_t* err) {
+__global__ void __launch_bounds__(kGatherThreads) gather_f16p_kernel(const uint16_t* __restrict__ x,
+                                                                      const int32_t* __restrict__ perm,
+                                                                      const int32_t* __restrict__ meta, int T, int D,
+                                                                      uint16_t* __restrict__ xg, uint32_t* err) {
+    // one block per row (rows past the routed groups + the shared group return)
     pdl_wait();
-    const int row_groups = D / 16;
-    const size_t ngroups = (size_t)(__ldg(meta) + T) * row_groups;
+    const int row = blockIdx.x;
+    if (row >= __ldg(meta) + T) return;
+    const uint16_t* xr = x + (size_t)__ldg(perm + row) * D;
+    uint16_t* dr = xg + (size_t)row * D;
     bool bad = false;
-    for (size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x; gi < ngroups; gi += (size_t)gridDim.x * blockDim.x) {
-        const size_t row = gi / row_groups, gc = gi % row_groups;
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)__ldg(perm + row) * D + gc * 16);
+    for (int gc = threadIdx.x; gc < D / 16; gc += kGatherThreads) {
+        const uint4* src = reinterpret_cast<const uint4*>(xr + gc * 16);
         const uint4 a = __ldg(src), b = __ldg(src + 1);
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
         uint32_t o[8];
@@ -363,7 +367,7 @@ __global__ void __launch_bounds__(256) gather_f16p_kernel(const uint16_t* __rest
             bad |= !(fabsf(lo) < 65520.f) || !(fabsf(hi) < 65520.f);
             o[i] = pack_f16x2(lo, hi);
         }
-        uint4* dst = reinterpret_cast<uint4*>(xg + row * D + gc * 16);
+        uint4* dst = reinterpret_cast<uint4*>(dr + gc * 16);
         dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
         dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
@@ -387,16 +391,18 @@ MOE_DEVINL uint32_t e4m3x2_of_f32(float lo, float hi) {
 // The e4m3 variant: x rows in group order as e4m3 bytes, K-permuted the same way
 // (bytes 2i, 2i + 1 of a 16-group = elements i, i + 8), rounded to nearest even
 // and saturated; |x| >= 448 sets the range bit.
-__global__ void __launch_bounds__(256) gather_f8p_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
-                                                         const int32_t* __restrict__ meta, int T, int D,
-                                                         uint8_t* __restrict__ xg, uint32_t* err) {
+__global__ void __launch_bounds__(kGatherThreads) gather_f8p_kernel(const uint16_t* __restrict__ x,
+                                                                     const int32_t* __restrict__ perm,
+                                                                     const int32_t* __restrict__ meta, int T, int D,
+                                                                     uint8_t* __restrict__ xg, uint32_t* err) {
     pdl_wait();
-    const int row_groups = D / 16;
-    const size_t ngroups = (size_t)(__ldg(meta) + T) * row_groups;
+    const int row = blockIdx.x;
+    if (row >= __ldg(meta) + T) return;
+    const uint16_t* xr = x + (size_t)__ldg(perm + row) * D;
+    uint8_t* dr = xg + (size_t)row * D;
     bool bad = false;
-    for (size_t gi = (size_t)blockIdx.x * blockDim.x + threadIdx.x; gi < ngroups; gi += (size_t)gridDim.x * blockDim.x) {
-        const size_t row = gi / row_groups, gc = gi % row_groups;
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)__ldg(perm + row) * D + gc * 16);
+    for (int gc = threadIdx.x; gc < D / 16; gc += kGatherThreads) {
+        const uint4* src = reinterpret_cast<const uint4*>(xr + gc * 16);
         const uint4 a = __ldg(src), b = __ldg(src + 1);
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
         uint32_t o[4] = {0, 0, 0, 0};
@@ -407,7 +413,7 @@ __global__ void __launch_bounds__(256) gather_f8p_kernel(const uint16_t* __restr
             bad |= !(fabsf(lo) < 448.f) || !(fabsf(hi) < 448.f);
             o[i >> 1] |= e4m3x2_of_f32(lo, hi) << (16 * (i & 1));
         }
-        *reinterpret_cast<uint4*>(xg + row * D + gc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(dr + gc * 16) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (bad) atomicOr(err, kErrRange);
 }
@@ -1170,11 +1176,10 @@ moe_status launch_prefill_forward(const PoolView& P, const int32_t* slot_table, 
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     e = launch_pdl(plan_scatter_kernel, dim3(nchunk), dim3(kChunk), 0, s, a);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    const size_t gblocks = ((size_t)T * (k + 1) * (P.D / 16) + 255) / 256;
-    const dim3 ggrid((unsigned)(gblocks < 2368 ? gblocks : 2368));
-    e = fp8 ? launch_pdl(gather_f8p_kernel, ggrid, dim3(256), 0, s, x, w.perm, w.meta, T, P.D,
+    const dim3 ggrid((unsigned)((size_t)T * (k + 1)));     // rows: at most T k routed + T shared
+    e = fp8 ? launch_pdl(gather_f8p_kernel, ggrid, dim3(kGatherThreads), 0, s, x, w.perm, w.meta, T, P.D,
                          reinterpret_cast<uint8_t*>(w.xg), w.err)
-            : launch_pdl(gather_f16p_kernel, ggrid, dim3(256), 0, s, x, w.perm, w.meta, T, P.D, w.xg, w.err);
+            : launch_pdl(gather_f16p_kernel, ggrid, dim3(kGatherThreads), 0, s, x, w.perm, w.meta, T, P.D, w.xg, w.err);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const WsSizes sz = ws_sizes(T, P.D, P.F, E, k);
     uint16_t* yrows = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(expert_out) + rowmap_bytes(T, k));
