@@ -133,16 +133,29 @@ __device__ __forceinline__ int plan_slot(const PlanArgs& a, int e) {
 
 // Per chunk of 256 tokens: a bitmask of the chunk's tokens for every expert
 // (bit t set when token t of the chunk selected the expert and it is resident).
-__device__ void chunk_masks(const PlanArgs& a, int chunk, uint32_t (*mask)[kChunk / 32], int& my_miss) {
+__device__ void chunk_masks(const PlanArgs& a, int chunk, uint32_t (*mask)[kChunk / 32], int& my_miss,
+                            int (&eid)[kMaxTopK], uint32_t& hit) {
     for (int i = threadIdx.x; i < a.E * (kChunk / 32); i += blockDim.x) mask[i / (kChunk / 32)][i % (kChunk / 32)] = 0;
-    __syncthreads();
     const int t = chunk * kChunk + threadIdx.x;
     my_miss = 0;
+    hit = 0;
+    // the token's ids, then their slots: all loads of one kind in flight together
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r) eid[r] = (t < a.T && r < a.k) ? __ldg(a.ids + (size_t)t * a.k + r) : -1;
+    int sl[kMaxTopK];
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r) sl[r] = r < a.k ? plan_slot(a, eid[r]) : -1;
+    __syncthreads();
     if (t < a.T) {
-        for (int r = 0; r < a.k; ++r) {
-            const int e = __ldg(a.ids + (size_t)t * a.k + r);
-            if (plan_slot(a, e) >= 0) atomicOr(&mask[e][threadIdx.x >> 5], 1u << (threadIdx.x & 31));
-            else ++my_miss;
+#pragma unroll
+        for (int r = 0; r < kMaxTopK; ++r) {
+            if (r >= a.k) break;
+            if (sl[r] >= 0) {
+                atomicOr(&mask[eid[r]][threadIdx.x >> 5], 1u << (threadIdx.x & 31));
+                hit |= 1u << r;
+            } else {
+                ++my_miss;
+            }
         }
     }
     __syncthreads();
@@ -153,7 +166,9 @@ __global__ void __launch_bounds__(kChunk) plan_count_kernel(PlanArgs a) {
     __shared__ int wsum[kChunk / 32];
     pdl_wait();
     int my_miss;
-    chunk_masks(a, blockIdx.x, mask, my_miss);
+    int eid[kMaxTopK];
+    uint32_t hit;
+    chunk_masks(a, blockIdx.x, mask, my_miss, eid, hit);
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int c = 0;
 #pragma unroll
@@ -299,7 +314,9 @@ __global__ void __launch_bounds__(kChunk) plan_scatter_kernel(PlanArgs a) {
     __shared__ int wsum[kChunk / 32];
     pdl_wait();
     int my_miss;
-    chunk_masks(a, blockIdx.x, mask, my_miss);
+    int eid[kMaxTopK];
+    uint32_t hit;
+    chunk_masks(a, blockIdx.x, mask, my_miss, eid, hit);
     // exclusive scan of misses over the chunk's threads
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int v = my_miss;
@@ -317,14 +334,20 @@ __global__ void __launch_bounds__(kChunk) plan_scatter_kernel(PlanArgs a) {
     if (t >= a.T) return;
     const int S = a.w.meta[0];
     const int k = a.k;
-    for (int r = 0; r < k; ++r) {
-        const int e = __ldg(a.ids + (size_t)t * k + r);
-        if (plan_slot(a, e) >= 0) {
+    // the chunk's base row of each hit expert: all loads in flight together
+    int hb[kMaxTopK];
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r) hb[r] = (hit >> r) & 1u ? a.w.hist[(size_t)blockIdx.x * a.E + eid[r]] : 0;
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r) {
+        if (r >= k) break;
+        const int e = eid[r];
+        if ((hit >> r) & 1u) {
             int below = 0;
             const int wi = threadIdx.x >> 5;
             for (int w = 0; w < wi; ++w) below += __popc(mask[e][w]);
             below += __popc(mask[e][wi] & ((1u << (threadIdx.x & 31)) - 1u));
-            const int row = a.w.hist[(size_t)blockIdx.x * a.E + e] + below;
+            const int row = hb[r] + below;
             a.w.perm[row] = t;
             a.rowmap[(size_t)t * (k + 1) + r] = row;
         } else {
