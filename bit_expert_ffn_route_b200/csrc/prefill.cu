@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
     for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
         if (e == a.E) { gslot[e] = a.shared_slot; continue; }
         int run = 0;
-#pragma unroll 4
+#pragma unroll 8
         for (int c = 0; c < nchunk; ++c) run += a.w.hist[(size_t)c * a.E + e];
         tot[e] = run;
         gslot[e] = plan_slot(a, e);
@@ -272,20 +272,34 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(PlanArgs a) {
         a.w.meta[0] = c_rows;
         a.w.meta[1] = c_t1 * (a.F / kGateFeat);
         a.w.meta[2] = c_t2 * (a.D / kDownRows);
-        // misses: exclusive scan over chunks (token-major order)
-        int m = 0;
-        for (int c = 0; c < nchunk; ++c) { const int v = a.w.miss_hist[c]; a.w.miss_hist[c] = m; m += v; }
-        a.miss_count[0] = m;
     }
+    // misses: exclusive scan over chunks (token-major order)
+    int c_miss = 0;
+    for (int base = 0; base < nchunk; base += 1024) {
+        const int c = base + (int)threadIdx.x;
+        int s_miss;
+        const int v = c < nchunk ? a.w.miss_hist[c] : 0;
+        const int x_miss = block_exscan1024(v, &s_miss);
+        if (c < nchunk) a.w.miss_hist[c] = c_miss + x_miss;
+        c_miss += s_miss;
+    }
+    if (threadIdx.x == 0) a.miss_count[0] = c_miss;
     __syncthreads();
-    // per-chunk base rows of every expert
+    // per-chunk base rows of every expert: eight chunks' counts loaded before their
+    // base rows are written back
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int run = off[e];
-#pragma unroll 4
-        for (int c = 0; c < nchunk; ++c) {
-            const int v = a.w.hist[(size_t)c * a.E + e];
-            a.w.hist[(size_t)c * a.E + e] = run;
-            run += v;
+        for (int c0 = 0; c0 < nchunk; c0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = c0 + i < nchunk ? a.w.hist[(size_t)(c0 + i) * a.E + e] : 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (c0 + i < nchunk) {
+                    a.w.hist[(size_t)(c0 + i) * a.E + e] = run;
+                    run += v[i];
+                }
+            }
         }
     }
     // tile lists
