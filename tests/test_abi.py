@@ -151,8 +151,10 @@ def test_operand_hook_argument_errors(L):
         ctypes.byref(pool), gemm, slot, m0, dump, ws, nb, None)
     assert op(gemm=3) == moe.MOE_ERR_INVALID_ARG
     assert op(slot=4) == moe.MOE_ERR_INVALID_ARG
-    assert op(m0=32) == moe.MOE_ERR_INVALID_ARG            # gate|up tiles start at multiples of 64
-    assert op(gemm=2, m0=64) == moe.MOE_ERR_INVALID_ARG    # down tiles start at multiples of 128
+    assert op(m0=32) == moe.MOE_ERR_INVALID_ARG            # gate|up tiles start at multiples of 128
+    assert op(m0=64) == moe.MOE_ERR_INVALID_ARG
+    assert op(gemm=2, m0=64) == moe.MOE_ERR_INVALID_ARG    # down tiles start at multiples of 256
+    assert op(gemm=2, m0=128) == moe.MOE_ERR_INVALID_ARG
     assert op(m0=512) == moe.MOE_ERR_INVALID_ARG           # beyond d_ff
     assert op(dump=None) == moe.MOE_ERR_INVALID_ARG
     assert op(nb=64) == moe.MOE_ERR_WORKSPACE
@@ -174,3 +176,25 @@ def test_layer_size_and_argument_errors(L):
     assert lf(_pool(), ws=16) == moe.MOE_ERR_WORKSPACE
     assert lf(_pool(), out=None) == moe.MOE_ERR_INVALID_ARG
     assert lf(_pool(), x=f, out=f) == moe.MOE_ERR_INVALID_ARG        # out may not alias x
+
+
+def test_small_batch_layout_and_fp8_entry(L):
+    """Batches of up to 24 tokens take the decode path (fp32 rows in expert_out,
+    a workspace for 8-token launches); the e4m3 entry takes only larger ones."""
+    D, F, E, k = 3072, 512, 512, 10
+    rowmap = lambda T: (T * (k + 1) * 4 + 255) // 256 * 256
+    assert L.moe_expert_out_size(24, D, k) == rowmap(24) + 24 * (k + 1) * D * 4
+    assert L.moe_expert_out_size(25, D, k) == rowmap(25) + 25 * (k + 1) * D * 2
+    assert L.moe_workspace_size(24, D, F, E, k, 0) == L.moe_workspace_size(8, D, F, E, k, 0)
+    assert L.moe_workspace_size(16, D, F, E, k, 0) == L.moe_workspace_size(8, D, F, E, k, 0)
+    assert L.moe_workspace_size(25, D, F, E, k, 0) > L.moe_workspace_size(24, D, F, E, k, 0)
+    assert L.moe_workspace_size_fp8(24, D, F, E, k, 0) == 0
+    assert L.moe_workspace_size_fp8(25, D, F, E, k, 0) == L.moe_workspace_size(25, D, F, E, k, 0)
+    f = _fake()
+    fw = lambda pool, T=32, eo=1 << 30, ws=1 << 30: L.moe_expert_forward_fp8(
+        ctypes.byref(pool), f, E, f, T, f, k, f, eo, f, f, f, ws, None)
+    assert fw(_pool(fmt=5)) == moe.MOE_ERR_INVALID_ARG
+    assert fw(_pool(), T=24) == moe.MOE_ERR_UNSUPPORTED
+    assert fw(_pool(), T=1) == moe.MOE_ERR_UNSUPPORTED
+    assert fw(_pool(), eo=16) == moe.MOE_ERR_WORKSPACE
+    assert fw(_pool(), ws=16) == moe.MOE_ERR_WORKSPACE
