@@ -189,9 +189,68 @@ __global__ void __launch_bounds__(256) wnorm_kernel(const uint16_t* __restrict__
 }
 
 constexpr int kSelWarps = 8;
+constexpr int kMaxRouterE = 1024;     // the largest expert count the selection takes
 
-// One warp per token: the k-th largest approximate logit, the candidates within
-// twice the margin, their canonical logits, then the exact top-k and gates.
+// Canonical logits (+ bias) of the n <= NC experts es[0..n) for one token
+// (bf16 row xrow): for each expert the order and arithmetic of
+// canon_logit_one, with the token row read and unpacked once for all of them
+// and the next 256-element chunk's router rows loaded while the current one is
+// summed.  Lane 0 stores expert es[j]'s logit into out[es[j]].
+template <int NC>
+__device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ xrow, int D,
+                                                   const uint16_t* __restrict__ Wr, const float* __restrict__ bias,
+                                                   const uint16_t* es, int n, float* out) {
+    const int lane = threadIdx.x & 31;
+    const uint16_t* wrow[NC];
+    float acc[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        wrow[j] = Wr + (size_t)es[j < n ? j : 0] * D + 8 * lane;
+        acc[j] = 0.0f;
+    }
+    const int nc = D >> 8;
+    uint4 wc[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) wc[j] = j < n ? ld_nc_u128(wrow[j]) : make_uint4(0, 0, 0, 0);
+    for (int c = 0; c < nc; ++c) {
+        uint4 wn[NC];
+#pragma unroll
+        for (int j = 0; j < NC; ++j)
+            wn[j] = (j < n && c + 1 < nc) ? ld_nc_u128(wrow[j] + 256 * (c + 1)) : make_uint4(0, 0, 0, 0);
+        const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow + 256 * c + 8 * lane);
+        const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+        float xf[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { xf[2 * q] = bf16lo(xv[q]); xf[2 * q + 1] = bf16hi(xv[q]); }
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            if (j < n) {
+                const uint32_t wv[4] = {wc[j].x, wc[j].y, wc[j].z, wc[j].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[j] = __fmaf_rn(xf[2 * q], bf16lo(wv[q]), acc[j]);
+                    acc[j] = __fmaf_rn(xf[2 * q + 1], bf16hi(wv[q]), acc[j]);
+                }
+            }
+            wc[j] = wn[j];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) acc[j] = __fadd_rn(acc[j], __shfl_xor_sync(0xffffffffu, acc[j], off));
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < NC; ++j)
+            if (j < n) out[es[j]] = bias ? __fadd_rn(acc[j], __ldg(bias + es[j])) : acc[j];
+    }
+}
+
+// One warp per token: the k-th largest approximate logit (by the warp top-k
+// on the approximate row), the candidates within twice the margin below it,
+// their canonical logits (four experts at a time), then the exact top-k and
+// gates over the canonical row (every other expert at -inf).
 __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uint16_t* __restrict__ x, int T, int D,
                                                                        const uint16_t* __restrict__ Wr,
                                                                        const float* __restrict__ bias, int E, int k,
@@ -199,7 +258,9 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
                                                                        const float* __restrict__ wn,
                                                                        int32_t* __restrict__ ids, float* __restrict__ gates,
                                                                        const uint32_t* err) {
-    extern __shared__ float rows[];          // [kSelWarps][E]
+    extern __shared__ float rows[];          // [kSelWarps][E] logits, then [kSelWarps][E] candidate ids (16-bit)
+    __shared__ int32_t s_kid[kSelWarps][kMaxTopK];
+    __shared__ float s_kg[kSelWarps][kMaxTopK];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kSelWarps + warp;
     pdl_wait();
@@ -209,8 +270,11 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
         return;
     }
     float* row = rows + (size_t)warp * E;
+    uint16_t* cl = reinterpret_cast<uint16_t*>(rows + (size_t)kSelWarps * E) + (size_t)warp * E;
     const float* ar = approx + (size_t)t * E;
     const uint16_t* xr = x + (size_t)t * D;
+    // the approximate row into shared memory (its loads in flight with the norms' below)
+    for (int e = lane; e < E; e += 32) row[e] = __ldg(ar + e);
     // |x_t|_2 and max_e |Wr_e|_2
     float sx = 0.f, wmax = 0.f;
     for (int i = 8 * lane; i < D; i += 256) {
@@ -229,44 +293,27 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
         wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, off));
     }
     const float margin2 = ldexpf(sqrtf(sx) * 1.0001f * wmax, -11);   // 2 M
-    // k-th largest approximate logit: k rounds of a warp max with removal
-    for (int e = lane; e < E; e += 32) row[e] = __ldg(ar + e);
     __syncwarp();
-    float kth = 0.f;
-    for (int r = 0; r < k; ++r) {
-        float best = -INFINITY;
-        int be = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            const float v = row[e];
-            if (v > best || (v == best && e < be)) { best = v; be = e; }
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (ov > best || (ov == best && oe < be)) { best = ov; be = oe; }
-        }
-        kth = best;
-        __syncwarp();
-        if (lane == 0 && be < E) row[be] = -INFINITY;
-        __syncwarp();
-    }
+    // k-th largest approximate logit: the expert the top-k of the approximate row ranks k-th
+    topk_row_warp(row, E, k, s_kid[warp], s_kg[warp]);
+    __syncwarp();
+    const int kid = s_kid[warp][k - 1];
+    const float kth = (unsigned)kid < (unsigned)E ? row[kid] : -INFINITY;
     const float thr = kth - margin2;
-    // candidates -> canonical logits; every other expert -> -inf
+    // candidates in ascending expert order
+    int n = 0;
     for (int base = 0; base < E; base += 32) {
         const int e = base + lane;
-        const bool cand = e < E && __ldg(ar + e) >= thr;
-        if (e < E) row[e] = -INFINITY;
-        uint32_t m = __ballot_sync(0xffffffffu, cand);
-        __syncwarp();
-        while (m) {
-            const int l = __ffs(m) - 1;
-            m &= m - 1;
-            const float v = canon_logit_one(xr, D, Wr, bias, base + l);
-            if (lane == 0) row[base + l] = v;
-        }
-        __syncwarp();
+        const bool cand = e < E && row[e] >= thr;
+        const uint32_t m = __ballot_sync(0xffffffffu, cand);
+        if (cand) cl[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)e;
+        n += __popc(m);
     }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) row[e] = -INFINITY;
+    __syncwarp();
+    for (int c0 = 0; c0 < n; c0 += 4) canon_logits_multi<4>(xr, D, Wr, bias, cl + c0, min(4, n - c0), row);
+    __syncwarp();
     topk_row_warp(row, E, k, ids + (size_t)t * k, gates + (size_t)t * k);
 }
 
@@ -296,7 +343,9 @@ moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t*
     static std::atomic<uint64_t> attr{0};
     if (!once_per_device(attr, [&] {
             return cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
-                   cudaSuccess;
+                       cudaSuccess &&
+                   cudaFuncSetAttribute(router_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)(kSelWarps * kMaxRouterE * (sizeof(float) + sizeof(uint16_t)))) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
     cudaError_t e = launch_pdl(wnorm_kernel, dim3((E + 7) / 8), dim3(256), 0, s, Wr, D, E, wnorm);
@@ -304,7 +353,7 @@ moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t*
     e = launch_pdl(router_tc_kernel, dim3((E + kRN - 1) / kRN, (T + kRM - 1) / kRM), dim3(kRThreads), smem, s, mx, mw,
                    bias, T, D, E, logits, err);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    const size_t sel_smem = (size_t)kSelWarps * E * sizeof(float);
+    const size_t sel_smem = (size_t)kSelWarps * E * (sizeof(float) + sizeof(uint16_t));
     e = launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), sel_smem, s, x,
                    T, D, Wr, bias, E, k, (const float*)logits, (const float*)wnorm, ids, gates, (const uint32_t*)err);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
