@@ -194,8 +194,8 @@ constexpr int kMaxRouterE = 1024;     // the largest expert count the selection 
 // Canonical logits (+ bias) of the n <= NC experts es[0..n) for one token
 // (bf16 row xrow): for each expert the order and arithmetic of
 // canon_logit_one, with the token row read and unpacked once for all of them
-// and the next 256-element chunk's router rows loaded while the current one is
-// summed.  Lane 0 stores expert es[j]'s logit into out[es[j]].
+// and the router rows of the next two 256-element chunks in flight while the
+// current one is summed.  Lane 0 stores expert es[j]'s logit into out[es[j]].
 template <int NC>
 __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ xrow, int D,
                                                    const uint16_t* __restrict__ Wr, const float* __restrict__ bias,
@@ -209,14 +209,16 @@ __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ 
         acc[j] = 0.0f;
     }
     const int nc = D >> 8;
-    uint4 wc[NC];
+    auto load = [&](uint4 (&w)[NC], int c) {
 #pragma unroll
-    for (int j = 0; j < NC; ++j) wc[j] = j < n ? ld_nc_u128(wrow[j]) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < NC; ++j) w[j] = (j < n && c < nc) ? ld_nc_u128(wrow[j] + 256 * c) : make_uint4(0, 0, 0, 0);
+    };
+    uint4 w0[NC], w1[NC];
+    load(w0, 0);
+    load(w1, 1);
     for (int c = 0; c < nc; ++c) {
-        uint4 wn[NC];
-#pragma unroll
-        for (int j = 0; j < NC; ++j)
-            wn[j] = (j < n && c + 1 < nc) ? ld_nc_u128(wrow[j] + 256 * (c + 1)) : make_uint4(0, 0, 0, 0);
+        uint4 w2[NC];
+        load(w2, c + 2);
         const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow + 256 * c + 8 * lane);
         const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
         float xf[8];
@@ -225,14 +227,15 @@ __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ 
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
             if (j < n) {
-                const uint32_t wv[4] = {wc[j].x, wc[j].y, wc[j].z, wc[j].w};
+                const uint32_t wv[4] = {w0[j].x, w0[j].y, w0[j].z, w0[j].w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     acc[j] = __fmaf_rn(xf[2 * q], bf16lo(wv[q]), acc[j]);
                     acc[j] = __fmaf_rn(xf[2 * q + 1], bf16hi(wv[q]), acc[j]);
                 }
             }
-            wc[j] = wn[j];
+            w0[j] = w1[j];
+            w1[j] = w2[j];
         }
     }
 #pragma unroll
@@ -247,10 +250,11 @@ __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ 
     }
 }
 
-// One warp per token: the k-th largest approximate logit (by the warp top-k
-// on the approximate row), the candidates within twice the margin below it,
-// their canonical logits (four experts at a time), then the exact top-k and
-// gates over the canonical row (every other expert at -inf).
+// One warp per token (E <= 32 NV): the k-th largest approximate logit (by the
+// warp top-k on the approximate row), the candidates within twice the margin
+// below it, their canonical logits (four experts at a time), then the exact
+// top-k and gates over the canonical row (every other expert at -inf).
+template <int NV>
 __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uint16_t* __restrict__ x, int T, int D,
                                                                        const uint16_t* __restrict__ Wr,
                                                                        const float* __restrict__ bias, int E, int k,
@@ -273,20 +277,41 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
     uint16_t* cl = reinterpret_cast<uint16_t*>(rows + (size_t)kSelWarps * E) + (size_t)warp * E;
     const float* ar = approx + (size_t)t * E;
     const uint16_t* xr = x + (size_t)t * D;
-    // the approximate row into shared memory (its loads in flight with the norms' below)
-    for (int e = lane; e < E; e += 32) row[e] = __ldg(ar + e);
-    // |x_t|_2 and max_e |Wr_e|_2
-    float sx = 0.f, wmax = 0.f;
-    for (int i = 8 * lane; i < D; i += 256) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + i));
-        const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+    // every load of the approximate row, the expert norms and the first 16
+    // chunks of x in flight together
+    float av[NV], wv[NV];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const float a = bf16lo(vv[h]), b = bf16hi(vv[h]);
-            sx = __fmaf_rn(a, a, __fmaf_rn(b, b, sx));
+    for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        av[i] = e < E ? __ldg(ar + e) : 0.f;
+        wv[i] = e < E ? __ldg(wn + e) : 0.f;
+    }
+    // |x_t|_2 (the same summation order as one chunk at a time) and max_e |Wr_e|_2
+    float sx = 0.f, wmax = 0.f;
+    constexpr int kXB = 8;
+    for (int c0 = 0; c0 < D / 256; c0 += kXB) {
+        uint4 v[kXB];
+#pragma unroll
+        for (int q = 0; q < kXB; ++q)
+            v[q] = c0 + q < D / 256 ? __ldg(reinterpret_cast<const uint4*>(xr + 256 * (c0 + q) + 8 * lane))
+                                    : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < kXB; ++q) {
+            if (c0 + q < D / 256) {
+                const uint32_t vv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float a = bf16lo(vv[h]), b = bf16hi(vv[h]);
+                    sx = __fmaf_rn(a, a, __fmaf_rn(b, b, sx));
+                }
+            }
         }
     }
-    for (int e = lane; e < E; e += 32) wmax = fmaxf(wmax, __ldg(wn + e));
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        if (lane + 32 * i < E) row[lane + 32 * i] = av[i];
+        wmax = fmaxf(wmax, wv[i]);
+    }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) {
         sx += __shfl_xor_sync(0xffffffffu, sx, off);
@@ -295,26 +320,27 @@ __global__ void __launch_bounds__(kSelWarps * 32) router_select_kernel(const uin
     const float margin2 = ldexpf(sqrtf(sx) * 1.0001f * wmax, -11);   // 2 M
     __syncwarp();
     // k-th largest approximate logit: the expert the top-k of the approximate row ranks k-th
-    topk_row_warp(row, E, k, s_kid[warp], s_kg[warp]);
+    topk_warp_n<NV, true>(row, E, k, s_kid[warp], s_kg[warp]);
     __syncwarp();
     const int kid = s_kid[warp][k - 1];
     const float kth = (unsigned)kid < (unsigned)E ? row[kid] : -INFINITY;
     const float thr = kth - margin2;
-    // candidates in ascending expert order
+    __syncwarp();                    // every lane has read row[kid] before the row is reset
+    // candidates in ascending expert order; the row is then reset to -inf
     int n = 0;
-    for (int base = 0; base < E; base += 32) {
-        const int e = base + lane;
-        const bool cand = e < E && row[e] >= thr;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        const bool cand = e < E && av[i] >= thr;
         const uint32_t m = __ballot_sync(0xffffffffu, cand);
         if (cand) cl[n + __popc(m & ((1u << lane) - 1u))] = (uint16_t)e;
         n += __popc(m);
+        if (e < E) row[e] = -INFINITY;
     }
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) row[e] = -INFINITY;
     __syncwarp();
     for (int c0 = 0; c0 < n; c0 += 4) canon_logits_multi<4>(xr, D, Wr, bias, cl + c0, min(4, n - c0), row);
     __syncwarp();
-    topk_row_warp(row, E, k, ids + (size_t)t * k, gates + (size_t)t * k);
+    topk_warp_n<NV, true>(row, E, k, ids + (size_t)t * k, gates + (size_t)t * k);
 }
 
 // bf16 [rows][D], boxes of 64 x 128 rows, 128B swizzle
@@ -344,7 +370,9 @@ moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t*
     if (!once_per_device(attr, [&] {
             return cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) ==
                        cudaSuccess &&
-                   cudaFuncSetAttribute(router_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                   cudaFuncSetAttribute(router_select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)(kSelWarps * 512 * (sizeof(float) + sizeof(uint16_t)))) == cudaSuccess &&
+                   cudaFuncSetAttribute(router_select_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)(kSelWarps * kMaxRouterE * (sizeof(float) + sizeof(uint16_t)))) == cudaSuccess;
         }))
         return MOE_ERR_CUDA;
@@ -354,7 +382,7 @@ moe_status launch_route_prefill(const uint16_t* x, int T, int D, const uint16_t*
                    bias, T, D, E, logits, err);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     const size_t sel_smem = (size_t)kSelWarps * E * (sizeof(float) + sizeof(uint16_t));
-    e = launch_pdl(router_select_kernel, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), sel_smem, s, x,
+    e = launch_pdl(E <= 512 ? router_select_kernel<16> : router_select_kernel<32>, dim3((T + kSelWarps - 1) / kSelWarps), dim3(kSelWarps * 32), sel_smem, s, x,
                    T, D, Wr, bias, E, k, (const float*)logits, (const float*)wnorm, ids, gates, (const uint32_t*)err);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
