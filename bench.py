@@ -1,6 +1,7 @@
 """Benchmark of the routed-MoE expert pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--only NAME] [--impl ours|reference]
+                    [--seed S]
 
 A step is one pass of the whole hot path — router logits + top-k + gates,
 slot lookup + miss list, expert FFNs, combine — over one batch of synthetic
@@ -13,17 +14,22 @@ per other workload, each measured the same way:
   prefill    one layer, 2,048 tokens, Q2_32, all resident, Zipf(0.8) loads
   decode48   48 chained layers, 1 token, Q3_32, 7,948 resident slots
   prefill48  48 chained layers, 4,096 tokens, Q3_S256, all 24,576 experts resident
+  decode_coder, prefill_coder
+             the decode and prefill workloads at the 256-expert Coder shape, all resident
 
 Timing: CUDA graphs of whole steps are replayed until exactly K steps ran;
 barrier + synchronize on both sides; CUDA events on the launching stream; max
 over ranks.  L2 (126 MB) is defeated by rotating over replicas of the expert
 pool, router weights and token batches for the one-layer workloads; the
 48-layer workloads read 19 GB / 50 GB of experts per step.  Per-kernel
-durations come from external event nodes inside the same graph.
+durations come from external event nodes inside the same graph; each roofline
+object also gives their p10 / p50 / p90.  --seed replaces every workload's
+seed (weights, router, tokens) to report other draws of the same recipe.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import gc
 import hashlib
 import json
@@ -46,11 +52,22 @@ METRIC = "MoE expert-pass tokens/s per layer"
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-EXTRA = ["prefill", "decode48", "prefill48"]
+EXTRA = ["prefill", "decode48", "prefill48", "decode_coder", "prefill_coder"]
 # kernels per layer and step: the one-call decode layer (T <= 8) 1; decode as
 # three calls: route 1, expert pass 1, combine 1; prefill route 3 (norms, tensor-core logits, selection), expert pass 6 (3
 # plan, gather, 2 GEMMs), combine 1
 LAUNCHES = {"layer": 1, "decode": 3, "prefill": 10}
+
+
+def _cfg(name, args):
+    """The workload's config, with --seed (when given) for every synthetic input."""
+    cfg = configs.CONFIGS[name]
+    return cfg if getattr(args, "seed", None) is None else dataclasses.replace(cfg, seed=args.seed)
+
+
+def _pct_us(ms):
+    """p10 / p50 / p90 of per-launch durations (ms) in microseconds."""
+    return [round(float(np.percentile(ms, q)) * 1e3, 3) for q in (10, 50, 90)]
 
 
 def _peaks():
@@ -257,7 +274,7 @@ def _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_
 
 # ---------------------------------------------------------------- one-layer workloads
 def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
-    cfg = configs.CONFIGS[name]
+    cfg = _cfg(name, args)
     T, D, F, E, k = cfg.T, cfg.D, cfg.F, cfg.E, cfg.k
     wl = configs.build(cfg, device=dev)
     L0 = wl.layers[0]
@@ -362,6 +379,7 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     else:
         roof = _roofline("tensor", float(np.mean([fwd_flops[i % R] for i in range(G)])), fwd_avg_ms, peaks, "prefill")
         roof["kernel"] = "moe_expert_forward (plan + gather + tcgen05 gate|up and down grouped GEMMs)"
+    roof["launch_us_p10_p50_p90"] = _pct_us(fwd_ms)
 
     # end to end through the public API: pinned host input -> device, the layer
     # call(s), device -> pinned host output, every step.  The copies run on a
@@ -445,7 +463,7 @@ def bench_small_batches(ws_, dev, local, args, Ts=(1, 4, 5, 8, 9, 12, 16, 24, 25
     per-step time and tokens/s of the three calls, and which expert-pass path
     ran (decode: T <= 24, tensor-core GEMV in launches of up to 8 tokens;
     prefill: T > 24, grouped GEMMs)."""
-    cfg = configs.CONFIGS["decode"]
+    cfg = _cfg("decode", args)
     wl = configs.build(cfg, device=dev, T=max(Ts))
     L0 = wl.layers[0]
     R = 8
@@ -532,7 +550,7 @@ class ChainBuffers:
 
 
 def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
-    cfg = configs.CONFIGS[name]
+    cfg = _cfg(name, args)
     T, D, F, E, k, NL = cfg.T, cfg.D, cfg.F, cfg.E, cfg.k, cfg.layers
     wl = configs.build(cfg, device=dev)
     buf = ChainBuffers(wl, dev)
@@ -580,6 +598,7 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
     else:
         roof = _roofline("tensor", float(np.sum(fwd_flops)) / NL, float(np.sum(fwd_ms)) / NL, peaks, "prefill48")
         roof["kernel"] = "moe_expert_forward (plan + gather + tcgen05 GEMMs), averaged over the 48 layers"
+    roof["launch_us_p10_p50_p90"] = _pct_us(fwd_ms)         # over the chain's layers
     # end to end: the first layer's input from pinned host memory, the last
     # layer's output back, every step
     xh = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
@@ -672,7 +691,7 @@ def run_reference(args, ws_, rank):
     cores."""
     if rank != 0:
         return
-    cfg = configs.CONFIGS["decode"]
+    cfg = _cfg("decode", args)
     wl = configs.build(cfg, device="cpu", T=1)
     from tests.harness import oracle_layer, u16
     ncores = os.cpu_count() or 1
@@ -701,7 +720,7 @@ def run_ours(args, ws_, rank, local):
     cpu = rank == 0 and ws_ == 1 and not args.no_cpu_baseline
     only = args.only
     head_name = only or "decode"
-    cfg = configs.CONFIGS[head_name]
+    cfg = _cfg(head_name, args)
     K, W = args.steps, args.warmup
     if cfg.layers == 1:
         head = bench_layer(head_name, K, W, ws_, dev, local, args, cpu)
@@ -729,11 +748,13 @@ def run_ours(args, ws_, rank, local):
         # the other workloads: fixed, small step counts (each is far above L2 or
         # rotates replicas); the decode chain at 48 layers x K steps
         plan = {"prefill": (max(8, min(K, 64)), 3), "decode48": (max(8, min(K, 64)), 3),
-                "prefill48": (3, 1)}
+                "prefill48": (3, 1), "decode_coder": (max(8, min(K, 64)), 3),
+                "prefill_coder": (max(8, min(K, 64)), 3)}
         for name in EXTRA:
             k_, w_ = plan[name]
             fn = bench_layer if configs.CONFIGS[name].layers == 1 else bench_chain
-            line[name] = fn(name, k_, max(w_, 1), ws_, dev, local, args, cpu)
+            # the Coder shape: no oracle timing of its own (the 512-expert lines carry it)
+            line[name] = fn(name, k_, max(w_, 1), ws_, dev, local, args, cpu and not name.endswith("_coder"))
             gc.collect()
             torch.cuda.empty_cache()
         line["small_batches"] = bench_small_batches(ws_, dev, local, args)
@@ -755,6 +776,8 @@ def main():
     ap.add_argument("--replicas", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=None,
+                    help="seed of every synthetic input (default: each workload's own, 0 except tiny)")
     args = ap.parse_args()
     ws_, rank, local = _dist()
     if args.impl == "reference":

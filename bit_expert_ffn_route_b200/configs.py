@@ -1,4 +1,4 @@
-"""The five synthetic workloads of the routed-MoE expert pass.
+"""The synthetic workloads of the routed-MoE expert pass.
 
 Model shapes follow the pages: 48 layers of 512 routed experts, 10 routed + 1
 shared expert per token (wiselychen RTX 5090 report, "30 秒定位"; greenbean-ai
@@ -16,6 +16,10 @@ shared expert per token (wiselychen RTX 5090 report, "30 秒定位"; greenbean-a
               (expert loads from 0 to ~1,450 tokens)
   prefill48   48 layers x 4,096 tokens, Q3_S256, all resident (~50 GB of experts),
               no bias (uniform routing), layer input = previous output + residual
+  decode_coder, prefill_coder
+              the "Coder" shape: 256 of the 512 routed experts kept per layer
+              (greenbean-ai §四, the Coder checkpoint), otherwise the decode and
+              prefill workloads' shapes, routing and bias; all 256 experts resident
 """
 from __future__ import annotations
 
@@ -63,7 +67,9 @@ CONFIGS = {
     "prefill48": Config("prefill48", 48, 3072, 512, 512, 10, 4096, synth.Q3_S256, None, None, None,
                         chained=True, weight_std=0.008),
 }
-ORDER = ["tiny", "decode", "decode48", "prefill", "prefill48"]
+CONFIGS["decode_coder"] = Config("decode_coder", 1, 3072, 512, 256, 10, 4, synth.Q2_32, None, 1.1, 0.47)
+CONFIGS["prefill_coder"] = Config("prefill_coder", 1, 3072, 512, 256, 10, 2048, synth.Q2_32, None, 0.8, 0.8)
+ORDER = ["tiny", "decode", "decode48", "prefill", "prefill48", "decode_coder", "prefill_coder"]
 
 
 @dataclass

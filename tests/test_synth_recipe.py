@@ -40,3 +40,16 @@ def test_prefill_loads_are_skewed():
     top = np.sort(load)[::-1]
     assert top[: cfg.E // 10].sum() > 0.5 * load.sum()    # a tenth of the experts take over half the rows
     assert np.allclose(gates.sum(axis=1), 1.0, atol=1e-12)
+
+
+def test_coder_shape_routes_over_256_experts():
+    """The Coder shape keeps 256 of the 512 routed experts: every id is below
+    256, and the 2,048-token chunk's loads stay skewed under the same bias."""
+    cfg = configs.CONFIGS["prefill_coder"]
+    assert cfg.E == 256 and configs.CONFIGS["decode_coder"].E == 256
+    ids, gates = _route(cfg, cfg.T)
+    assert ids.min() >= 0 and ids.max() < 256
+    assert all(len(set(row)) == cfg.k for row in ids.tolist())
+    load = np.bincount(ids.ravel(), minlength=cfg.E)
+    assert load.max() >= 200
+    assert np.allclose(gates.sum(axis=1), 1.0, atol=1e-12)
