@@ -80,8 +80,9 @@ def _peaks():
 
 
 def _traffic(kind):
-    """DRAM bytes per launch from the committed ncu capture of this kernel, or
-    None when the kernel's sources changed since the counters were taken."""
+    """DRAM bytes per launch from the committed ncu capture of this workload's
+    dominant launch (keyed by workload name), or None when there is none or the
+    kernel's sources changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -233,7 +234,7 @@ def _roofline(kind, per_launch, avg_ms, peaks, traffic_kind):
             "algorithmic_flops_per_launch": round(per_launch), "avg_launch_us": round(avg_ms * 1e3, 3)}
 
 
-def _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_flops, peaks):
+def _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_flops, peaks, traffic_key):
     """The same prefill steps with the e4m3-operand expert pass
     (moe_expert_forward_fp8): step time and the expert pass against the e4m3
     tensor peak (the measured bf16 peak x 2, the nominal dense ratio)."""
@@ -263,7 +264,7 @@ def _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_
     fwd8 = float(np.mean([ev[i][0].elapsed_time(ev[i][1]) for i in range(G)]))
     hbm, tf, tf_sus, kind = peaks
     roof8 = _roofline("tensor", float(np.mean([fwd_flops[i % R] for i in range(G)])), fwd8,
-                      (hbm, round(2 * tf, 1), round(2 * tf_sus, 1), kind), "prefill_fp8")
+                      (hbm, round(2 * tf, 1), round(2 * tf_sus, 1), kind), traffic_key)
     roof8["peak_kind"] = f"measured bf16 burst x 2 (e4m3 nominal dense ratio); sustained {round(2 * tf_sus, 1)}"
     roof8["kernel"] = "moe_expert_forward_fp8 (plan + e4m3 gather + tcgen05 kind::f8f6f4 grouped GEMMs)"
     del g8, g8e
@@ -370,14 +371,15 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
         three = {"ms_per_step": round(ms3 / K, 6), "value": round(ws_ * T * K / (ms3 / 1e3), 1),
                  "calls": "moe_route_topk + moe_expert_forward + moe_combine"}
         del g3
-        roof = _roofline("hbm", float(np.mean([step_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks, "decode")
+        roof = _roofline("hbm", float(np.mean([step_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks, name)
         roof["kernel"] = ("moe_layer_forward (decode_ffn_kernel, one-call layer: logits + top-k, gate|up and down "
                           "dequant-GEMV, combine); bytes = Wr + resident experts read + x + out")
     elif T <= 8:
-        roof = _roofline("hbm", float(np.mean([fwd_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks, "decode")
+        roof = _roofline("hbm", float(np.mean([fwd_bytes[i % R] for i in range(G)])), fwd_avg_ms, peaks,
+                         name + "_three_calls")
         roof["kernel"] = "moe_expert_forward (decode_ffn_kernel: gate|up + down dequant-GEMV)"
     else:
-        roof = _roofline("tensor", float(np.mean([fwd_flops[i % R] for i in range(G)])), fwd_avg_ms, peaks, "prefill")
+        roof = _roofline("tensor", float(np.mean([fwd_flops[i % R] for i in range(G)])), fwd_avg_ms, peaks, name)
         roof["kernel"] = "moe_expert_forward (plan + gather + tcgen05 gate|up and down grouped GEMMs)"
     roof["launch_us_p10_p50_p90"] = _pct_us(fwd_ms)
 
@@ -446,7 +448,8 @@ def bench_layer(name, K, W, ws_, dev, local, args, with_cpu):
     if three is not None:
         res["three_calls"] = three
     if T > 8:
-        res["fp8_variant"] = _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_flops, peaks)
+        res["fp8_variant"] = _fp8_variant(layers, xs, R, G, K, k, T, D, stream, ev, ws_, dev, local, fwd_flops, peaks,
+                                          name + "_fp8")
     if T > 8:
         loads = np.bincount(layers[0].ids.cpu().numpy().ravel(), minlength=E)
         res["expert_loads"] = {"max": int(loads.max()), "zero": int((loads == 0).sum()),
@@ -592,11 +595,11 @@ def bench_chain(name, K, W, ws_, dev, local, args, with_cpu):
     fwd_ms = [ev[l][0].elapsed_time(ev[l][1]) for l in range(NL)]
     peaks = _peaks()
     if T <= 8:
-        roof = _roofline("hbm", float(np.sum(fwd_bytes)) / NL, float(np.sum(fwd_ms)) / NL, peaks, "decode48")
+        roof = _roofline("hbm", float(np.sum(fwd_bytes)) / NL, float(np.sum(fwd_ms)) / NL, peaks, name)
         roof["kernel"] = ("moe_layer_forward (decode_ffn_kernel, one-call layer), averaged over the 48 layers; "
                           "bytes = Wr + resident experts read + x + out")
     else:
-        roof = _roofline("tensor", float(np.sum(fwd_flops)) / NL, float(np.sum(fwd_ms)) / NL, peaks, "prefill48")
+        roof = _roofline("tensor", float(np.sum(fwd_flops)) / NL, float(np.sum(fwd_ms)) / NL, peaks, name)
         roof["kernel"] = "moe_expert_forward (plan + gather + tcgen05 GEMMs), averaged over the 48 layers"
     roof["launch_us_p10_p50_p90"] = _pct_us(fwd_ms)         # over the chain's layers
     # end to end: the first layer's input from pinned host memory, the last
