@@ -1,7 +1,7 @@
 """Host-side helpers of bench.py (CPU only): the DRAM-traffic records are looked
 up by workload name and reported only while the kernels' sources are the
-captured ones; --seed replaces
-every workload's seed and nothing else; the per-launch percentiles."""
+captured ones; --seed replaces every workload's seed and nothing else; the
+per-launch percentiles."""
 import argparse
 import hashlib
 import json
