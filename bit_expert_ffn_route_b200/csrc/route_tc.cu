@@ -194,7 +194,7 @@ constexpr int kMaxRouterE = 1024;     // the largest expert count the selection 
 // Canonical logits (+ bias) of the n <= NC experts es[0..n) for one token
 // (bf16 row xrow): for each expert the order and arithmetic of
 // canon_logit_one, with the token row read and unpacked once for all of them
-// and the router rows of the next two 256-element chunks in flight while the
+// and the router rows of the next 256-element chunk in flight while the
 // current one is summed.  Lane 0 stores expert es[j]'s logit into out[es[j]].
 template <int NC>
 __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ xrow, int D,
@@ -213,12 +213,7 @@ __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ 
 #pragma unroll
         for (int j = 0; j < NC; ++j) w[j] = (j < n && c < nc) ? ld_nc_u128(wrow[j] + 256 * c) : make_uint4(0, 0, 0, 0);
     };
-    uint4 w0[NC], w1[NC];
-    load(w0, 0);
-    load(w1, 1);
-    for (int c = 0; c < nc; ++c) {
-        uint4 w2[NC];
-        load(w2, c + 2);
+    auto sum = [&](const uint4 (&w)[NC], int c) {
         const uint4 xv4 = *reinterpret_cast<const uint4*>(xrow + 256 * c + 8 * lane);
         const uint32_t xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
         float xf[8];
@@ -227,15 +222,26 @@ __device__ __forceinline__ void canon_logits_multi(const uint16_t* __restrict__ 
 #pragma unroll
         for (int j = 0; j < NC; ++j) {
             if (j < n) {
-                const uint32_t wv[4] = {w0[j].x, w0[j].y, w0[j].z, w0[j].w};
+                const uint32_t wv[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     acc[j] = __fmaf_rn(xf[2 * q], bf16lo(wv[q]), acc[j]);
                     acc[j] = __fmaf_rn(xf[2 * q + 1], bf16hi(wv[q]), acc[j]);
                 }
             }
-            w0[j] = w1[j];
-            w1[j] = w2[j];
+        }
+    };
+    // two buffers in turn: chunk c is summed while chunk c + 1 is in flight,
+    // then its buffer is refilled with chunk c + 2
+    uint4 wa[NC], wb[NC];
+    load(wa, 0);
+    load(wb, 1);
+    for (int c = 0; c < nc; c += 2) {
+        sum(wa, c);
+        load(wa, c + 2);
+        if (c + 1 < nc) {
+            sum(wb, c + 1);
+            load(wb, c + 3);
         }
     }
 #pragma unroll
