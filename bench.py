@@ -1,7 +1,7 @@
 """Benchmark of the routed-MoE expert pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--only NAME] [--impl ours|reference]
-                    [--seed S]
+                    [--seed S] [--nvtx]
 
 A step is one pass of the whole hot path — router logits + top-k + gates,
 slot lookup + miss list, expert FFNs, combine — over one batch of synthetic
@@ -24,11 +24,13 @@ pool, router weights and token batches for the one-layer workloads; the
 48-layer workloads read 19 GB / 50 GB of experts per step.  Per-kernel
 durations come from external event nodes inside the same graph; each roofline
 object also gives their p10 / p50 / p90.  --seed replaces every workload's
-seed (weights, router, tokens) to report other draws of the same recipe.
+seed (weights, router, tokens) to report other draws of the same recipe;
+--nvtx puts NVTX ranges around each workload and each timed region.
 """
 from __future__ import annotations
 
 import argparse
+import contextlib
 import dataclasses
 import gc
 import hashlib
@@ -190,12 +192,27 @@ def _barrier(ws_):
     torch.cuda.synchronize()
 
 
+NVTX = False            # --nvtx: host ranges around each workload and each timed region
+
+
+@contextlib.contextmanager
+def _nvtx(name):
+    """An NVTX range (for `ncu --nvtx --nvtx-include`) when --nvtx is given."""
+    if NVTX:
+        torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        if NVTX:
+            torch.cuda.nvtx.range_pop()
+
+
 def _timed_replays(graph, n, stream, ws_, dev, local, clocks=True):
     """Replay `graph` n times on `stream` between barriers; returns (max-over-ranks
     ms, clock summary)."""
     _barrier(ws_)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) if clocks else _NoClock() as clk, torch.cuda.stream(stream):
+    with ClockSampler(local) if clocks else _NoClock() as clk, torch.cuda.stream(stream), _nvtx("timed"):
         t0.record(stream)
         for _ in range(n):
             graph.replay()
@@ -725,10 +742,11 @@ def run_ours(args, ws_, rank, local):
     head_name = only or "decode"
     cfg = _cfg(head_name, args)
     K, W = args.steps, args.warmup
-    if cfg.layers == 1:
-        head = bench_layer(head_name, K, W, ws_, dev, local, args, cpu)
-    else:
-        head = bench_chain(head_name, K, W, ws_, dev, local, args, cpu)
+    with _nvtx(head_name):
+        if cfg.layers == 1:
+            head = bench_layer(head_name, K, W, ws_, dev, local, args, cpu)
+        else:
+            head = bench_chain(head_name, K, W, ws_, dev, local, args, cpu)
     gc.collect()
     torch.cuda.empty_cache()
     line = {
@@ -757,10 +775,12 @@ def run_ours(args, ws_, rank, local):
             k_, w_ = plan[name]
             fn = bench_layer if configs.CONFIGS[name].layers == 1 else bench_chain
             # the Coder shape: no oracle timing of its own (the 512-expert lines carry it)
-            line[name] = fn(name, k_, max(w_, 1), ws_, dev, local, args, cpu and not name.endswith("_coder"))
+            with _nvtx(name):
+                line[name] = fn(name, k_, max(w_, 1), ws_, dev, local, args, cpu and not name.endswith("_coder"))
             gc.collect()
             torch.cuda.empty_cache()
-        line["small_batches"] = bench_small_batches(ws_, dev, local, args)
+        with _nvtx("small_batches"):
+            line["small_batches"] = bench_small_batches(ws_, dev, local, args)
         gc.collect()
         torch.cuda.empty_cache()
     if rank == 0:
@@ -779,9 +799,13 @@ def main():
     ap.add_argument("--replicas", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="NVTX ranges around each workload and each timed region (ncu --nvtx-include)")
     ap.add_argument("--seed", type=int, default=None,
                     help="seed of every synthetic input (default: each workload's own, 0 except tiny)")
     args = ap.parse_args()
+    global NVTX
+    NVTX = args.nvtx
     ws_, rank, local = _dist()
     if args.impl == "reference":
         run_reference(args, ws_, rank)

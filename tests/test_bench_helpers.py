@@ -1,7 +1,7 @@
 """Host-side helpers of bench.py (CPU only): the DRAM-traffic records are looked
 up by workload name and reported only while the kernels' sources are the
 captured ones; --seed replaces every workload's seed and nothing else; the
-per-launch percentiles."""
+per-launch percentiles; --nvtx ranges, off unless asked for and balanced."""
 import argparse
 import hashlib
 import json
@@ -46,3 +46,25 @@ def test_seed_option_replaces_only_the_seed():
 def test_percentiles_in_microseconds():
     ms = np.linspace(0.010, 0.020, 101)           # 10 .. 20 us
     assert bench._pct_us(ms) == [11.0, 15.0, 19.0]
+
+
+def test_nvtx_ranges_are_opt_in_and_balanced():
+    calls = []
+    push, pop = bench.torch.cuda.nvtx.range_push, bench.torch.cuda.nvtx.range_pop
+    try:
+        bench.torch.cuda.nvtx.range_push = lambda name: calls.append(("push", name))
+        bench.torch.cuda.nvtx.range_pop = lambda: calls.append(("pop",))
+        with bench._nvtx("off"):
+            pass
+        assert calls == []
+        bench.NVTX = True
+        try:
+            with bench._nvtx("workload"):
+                with bench._nvtx("timed"):
+                    raise KeyError("inside")
+        except KeyError:
+            pass
+        assert calls == [("push", "workload"), ("push", "timed"), ("pop",), ("pop",)]
+    finally:
+        bench.NVTX = False
+        bench.torch.cuda.nvtx.range_push, bench.torch.cuda.nvtx.range_pop = push, pop
