@@ -179,7 +179,7 @@ def moe_expert_forward(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_l
 
 def moe_expert_forward_fp8(pool: moe_pool, slot_table, x, ids, k, expert_out, miss_list, miss_count, ws,
                            stream=None):
-    """The expert pass with e4m3 tensor-core operands (lossy; any T)."""
+    """The expert pass with e4m3 tensor-core operands (lossy; T > 24: smaller batches take the decode path)."""
     T = x.shape[0]
     E = slot_table.shape[0]
     st = lib().moe_expert_forward_fp8(ctypes.byref(pool), _p(slot_table), E, _p(x), T, _p(ids), k,
