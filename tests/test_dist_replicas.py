@@ -32,7 +32,7 @@ def _rank(rank, ws, port, out):
 
 def test_max_over_ranks_two_gloo_ranks():
     ws = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:        # no fork of this (threaded) process
         out = m.dict()
         mp.start_processes(_rank, args=(ws, _free_port(), out), nprocs=ws, start_method="spawn")
         res = dict(out)
